@@ -1,0 +1,53 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle checks.
+
+This module holds no arithmetic of the attention method: it only draws random numbers.
+Recipe (same for every workload): a torch Generator seeded with `seed` draws, in this
+order, q ~ N(0,1) [B,T,Hq,d], k ~ N(0,1) [B,T,Hkv,d], v ~ N(0,1) [B,T,Hkv,d] (only for
+layers with a separate value), then gamma_q = 1 + 0.1 N(0,1) [d] and
+gamma_k = 1 + 0.1 N(0,1) [d] in fp32.  q, k and v are rounded to bf16 (round to nearest
+even).  On the CPU the bytes are reproducible across machines; `device="cuda"` uses the
+CUDA generator instead (fast for the largest workloads, different bytes for the same seed).
+"""
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+
+@dataclass
+class LayerInputs:
+    q: torch.Tensor
+    k: torch.Tensor
+    v: Optional[torch.Tensor]
+    gamma_q: torch.Tensor
+    gamma_k: torch.Tensor
+
+
+def _randn(shape, gen, device):
+    return torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+
+
+def layer_inputs(B, T, n_q_heads, n_kv_heads, head_dim, separate_v, seed, device="cpu"):
+    gen = torch.Generator(device=device).manual_seed(int(seed))
+    q = _randn((B, T, n_q_heads, head_dim), gen, device).to(torch.bfloat16)
+    k = _randn((B, T, n_kv_heads, head_dim), gen, device).to(torch.bfloat16)
+    v = None
+    if separate_v:
+        v = _randn((B, T, n_kv_heads, head_dim), gen, device).to(torch.bfloat16)
+    gamma_q = 1.0 + 0.1 * _randn((head_dim,), gen, device)
+    gamma_k = 1.0 + 0.1 * _randn((head_dim,), gen, device)
+    return LayerInputs(q, k, v, gamma_q.contiguous(), gamma_k.contiguous())
+
+
+def decode_inputs(B, L, n_q_heads, n_kv_heads, head_dim, separate_v, seed, device="cpu"):
+    """A decode step: q [B,1,Hq,d] and a cache [B,L,Hkv,d] of N(0,1) bf16 values that is
+    used as if it already held normalised keys (the cache of the decode workload)."""
+    gen = torch.Generator(device=device).manual_seed(int(seed))
+    q = _randn((B, 1, n_q_heads, head_dim), gen, device).to(torch.bfloat16)
+    kcache = _randn((B, L, n_kv_heads, head_dim), gen, device).to(torch.bfloat16)
+    vcache = None
+    if separate_v:
+        vcache = _randn((B, L, n_kv_heads, head_dim), gen, device).to(torch.bfloat16)
+    gamma_q = 1.0 + 0.1 * _randn((head_dim,), gen, device)
+    gamma_k = 1.0 + 0.1 * _randn((head_dim,), gen, device)
+    return LayerInputs(q, kcache, vcache, gamma_q.contiguous(), gamma_k.contiguous())

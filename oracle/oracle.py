@@ -1,0 +1,174 @@
+"""ctypes front end of the fp64 CPU oracle (test infrastructure only).
+
+Inputs arrive as bf16 bit patterns (numpy uint16) or as torch bf16 CPU tensors; the C side
+widens them exactly to double.  Outputs are float64 numpy arrays.
+"""
+import ctypes
+import math
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [
+        ("n_q_heads", ctypes.c_int),
+        ("n_kv_heads", ctypes.c_int),
+        ("head_dim", ctypes.c_int),
+        ("rope_p", ctypes.c_double),
+        ("rope_base", ctypes.c_double),
+        ("window", ctypes.c_int),
+        ("scale", ctypes.c_double),
+        ("kv_is_k", ctypes.c_int),
+        ("qk_norm", ctypes.c_int),
+        ("qk_norm_eps", ctypes.c_double),
+    ]
+
+
+@dataclass
+class OracleCfg:
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    rope_p: float
+    rope_base: float
+    window: int = 0
+    scale: float = None
+    kv_is_k: int = 1
+    qk_norm: int = 1
+    qk_norm_eps: float = 1e-6
+
+    def c(self) -> _Cfg:
+        scale = self.scale if self.scale is not None else 1.0 / math.sqrt(self.head_dim)
+        return _Cfg(self.n_q_heads, self.n_kv_heads, self.head_dim, float(self.rope_p),
+                    float(self.rope_base), int(self.window), float(scale), int(self.kv_is_k),
+                    int(self.qk_norm), float(self.qk_norm_eps))
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        P = ctypes.c_void_p
+        lib.g4o_rope_pairs.argtypes = [ctypes.c_int, ctypes.c_double]
+        lib.g4o_rope_pairs.restype = ctypes.c_int
+        lib.g4o_rmsnorm.argtypes = [P, P, ctypes.c_int, ctypes.c_double, P]
+        lib.g4o_rmsnorm.restype = None
+        lib.g4o_rope.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+                                 ctypes.c_int64, P]
+        lib.g4o_rope.restype = None
+        lib.g4o_qknorm_rope.argtypes = [P, P, P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int64,
+                                        ctypes.POINTER(_Cfg), P, P, P]
+        lib.g4o_qknorm_rope.restype = ctypes.c_int
+        lib.g4o_prefill_rows.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                         ctypes.POINTER(_Cfg), P, ctypes.c_int, ctypes.c_int,
+                                         P, P]
+        lib.g4o_prefill_rows.restype = ctypes.c_int
+        lib.g4o_decode.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cfg),
+                                   P, ctypes.c_int, ctypes.c_int, P, P]
+        lib.g4o_decode.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def bf16_bits(x) -> np.ndarray:
+    """Return the bf16 bit patterns of a torch bf16 tensor (CPU) or pass uint16 through."""
+    if isinstance(x, np.ndarray):
+        assert x.dtype == np.uint16
+        return np.ascontiguousarray(x)
+    import torch
+    assert x.dtype == torch.bfloat16
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy()
+                                .view(np.uint16))
+
+
+def _f32(x):
+    if x is None:
+        return None
+    if not isinstance(x, np.ndarray):
+        x = x.detach().cpu().numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def rope_pairs(head_dim: int, p: float) -> int:
+    return _load().g4o_rope_pairs(head_dim, p)
+
+
+def rmsnorm(x: np.ndarray, gamma=None, eps: float = 1e-6) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    g = None if gamma is None else np.ascontiguousarray(gamma, dtype=np.float64)
+    y = np.empty_like(x)
+    _load().g4o_rmsnorm(_ptr(x), _ptr(g), x.shape[-1], eps, _ptr(y))
+    return y
+
+
+def rope(x: np.ndarray, R: int, base: float, pos: int) -> np.ndarray:
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    y = np.empty_like(x)
+    _load().g4o_rope(_ptr(x), x.shape[-1], R, base, pos, _ptr(y))
+    return y
+
+
+def qknorm_rope(q, k, gamma_q, gamma_k, cfg: OracleCfg, pos0: int = 0, want_krot=True):
+    """Returns (q_out, k_out, krot_out) as float64 arrays shaped like the inputs."""
+    qb = None if q is None else bf16_bits(q)
+    kb = None if k is None else bf16_bits(k)
+    ref = qb if qb is not None else kb
+    B, T = ref.shape[0], ref.shape[1]
+    qo = None if qb is None else np.empty(qb.shape, np.float64)
+    ko = None if kb is None else np.empty(kb.shape, np.float64)
+    kr = None if (kb is None or not want_krot) else np.empty(kb.shape, np.float64)
+    c = cfg.c()
+    rc = _load().g4o_qknorm_rope(_ptr(qb), _ptr(kb), _ptr(_f32(gamma_q)), _ptr(_f32(gamma_k)),
+                                 B, T, pos0, ctypes.byref(c), _ptr(qo), _ptr(ko), _ptr(kr))
+    if rc != 0:
+        raise ValueError("oracle qknorm_rope rejected its arguments (%d)" % rc)
+    return qo, ko, kr
+
+
+def prefill_rows(q, k, v, gamma_q, gamma_k, cfg: OracleCfg, rows=None, nthreads: int = 0):
+    """Attention output for query positions `rows` (all by default).
+
+    Returns (out [B, nrows, Hq, d], lse [B, Hq, nrows]) in float64."""
+    qb, kb = bf16_bits(q), bf16_bits(k)
+    vb = None if v is None else bf16_bits(v)
+    B, T = qb.shape[0], qb.shape[1]
+    if rows is None:
+        rows = np.arange(T, dtype=np.int32)
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    out = np.zeros((B, len(rows), cfg.n_q_heads, cfg.head_dim), np.float64)
+    lse = np.zeros((B, cfg.n_q_heads, len(rows)), np.float64)
+    c = cfg.c()
+    rc = _load().g4o_prefill_rows(_ptr(qb), _ptr(kb), _ptr(vb), _ptr(_f32(gamma_q)),
+                                  _ptr(_f32(gamma_k)), B, T, ctypes.byref(c), _ptr(rows),
+                                  len(rows), nthreads, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle prefill rejected its arguments (%d)" % rc)
+    return out, lse
+
+
+def decode(q, kcache, vcache, cfg: OracleCfg, items=None, nthreads: int = 0):
+    """One query per (b, h) at position L-1.  Returns (out [B, Hq, d], lse [B, Hq]).
+
+    `items` optionally restricts the work to b * Hkv + g entries (others stay NaN)."""
+    qb, kb = bf16_bits(q), bf16_bits(kcache)
+    vb = None if vcache is None else bf16_bits(vcache)
+    B, L = kb.shape[0], kb.shape[1]
+    out = np.full((B, cfg.n_q_heads, cfg.head_dim), np.nan)
+    lse = np.full((B, cfg.n_q_heads), np.nan)
+    it = None if items is None else np.ascontiguousarray(items, dtype=np.int32)
+    c = cfg.c()
+    rc = _load().g4o_decode(_ptr(qb), _ptr(kb), _ptr(vb), B, L, ctypes.byref(c), _ptr(it),
+                            0 if it is None else len(it), nthreads, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle decode rejected its arguments (%d)" % rc)
+    return out, lse

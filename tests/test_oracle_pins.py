@@ -1,0 +1,334 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself:
+the pages' worked example (4-token sliding window), closed forms (textbook complex RoPE,
+RMS of a constant vector, the two-key logistic softmax, uniform attention when q = 0),
+invariants (relative-position dependence of RoPE scores, norm preservation, head
+repetition for GQA) and a second, unblocked formulation on tiny inputs.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import bruteforce as bf
+import oracle
+from oracle import OracleCfg
+from attention_g4attn_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _bits(t):
+    return oracle.bf16_bits(t)
+
+
+# ----------------------------------------------------------------------------- RoPE
+
+def test_rope_pairs_match_pages():
+    for case in _golden("prope_rotated_pairs.json")["cases"]:
+        d, p = case["head_dim"], case["p"]
+        R = oracle.rope_pairs(d, p)
+        assert R == case["R"]
+        # which dims move: rotate a vector of ones at a large position and compare
+        x = np.ones(d)
+        y = oracle.rope(x, R, 1e4, 7)
+        moved = np.nonzero(np.abs(y - x) > 1e-12)[0]
+        want = [c for lo, hi in case["rotated_dims"] for c in range(lo, hi)]
+        # pair 0 turns by 7 rad at theta 1, every rotated pair moves for this input
+        assert sorted(moved.tolist()) == want
+        assert len(want) / d == pytest.approx(case["fraction_of_dims"])
+
+
+def test_rope_frequencies_golden():
+    for case in _golden("rope_frequencies.json")["cases"]:
+        d, base = case["head_dim"], case["base"]
+        half = d // 2
+        for i, th in enumerate(case["theta"]):
+            e = np.zeros(d)
+            e[i] = 1.0
+            y = oracle.rope(e, half, base, 1)
+            # unit vector on the first slot of pair i turns by angle theta_i
+            assert y[i] == pytest.approx(math.cos(th), abs=1e-15)
+            assert y[i + half] == pytest.approx(math.sin(th), abs=1e-15)
+
+
+@pytest.mark.parametrize("d,base", [(8, 1e4), (64, 1e6), (512, 1e6), (256, 1e4)])
+def test_full_rope_equals_textbook_complex_rotation(d, base):
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal(d)
+    for pos in (0, 1, 5, 1000, 131071):
+        y = oracle.rope(x, d // 2, base, pos)
+        want = bf.rope_complex(x[None, None, :], np.array([pos]), d // 2, base)[0, 0]
+        # fp64 angles of size pos carry ~pos * 2^-52 rad of rounding on either side
+        np.testing.assert_allclose(y, want, rtol=0, atol=1e-13 * max(1, pos))
+
+
+def test_rope_p0_is_identity():
+    x = np.random.default_rng(2).standard_normal(512)
+    R = oracle.rope_pairs(512, 0.0)
+    assert R == 0
+    np.testing.assert_array_equal(oracle.rope(x, R, 1e6, 12345), x)
+
+
+@pytest.mark.parametrize("p", [0.25, 1.0])
+def test_rope_score_depends_only_on_offset(p):
+    rng = np.random.default_rng(3)
+    d = 64
+    R = oracle.rope_pairs(d, p)
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    for m, n in [(10, 3), (100, 99), (7, 7), (5000, 17)]:
+        ref = oracle.rope(q, R, 1e4, m) @ oracle.rope(k, R, 1e4, n)
+        for shift in (1, 37, 4096):
+            got = oracle.rope(q, R, 1e4, m + shift) @ oracle.rope(k, R, 1e4, n + shift)
+            assert got == pytest.approx(ref, abs=1e-9)
+
+
+def test_rope_preserves_pair_norms():
+    rng = np.random.default_rng(4)
+    d = 512
+    x = rng.standard_normal(d)
+    y = oracle.rope(x, 64, 1e6, 31337)
+    half = d // 2
+    np.testing.assert_allclose(x[:half] ** 2 + x[half:] ** 2, y[:half] ** 2 + y[half:] ** 2,
+                               rtol=1e-13)
+
+
+def test_rope_turns_counterclockwise():
+    # (1, 0) at angle phi goes to (cos phi, sin phi): the (cos -sin; sin cos) reading
+    e = np.array([1.0, 0.0])
+    y = oracle.rope(e, 1, 1e4, 1)
+    assert y[0] == pytest.approx(math.cos(1.0), abs=1e-15)
+    assert y[1] == pytest.approx(math.sin(1.0), abs=1e-15)
+
+
+# ----------------------------------------------------------------------------- RMSNorm
+
+def test_rmsnorm_constant_vector_closed_form():
+    d, c, eps = 16, -3.0, 1e-6
+    gamma = np.linspace(0.5, 2.0, d)
+    y = oracle.rmsnorm(np.full(d, c), gamma, eps)
+    np.testing.assert_allclose(y, gamma * c / math.sqrt(c * c + eps), rtol=1e-15)
+
+
+def test_rmsnorm_unit_rms_and_scale_invariance():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal(512) * 7.0
+    y = oracle.rmsnorm(x, None, 0.0)
+    assert math.sqrt(np.mean(y * y)) == pytest.approx(1.0, abs=1e-14)
+    np.testing.assert_allclose(oracle.rmsnorm(x * 1000.0, None, 0.0), y, rtol=1e-13)
+
+
+def test_rmsnorm_zero_vector_stays_zero():
+    y = oracle.rmsnorm(np.zeros(8), np.ones(8), 1e-6)
+    np.testing.assert_array_equal(y, np.zeros(8))
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _cfg(Hq, Hkv, d, p=0.25, base=1e6, window=0, kv_is_k=1, qk_norm=1, scale=None):
+    return OracleCfg(Hq, Hkv, d, p, base, window, scale, kv_is_k, qk_norm, 1e-6)
+
+
+def test_window_toy_example_support():
+    g = _golden("window_toy_w4.json")
+    T, W = g["T"], g["window"]
+    d = T
+    q = torch.zeros(1, T, 1, d, dtype=torch.bfloat16)          # q = 0: uniform weights
+    k = torch.randn(1, T, 1, d, generator=torch.Generator().manual_seed(0)).bfloat16()
+    v = torch.eye(T, dtype=torch.bfloat16).reshape(1, T, 1, d)  # v_j = e_j
+    out, lse = oracle.prefill_rows(q, k, v, None, None, _cfg(1, 1, d, p=1.0, base=1e4,
+                                                             window=W, kv_is_k=0))
+    for i, vis in enumerate(g["visible"]):
+        want = np.zeros(d)
+        want[vis] = 1.0 / len(vis)
+        np.testing.assert_allclose(out[0, i, 0], want, atol=1e-15)
+        assert lse[0, 0, i] == pytest.approx(math.log(len(vis)), abs=1e-14)
+
+
+def test_causal_support_and_uniform_mean():
+    T, d = 12, 16
+    gen = torch.Generator().manual_seed(6)
+    q = torch.zeros(2, T, 4, d, dtype=torch.bfloat16)
+    k = torch.randn(2, T, 2, d, generator=gen).bfloat16()
+    v = torch.randn(2, T, 2, d, generator=gen).bfloat16()
+    out, lse = oracle.prefill_rows(q, k, v, None, None, _cfg(4, 2, d, kv_is_k=0))
+    vf = v.double().numpy()
+    for b in range(2):
+        for h in range(4):
+            for i in range(T):
+                want = vf[b, :i + 1, h // 2].mean(axis=0)
+                np.testing.assert_allclose(out[b, i, h], want, atol=1e-13)
+                assert lse[b, h, i] == pytest.approx(math.log(i + 1), abs=1e-13)
+
+
+def test_two_key_logistic_closed_form():
+    # T=2, no norm, no rotation: row 1 scores [0, scale*a] -> weight sigma(scale*a) on v_1
+    a, scale = 2.0, 0.75
+    q = torch.tensor([[[[0.0, 0.0]]], [[[a, 0.0]]]]).reshape(1, 2, 1, 2).bfloat16()
+    k = torch.tensor([[0.0, 0.0], [1.0, 0.0]]).reshape(1, 2, 1, 2).bfloat16()
+    v = torch.tensor([[0.0, 0.0], [1.0, -2.0]]).reshape(1, 2, 1, 2).bfloat16()
+    cfg = _cfg(1, 1, 2, p=0.0, kv_is_k=0, qk_norm=0, scale=scale)
+    out, lse = oracle.prefill_rows(q, k, v, None, None, cfg)
+    sig = 1.0 / (1.0 + math.exp(-scale * a))
+    np.testing.assert_allclose(out[0, 1, 0], [sig, -2.0 * sig], rtol=1e-14)
+    assert lse[0, 0, 1] == pytest.approx(math.log1p(math.exp(scale * a)), rel=1e-14)
+
+
+def test_single_token_returns_its_value():
+    gen = torch.Generator().manual_seed(7)
+    q = torch.randn(1, 1, 8, 512, generator=gen).bfloat16()
+    k = torch.randn(1, 1, 1, 512, generator=gen).bfloat16()
+    gk = 1 + 0.1 * torch.randn(512, generator=gen)
+    out, lse = oracle.prefill_rows(q, k, None, None, gk, _cfg(8, 1, 512))
+    khat = bf.rms(bf.bf16_to_f64(oracle.bf16_bits(k))[0, 0, 0], gk.double().numpy(), 1e-6)
+    for h in range(8):
+        np.testing.assert_allclose(out[0, 0, h], khat, rtol=1e-13, atol=1e-15)
+
+
+def test_window_at_least_T_equals_global_causal():
+    inp = synth.layer_inputs(1, 40, 4, 2, 64, True, seed=8)
+    c0 = _cfg(4, 2, 64, p=1.0, base=1e4, window=0, kv_is_k=0)
+    cw = _cfg(4, 2, 64, p=1.0, base=1e4, window=40, kv_is_k=0)
+    cbig = _cfg(4, 2, 64, p=1.0, base=1e4, window=1000, kv_is_k=0)
+    o0, l0 = oracle.prefill_rows(inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, c0)
+    for c in (cw, cbig):
+        o, l = oracle.prefill_rows(inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, c)
+        np.testing.assert_array_equal(o, o0)
+        np.testing.assert_array_equal(l, l0)
+
+
+@pytest.mark.parametrize("kv_is_k", [0, 1, 2])
+def test_gqa_equals_repeated_kv_heads(kv_is_k):
+    Hq, Hkv, G = 8, 2, 4
+    inp = synth.layer_inputs(2, 20, Hq, Hkv, 32, kv_is_k == 0, seed=9)
+    k_rep = inp.k.repeat_interleave(G, dim=2)      # kv head of query head h is h // G
+    v_rep = None if inp.v is None else inp.v.repeat_interleave(G, dim=2)
+    a = oracle.prefill_rows(inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k,
+                            _cfg(Hq, Hkv, 32, kv_is_k=kv_is_k))
+    b = oracle.prefill_rows(inp.q, k_rep, v_rep, inp.gamma_q, inp.gamma_k,
+                            _cfg(Hq, Hq, 32, kv_is_k=kv_is_k))
+    np.testing.assert_allclose(a[0], b[0], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(a[1], b[1], rtol=0, atol=1e-14)
+
+
+def test_keys_as_values_equals_supplied_values():
+    # without QKNorm the normalised key is the raw key, so kv_is_k=1 must equal v := k
+    inp = synth.layer_inputs(1, 24, 8, 1, 64, False, seed=10)
+    a = oracle.prefill_rows(inp.q, inp.k, None, None, None, _cfg(8, 1, 64, qk_norm=0))
+    b = oracle.prefill_rows(inp.q, inp.k, inp.k, None, None,
+                            _cfg(8, 1, 64, qk_norm=0, kv_is_k=0))
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+CASES = [
+    dict(Hq=8, Hkv=1, d=64, p=0.25, base=1e6, window=0, kv_is_k=1),
+    dict(Hq=4, Hkv=2, d=32, p=1.0, base=1e4, window=5, kv_is_k=0),
+    dict(Hq=4, Hkv=4, d=16, p=0.5, base=1e4, window=0, kv_is_k=2),
+    dict(Hq=6, Hkv=3, d=24, p=0.25, base=1e6, window=3, kv_is_k=1),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+@pytest.mark.parametrize("T", [1, 2, 7, 16])
+def test_oracle_equals_bruteforce(case, T):
+    inp = synth.layer_inputs(2, T, case["Hq"], case["Hkv"], case["d"], case["kv_is_k"] == 0,
+                             seed=11 + T)
+    scale = 1.0 / math.sqrt(case["d"])
+    cfg = _cfg(case["Hq"], case["Hkv"], case["d"], case["p"], case["base"], case["window"],
+               case["kv_is_k"])
+    out, lse = oracle.prefill_rows(inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, cfg)
+    vb = None if inp.v is None else _bits(inp.v)
+    bo, bl = bf.attention(_bits(inp.q), _bits(inp.k), vb, inp.gamma_q.double().numpy(),
+                          inp.gamma_k.double().numpy(), case["Hq"], case["Hkv"], case["d"],
+                          case["p"], case["base"], case["window"], scale, case["kv_is_k"])
+    np.testing.assert_allclose(out, bo, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, bl, rtol=0, atol=1e-12)
+
+
+def test_row_subset_matches_full_run():
+    inp = synth.layer_inputs(1, 33, 8, 1, 64, False, seed=12)
+    cfg = _cfg(8, 1, 64)
+    full, lf = oracle.prefill_rows(inp.q, inp.k, None, inp.gamma_q, inp.gamma_k, cfg)
+    rows = np.array([32, 0, 17], np.int32)
+    sub, ls = oracle.prefill_rows(inp.q, inp.k, None, inp.gamma_q, inp.gamma_k, cfg, rows)
+    np.testing.assert_array_equal(sub, full[:, rows])
+    np.testing.assert_array_equal(ls, lf[:, :, rows])
+
+
+# ----------------------------------------------------------------------------- prologue
+
+def test_qknorm_rope_matches_bruteforce():
+    inp = synth.layer_inputs(2, 9, 8, 2, 64, False, seed=13)
+    cfg = _cfg(8, 2, 64, p=0.25, base=1e6)
+    qo, ko, kr = oracle.qknorm_rope(inp.q, inp.k, inp.gamma_q, inp.gamma_k, cfg, pos0=5)
+    pos = np.arange(5, 14)
+    qh = bf.rms(bf.bf16_to_f64(_bits(inp.q)), inp.gamma_q.double().numpy(), 1e-6)
+    kh = bf.rms(bf.bf16_to_f64(_bits(inp.k)), inp.gamma_k.double().numpy(), 1e-6)
+    np.testing.assert_allclose(qo, bf.rope_complex(qh, pos, 8, 1e6), atol=1e-13)
+    np.testing.assert_allclose(ko, kh, atol=1e-14)
+    np.testing.assert_allclose(kr, bf.rope_complex(kh, pos, 8, 1e6), atol=1e-13)
+
+
+# ----------------------------------------------------------------------------- decode
+
+def test_decode_equals_last_prefill_row_exactly_without_norm_or_rotation():
+    inp = synth.layer_inputs(2, 30, 8, 2, 64, False, seed=14)
+    cfg = _cfg(8, 2, 64, p=0.0, qk_norm=0)
+    out, lse = oracle.prefill_rows(inp.q, inp.k, None, None, None, cfg,
+                                   np.array([29], np.int32))
+    dq = inp.q[:, 29]                                        # [B, Hq, d]
+    dout, dlse = oracle.decode(dq, inp.k, None, cfg)
+    np.testing.assert_allclose(dout, out[:, 0], rtol=0, atol=1e-14)
+    np.testing.assert_allclose(dlse, lse[:, :, 0], rtol=0, atol=1e-13)
+
+
+@pytest.mark.parametrize("kv_is_k", [0, 1, 2])
+def test_decode_matches_bruteforce_with_rotation(kv_is_k):
+    B, L, Hq, Hkv, d = 2, 21, 8, 2, 64
+    dec = synth.decode_inputs(B, L, Hq, Hkv, d, kv_is_k == 0, seed=15)
+    cfg = _cfg(Hq, Hkv, d, p=0.25, base=1e6, kv_is_k=kv_is_k)
+    out, lse = oracle.decode(dec.q[:, 0], dec.k, dec.v, cfg)
+    # brute force: rotate the bf16 query back to "unrotated" is not needed: compare with
+    # an explicit score computation against keys rotated by position (complex form)
+    R = oracle.rope_pairs(d, 0.25)
+    kf = bf.bf16_to_f64(_bits(dec.k))
+    kr = bf.rope_complex(kf, np.arange(L), R, 1e6)
+    vals = {1: kf, 2: kr, 0: None}[kv_is_k]
+    if vals is None:
+        vals = bf.bf16_to_f64(_bits(dec.v))
+    qf = bf.bf16_to_f64(_bits(dec.q))[:, 0]
+    G = Hq // Hkv
+    for b in range(B):
+        for h in range(Hq):
+            s = (kr[b, :, h // G] @ qf[b, h]) / math.sqrt(d)
+            w = np.exp(s - s.max())
+            np.testing.assert_allclose(out[b, h], (w / w.sum()) @ vals[b, :, h // G],
+                                       atol=1e-13)
+            assert lse[b, h] == pytest.approx(s.max() + math.log(w.sum()), abs=1e-12)
+
+
+def test_decode_item_subset():
+    dec = synth.decode_inputs(3, 17, 8, 2, 32, False, seed=16)
+    cfg = _cfg(8, 2, 32)
+    full, _ = oracle.decode(dec.q[:, 0], dec.k, None, cfg)
+    part, _ = oracle.decode(dec.q[:, 0], dec.k, None, cfg, items=[5, 0])
+    for item in (5, 0):
+        b, g = divmod(item, 2)
+        np.testing.assert_array_equal(part[b, g * 4:(g + 1) * 4], full[b, g * 4:(g + 1) * 4])
+    assert np.isnan(part[1, 0]).all()
+
+
+def test_invalid_arguments_rejected():
+    inp = synth.layer_inputs(1, 4, 6, 4, 8, True, seed=17)
+    with pytest.raises(ValueError):   # Hq % Hkv != 0
+        oracle.prefill_rows(inp.q, inp.k, inp.v, None, None, _cfg(6, 4, 8, kv_is_k=0))
+    with pytest.raises(ValueError):   # separate values requested but none given
+        oracle.prefill_rows(inp.q, inp.k, None, None, None, _cfg(6, 6, 8, kv_is_k=0))
