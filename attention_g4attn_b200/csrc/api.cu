@@ -1,0 +1,390 @@
+// api.cu -- the C ABI of g4attn: argument validation, workspace layout, TMA tensor-map
+// encoding and stream-ordered launches.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "g4attn.h"
+#include "kernels.h"
+
+namespace {
+
+__device__ int g_device_status = 0;   // written by bounded waits that give up
+
+constexpr long long kDefaultWaitLimit = 1LL << 62;   // polls; the 2 s time bound rules
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+    bool probed = false;
+    bool supported = false;
+    int sms = 0;
+    int* status = nullptr;   // device address of g_device_status
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+// Probe the current device once: compute capability 10.0, SM count, status word address.
+int current_device(DeviceInfo** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return G4ATTN_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.probed) {
+        d.probed = true;
+        int major = 0, minor = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        d.supported = (major == 10 && minor == 0);
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
+            cudaGetLastError();
+            d.supported = false;
+        }
+        d.status = static_cast<int*>(p);
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                    cudaSuccess &&
+                q == cudaDriverEntryPointSuccess)
+                g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+            else
+                cudaGetLastError();
+        }
+        if (!g_encode) d.supported = false;
+    }
+    if (!d.supported) return G4ATTN_ERR_UNSUPPORTED;
+    *out = &d;
+    return G4ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int rope_pairs(const g4attn_layer_cfg* c) {
+    double r = std::floor((double)c->rope_p * (double)c->head_dim / 2.0);
+    if (r < 0) r = 0;
+    if (r > c->head_dim / 2) r = c->head_dim / 2;
+    return (int)r;
+}
+
+bool chunk_rotated(int c, int d, int R) {
+    const int lo = c * 64, hi = lo + 64, h = d / 2;
+    return (lo < R) || (lo < h + R && hi > h);
+}
+
+// Configuration checks shared by every entry point.
+int check_cfg(const g4attn_layer_cfg* c, bool tensor_core_path) {
+    if (!c) return G4ATTN_ERR_INVALID_ARG;
+    if (c->n_q_heads <= 0 || c->n_kv_heads <= 0 || c->n_q_heads % c->n_kv_heads != 0)
+        return G4ATTN_ERR_INVALID_ARG;
+    if (c->head_dim <= 0 || (c->head_dim & 1)) return G4ATTN_ERR_INVALID_ARG;
+    if (!(c->rope_p >= 0.f && c->rope_p <= 1.f)) return G4ATTN_ERR_INVALID_ARG;
+    if (!(c->rope_base > 0.0) || !std::isfinite(c->rope_base)) return G4ATTN_ERR_INVALID_ARG;
+    if (c->window < 0) return G4ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(c->scale)) return G4ATTN_ERR_INVALID_ARG;
+    if (c->kv_is_k < 0 || c->kv_is_k > 2) return G4ATTN_ERR_INVALID_ARG;
+    if (c->qk_norm != 0 && c->qk_norm != 1) return G4ATTN_ERR_INVALID_ARG;
+    if (c->qk_norm && !(c->qk_norm_eps >= 0.f)) return G4ATTN_ERR_INVALID_ARG;
+    if (tensor_core_path) {
+        if (c->head_dim != 256 && c->head_dim != 512) return G4ATTN_ERR_UNSUPPORTED;
+        const int G = c->n_q_heads / c->n_kv_heads;
+        if (128 % G != 0) return G4ATTN_ERR_UNSUPPORTED;
+    } else if (c->head_dim != 128 && c->head_dim != 256 && c->head_dim != 512) {
+        return G4ATTN_ERR_UNSUPPORTED;
+    }
+    return G4ATTN_OK;
+}
+
+// 4-D map over a [B, T, H, d] bf16 tensor: dims (d, H, T, B), box (64, 1, 128, 1),
+// 128-byte swizzle, zero fill outside the tensor.
+int encode_rows(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? G4ATTN_OK : G4ATTN_ERR_CUDA;
+}
+
+struct PrefillWs {
+    size_t kn_off, kr_off, cs_off, total;
+    bool need_kn;
+};
+
+PrefillWs prefill_ws(int B, int T, const g4attn_layer_cfg* c) {
+    PrefillWs w{};
+    const int d = c->head_dim, R = rope_pairs(c);
+    bool any_plain = false;
+    for (int ch = 0; ch < d / 64; ++ch) any_plain |= !chunk_rotated(ch, d, R);
+    w.need_kn = any_plain || c->kv_is_k == 1;
+    const size_t rows = (size_t)B * T * c->n_kv_heads * d * 2;
+    w.kn_off = 0;
+    w.kr_off = w.need_kn ? align256(rows) : 0;
+    w.cs_off = w.kr_off + align256(rows);
+    w.total = w.cs_off + align256((size_t)T * (R > 0 ? R : 1) * sizeof(float2));
+    return w;
+}
+
+struct DecodePlan {
+    int key_lo, splits, keys_per_split;
+    size_t o_off, ml_off, total;
+};
+
+DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms) {
+    DecodePlan p{};
+    p.key_lo = (c->window > 0 && L > c->window) ? L - c->window : 0;
+    const int len = L - p.key_lo;
+    const int tiles = (len + 127) / 128;
+    const int nbg = B * c->n_kv_heads;
+    int S = 1;
+    if (tiles > 0 && nbg > 0) {
+        // enough items that every SM holds the same number of them
+        int a = nbg, b = sms > 0 ? sms : 148;
+        while (b) { int t = a % b; a = b; b = t; }
+        const int base = (sms > 0 ? sms : 148) / a;
+        S = base;
+        while (S > tiles) S = (S + 1) / 2;
+        if (S < 1) S = 1;
+    }
+    const int tps = tiles > 0 ? (tiles + S - 1) / S : 1;
+    p.keys_per_split = tps * 128;
+    p.splits = len > 0 ? (len + p.keys_per_split - 1) / p.keys_per_split : 0;
+    const size_t n = (size_t)(p.splits > 0 ? p.splits : 1) * B * c->n_q_heads;
+    p.o_off = 0;
+    p.ml_off = align256(n * c->head_dim * sizeof(float));
+    p.total = p.ml_off + align256(n * 2 * sizeof(float));
+    return p;
+}
+
+g4::Rope make_rope(const g4attn_layer_cfg* c) {
+    g4::Rope r;
+    r.R = rope_pairs(c);
+    r.log2_base = std::log2(c->rope_base);
+    return r;
+}
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return G4ATTN_OK;
+    cudaGetLastError();
+    return G4ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* g4attn_version(void) { return "g4attn 0.1 (sm_100a)"; }
+
+const char* g4attn_status_string(int s) {
+    switch (s) {
+        case G4ATTN_OK: return "ok";
+        case G4ATTN_ERR_INVALID_ARG: return "invalid argument";
+        case G4ATTN_ERR_UNSUPPORTED: return "unsupported configuration or device";
+        case G4ATTN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case G4ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+        case G4ATTN_ERR_CUDA: return "CUDA error";
+        case G4ATTN_ERR_TIMEOUT: return "device wait timed out";
+        default: return "unknown status";
+    }
+}
+
+long long g4attn_set_wait_limit(long long polls) {
+    return g_wait_limit.exchange(polls < 1 ? kDefaultWaitLimit : polls);
+}
+
+int g4attn_device_status(g4attn_stream_t stream) {
+    DeviceInfo* dev = nullptr;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(st) != cudaSuccess) return cuda_status(cudaErrorUnknown);
+    int v = 0;
+    if (cudaMemcpy(&v, dev->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return cuda_status(cudaErrorUnknown);
+    const int zero = 0;
+    if (cudaMemcpy(dev->status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+        return cuda_status(cudaErrorUnknown);
+    return v;
+}
+
+int g4attn_qknorm_rope(const g4attn_bf16* q_in, const g4attn_bf16* k_in, g4attn_bf16* q_out,
+                       g4attn_bf16* kcache_out, g4attn_bf16* krot_out, const float* gamma_q,
+                       const float* gamma_k, int B, int T, long long pos0,
+                       const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
+    int rc = check_cfg(cfg, false);
+    if (rc) return rc;
+    if (B < 0 || T < 0 || pos0 < 0) return G4ATTN_ERR_INVALID_ARG;
+    if ((q_in && !q_out) || (k_in && !kcache_out && !krot_out)) return G4ATTN_ERR_INVALID_ARG;
+    if (cfg->qk_norm && ((q_in && !gamma_q) || (k_in && !gamma_k))) return G4ATTN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q_in, k_in, q_out, kcache_out, krot_out, gamma_q, gamma_k};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;
+    if ((long long)B * T == 0 || (!q_in && !k_in)) return G4ATTN_OK;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    g4::QkNormRopeArgs a{};
+    a.q_in = q_in;
+    a.k_in = k_in;
+    a.q_out = q_out;
+    a.k_out = k_in ? kcache_out : nullptr;
+    a.krot_out = k_in ? krot_out : nullptr;
+    a.gamma_q = gamma_q;
+    a.gamma_k = gamma_k;
+    a.cs_out = nullptr;
+    a.B = B; a.T = T; a.Hq = cfg->n_q_heads; a.Hkv = cfg->n_kv_heads; a.d = cfg->head_dim;
+    a.pos0 = pos0;
+    a.rope = make_rope(cfg);
+    a.qk_norm = cfg->qk_norm;
+    a.eps = cfg->qk_norm_eps;
+    return cuda_status(g4::launch_qknorm_rope(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t g4attn_prefill_workspace_size(int B, int T, const g4attn_layer_cfg* cfg) {
+    if (check_cfg(cfg, true) || B < 0 || T < 0) return 0;
+    return prefill_ws(B, T, cfg).total;
+}
+
+int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16* v,
+                   const float* gamma_q, const float* gamma_k, g4attn_bf16* out, float* lse,
+                   void* workspace, size_t ws_bytes, int B, int T, const g4attn_layer_cfg* cfg,
+                   g4attn_stream_t stream) {
+    int rc = check_cfg(cfg, true);
+    if (rc) return rc;
+    if (B < 0 || T < 0) return G4ATTN_ERR_INVALID_ARG;
+    if ((long long)B * T == 0) return G4ATTN_OK;
+    if (!q || !k || !out) return G4ATTN_ERR_INVALID_ARG;
+    if ((cfg->kv_is_k == 0) != (v != nullptr)) return G4ATTN_ERR_INVALID_ARG;
+    if (cfg->qk_norm && (!gamma_q || !gamma_k)) return G4ATTN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, gamma_q, gamma_k, out, lse};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;
+    const PrefillWs ws = prefill_ws(B, T, cfg);
+    if (!workspace || ws_bytes < ws.total) return G4ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    uint16_t* kn = ws.need_kn ? reinterpret_cast<uint16_t*>(w + ws.kn_off) : nullptr;
+    uint16_t* kr = reinterpret_cast<uint16_t*>(w + ws.kr_off);
+    float2* cs = reinterpret_cast<float2*>(w + ws.cs_off);
+    const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
+
+    // 1) normalise the keys once: pre-RoPE copy (the K(=V) cache) and the rotated copy,
+    //    plus the (cos, sin) table of every position for the query prologue
+    g4::QkNormRopeArgs ka{};
+    ka.k_in = k;
+    ka.k_out = kn;
+    ka.krot_out = kr;
+    ka.gamma_k = gamma_k;
+    ka.cs_out = cs;
+    ka.B = B; ka.T = T; ka.Hq = cfg->n_q_heads; ka.Hkv = Hkv; ka.d = d;
+    ka.pos0 = 0;
+    ka.rope = make_rope(cfg);
+    ka.qk_norm = cfg->qk_norm;
+    ka.eps = cfg->qk_norm_eps;
+    if ((rc = cuda_status(g4::launch_qknorm_rope(ka, st)))) return rc;
+
+    // 2) the fused flash-attention kernel
+    g4::PrefillArgs a{};
+    if ((rc = encode_rows(&a.tm_kr, kr, B, T, Hkv, d))) return rc;
+    if ((rc = encode_rows(&a.tm_kn, kn ? kn : kr, B, T, Hkv, d))) return rc;
+    if ((rc = encode_rows(&a.tm_v, v ? v : (kn ? kn : kr), B, T, Hkv, d))) return rc;
+    a.q = q;
+    a.gamma_q = gamma_q;
+    a.rope_cs = cs;
+    a.out = out;
+    a.lse = lse;
+    a.B = B; a.T = T; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d;
+    a.G = cfg->n_q_heads / Hkv;
+    a.window = cfg->window;
+    a.rope = make_rope(cfg);
+    a.qk_norm = cfg->qk_norm;
+    a.eps = cfg->qk_norm_eps;
+    a.scale_log2 = cfg->scale * 1.4426950408889634f;
+    a.kv_is_k = cfg->kv_is_k;
+    a.wait_limit = g_wait_limit.load();
+    a.status = dev->status;
+    return cuda_status(g4::launch_prefill(a, st));
+}
+
+size_t g4attn_decode_workspace_size(int B, int L, const g4attn_layer_cfg* cfg) {
+    if (check_cfg(cfg, true) || B < 0 || L < 0) return 0;
+    DeviceInfo* dev = nullptr;
+    int sms = 148;
+    if (current_device(&dev) == G4ATTN_OK) sms = dev->sms;
+    else cudaGetLastError();
+    return decode_plan(B, L, cfg, sms).total;
+}
+
+int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_bf16* vcache,
+                  int L, g4attn_bf16* out, float* lse, void* workspace, size_t ws_bytes, int B,
+                  const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
+    int rc = check_cfg(cfg, true);
+    if (rc) return rc;
+    if (B < 0 || L < 0) return G4ATTN_ERR_INVALID_ARG;
+    if (B == 0) return G4ATTN_OK;
+    if (!q || !out || (L > 0 && !kcache)) return G4ATTN_ERR_INVALID_ARG;
+    if ((cfg->kv_is_k == 0) != (vcache != nullptr)) return G4ATTN_ERR_INVALID_ARG;
+    const int G = cfg->n_q_heads / cfg->n_kv_heads;
+    if (G > 16) return G4ATTN_ERR_UNSUPPORTED;
+    const int R = rope_pairs(cfg);
+    if (cfg->kv_is_k == 1) {   // side buffers for the turned copy of at most two chunks
+        int n = 0;
+        for (int c = 0; c < cfg->head_dim / 64; ++c) n += chunk_rotated(c, cfg->head_dim, R);
+        if (n > 2) return G4ATTN_ERR_UNSUPPORTED;
+    }
+    const void* ptrs[] = {q, kcache, vcache, out, lse};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    const DecodePlan plan = decode_plan(B, L, cfg, dev->sms);
+    if (!workspace || ws_bytes < plan.total) return G4ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    g4::DecodeArgs a{};
+    const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
+    if (L > 0) {
+        if ((rc = encode_rows(&a.tm_k, kcache, B, L, Hkv, d))) return rc;
+        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, L, Hkv, d))) return rc;
+    }
+    a.q = q;
+    a.part_o = reinterpret_cast<float*>(w + plan.o_off);
+    a.part_ml = reinterpret_cast<float*>(w + plan.ml_off);
+    a.out = out;
+    a.lse = lse;
+    a.B = B; a.L = L; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d; a.G = G;
+    a.key_lo = plan.key_lo;
+    a.splits = plan.splits;
+    a.keys_per_split = plan.keys_per_split;
+    a.rope = make_rope(cfg);
+    a.scale_log2 = cfg->scale * 1.4426950408889634f;
+    a.kv_is_k = cfg->kv_is_k;
+    a.wait_limit = g_wait_limit.load();
+    a.status = dev->status;
+    return cuda_status(g4::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

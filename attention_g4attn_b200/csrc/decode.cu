@@ -1,0 +1,505 @@
+// decode.cu -- split-KV flash decoding for one new token per sequence against a bf16
+// K(=V) cache, on the 5th-generation tensor core (tcgen05) with TMA-fed shared memory.
+//
+// Work item = (split s, kv head g, batch b): keys [k0, k1) of one sequence and all G query
+// heads that share kv head g (GQA; explainer "GQA": 8 query heads per KV head in global
+// layers).  Per tile of 128 keys:
+//   S^T[key, head]  = K_tile . Q^T         M = 128 keys, N = 16 (heads, zero padded), K = d
+//   O^T[d, head]   += K_tile^T . P^T        M = 128 d-rows per chunk, N = 16, K = 128 keys
+// Keys sit on the MMA's M side, so one 128-key tile in shared memory is the K operand of
+// the first product and, read MN-major, the V operand of the second (keys reused as
+// values, report section 2 / explainer "K=V": one cache read serves both).  The cache
+// holds pre-RoPE keys; the rotated pairs (i, i + d/2), i < R, of every key are turned to
+// the key's position on the fly (report section 2, p-RoPE) by the softmax warps, into a
+// side buffer when the values are the pre-RoPE keys, in place otherwise.
+//
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// warps 2..5 rotation / softmax / epilogue (thread = TMEM lane = key row or d-row).
+// The CTA is persistent over work items blockIdx.x, +gridDim.x, ...  Every mbarrier wait
+// is bounded (sm100.cuh); on a timeout all roles drain their in-flight work and exit.
+#include <cuda_bf16.h>
+
+#include "kernels.h"
+#include "rope.cuh"
+#include "sm100.cuh"
+
+namespace g4 {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kTileKeys = 128;
+constexpr int kNSlots = 5;           // ring of 32 KB slots: 128 keys x 128 dims (2 chunks)
+constexpr int kSlotBytes = 32768;
+constexpr int kChunkBytes = 16384;   // 128 keys x 64 dims, 128-byte swizzled rows
+constexpr int kMaxRotChunks = 2;     // side buffers when values are the pre-RoPE keys
+constexpr int kN = 16;               // MMA N: query heads of one KV head, zero padded
+constexpr uint32_t kTmemCols = 128;
+constexpr int kBarWG = 1;            // named barrier of the softmax warpgroup
+
+struct __align__(1024) DecodeSmem {
+    uint8_t ring[kNSlots][kSlotBytes];
+    uint8_t rot[kMaxRotChunks][kChunkBytes];
+    uint8_t q[8][kN * 128];          // B operand of S^T: per 64-dim chunk, 16 rows x 128 B
+    uint8_t p[2][kN * 128];          // B operand of O^T: P^T, K-major, 2 chunks of 64 keys
+    float theta[256];                // base^(-2i/d) in fp32, i < R
+    float2 base_cs[256];             // cos/sin of tile_start * theta_i (fp64-reduced angle)
+    float red[4][kN];                // cross-warp reductions
+    uint64_t full[kNSlots];
+    uint64_t empty[kNSlots];
+    uint64_t s_full, p_full, rot_ready, q_ready, o_done, drain;
+    uint32_t tmem_base;
+    int abort;
+};
+
+__device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+struct Item {
+    int s, g, b, k0, k1;
+};
+
+// Splits of one sequence are consecutive items, so concurrent CTAs stream neighbouring
+// key ranges of the same (b, g).
+__device__ __forceinline__ Item item_of(const DecodeArgs& a, int it) {
+    Item r;
+    r.s = it % a.splits;
+    const int bg = it / a.splits;
+    r.g = bg % a.Hkv;
+    r.b = bg / a.Hkv;
+    r.k0 = a.key_lo + r.s * a.keys_per_split;
+    r.k1 = min(a.L, r.k0 + a.keys_per_split);
+    if (r.k1 < r.k0) r.k1 = r.k0;
+    return r;
+}
+
+// Does 64-dim chunk c hold rotated dims?  Rotated dims: [0, R) and [d/2, d/2 + R).
+__device__ __forceinline__ bool chunk_rotated(int c, int d, int R) {
+    const int lo = c * 64, hi = lo + 64, h = d / 2;
+    return (lo < R) || (lo < h + R && hi > h);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    decode_kernel(const __grid_constant__ DecodeArgs a) {
+    constexpr int NCH = D / 64;     // 64-dim chunks per key row
+    constexpr int NPAIR = D / 128;  // 32 KB ring slots per tile and tensor
+    extern __shared__ uint8_t smem_raw[];
+    DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const WaitCtl wc{a.wait_limit, a.status};
+    volatile int* abort = &sm.abort;
+    const int R = a.rope.R;
+    const bool sep_v = a.kv_is_k == 0;
+    const bool side_rot = a.kv_is_k == 1;
+    const int n_items = a.splits * a.Hkv * a.B;
+    const int slots_per_tile = sep_v ? 2 * NPAIR : NPAIR;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kNSlots; ++i) {
+            mbar_init(&sm.full[i], 1);
+            mbar_init(&sm.empty[i], 1);
+        }
+        mbar_init(&sm.s_full, 1);
+        mbar_init(&sm.p_full, 1);
+        mbar_init(&sm.rot_ready, 1);
+        mbar_init(&sm.q_ready, 1);
+        mbar_init(&sm.o_done, 1);
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
+    if (warp >= 2)
+        for (int i = threadIdx.x - 64; i < R; i += 128)
+            sm.theta[i] = (float)exp2(-(2.0 * (double)i / (double)D) * a.rope.log2_base);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const uint32_t tm_s = tmem;          // S^T: 16 columns
+    const uint32_t tm_o = tmem + 16;     // O^T: NPAIR blocks of 16 columns
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            prefetch_tmap(&a.tm_k);
+            if (sep_v) prefetch_tmap(&a.tm_v);
+            uint32_t q = 0;   // ring slots filled so far
+            for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
+                const Item w = item_of(a, it);
+                const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+                for (int t = 0; t < nt && !*abort; ++t) {
+                    const int key = w.k0 + t * kTileKeys;
+                    // keep HBM busy beyond the ring: pull the tile two steps ahead into L2
+                    if (t + 2 < nt)
+                        for (int c = 0; c < NCH; ++c) {
+                            tma_prefetch_l2_4d(&a.tm_k, c * 64, w.g, key + 2 * kTileKeys, w.b);
+                            if (sep_v)
+                                tma_prefetch_l2_4d(&a.tm_v, c * 64, w.g, key + 2 * kTileKeys, w.b);
+                        }
+                    for (int pass = 0; pass < (sep_v ? 2 : 1) && !*abort; ++pass) {
+                        const CUtensorMap* map = pass ? &a.tm_v : &a.tm_k;
+                        for (int pr = 0; pr < NPAIR; ++pr) {
+                            const int slot = q % kNSlots;
+                            if (!mbar_wait(&sm.empty[slot], ((q / kNSlots) & 1) ^ 1, wc, abort))
+                                break;
+                            mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes);
+                            tma_load_4d(sm.ring[slot], map, &sm.full[slot], pr * 128, w.g, key, w.b);
+                            tma_load_4d(sm.ring[slot] + kChunkBytes, map, &sm.full[slot],
+                                        pr * 128 + 64, w.g, key, w.b);
+                            ++q;
+                        }
+                    }
+                }
+            }
+            // before the CTA exits, every copy it started must have landed
+            if (*abort) {
+                const uint32_t first = q > (uint32_t)kNSlots ? q - kNSlots : 0;
+                for (uint32_t k = first; k < q; ++k)
+                    mbar_wait_drain(&sm.full[k % kNSlots], (k / kNSlots) & 1, a.wait_limit);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t idesc_s = idesc_bf16_f32(128, kN, false, false);
+            const uint32_t idesc_o = idesc_bf16_f32(128, kN, true, false);  // A = V^T, MN-major
+            uint32_t q = 0, tile = 0, item_n = 0;
+            for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++item_n) {
+                const Item w = item_of(a, it);
+                const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+                if (!mbar_wait(&sm.q_ready, item_n & 1, wc, abort)) goto done;
+                for (int t = 0; t < nt; ++t, ++tile) {
+                    const uint32_t qk = q;
+                    const uint32_t qv = sep_v ? q + NPAIR : q;
+                    bool first = true;
+                    // S^T over the chunks that need no rotation, as soon as they land
+                    for (int pr = 0; pr < NPAIR; ++pr) {
+                        const uint32_t k = qk + pr, slot = k % kNSlots;
+                        if (!mbar_wait(&sm.full[slot], (k / kNSlots) & 1, wc, abort)) goto done;
+                        tc_fence_after();
+                        for (int h = 0; h < 2; ++h) {
+                            const int c = pr * 2 + h;
+                            if (chunk_rotated(c, D, R)) continue;
+                            const uint32_t ab = smem_u32(sm.ring[slot] + h * kChunkBytes);
+                            const uint32_t bb = smem_u32(sm.q[c]);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
+                                            sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
+                                            first ? 0u : 1u);
+                                first = false;
+                            }
+                        }
+                    }
+                    // then the rotated chunks, once the softmax warps have turned them
+                    if (R > 0) {
+                        if (!mbar_wait(&sm.rot_ready, tile & 1, wc, abort)) goto done;
+                        tc_fence_after();
+                        int ri = 0;
+                        for (int c = 0; c < NCH; ++c) {
+                            if (!chunk_rotated(c, D, R)) continue;
+                            const uint32_t slot = (qk + c / 2) % kNSlots;
+                            const uint8_t* src = side_rot ? sm.rot[ri++]
+                                                          : sm.ring[slot] + (c & 1) * kChunkBytes;
+                            const uint32_t ab = smem_u32(src);
+                            const uint32_t bb = smem_u32(sm.q[c]);
+                            for (int kk = 0; kk < 4; ++kk) {
+                                mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
+                                            sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
+                                            first ? 0u : 1u);
+                                first = false;
+                            }
+                        }
+                    }
+                    mma_commit(&sm.s_full);
+                    if (sep_v)   // key slots are free once S^T has read them
+                        for (int pr = 0; pr < NPAIR; ++pr) mma_commit(&sm.empty[(qk + pr) % kNSlots]);
+                    // O^T += V^T . P^T once the softmax warps have written P
+                    if (!mbar_wait(&sm.p_full, tile & 1, wc, abort)) goto done;
+                    tc_fence_after();
+                    for (int pr = 0; pr < NPAIR; ++pr) {
+                        const uint32_t k = qv + pr, slot = k % kNSlots;
+                        if (sep_v && !mbar_wait(&sm.full[slot], (k / kNSlots) & 1, wc, abort))
+                            goto done;
+                        tc_fence_after();
+                        const uint32_t ab = smem_u32(sm.ring[slot]);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            // 16 keys per step = two 8-row groups of 1024 B; the slot's second
+                            // 64-dim chunk is the next 64-element MN block (LBO)
+                            const uint64_t ad = sdesc_sw128(ab + kk * 2048, kChunkBytes, 1024);
+                            const uint32_t pb = smem_u32(sm.p[kk >> 2]) + (kk & 3) * 32;
+                            mma_bf16_ss(tm_o + pr * 16, ad, sdesc_sw128(pb, 16, 1024), idesc_o,
+                                        (t > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                    for (int pr = 0; pr < NPAIR; ++pr) mma_commit(&sm.empty[(qv + pr) % kNSlots]);
+                    q += slots_per_tile;
+                }
+                mma_commit(&sm.o_done);
+            }
+        done:
+            // all issued MMAs must finish before the tensor memory is released
+            mma_commit(&sm.drain);
+            mbar_wait_drain(&sm.drain, 0, a.wait_limit);
+        }
+    } else {
+        // ---------------------------------------------- rotation / softmax / epilogue
+        const int t128 = threadIdx.x - 64;            // 0..127
+        const int quarter = warp & 3;                 // TMEM lane quarter of this warp
+        const int row = quarter * 32 + lane;          // TMEM lane: key row or d-row
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int G = a.G;
+        uint32_t q = 0, tile = 0, item_n = 0;
+        bool ok = true;
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++item_n) {
+            const Item w = item_of(a, it);
+            const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+            // stage the G queries of (b, g) as the B operand of S^T (K-major, swizzled)
+            for (int e = t128; e < kN * (D / 8); e += 128) {
+                const int h = e / (D / 8), c8 = e % (D / 8);
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (h < G)
+                    v = *reinterpret_cast<const uint4*>(
+                        a.q + ((size_t)w.b * a.Hq + (size_t)w.g * G + h) * D + c8 * 8);
+                *reinterpret_cast<uint4*>(sm.q[c8 / 8] + sw128_offset(h, (c8 % 8) * 8)) = v;
+            }
+            fence_proxy_async_smem();
+            group_sync(kBarWG, 128);
+            if (t128 == 0) mbar_arrive(&sm.q_ready);
+
+            float m_run[kN], l_part[kN];
+#pragma unroll
+            for (int h = 0; h < kN; ++h) {
+                m_run[h] = -INFINITY;
+                l_part[h] = 0.f;
+            }
+            for (int t = 0; t < nt; ++t, ++tile) {
+                const int key0 = w.k0 + t * kTileKeys;
+                const uint32_t qk = q;
+                q += slots_per_tile;
+                // ---- turn the rotated pairs of this tile's keys to their positions
+                if (R > 0) {
+                    for (int i = t128; i < R; i += 128)
+                        sm.base_cs[i] = rope_cos_sin((long long)key0, i, D, a.rope.log2_base);
+                    bool got = true;
+                    for (int pr = 0; pr < NPAIR && got; ++pr)
+                        if (chunk_rotated(2 * pr, D, R) || chunk_rotated(2 * pr + 1, D, R))
+                            got = mbar_wait(&sm.full[(qk + pr) % kNSlots],
+                                            ((qk + pr) / kNSlots) & 1, wc, abort);
+                    ok = group_all(got, kBarWG, 128);   // also orders base_cs writes
+                    if (!ok) break;
+                    const float fr = (float)row;
+                    int ri = 0;
+                    for (int c = 0; c < NCH / 2; ++c) {
+                        if (!chunk_rotated(c, D, R)) continue;
+                        const int c2 = c + NCH / 2;   // partner chunk: dims + d/2
+                        uint8_t* src1 = sm.ring[(qk + c / 2) % kNSlots] + (c & 1) * kChunkBytes;
+                        uint8_t* src2 = sm.ring[(qk + c2 / 2) % kNSlots] + (c2 & 1) * kChunkBytes;
+                        uint8_t* dst1 = side_rot ? sm.rot[ri] : src1;
+                        uint8_t* dst2 = side_rot ? sm.rot[ri + 1] : src2;
+                        ri += 2;
+                        for (int g8 = 0; g8 < 8; ++g8) {
+                            const uint32_t off = sw128_offset(row, g8 * 8);
+                            uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
+                            uint4 x2 = *reinterpret_cast<const uint4*>(src2 + off);
+                            __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&x1);
+                            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x2);
+#pragma unroll
+                            for (int e2 = 0; e2 < 4; ++e2) {
+                                const float2 u = __bfloat1622float2(h1[e2]);
+                                const float2 v = __bfloat1622float2(h2[e2]);
+                                float uo[2] = {u.x, u.y}, vo[2] = {v.x, v.y};
+#pragma unroll
+                                for (int e = 0; e < 2; ++e) {
+                                    const int i = c * 64 + g8 * 8 + e2 * 2 + e;
+                                    if (i < R) {
+                                        // angle(key0 + row) = angle(key0) + row * theta_i
+                                        float x = fr * sm.theta[i];
+                                        x = fmaf(-6.2831853f, rintf(x * 0.15915494f), x);
+                                        float so, co;
+                                        __sincosf(x, &so, &co);
+                                        const float2 b = sm.base_cs[i];
+                                        const float cc = b.x * co - b.y * so;
+                                        const float ss = b.y * co + b.x * so;
+                                        const float p0 = uo[e], p1 = vo[e];
+                                        uo[e] = p0 * cc - p1 * ss;
+                                        vo[e] = p0 * ss + p1 * cc;
+                                    }
+                                }
+                                h1[e2] = __floats2bfloat162_rn(uo[0], uo[1]);
+                                h2[e2] = __floats2bfloat162_rn(vo[0], vo[1]);
+                            }
+                            *reinterpret_cast<uint4*>(dst1 + off) = x1;
+                            *reinterpret_cast<uint4*>(dst2 + off) = x2;
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    group_sync(kBarWG, 128);
+                    if (t128 == 0) mbar_arrive(&sm.rot_ready);
+                }
+                // ---- softmax over the 128 keys of the tile (thread = key)
+                ok = group_all(mbar_wait(&sm.s_full, tile & 1, wc, abort), kBarWG, 128);
+                if (!ok) break;
+                tc_fence_after();
+                float s[kN];
+                tmem_ld16(tm_s + lane_off, s);
+                tmem_ld_wait();
+                const bool valid = key0 + row < w.k1;
+                float mt[kN];
+#pragma unroll
+                for (int h = 0; h < kN; ++h) {
+                    s[h] = (valid && h < G) ? s[h] * a.scale_log2 : -INFINITY;
+                    mt[h] = s[h];
+                }
+#pragma unroll
+                for (int h = 0; h < kN; ++h)
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1)
+                        mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], o));
+                if (lane == 0)
+#pragma unroll
+                    for (int h = 0; h < kN; ++h) sm.red[quarter][h] = mt[h];
+                group_sync(kBarWG, 128);
+                float alpha[kN];
+                bool rescale = false;
+#pragma unroll
+                for (int h = 0; h < kN; ++h) {
+                    const float tmax = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]),
+                                             fmaxf(sm.red[2][h], sm.red[3][h]));
+                    const float mn = fmaxf(m_run[h], tmax);
+                    alpha[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mn);
+                    rescale |= (t > 0) && (alpha[h] != 1.f);
+                    m_run[h] = mn;
+                }
+                // P^T: row = head, K-major, 64 keys per 128-byte row, two chunks
+                {
+                    uint8_t* pb = sm.p[row >> 6];
+                    const int kc = row & 63;
+#pragma unroll
+                    for (int h = 0; h < kN; ++h) {
+                        const float p = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m_run[h]);
+                        l_part[h] = l_part[h] * alpha[h] + p;
+                        *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(h, kc)) =
+                            __float2bfloat16_rn(p);
+                    }
+                }
+                // rescale O^T when a running max moved.  O is idle: the MMA that wrote S for
+                // this tile was issued after the previous tile's O update, and commits track
+                // every earlier MMA.  Thread = d-row, column = head.
+                if (!group_all(!rescale, kBarWG, 128)) {
+                    for (int pr = 0; pr < NPAIR; ++pr) {
+                        float o[kN];
+                        tmem_ld16(tm_o + pr * 16 + lane_off, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h = 0; h < kN; ++h) o[h] *= alpha[h];
+                        tmem_st16(tm_o + pr * 16 + lane_off, o);
+                    }
+                    tmem_st_wait();
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                group_sync(kBarWG, 128);
+                if (t128 == 0) mbar_arrive(&sm.p_full);
+            }
+            if (!ok) break;
+            // ---- item epilogue: partial O^T, running max and sum
+            ok = group_all(mbar_wait(&sm.o_done, item_n & 1, wc, abort), kBarWG, 128);
+            if (!ok) break;
+            tc_fence_after();
+            const size_t obase = ((size_t)w.s * a.B + w.b) * a.Hq + (size_t)w.g * G;
+            for (int pr = 0; pr < NPAIR; ++pr) {
+                float o[kN];
+                tmem_ld16(tm_o + pr * 16 + lane_off, o);
+                tmem_ld_wait();
+                for (int h = 0; h < G; ++h)
+                    a.part_o[(obase + h) * D + pr * 128 + row] = nt > 0 ? o[h] : 0.f;
+            }
+#pragma unroll
+            for (int h = 0; h < kN; ++h)
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1)
+                    l_part[h] += __shfl_xor_sync(0xffffffffu, l_part[h], o);
+            if (lane == 0)
+#pragma unroll
+                for (int h = 0; h < kN; ++h) sm.red[quarter][h] = l_part[h];
+            group_sync(kBarWG, 128);
+            if (t128 < G) {
+                const float l = sm.red[0][t128] + sm.red[1][t128] + sm.red[2][t128] +
+                                sm.red[3][t128];
+                float mv = m_run[0];
+#pragma unroll
+                for (int h = 1; h < kN; ++h) mv = (t128 == h) ? m_run[h] : mv;
+                a.part_ml[(obase + t128) * 2 + 0] = mv;
+                a.part_ml[(obase + t128) * 2 + 1] = l;
+            }
+            tc_fence_before();
+            group_sync(kBarWG, 128);   // red[] and O^T are reused by the next item
+        }
+    }
+
+    // -------------------------------------------------------------------- teardown
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// Merge the split partials of one (b, h):
+//   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,   M = max_s m_s (log2 units).
+__global__ void decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
+    const int bh = blockIdx.x;   // b * Hq + h
+    const size_t stride = (size_t)a.B * a.Hq;
+    float M = -INFINITY;
+    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[(s * stride + bh) * 2]);
+    float den = 0.f;
+    for (int s = 0; s < a.splits; ++s) {
+        const float m = a.part_ml[(s * stride + bh) * 2];
+        if (m != -INFINITY) den += exp2f(m - M) * a.part_ml[(s * stride + bh) * 2 + 1];
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+    for (int c = threadIdx.x; c < a.d; c += blockDim.x) {
+        float acc = 0.f;
+        for (int s = 0; s < a.splits; ++s) {
+            const float m = a.part_ml[(s * stride + bh) * 2];
+            if (m != -INFINITY) acc += exp2f(m - M) * a.part_o[(s * stride + bh) * a.d + c];
+        }
+        a.out[(size_t)bh * a.d + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc * inv));
+    }
+    if (threadIdx.x == 0 && a.lse)
+        a.lse[bh] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
+}
+
+template <int D>
+cudaError_t run_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
+    cudaError_t e =
+        cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    decode_kernel<D><<<grid, kThreads, smem, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t decode_smem_bytes() { return sizeof(DecodeSmem) + 1024; }
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
+    const size_t smem = decode_smem_bytes();
+    const int n_items = a.splits * a.Hkv * a.B;
+    if (n_items > 0) {
+        int dev = 0, sms = 148;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        const int grid = n_items < sms ? n_items : sms;
+        cudaError_t e = a.d == 512 ? run_decode<512>(a, grid, smem, stream)
+                        : a.d == 256 ? run_decode<256>(a, grid, smem, stream)
+                                     : cudaErrorInvalidValue;
+        if (e != cudaSuccess) return e;
+    }
+    if (a.B * a.Hq > 0) decode_combine_kernel<<<a.B * a.Hq, 128, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+}  // namespace g4

@@ -1,0 +1,82 @@
+// kernels.h -- launcher interfaces between the C-ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "g4attn.h"
+
+namespace g4 {
+
+// RoPE geometry of a layer: R rotated pairs (i, i + d/2), i < R.
+struct Rope {
+    int R;
+    double log2_base;   // log2(rope_base)
+};
+
+struct QkNormRopeArgs {
+    const uint16_t* q_in;
+    const uint16_t* k_in;
+    uint16_t* q_out;
+    uint16_t* k_out;      // normalised, not rotated
+    uint16_t* krot_out;   // normalised and rotated
+    const float* gamma_q;
+    const float* gamma_k;
+    float2* cs_out;       // optional [T, R] (cos, sin) table of positions pos0 + t
+    int B, T, Hq, Hkv, d;
+    long long pos0;
+    Rope rope;
+    int qk_norm;
+    float eps;
+};
+
+cudaError_t launch_qknorm_rope(const QkNormRopeArgs& a, cudaStream_t stream);
+
+// Split-KV decode (one query per (b, h) at position L-1) and its combine pass.
+struct DecodeArgs {
+    CUtensorMap tm_k;       // kcache [B, L, Hkv, d] as a 4-D map (d, Hkv, L, B), box (64, 1, 128, 1)
+    CUtensorMap tm_v;       // vcache, same geometry (kv_is_k == 0), else a copy of tm_k
+    const uint16_t* q;      // [B, Hq, d], normalised and rotated
+    float* part_o;          // [S, B, Hq, d]
+    float* part_ml;         // [S, B, Hq, 2]  (running max in log2 units, sum)
+    uint16_t* out;          // [B, Hq, d]
+    float* lse;             // [B, Hq] or null
+    int B, L, Hq, Hkv, d, G;
+    int key_lo;             // first visible key (window), 0 for full attention
+    int splits, keys_per_split;  // multiples of 128
+    Rope rope;
+    float scale_log2;       // scale * log2(e)
+    int kv_is_k;
+    long long wait_limit;
+    int* status;
+};
+
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
+size_t decode_smem_bytes();
+
+// Flash-attention prefill.
+struct PrefillArgs {
+    CUtensorMap tm_kn;      // normalised pre-RoPE keys  (d, Hkv, T, B), box (64, 1, 128, 1)
+    CUtensorMap tm_kr;      // normalised rotated keys, same geometry
+    CUtensorMap tm_v;       // separate values, same geometry (kv_is_k == 0), else = tm_kn
+    const uint16_t* q;      // raw queries [B, T, Hq, d]
+    const float* gamma_q;
+    const float2* rope_cs;  // [T, R] (cos, sin) of position t, pair i
+    uint16_t* out;          // [B, T, Hq, d]
+    float* lse;             // [B, Hq, T] or null
+    int B, T, Hq, Hkv, d, G;
+    int window;
+    Rope rope;
+    int qk_norm;
+    float eps;
+    float scale_log2;
+    int kv_is_k;
+    long long wait_limit;
+    int* status;
+};
+
+cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
+size_t prefill_smem_bytes(int d);
+
+}  // namespace g4

@@ -1,0 +1,166 @@
+/*
+ * g4attn.h -- C ABI of the g4attn library: the Gemma-4-style attention layer as
+ * hand-written sm_100a (B200) CUDA kernels.
+ *
+ * The operation (Gemma 4 Technical Report, section 2 "Model Architecture"; the
+ * yunpan.plus explainer sections "GQA", "K=V", "p-RoPE" and "interleaved layers";
+ * the AI Engineer talk notes on GQA 2:1 / 8:1 and head_dim 256 -> 512):
+ *   QKNorm   q^ = RMS(q; gamma_q), k^ = RMS(k; gamma_k)  over head_dim, with
+ *            RMS(x; g)_c = x_c / sqrt(mean(x^2) + eps) * g_c
+ *   p-RoPE   pairs (x_i, x_{i+d/2}), i < R = floor(p*d/2), turn by pos * base^(-2i/d)
+ *            ((cos -sin; sin cos)); the other pairs do not turn.  Global layers:
+ *            p = 0.25, base 1e6; local layers: p = 1, base 1e4.
+ *   GQA      query head h reads kv head h / (Hq/Hkv).
+ *   scores   s_ij = scale * rot(q^_i, i) . rot(k^_j, j) for j visible to i: causal
+ *            (window = 0: j <= i) or sliding window (window = W: i - W < j <= i).
+ *   values   kv_is_k = 1: v_j = k^_j (keys reused as values, the pre-RoPE normed key);
+ *            kv_is_k = 2: v_j = rot(k^_j, j); kv_is_k = 0: the supplied v_j.
+ *   output   out_i = sum_j softmax_j(s_ij) v_j;   lse_i = log sum_j exp(s_ij).
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major, contiguous, [B, T, H, d] with d fastest, in device
+ *     memory.  bf16 tensors hold IEEE bfloat16 bit patterns.  Device pointers must be
+ *     16-byte aligned (G4ATTN_ERR_MISALIGNED otherwise).
+ *   - The caller owns every buffer.  The library never allocates device memory on
+ *     these paths; it keeps a small host-side cache only (kernel attributes).
+ *   - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL = the
+ *     legacy default stream).  Arguments are validated before any launch; on an error
+ *     nothing is launched.
+ *   - The current CUDA device must be an sm_100 part (G4ATTN_ERR_UNSUPPORTED otherwise).
+ *   - Return value: G4ATTN_OK or one of the negative codes below.
+ */
+#ifndef G4ATTN_H
+#define G4ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define G4ATTN_API __attribute__((visibility("default")))
+#else
+#define G4ATTN_API
+#endif
+
+typedef uint16_t g4attn_bf16;          /* IEEE bfloat16 bit pattern */
+typedef struct CUstream_st* g4attn_stream_t;  /* same type as cudaStream_t */
+
+enum {
+    G4ATTN_OK = 0,
+    G4ATTN_ERR_INVALID_ARG = -1,   /* null pointer, bad size, inconsistent config */
+    G4ATTN_ERR_UNSUPPORTED = -2,   /* head_dim / group / device not handled by the kernels */
+    G4ATTN_ERR_MISALIGNED = -3,    /* a pointer is not 16-byte aligned */
+    G4ATTN_ERR_WORKSPACE = -4,     /* workspace missing or smaller than *_workspace_size */
+    G4ATTN_ERR_CUDA = -5,          /* a CUDA runtime / driver call or launch failed */
+    G4ATTN_ERR_TIMEOUT = -6        /* a device wait gave up (see g4attn_device_status) */
+};
+
+/* Layer configuration (one attention layer). */
+typedef struct g4attn_layer_cfg {
+    int n_q_heads;      /* Hq > 0 */
+    int n_kv_heads;     /* Hkv > 0, Hq % Hkv == 0; G = Hq / Hkv must divide 128 */
+    int head_dim;       /* d: 256 or 512 for the tensor-core kernels */
+    float rope_p;       /* fraction of rotary pairs that turn, 0 <= p <= 1 (0.25 global, 1 local) */
+    double rope_base;   /* RoPE base > 0 (1e6 global, 1e4 local) */
+    int window;         /* 0 = full causal; W > 0 = sliding window i - W < j <= i */
+    float scale;        /* softmax scale (1/sqrt(d) for the pages' layers) */
+    int kv_is_k;        /* 0 separate v; 1 v = normed pre-RoPE key; 2 v = normed rotated key */
+    int qk_norm;        /* 1 = apply QKNorm (the layers on the pages), 0 = inputs are used as is */
+    float qk_norm_eps;  /* eps inside the RMS (1e-6) */
+} g4attn_layer_cfg;
+
+/*
+ * Standalone prologue: QKNorm and p-RoPE of one block of tokens at positions
+ * pos0 .. pos0+T-1 (report section 2: QKNorm, p-RoPE / RoPE; explainer "K=V": the
+ * cache of a global layer holds keys only).
+ *   q_in       [B, T, Hq, d] bf16, or NULL (then q_out is ignored)
+ *   k_in       [B, T, Hkv, d] bf16, or NULL (then kcache_out / krot_out are ignored)
+ *   q_out      [B, T, Hq, d] bf16: rot(RMS(q), pos)            (NULL = not written)
+ *   kcache_out [B, T, Hkv, d] bf16: RMS(k), not rotated: the K(=V) cache rows
+ *   krot_out   [B, T, Hkv, d] bf16: rot(RMS(k), pos)           (NULL = not written)
+ *   gamma_q / gamma_k  [d] fp32 device arrays (required when cfg->qk_norm = 1)
+ * Writes only.  With qk_norm = 0 the norm step is skipped (pure RoPE).
+ */
+G4ATTN_API int g4attn_qknorm_rope(const g4attn_bf16* q_in, const g4attn_bf16* k_in,
+                       g4attn_bf16* q_out, g4attn_bf16* kcache_out, g4attn_bf16* krot_out,
+                       const float* gamma_q, const float* gamma_k,
+                       int B, int T, long long pos0,
+                       const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/*
+ * Bytes of device workspace g4attn_prefill needs for (B, T, cfg): the normalised key
+ * cache and its rotated copy.  Returns 0 when the configuration is invalid.
+ */
+G4ATTN_API size_t g4attn_prefill_workspace_size(int B, int T, const g4attn_layer_cfg* cfg);
+
+/*
+ * Prefill: causal or sliding-window attention of T new tokens at positions 0..T-1
+ * over themselves (report section 2; explainer "interleaved layers", "K=V", "p-RoPE").
+ *   q      [B, T, Hq, d] bf16, raw (QKNorm and RoPE are applied inside, fused into
+ *          the query tile load)
+ *   k      [B, T, Hkv, d] bf16, raw
+ *   v      [B, T, Hkv, d] bf16 raw values; must be NULL when kv_is_k != 0 and
+ *          non-NULL when kv_is_k == 0
+ *   gamma_q, gamma_k  [d] fp32
+ *   out    [B, T, Hq, d] bf16 (written)
+ *   lse    [B, Hq, T] fp32 natural-log sum of exp of the scaled scores, or NULL
+ *   workspace / ws_bytes  >= g4attn_prefill_workspace_size(B, T, cfg), 256-byte aligned
+ * T = 0 or B = 0 is a no-op.  window >= T behaves as full causal attention.
+ */
+G4ATTN_API int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16* v,
+                   const float* gamma_q, const float* gamma_k,
+                   g4attn_bf16* out, float* lse, void* workspace, size_t ws_bytes,
+                   int B, int T, const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/*
+ * Bytes of device workspace g4attn_decode needs for (B, L, cfg): fp32 partial outputs
+ * and softmax statistics of the split-KV pass.  Returns 0 for an invalid configuration.
+ */
+G4ATTN_API size_t g4attn_decode_workspace_size(int B, int L, const g4attn_layer_cfg* cfg);
+
+/*
+ * Decode: one new token per sequence, at position L-1, against a cache of L keys that
+ * already includes it (explainer "K=V": the global layer keeps a single K cache).
+ *   q       [B, 1, Hq, d] bf16: the new queries, already normalised and rotated to
+ *           position L-1 (g4attn_qknorm_rope with pos0 = L-1 produces it)
+ *   kcache  [B, L, Hkv, d] bf16: normalised, NOT rotated keys; the kernel turns key j
+ *           to position j on the fly
+ *   vcache  [B, L, Hkv, d] bf16 or NULL: separate values (kv_is_k = 0 only)
+ *   out     [B, 1, Hq, d] bf16 (written);  lse [B, Hq] fp32 or NULL
+ *   workspace / ws_bytes  >= g4attn_decode_workspace_size(B, L, cfg), 256-byte aligned
+ * With window W > 0 only the last W cache rows are read.  L = 0 writes out = 0 and
+ * lse = -inf.
+ */
+G4ATTN_API int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_bf16* vcache,
+                  int L, g4attn_bf16* out, float* lse, void* workspace, size_t ws_bytes,
+                  int B, const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+G4ATTN_API const char* g4attn_status_string(int status);
+
+/*
+ * Device-side status word.  Every bounded wait inside the kernels (mbarrier spins)
+ * gives up after the current wait limit, records G4ATTN_ERR_TIMEOUT here and lets the
+ * kernel finish early.  g4attn_device_status synchronises `stream`, returns the word
+ * (G4ATTN_OK if no wait gave up since the last reset) and clears it.
+ */
+G4ATTN_API int g4attn_device_status(g4attn_stream_t stream);
+
+/*
+ * Upper bound on the polls of one device wait.  Independently of it, every wait gives
+ * up after 2 seconds of wall-clock time (legal waits last microseconds).  The default
+ * poll bound is effectively unlimited; tests of the timeout path set a small one.
+ * Values < 1 restore the default.  Returns the previous bound.
+ */
+G4ATTN_API long long g4attn_set_wait_limit(long long polls);
+
+/* Library version string. */
+G4ATTN_API const char* g4attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* G4ATTN_H */

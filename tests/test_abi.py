@@ -1,0 +1,143 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports every entry
+point declared in include/g4attn.h, and rejects bad arguments before any launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "g4attn.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from attention_g4attn_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+@pytest.fixture(scope="module")
+def b():
+    from attention_g4attn_b200 import build
+    build.build()
+    from attention_g4attn_b200 import binding
+    return binding
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    return re.findall(r"G4ATTN_API\s+[\w\s\*]+?\b(g4attn_\w+)\s*\(", src)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    for n in ("g4attn_qknorm_rope", "g4attn_prefill", "g4attn_decode",
+              "g4attn_prefill_workspace_size", "g4attn_decode_workspace_size",
+              "g4attn_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(b):
+    assert b.g4attn_status_string(0) == "ok"
+    for code in range(-6, 0):
+        s = b.g4attn_status_string(code)
+        assert s and s != "unknown status"
+    assert b.g4attn_status_string(-99) == "unknown status"
+    assert "sm_100a" in b.g4attn_version()
+
+
+def test_wait_limit_roundtrip(b):
+    old = b.g4attn_set_wait_limit(1234)
+    assert b.g4attn_set_wait_limit(0) == 1234       # < 1 restores the default
+    assert b.g4attn_set_wait_limit(old) == old
+
+
+def _align(x):
+    return (x + 255) // 256 * 256
+
+
+def test_prefill_workspace_formula(b):
+    # normalised keys + rotated keys (bf16) + the (cos, sin) table of every position
+    g = b.LayerCfg(32, 4, 512, 0.25, 1e6, 0, None, 1)
+    B, T = 1, 32768
+    rows = B * T * 4 * 512 * 2
+    assert b.g4attn_prefill_workspace_size(B, T, g) == 2 * _align(rows) + _align(T * 64 * 8)
+    # local layer: every chunk rotated and separate values -> no pre-RoPE copy
+    loc = b.LayerCfg(16, 8, 256, 1.0, 1e4, 512, None, 0)
+    rows = 2 * 4096 * 8 * 256 * 2
+    assert b.g4attn_prefill_workspace_size(2, 4096, loc) == _align(rows) + _align(4096 * 128 * 8)
+
+
+def test_invalid_configs_are_rejected(b):
+    bad = [
+        b.LayerCfg(6, 4, 512, 0.25, 1e6),        # Hq % Hkv != 0
+        b.LayerCfg(8, 1, 384, 0.25, 1e6),        # head_dim not handled by the kernels
+        b.LayerCfg(8, 1, 512, 1.5, 1e6),         # p outside [0, 1]
+        b.LayerCfg(8, 1, 512, 0.25, -1.0),       # base <= 0
+        b.LayerCfg(8, 1, 512, 0.25, 1e6, -3),    # negative window
+        b.LayerCfg(8, 1, 512, 0.25, 1e6, 0, None, 3),   # kv_is_k out of range
+        b.LayerCfg(256, 1, 512, 0.25, 1e6),      # G = 256 does not divide 128
+    ]
+    for cfg in bad:
+        assert b.g4attn_prefill_workspace_size(1, 16, cfg) == 0
+        assert b.g4attn_decode_workspace_size(1, 16, cfg) == 0
+
+
+def _call_prefill(lib, b, cfg, q=0x1000, k=0x2000, v=None, gq=0x3000, gk=0x4000, out=0x5000,
+                  ws=0x100000, ws_bytes=1 << 40, B=1, T=16):
+    c = cfg.c()
+    P = ctypes.c_void_p
+    f = lib.g4attn_prefill
+    f.restype = ctypes.c_int
+    f.argtypes = [P, P, P, P, P, P, P, P, ctypes.c_size_t, ctypes.c_int, ctypes.c_int,
+                  ctypes.POINTER(type(c)), P]
+    return f(q, k, v, gq, gk, out, None, ws, ws_bytes, B, T, ctypes.byref(c), None)
+
+
+def test_prefill_argument_checks_without_gpu(lib, b):
+    g = b.LayerCfg(8, 1, 512, 0.25, 1e6)
+    assert _call_prefill(lib, b, b.LayerCfg(6, 4, 512, 0.25, 1e6)) == b.G4ATTN_ERR_INVALID_ARG
+    assert _call_prefill(lib, b, g, v=0x6000) == b.G4ATTN_ERR_INVALID_ARG     # K=V takes no v
+    assert _call_prefill(lib, b, b.LayerCfg(8, 1, 512, 1.0, 1e4, 0, None, 0)) == \
+        b.G4ATTN_ERR_INVALID_ARG                                              # v missing
+    assert _call_prefill(lib, b, g, q=0x1001) == b.G4ATTN_ERR_MISALIGNED
+    assert _call_prefill(lib, b, g, ws_bytes=16) == b.G4ATTN_ERR_WORKSPACE
+    assert _call_prefill(lib, b, g, ws=None) == b.G4ATTN_ERR_WORKSPACE
+    assert _call_prefill(lib, b, g, ws=0x100010) == b.G4ATTN_ERR_MISALIGNED  # 256 B rule
+    assert _call_prefill(lib, b, g, gq=None) == b.G4ATTN_ERR_INVALID_ARG      # QKNorm gains
+    assert _call_prefill(lib, b, g, B=-1) == b.G4ATTN_ERR_INVALID_ARG
+    assert _call_prefill(lib, b, g, T=0) == b.G4ATTN_OK                       # empty: no-op
+
+
+def test_decode_argument_checks_without_gpu(lib, b):
+    P = ctypes.c_void_p
+    f = lib.g4attn_decode
+    f.restype = ctypes.c_int
+    g = b.LayerCfg(32, 4, 512, 0.25, 1e6).c()
+    f.argtypes = [P, P, P, ctypes.c_int, P, P, P, ctypes.c_size_t, ctypes.c_int,
+                  ctypes.POINTER(type(g)), P]
+    assert f(0x1000, 0x2000, 0x3000, 16, 0x4000, None, 0x10000, 1 << 30, 1, ctypes.byref(g),
+             None) == b.G4ATTN_ERR_INVALID_ARG   # K=V layer given a value cache
+    assert f(0x1000, 0x2000, None, -1, 0x4000, None, 0x10000, 1 << 30, 1, ctypes.byref(g),
+             None) == b.G4ATTN_ERR_INVALID_ARG
+    g32 = b.LayerCfg(64, 2, 512, 0.25, 1e6).c()     # 32 query heads per KV head
+    assert f(0x1000, 0x2000, None, 16, 0x4000, None, 0x10000, 1 << 30, 1, ctypes.byref(g32),
+             None) == b.G4ATTN_ERR_UNSUPPORTED
+    assert f(0x1000, 0x2001, None, 16, 0x4000, None, 0x10000, 1 << 30, 1, ctypes.byref(g),
+             None) == b.G4ATTN_ERR_MISALIGNED
+
+
+def test_binding_refuses_host_tensors(b):
+    import torch
+    q = torch.zeros(1, 4, 8, 512, dtype=torch.bfloat16)
+    k = torch.zeros(1, 4, 1, 512, dtype=torch.bfloat16)
+    g = torch.ones(512)
+    with pytest.raises(b.G4AttnError):
+        b.g4attn_prefill(q, k, None, g, g, b.LayerCfg(8, 1, 512, 0.25, 1e6), out=q.clone(),
+                         workspace=torch.zeros(16, dtype=torch.uint8))

@@ -1,0 +1,101 @@
+"""GPU parity of split-KV decode (g4attn_decode) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from attention_g4attn_b200 import synth, workloads
+from gpu_common import binding, ocfg
+from parity import assert_parity, to_np
+
+pytestmark = pytest.mark.gpu
+
+GLOBAL = workloads.GLOBAL_8TO1
+
+
+def run_decode(dec, layer, **kw):
+    b = binding()
+    dev = torch.device("cuda:0")
+    cfg = b.LayerCfg.from_layer(layer, **kw)
+    v = dec.v.to(dev) if dec.v is not None else None
+    out, lse = b.g4attn_decode(dec.q.to(dev), dec.k.to(dev), v, cfg, want_lse=True)
+    torch.cuda.synchronize()
+    assert b.g4attn_device_status() == 0
+    return out.cpu(), lse.cpu()
+
+
+def check(dec, layer, items=None, what="decode", **kw):
+    out, lse = run_decode(dec, layer, **kw)
+    ro, rl = oracle.decode(dec.q[:, 0], dec.k, dec.v, ocfg(layer, **kw), items=items)
+    go, gl = to_np(out)[:, 0], to_np(lse)
+    assert np.all(np.isfinite(go)) and np.all(np.isfinite(gl))
+    if items is not None:
+        G = layer.n_q_heads // layer.n_kv_heads
+        sel = [(it // layer.n_kv_heads, (it % layer.n_kv_heads) * G + h)
+               for it in items for h in range(G)]
+        bi = [s[0] for s in sel]
+        hi = [s[1] for s in sel]
+        go, ro, gl, rl = go[bi, hi], ro[bi, hi], gl[bi, hi], rl[bi, hi]
+    assert_parity(go, ro, what + " out")
+    assert_parity(gl, rl, what + " lse")
+
+
+@pytest.mark.parametrize("L", [1, 100, 128, 129, 1000, 3001])
+def test_decode_global_small(L):
+    dec = synth.decode_inputs(2, L, 32, 4, 512, False, seed=L)
+    check(dec, GLOBAL, what="decode L=%d" % L)
+
+
+def test_decode_rotated_values_variant():
+    dec = synth.decode_inputs(2, 777, 32, 4, 512, False, seed=5)
+    check(dec, GLOBAL, kv_is_k=2, what="decode kv_is_k=2")
+
+
+def test_decode_separate_values_and_window():
+    dec = synth.decode_inputs(2, 1500, 32, 4, 512, True, seed=6)
+    check(dec, GLOBAL, kv_is_k=0, what="decode separate v")
+    check(dec, GLOBAL, kv_is_k=0, window=300, what="decode separate v, window 300")
+
+
+def test_decode_local_layer_shape():
+    loc = workloads.LOCAL_W1024
+    dec = synth.decode_inputs(2, 2000, loc.n_q_heads, loc.n_kv_heads, loc.head_dim, True, seed=9)
+    check(dec, loc, what="decode local")
+
+
+def test_decode_empty_cache():
+    b = binding()
+    dev = torch.device("cuda:0")
+    q = torch.randn(2, 1, 32, 512, device=dev).bfloat16()
+    k = torch.empty(2, 0, 4, 512, dtype=torch.bfloat16, device=dev)
+    out, lse = b.g4attn_decode(q, k, None, b.LayerCfg.from_layer(GLOBAL), want_lse=True)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0)
+    assert torch.all(torch.isinf(lse)) and torch.all(lse < 0)
+
+
+@pytest.mark.parametrize("wl", [workloads.GLOBAL_DECODE_32K, workloads.GLOBAL_DECODE_128K])
+def test_decode_full_size_sampled(wl):
+    ly = wl.layer
+    dec = synth.decode_inputs(wl.B, wl.L, ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False,
+                              seed=wl.seed)
+    items = [0, 17, wl.B * ly.n_kv_heads - 1]      # (b, g) = (0,0), (4,1), (15,3)
+    check(dec, ly, items=items, what=wl.name)
+
+
+def test_decode_matches_last_prefill_row():
+    """Decode at position T-1 against the normalised cache equals prefill row T-1."""
+    b = binding()
+    dev = torch.device("cuda:0")
+    T = 517
+    inp = synth.layer_inputs(1, T, 32, 4, 512, False, seed=21)
+    cfg = b.LayerCfg.from_layer(GLOBAL)
+    q, k, gq, gk = (x.to(dev) for x in (inp.q, inp.k, inp.gamma_q, inp.gamma_k))
+    pre, pre_lse = b.g4attn_prefill(q, k, None, gq, gk, cfg, want_lse=True)
+    _, kc, _ = b.g4attn_qknorm_rope(None, k, None, gk, cfg, pos0=0, want_krot=False)
+    # the query of the last token sits at position T-1
+    qn, _, _ = b.g4attn_qknorm_rope(q[:, T - 1:T].contiguous(), None, gq, None, cfg, pos0=T - 1)
+    dout, dlse = b.g4attn_decode(qn, kc, None, cfg, want_lse=True)
+    torch.cuda.synchronize()
+    assert_parity(to_np(dout)[:, 0], to_np(pre)[:, T - 1], "decode vs prefill row")
+    assert_parity(to_np(dlse), to_np(pre_lse)[:, :, T - 1], "decode vs prefill lse")
