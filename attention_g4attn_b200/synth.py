@@ -4,8 +4,8 @@ This module holds no arithmetic of the attention method: it only draws random nu
 Recipe (same for every workload): a torch Generator seeded with `seed` draws, in this
 order, q ~ N(0,1) [B,T,Hq,d], k ~ N(0,1) [B,T,Hkv,d], v ~ N(0,1) [B,T,Hkv,d] (only for
 layers with a separate value), then gamma_q = 1 + 0.1 N(0,1) [d] and
-gamma_k = 1 + 0.1 N(0,1) [d] in fp32.  q, k and v are rounded to bf16 (round to nearest
-even).  On the CPU the bytes are reproducible across machines; `device="cuda"` uses the
+gamma_k = 1 + 0.1 N(0,1) [d] in fp32.  q, k and v are drawn in fp32 (in pieces of 2^24
+elements for tensors larger than that) and rounded to bf16 (round to nearest even).  On the CPU the bytes are reproducible across machines; `device="cuda"` uses the
 CUDA generator instead (fast for the largest workloads, different bytes for the same seed).
 """
 from dataclasses import dataclass
@@ -23,17 +23,36 @@ class LayerInputs:
     gamma_k: torch.Tensor
 
 
+_CHUNK = 1 << 24
+
+
 def _randn(shape, gen, device):
     return torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
 
 
+def _randn_bf16(shape, gen, device):
+    """N(0,1) draws rounded to bf16.  Large tensors are drawn in fixed 2^24-element pieces
+    (fp32, then rounded) so host memory stays bounded; the piece size is part of the
+    recipe, so the bytes are the same on every run."""
+    n = 1
+    for x in shape:
+        n *= x
+    if n <= _CHUNK:
+        return _randn(shape, gen, device).to(torch.bfloat16)
+    out = torch.empty(n, dtype=torch.bfloat16, device=device)
+    for i in range(0, n, _CHUNK):
+        m = min(_CHUNK, n - i)
+        out[i:i + m] = _randn((m,), gen, device).to(torch.bfloat16)
+    return out.view(shape)
+
+
 def layer_inputs(B, T, n_q_heads, n_kv_heads, head_dim, separate_v, seed, device="cpu"):
     gen = torch.Generator(device=device).manual_seed(int(seed))
-    q = _randn((B, T, n_q_heads, head_dim), gen, device).to(torch.bfloat16)
-    k = _randn((B, T, n_kv_heads, head_dim), gen, device).to(torch.bfloat16)
+    q = _randn_bf16((B, T, n_q_heads, head_dim), gen, device)
+    k = _randn_bf16((B, T, n_kv_heads, head_dim), gen, device)
     v = None
     if separate_v:
-        v = _randn((B, T, n_kv_heads, head_dim), gen, device).to(torch.bfloat16)
+        v = _randn_bf16((B, T, n_kv_heads, head_dim), gen, device)
     gamma_q = 1.0 + 0.1 * _randn((head_dim,), gen, device)
     gamma_k = 1.0 + 0.1 * _randn((head_dim,), gen, device)
     return LayerInputs(q, k, v, gamma_q.contiguous(), gamma_k.contiguous())
@@ -43,11 +62,11 @@ def decode_inputs(B, L, n_q_heads, n_kv_heads, head_dim, separate_v, seed, devic
     """A decode step: q [B,1,Hq,d] and a cache [B,L,Hkv,d] of N(0,1) bf16 values that is
     used as if it already held normalised keys (the cache of the decode workload)."""
     gen = torch.Generator(device=device).manual_seed(int(seed))
-    q = _randn((B, 1, n_q_heads, head_dim), gen, device).to(torch.bfloat16)
-    kcache = _randn((B, L, n_kv_heads, head_dim), gen, device).to(torch.bfloat16)
+    q = _randn_bf16((B, 1, n_q_heads, head_dim), gen, device)
+    kcache = _randn_bf16((B, L, n_kv_heads, head_dim), gen, device)
     vcache = None
     if separate_v:
-        vcache = _randn((B, L, n_kv_heads, head_dim), gen, device).to(torch.bfloat16)
+        vcache = _randn_bf16((B, L, n_kv_heads, head_dim), gen, device)
     gamma_q = 1.0 + 0.1 * _randn((head_dim,), gen, device)
     gamma_k = 1.0 + 0.1 * _randn((head_dim,), gen, device)
     return LayerInputs(q, kcache, vcache, gamma_q.contiguous(), gamma_k.contiguous())
