@@ -115,12 +115,13 @@ int check_cfg(const g4attn_layer_cfg* c, bool tensor_core_path) {
 
 // 4-D map over a [B, T, H, d] bf16 tensor: dims (d, H, T, B), box (64, 1, 128, 1),
 // 128-byte swizzle, zero fill outside the tensor.
-int encode_rows(CUtensorMap* m, const void* base, int B, int T, int H, int d) {
+int encode_rows(CUtensorMap* m, const void* base, int B, int T, int H, int d, bool f16 = false) {
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
     cuuint32_t box[4] = {64, 1, 128, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+    CUresult r = g_encode(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                          4, const_cast<void*>(base), dims,
                           strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -291,14 +292,15 @@ int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16
     float2* cs = reinterpret_cast<float2*>(w + ws.cs_off);
     const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
 
-    // 1) normalise the keys once: pre-RoPE copy (the K(=V) cache) and the rotated copy,
-    //    plus the (cos, sin) table of every position for the query prologue
+    // 1) normalise the keys once: pre-RoPE copy (the K(=V) values) and the rotated copy,
+    //    both fp16, plus the (cos, sin) table of every position for the query prologue
     g4::QkNormRopeArgs ka{};
     ka.k_in = k;
     ka.k_out = kn;
     ka.krot_out = kr;
     ka.gamma_k = gamma_k;
     ka.cs_out = cs;
+    ka.k_f16 = 1;   // the prefill keeps its normalised key copies in fp16
     ka.B = B; ka.T = T; ka.Hq = cfg->n_q_heads; ka.Hkv = Hkv; ka.d = d;
     ka.pos0 = 0;
     ka.rope = make_rope(cfg);
@@ -308,9 +310,11 @@ int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16
 
     // 2) the fused flash-attention kernel
     g4::PrefillArgs a{};
-    if ((rc = encode_rows(&a.tm_kr, kr, B, T, Hkv, d))) return rc;
-    if ((rc = encode_rows(&a.tm_kn, kn ? kn : kr, B, T, Hkv, d))) return rc;
-    if ((rc = encode_rows(&a.tm_v, v ? v : (kn ? kn : kr), B, T, Hkv, d))) return rc;
+    if ((rc = encode_rows(&a.tm_kr, kr, B, T, Hkv, d, true))) return rc;
+    if ((rc = encode_rows(&a.tm_kn, kn ? kn : kr, B, T, Hkv, d, true))) return rc;
+    if (v) rc = encode_rows(&a.tm_v, v, B, T, Hkv, d, false);
+    else rc = encode_rows(&a.tm_v, kn ? kn : kr, B, T, Hkv, d, true);
+    if (rc) return rc;
     a.q = q;
     a.gamma_q = gamma_q;
     a.rope_cs = cs;

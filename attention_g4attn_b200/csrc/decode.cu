@@ -367,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float tmax = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]),
                                              fmaxf(sm.red[2][h], sm.red[3][h]));
                     const float mn = fmaxf(m_run[h], tmax);
-                    alpha[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - mn);
+                    alpha[h] = (m_run[h] == mn) ? 1.f : exp2f(m_run[h] - mn);
                     rescale |= (t > 0) && (alpha[h] != 1.f);
                     m_run[h] = mn;
                 }
@@ -378,9 +378,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int h = 0; h < kN; ++h) {
                         const float p = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m_run[h]);
-                        l_part[h] = l_part[h] * alpha[h] + p;
-                        *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(h, kc)) =
-                            __float2bfloat16_rn(p);
+                        const __nv_bfloat16 pr = __float2bfloat16_rn(p);
+                        // the running sum uses the rounded weight the MMA sees
+                        l_part[h] = l_part[h] * alpha[h] + __bfloat162float(pr);
+                        *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(h, kc)) = pr;
                     }
                 }
                 // rescale O^T when a running max moved.  O is idle: the MMA that wrote S for

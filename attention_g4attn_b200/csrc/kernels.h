@@ -24,6 +24,7 @@ struct QkNormRopeArgs {
     const float* gamma_q;
     const float* gamma_k;
     float2* cs_out;       // optional [T, R] (cos, sin) table of positions pos0 + t
+    int k_f16;            // 1: k_out / krot_out are written as fp16 instead of bf16
     int B, T, Hq, Hkv, d;
     long long pos0;
     Rope rope;

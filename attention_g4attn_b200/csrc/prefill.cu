@@ -3,15 +3,18 @@
 // One CTA computes one 128-row tile of packed query rows: row r is token m0 + r / G of
 // query head g*G + r % G, i.e. the G query heads that share kv head g sit in the MMA M
 // dimension (GQA; explainer "GQA": 8:1 in global layers, 2:1 in local layers).
-//   prologue  raw q rows -> RMSNorm * gamma -> RoPE / p-RoPE -> bf16, 128-byte-swizzled
+//   prologue  raw q rows -> RMSNorm * gamma -> RoPE / p-RoPE -> fp16, 128-byte-swizzled
 //             K-major tile in shared memory (report section 2: QKNorm, p-RoPE)
+//   The normalised key copies written by the key pre-pass are fp16 too: QKNorm bounds
+//   their range, and fp16 keeps 3 more mantissa bits than bf16 for the values that
+//   keys-as-values layers feed straight into the output.
 //   per key tile of 128 keys (causal / sliding-window tiles outside the band are skipped):
 //     S  = Q K^T        tcgen05.mma M=128 N=128, fp32 in TMEM, K streamed in 64-dim chunks
 //                       (rotated chunks from the rotated key copy, the rest from the
 //                       normalised pre-RoPE keys)
 //     softmax           thread = row: masked row max (lazy: the reference max only moves
-//                       when the tile max exceeds it by more than 2^8), P = exp2 -> bf16
-//                       into shared memory, running sum
+//                       when the tile max exceeds it by more than 2^8), P = exp2 rounded to
+//                       the format of V into shared memory, running sum of the rounded P
 //     O += P V          tcgen05.mma M=128 N=256, V read MN-major from the same 64-dim
 //                       chunk layout; V is the pre-RoPE normalised key (keys reused as
 //                       values), the rotated key, or the separate values
@@ -168,8 +171,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16_f32(128, kBN, false, false);
-            const uint32_t idesc_o = idesc_bf16_f32(128, 256, false, true);   // B = V, MN-major
+            // S in fp16 (normalised q and k copies); P.V in fp16 when V is the normalised key
+            // copy, in bf16 when V is the caller's bf16 values
+            const uint32_t idesc_s = idesc_f16kind_f32(128, kBN, false, false, false);
+            const uint32_t idesc_o = idesc_f16kind_f32(128, 256, false, true, a.kv_is_k == 0);
             uint32_t q = 0;
             for (int n = 0; n < ntiles; ++n) {
                 if (!mbar_wait(&sm.s_free, n & 1, wc, abort)) goto done;
@@ -273,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int col = hh * half + lane * E;
                     uint32_t w[E / 2];
 #pragma unroll
-                    for (int e = 0; e < E; e += 2) w[e / 2] = pack_bf16x2(x[e], x[e + 1]);
+                    for (int e = 0; e < E; e += 2) w[e / 2] = pack_f16x2(x[e], x[e + 1]);
                     uint8_t* base = sm.q[col / 64];
                     const uint32_t off = sw128_offset(r, col % 64);
                     if constexpr (E == 8)
@@ -290,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 
         // ---- main loop
+        const bool p_f16 = a.kv_is_k != 0;           // P in the format of V
         const int tok_r = tg.m0 + row / G;          // token of this row
         const bool row_valid = (row / G) < tg.tq;
         float m_ref = -INFINITY, l_sum = 0.f;
@@ -362,9 +368,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int j = key0 + c * 16 + e + u;
                         const bool vis = row_valid && (!need_mask || (j <= tok_r && j >= lo_r));
                         pv[u] = vis ? exp2f(fmaf(s[e + u], a.scale_log2, -m_ref)) : 0.f;
-                        psum += pv[u];
                     }
-                    w[e / 2] = pack_bf16x2(pv[0], pv[1]);
+                    // the row sum uses the rounded weights the MMA sees
+                    if (p_f16) {
+                        const __half2 h = __floats2half2_rn(pv[0], pv[1]);
+                        const float2 f = __half22float2(h);
+                        psum += f.x + f.y;
+                        w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+                    } else {
+                        const __nv_bfloat162 h = __floats2bfloat162_rn(pv[0], pv[1]);
+                        const float2 f = __bfloat1622float2(h);
+                        psum += f.x + f.y;
+                        w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+                    }
                 }
                 uint8_t* pb = sm.p[c >> 2];
                 const int col = (c & 3) * 16;

@@ -6,6 +6,7 @@
 // QKNorm), then turns the pairs (i, i + d/2), i < R (p-RoPE).  Lane l owns elements
 // [l*E, l*E + E) of both halves of the row, so a pair never leaves its lane.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.h"
 #include "rope.cuh"
@@ -43,6 +44,21 @@ __device__ __forceinline__ void store_bf16(uint16_t* p, const float* v) {
 #pragma unroll
     for (int i = 0; i < E / 2; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
     *reinterpret_cast<typename Vec<E>::T*>(p) = raw;
+}
+
+template <int E>
+__device__ __forceinline__ void store_f16(uint16_t* p, const float* v) {
+    typename Vec<E>::T raw;
+    __half2* h = reinterpret_cast<__half2*>(&raw);
+#pragma unroll
+    for (int i = 0; i < E / 2; ++i) h[i] = __floats2half2_rn(v[2 * i], v[2 * i + 1]);
+    *reinterpret_cast<typename Vec<E>::T*>(p) = raw;
+}
+
+template <int E>
+__device__ __forceinline__ void store_row_half(uint16_t* p, const float* v, bool f16) {
+    if (f16) store_f16<E>(p, v);
+    else store_bf16<E>(p, v);
 }
 
 template <int E>
@@ -84,10 +100,11 @@ __global__ void __launch_bounds__(kThreads) qknorm_rope_kernel(QkNormRopeArgs a)
                 x1[e] = x1[e] * inv * gamma[half + lane * E + e];
             }
         }
+        const bool f16 = !is_q && a.k_f16;
         if (!is_q && a.k_out) {
             uint16_t* dst = a.k_out + (bt * a.Hkv + h) * (long long)d;
-            store_bf16<E>(dst + lane * E, x0);
-            store_bf16<E>(dst + half + lane * E, x1);
+            store_row_half<E>(dst + lane * E, x0, f16);
+            store_row_half<E>(dst + half + lane * E, x1, f16);
         }
         uint16_t* rdst = is_q ? (a.q_out ? a.q_out + (bt * a.Hq + h) * (long long)d : nullptr)
                               : (a.krot_out ? a.krot_out + (bt * a.Hkv + h) * (long long)d
@@ -103,8 +120,8 @@ __global__ void __launch_bounds__(kThreads) qknorm_rope_kernel(QkNormRopeArgs a)
                     x1[e] = u * c.y + w * c.x;
                 }
             }
-            store_bf16<E>(rdst + lane * E, x0);
-            store_bf16<E>(rdst + half + lane * E, x1);
+            store_row_half<E>(rdst + lane * E, x0, f16);
+            store_row_half<E>(rdst + half + lane * E, x1, f16);
         }
     }
 }
