@@ -113,12 +113,13 @@ int check_cfg(const g4attn_layer_cfg* c, bool tensor_core_path) {
     return G4ATTN_OK;
 }
 
-// 4-D map over a [B, T, H, d] bf16 tensor: dims (d, H, T, B), box (64, 1, 128, 1),
+// 4-D map over a [B, T, H, d] 16-bit tensor: dims (d, H, T, B), box (64, 1, box_rows, 1),
 // 128-byte swizzle, zero fill outside the tensor.
-int encode_rows(CUtensorMap* m, const void* base, int B, int T, int H, int d, bool f16 = false) {
+int encode_rows(CUtensorMap* m, const void* base, int B, int T, int H, int d, bool f16 = false,
+                int box_rows = 128) {
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
-    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
     CUresult r = g_encode(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                           4, const_cast<void*>(base), dims,
@@ -310,10 +311,13 @@ int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16
 
     // 2) the fused flash-attention kernel
     g4::PrefillArgs a{};
-    if ((rc = encode_rows(&a.tm_kr, kr, B, T, Hkv, d, true))) return rc;
-    if ((rc = encode_rows(&a.tm_kn, kn ? kn : kr, B, T, Hkv, d, true))) return rc;
-    if (v) rc = encode_rows(&a.tm_v, v, B, T, Hkv, d, false);
-    else rc = encode_rows(&a.tm_v, kn ? kn : kr, B, T, Hkv, d, true);
+    const uint16_t* kn_or_kr = kn ? kn : kr;
+    if ((rc = encode_rows(&a.tm_kr_s, kr, B, T, Hkv, d, true, 64))) return rc;
+    if ((rc = encode_rows(&a.tm_kn_s, kn_or_kr, B, T, Hkv, d, true, 64))) return rc;
+    if ((rc = encode_rows(&a.tm_kr_v, kr, B, T, Hkv, d, true, 128))) return rc;
+    if ((rc = encode_rows(&a.tm_kn_v, kn_or_kr, B, T, Hkv, d, true, 128))) return rc;
+    if (v) rc = encode_rows(&a.tm_v, v, B, T, Hkv, d, false, 128);
+    else rc = encode_rows(&a.tm_v, kn_or_kr, B, T, Hkv, d, true, 128);
     if (rc) return rc;
     a.q = q;
     a.gamma_q = gamma_q;

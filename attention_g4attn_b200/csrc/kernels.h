@@ -58,9 +58,14 @@ size_t decode_smem_bytes();
 
 // Flash-attention prefill.
 struct PrefillArgs {
-    CUtensorMap tm_kn;      // normalised pre-RoPE keys  (d, Hkv, T, B), box (64, 1, 128, 1)
-    CUtensorMap tm_kr;      // normalised rotated keys, same geometry
-    CUtensorMap tm_v;       // separate values, same geometry (kv_is_k == 0), else = tm_kn
+    // 4-D maps over [B, T, Hkv, d] as (d, Hkv, T, B), 128-byte swizzle.  The *_s maps load
+    // 64 dims x 64 keys (the score operand, half a key tile per CTA of a pair); the *_v
+    // maps load 64 dims x 128 keys (the value operand).
+    CUtensorMap tm_kn_s;    // normalised pre-RoPE keys (fp16)
+    CUtensorMap tm_kr_s;    // normalised rotated keys (fp16)
+    CUtensorMap tm_kn_v;
+    CUtensorMap tm_kr_v;
+    CUtensorMap tm_v;       // separate values (bf16, kv_is_k == 0), else a copy of tm_kn_v
     const uint16_t* q;      // raw queries [B, T, Hq, d]
     const float* gamma_q;
     const float2* rope_cs;  // [T, R] (cos, sin) of position t, pair i

@@ -1,31 +1,35 @@
-// prefill.cu -- flash-attention prefill for the Gemma-4-style layer on tcgen05 / TMEM.
+// prefill.cu -- flash-attention prefill for the Gemma-4-style layer on tcgen05 / TMEM,
+// run by pairs of CTAs (a 2-CTA cluster issuing cta_group::2 MMAs).
 //
-// One CTA computes one 128-row tile of packed query rows: row r is token m0 + r / G of
-// query head g*G + r % G, i.e. the G query heads that share kv head g sit in the MMA M
-// dimension (GQA; explainer "GQA": 8:1 in global layers, 2:1 in local layers).
+// Each CTA owns one 128-row tile of packed query rows: row r is token m0 + r / G of query
+// head g*G + r % G, so the G query heads that share kv head g sit in the MMA M dimension
+// (GQA; explainer "GQA": 8:1 in global layers, 2:1 in local layers).  The two CTAs of a
+// pair hold consecutive row tiles of the same (batch, kv head) and share every key tile:
+// one MMA of M = 256 covers both row tiles while each CTA stages only half of the key
+// tile (S: 64 of the 128 keys; P.V: 128 of the 256 value dims of an N=256 block), which
+// halves the shared-memory and L2 traffic per CTA.
 //   prologue  raw q rows -> RMSNorm * gamma -> RoPE / p-RoPE -> fp16, 128-byte-swizzled
-//             K-major tile in shared memory (report section 2: QKNorm, p-RoPE)
-//   The normalised key copies written by the key pre-pass are fp16 too: QKNorm bounds
-//   their range, and fp16 keeps 3 more mantissa bits than bf16 for the values that
-//   keys-as-values layers feed straight into the output.
+//             K-major tile in shared memory (report section 2: QKNorm, p-RoPE).  The key
+//             pre-pass writes the normalised keys (pre-RoPE and rotated) as fp16 too:
+//             QKNorm bounds their range and fp16 keeps 3 more mantissa bits than bf16 for
+//             the values that keys-as-values layers feed straight into the output.
 //   per key tile of 128 keys (causal / sliding-window tiles outside the band are skipped):
-//     S  = Q K^T        tcgen05.mma M=128 N=128, fp32 in TMEM, K streamed in 64-dim chunks
-//                       (rotated chunks from the rotated key copy, the rest from the
-//                       normalised pre-RoPE keys)
-//     softmax           thread = row: masked row max (lazy: the reference max only moves
+//     S  = Q K^T        M=256 N=128, fp32 in TMEM; rotated 64-dim chunks come from the
+//                       rotated key copy, the others from the pre-RoPE copy
+//     softmax           thread = row: masked row max with a lazy reference (it only moves
 //                       when the tile max exceeds it by more than 2^8), P = exp2 rounded to
 //                       the format of V into shared memory, running sum of the rounded P
-//     O += P V          tcgen05.mma M=128 N=256, V read MN-major from the same 64-dim
-//                       chunk layout; V is the pre-RoPE normalised key (keys reused as
-//                       values), the rotated key, or the separate values
-//   epilogue  O / l -> bf16 rows; lse = m + log2(l) (natural log on output)
-// head_dim 512: the 128 x 512 fp32 O accumulator fills all 512 TMEM columns, so the S
-// tile borrows columns [128, 256): the softmax warps hold that quarter of O in registers
-// while S lives there and put it back before the PV product.
+//     O += P V          M=256 N=256 per 256-dim block, V read MN-major; V is the pre-RoPE
+//                       key (keys reused as values), the rotated key, or the caller's values
+//   epilogue  O / l -> bf16 rows; lse = (m + log2 l) ln 2
+// head_dim 512: a 128 x 512 fp32 O fills all 512 TMEM columns, so S borrows columns
+// [128, 256): the softmax warps hold that quarter of O in registers while S lives there.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer + TMEM owner,
-// warps 2..5 prologue / softmax / correction / epilogue.  Every wait is bounded.
+// Warp roles (192 threads per CTA): warp 0 TMA producer (both CTAs), warp 1 TMEM owner and,
+// in the leader CTA, the MMA issuer; warps 2..5 prologue / softmax / epilogue.  Every wait
+// is bounded; a CTA that gives up raises the abort flag of both CTAs of its pair.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.h"
 #include "sm100.cuh"
@@ -35,8 +39,8 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kBM = 128;               // packed query rows per CTA
-constexpr int kBN = 128;               // keys per tile
-constexpr int kChunkBytes = 16384;     // 128 keys x 64 dims bf16, 128-byte swizzle
+constexpr int kBN = 128;               // keys per tile (shared by the pair)
+constexpr int kSlot = 16384;           // ring slot: 64 keys x 128 dims (S) or 128 keys x 64 dims (V)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kBarWG = 1;
 constexpr float kLazyMax = 8.0f;       // log2 units
@@ -47,15 +51,17 @@ struct PrefillCfg {
     static constexpr bool SWAP = (D == 512);
     static constexpr int NSLOT = (D == 512) ? 4 : 8;
     static constexpr uint32_t S_COL = (D == 512) ? 128 : 256;
+    static constexpr int NS = D / 128;     // S stages per tile (128 dims each)
+    static constexpr int NV = D / 256;     // P.V blocks per tile (2 slots each)
 };
 
 template <int D>
 struct __align__(1024) PrefillSmem {
-    uint8_t q[PrefillCfg<D>::NCH][kChunkBytes];    // 128 rows x 64 dims per chunk
-    uint8_t p[2][kChunkBytes];                     // P: 128 rows x 64 keys per chunk
-    uint8_t ring[PrefillCfg<D>::NSLOT][kChunkBytes];
-    uint64_t full[PrefillCfg<D>::NSLOT];
-    uint64_t empty[PrefillCfg<D>::NSLOT];
+    uint8_t q[PrefillCfg<D>::NCH][16384];  // 128 rows x 64 dims per chunk
+    uint8_t p[2][16384];                   // P: 128 rows x 64 keys per chunk
+    uint8_t ring[PrefillCfg<D>::NSLOT][kSlot];
+    uint64_t full[PrefillCfg<D>::NSLOT];   // used in the leader: both CTAs' bytes land here
+    uint64_t empty[PrefillCfg<D>::NSLOT];  // per CTA, released by the leader's MMA commits
     uint64_t s_free, s_full, p_full, o_done, drain;
     uint32_t tmem_base;
     int abort;
@@ -66,29 +72,32 @@ __device__ __forceinline__ bool chunk_rotated(int c, int d, int R) {
     return (lo < R) || (lo < h + R && hi > h);
 }
 
-struct TileGeom {
-    int b, g, m0;      // batch, kv head, first token of the tile
-    int tq;            // tokens in the tile (<= 128 / G)
-    int j_lo, j_hi;    // key tiles visited (inclusive)
+struct PairGeom {
+    int b, g;
+    int m0, tq;        // this CTA: first token, valid tokens (<= 0: no valid row)
+    int j_lo, j_hi;    // key tiles visited by the pair (inclusive)
 };
 
-__device__ __forceinline__ TileGeom tile_geom(const PrefillArgs& a) {
-    TileGeom g;
-    const int tpt = kBM / a.G;                         // tokens per tile
+__device__ __forceinline__ PairGeom pair_geom(const PrefillArgs& a, uint32_t rank) {
+    PairGeom g;
+    const int tpt = kBM / a.G;                          // tokens per row tile
     const int mt_count = (a.T + tpt - 1) / tpt;
-    // heavy tiles first: the last query tiles of a causal layer see the most keys
-    const int idx = blockIdx.x;
-    const int mt = mt_count - 1 - idx / (a.B * a.Hkv);
-    const int bg = idx % (a.B * a.Hkv);
+    const int pairs = (mt_count + 1) / 2;
+    const int c = blockIdx.x >> 1;                      // cluster index
+    const int bgn = a.B * a.Hkv;
+    const int pr = pairs - 1 - c / bgn;                 // heavy (late) row tiles first
+    const int bg = c % bgn;
     g.b = bg / a.Hkv;
     g.g = bg % a.Hkv;
+    const int mt = 2 * pr + (int)rank;
     g.m0 = mt * tpt;
     g.tq = min(tpt, a.T - g.m0);
-    const int t_last = g.m0 + g.tq - 1;
+    const int first_tok = 2 * pr * tpt;
+    const int last_tok = min(a.T, (2 * pr + 2) * tpt) - 1;
     int k_first = 0;
-    if (a.window > 0) k_first = max(0, g.m0 - a.window + 1);
+    if (a.window > 0) k_first = max(0, first_tok - a.window + 1);
     g.j_lo = k_first / kBN;
-    g.j_hi = t_last / kBN;
+    g.j_hi = last_tok / kBN;
     return g;
 }
 
@@ -102,118 +111,124 @@ __global__ void __launch_bounds__(kThreads, 1)
     PrefillSmem<D>& sm = *reinterpret_cast<PrefillSmem<D>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
     const WaitCtl wc{a.wait_limit, a.status};
     volatile int* abort = &sm.abort;
     const int R = a.rope.R;
-    const TileGeom tg = tile_geom(a);
-    const int ntiles = tg.j_hi - tg.j_lo + 1;
+    const PairGeom pg = pair_geom(a, rank);
+    const int ntiles = pg.j_hi - pg.j_lo + 1;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NSLOT; ++i) {
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], 1);
         }
-        mbar_init(&sm.s_free, 1);
+        mbar_init(&sm.s_free, 2);   // one arrival per CTA of the pair
         mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.p_full, 1);
+        mbar_init(&sm.p_full, 2);
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
+    if (warp == 1) tmem_alloc_pair(&sm.tmem_base, kTmemCols);
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t tm_o = tmem;
     const uint32_t tm_s = tmem + C::S_COL;
 
     if (warp == 0) {
-        // ---------------------------------------------------------------- TMA producer
+        // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            prefetch_tmap(&a.tm_kn);
-            prefetch_tmap(&a.tm_kr);
+            prefetch_tmap(&a.tm_kn_s);
+            prefetch_tmap(&a.tm_kr_s);
+            prefetch_tmap(&a.tm_kn_v);
+            prefetch_tmap(&a.tm_kr_v);
             prefetch_tmap(&a.tm_v);
             uint32_t q = 0;
             for (int n = 0; n < ntiles && !*abort; ++n) {
-                const int key = (tg.j_lo + n) * kBN;
-                if (n + 2 < ntiles)
-                    for (int c = 0; c < NCH; ++c) {
-                        const bool rot = chunk_rotated(c, D, R);
-                        const CUtensorMap* ms = rot ? &a.tm_kr : &a.tm_kn;
-                        const CUtensorMap* mv = a.kv_is_k == 0 ? &a.tm_v
-                                                : (a.kv_is_k == 2 && rot) ? &a.tm_kr : &a.tm_kn;
-                        tma_prefetch_l2_4d(ms, c * 64, tg.g, key + 2 * kBN, tg.b);
-                        if (mv != ms) tma_prefetch_l2_4d(mv, c * 64, tg.g, key + 2 * kBN, tg.b);
+                const int key0 = (pg.j_lo + n) * kBN;
+                if (n + 2 < ntiles) {   // pull this CTA's share of a later tile into L2
+                    const int kp = key0 + 2 * kBN;
+                    for (int c = 0; c < NCH; ++c)
+                        tma_prefetch_l2_4d(chunk_rotated(c, D, R) ? &a.tm_kr_s : &a.tm_kn_s,
+                                           c * 64, pg.g, kp + 64 * (int)rank, pg.b);
+                }
+                for (int s = 0; s < C::NS && !*abort; ++s, ++q) {
+                    const int slot = q % NSLOT;
+                    if (!mbar_wait(&sm.empty[slot], ((q / NSLOT) & 1) ^ 1, wc, abort)) break;
+                    if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlot);
+                    for (int h = 0; h < 2; ++h) {
+                        const int c = 2 * s + h;
+                        const CUtensorMap* map = chunk_rotated(c, D, R) ? &a.tm_kr_s : &a.tm_kn_s;
+                        tma_load_4d_pair(sm.ring[slot] + h * (kSlot / 2), map, &sm.full[slot],
+                                         c * 64, pg.g, key0 + 64 * (int)rank, pg.b);
                     }
-                // S chunks then V chunks, in consumption order
-                for (int pass = 0; pass < 2 && !*abort; ++pass)
-                    for (int c = 0; c < NCH; ++c) {
-                        const bool rot = chunk_rotated(c, D, R);
-                        const CUtensorMap* map;
-                        if (pass == 0) map = rot ? &a.tm_kr : &a.tm_kn;
-                        else if (a.kv_is_k == 0) map = &a.tm_v;
-                        else map = (a.kv_is_k == 2 && rot) ? &a.tm_kr : &a.tm_kn;
+                }
+                for (int v = 0; v < C::NV && !*abort; ++v)
+                    for (int u = 0; u < 2 && !*abort; ++u, ++q) {
                         const int slot = q % NSLOT;
                         if (!mbar_wait(&sm.empty[slot], ((q / NSLOT) & 1) ^ 1, wc, abort)) break;
-                        mbar_arrive_expect_tx(&sm.full[slot], kChunkBytes);
-                        tma_load_4d(sm.ring[slot], map, &sm.full[slot], c * 64, tg.g, key, tg.b);
-                        ++q;
+                        if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlot);
+                        const int c = 4 * v + 2 * (int)rank + u;   // this CTA's half of the block
+                        const bool rot = chunk_rotated(c, D, R);
+                        const CUtensorMap* map = a.kv_is_k == 0 ? &a.tm_v
+                                                 : (a.kv_is_k == 2 && rot) ? &a.tm_kr_v
+                                                                           : &a.tm_kn_v;
+                        tma_load_4d_pair(sm.ring[slot], map, &sm.full[slot], c * 64, pg.g, key0,
+                                         pg.b);
                     }
-            }
-            if (*abort) {
-                const uint32_t first = q > (uint32_t)NSLOT ? q - NSLOT : 0;
-                for (uint32_t k = first; k < q; ++k)
-                    mbar_wait_drain(&sm.full[k % NSLOT], (k / NSLOT) & 1, a.wait_limit);
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            // S in fp16 (normalised q and k copies); P.V in fp16 when V is the normalised key
-            // copy, in bf16 when V is the caller's bf16 values
-            const uint32_t idesc_s = idesc_f16kind_f32(128, kBN, false, false, false);
-            const uint32_t idesc_o = idesc_f16kind_f32(128, 256, false, true, a.kv_is_k == 0);
+        // ------------------------------------------------ MMA issuer (leader CTA only)
+        if (lane == 0 && leader) {
+            const uint32_t idesc_s = idesc_f16kind_f32(256, kBN, false, false, false);
+            const uint32_t idesc_o = idesc_f16kind_f32(256, 256, false, true, a.kv_is_k == 0);
             uint32_t q = 0;
             for (int n = 0; n < ntiles; ++n) {
-                if (!mbar_wait(&sm.s_free, n & 1, wc, abort)) goto done;
+                if (!mbar_wait_cluster(&sm.s_free, n & 1, wc, abort)) goto done;
                 tc_fence_after();
-                for (int c = 0; c < NCH; ++c, ++q) {
+                for (int s = 0; s < C::NS; ++s, ++q) {
                     const uint32_t slot = q % NSLOT;
-                    if (!mbar_wait(&sm.full[slot], (q / NSLOT) & 1, wc, abort)) goto done;
+                    if (!mbar_wait_cluster(&sm.full[slot], (q / NSLOT) & 1, wc, abort)) goto done;
                     tc_fence_after();
-                    const uint32_t ab = smem_u32(sm.q[c]);
-                    const uint32_t bb = smem_u32(sm.ring[slot]);
-                    for (int kk = 0; kk < 4; ++kk)
-                        mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
-                                    sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
-                                    (c | kk) != 0 ? 1u : 0u);
-                    mma_commit(&sm.empty[slot]);
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const uint32_t ab = smem_u32(sm.q[2 * s + (kk >> 2)]) + (kk & 3) * 32;
+                        const uint32_t bb =
+                            smem_u32(sm.ring[slot]) + (kk >> 2) * (kSlot / 2) + (kk & 3) * 32;
+                        mma_pair_f16(tm_s, sdesc_sw128(ab, 16, 1024), sdesc_sw128(bb, 16, 1024),
+                                     idesc_s, (s | kk) != 0 ? 1u : 0u);
+                    }
+                    mma_commit_pair(&sm.empty[slot]);
                 }
-                mma_commit(&sm.s_full);
-                if (!mbar_wait(&sm.p_full, n & 1, wc, abort)) goto done;
+                mma_commit_pair(&sm.s_full);
+                if (!mbar_wait_cluster(&sm.p_full, n & 1, wc, abort)) goto done;
                 tc_fence_after();
-                // O[:, 256*grp + 0..255] += P . V[:, 256*grp ...]: four consecutive ring slots
-                for (int grp = 0; grp < NCH / 4; ++grp) {
-                    const uint32_t q0 = q;
-                    for (int u = 0; u < 4; ++u, ++q)
-                        if (!mbar_wait(&sm.full[q % NSLOT], (q / NSLOT) & 1, wc, abort)) goto done;
+                for (int v = 0; v < C::NV; ++v, q += 2) {
+                    const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
+                    if (!mbar_wait_cluster(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
+                    if (!mbar_wait_cluster(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
+                        goto done;
                     tc_fence_after();
-                    const uint32_t vb = smem_u32(sm.ring[q0 % NSLOT]);
+                    const uint32_t vb = smem_u32(sm.ring[s0]);
                     for (int kk = 0; kk < 8; ++kk) {
                         const uint32_t pa = smem_u32(sm.p[kk >> 2]) + (kk & 3) * 32;
-                        mma_bf16_ss(tm_o + grp * 256, sdesc_sw128(pa, 16, 1024),
-                                    sdesc_sw128(vb + kk * 2048, kChunkBytes, 1024), idesc_o,
-                                    (n > 0 || kk > 0) ? 1u : 0u);
+                        // V: 16 keys per step (two 8-row groups of 1024 B); the CTA's second
+                        // 64-dim chunk sits in the next slot (LBO)
+                        mma_pair_f16(tm_o + v * 256, sdesc_sw128(pa, 16, 1024),
+                                     sdesc_sw128(vb + kk * 2048, kSlot, 1024), idesc_o,
+                                     (n > 0 || kk > 0) ? 1u : 0u);
                     }
-                    for (int u = 0; u < 4; ++u) mma_commit(&sm.empty[(q0 + u) % NSLOT]);
+                    mma_commit_pair(&sm.empty[s0]);
+                    mma_commit_pair(&sm.empty[s1]);
                 }
-                if (C::SWAP || n == ntiles - 1) mma_commit(&sm.o_done);
+                if (C::SWAP || n == ntiles - 1) mma_commit_pair(&sm.o_done);
             }
-        done:
-            mma_commit(&sm.drain);
-            mbar_wait_drain(&sm.drain, 0, a.wait_limit);
+        done:;
         }
     } else {
         // ------------------------------------ prologue / softmax / correction / epilogue
@@ -230,11 +245,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int half = D / 2;
             for (int r = wq; r < kBM; r += 4) {
                 const int tl = r / G, hl = r % G;
-                const int tok = tg.m0 + tl;
+                const int tok = pg.m0 + tl;
                 float x0[E], x1[E];
-                if (tl < tg.tq) {
+                if (tl < pg.tq) {
                     const uint16_t* src =
-                        a.q + (((size_t)tg.b * a.T + tok) * a.Hq + (size_t)tg.g * G + hl) * D;
+                        a.q + (((size_t)pg.b * a.T + tok) * a.Hq + (size_t)pg.g * G + hl) * D;
 #pragma unroll
                     for (int e = 0; e < E; e += 2) {
                         const float2 f0 = __bfloat1622float2(
@@ -271,7 +286,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < E; ++e) x0[e] = x1[e] = 0.f;
                 }
-                // store: element (r, col) of chunk col / 64
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     const float* x = hh ? x1 : x0;
@@ -291,13 +305,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             group_sync(kBarWG, 128);
-            if (t128 == 0) mbar_arrive(&sm.s_free);   // Q ready, S region free for tile 0
+            if (t128 == 0) mbar_arrive_remote(&sm.s_free, 0);   // Q ready, S free for tile 0
         }
 
         // ---- main loop
         const bool p_f16 = a.kv_is_k != 0;           // P in the format of V
-        const int tok_r = tg.m0 + row / G;          // token of this row
-        const bool row_valid = (row / G) < tg.tq;
+        const int tok_r = pg.m0 + row / G;          // token of this row
+        const bool row_valid = (row / G) < pg.tq;
+        const int t_first = pg.m0, t_last = pg.m0 + pg.tq - 1;
         float m_ref = -INFINITY, l_sum = 0.f;
         float o1[C::SWAP ? 128 : 1];
         if constexpr (C::SWAP) {
@@ -306,7 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         bool ok = true;
         for (int n = 0; n < ntiles && ok; ++n) {
-            const int key0 = (tg.j_lo + n) * kBN;
+            const int key0 = (pg.j_lo + n) * kBN;
             if constexpr (C::SWAP) {
                 if (n > 0) {
                     // O[:, 128..255] leaves TMEM so S(n) can use those columns
@@ -318,16 +333,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_wait();
                     tc_fence_before();
                     group_sync(kBarWG, 128);
-                    if (t128 == 0) mbar_arrive(&sm.s_free);
+                    if (t128 == 0) mbar_arrive_remote(&sm.s_free, 0);
                 }
             } else {
-                if (n > 0 && t128 == 0) mbar_arrive(&sm.s_free);
+                if (n > 0 && t128 == 0) mbar_arrive_remote(&sm.s_free, 0);
             }
             ok = group_all(mbar_wait(&sm.s_full, n & 1, wc, abort), kBarWG, 128);
             if (!ok) break;
             tc_fence_after();
-            // does any key of this tile need masking for any row of the CTA?
-            const int t_first = tg.m0, t_last = tg.m0 + tg.tq - 1;
             const bool need_mask = (key0 + kBN - 1 > t_first) ||
                                    (a.window > 0 && key0 <= t_last - a.window);
             const int lo_r = a.window > 0 ? tok_r - a.window + 1 : 0;
@@ -346,13 +359,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (!row_valid) mx = -INFINITY;
-            // lazy reference max: move it only when the tile max exceeds it by > 2^8
             float alpha = 1.f;
             if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
                 alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
                 m_ref = mx;
             }
-            // pass 2: P = exp2(s * scale_log2 - m_ref) as bf16 into the A tile of P.V
+            // pass 2: P = exp2(s * scale_log2 - m_ref), rounded, into the A tile of P.V
             float psum = 0.f;
 #pragma unroll 1
             for (int c = 0; c < 8; ++c) {
@@ -369,7 +381,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const bool vis = row_valid && (!need_mask || (j <= tok_r && j >= lo_r));
                         pv[u] = vis ? exp2f(fmaf(s[e + u], a.scale_log2, -m_ref)) : 0.f;
                     }
-                    // the row sum uses the rounded weights the MMA sees
                     if (p_f16) {
                         const __half2 h = __floats2half2_rn(pv[0], pv[1]);
                         const float2 f = __half22float2(h);
@@ -417,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             group_sync(kBarWG, 128);
-            if (t128 == 0) mbar_arrive(&sm.p_full);
+            if (t128 == 0) mbar_arrive_remote(&sm.p_full, 0);
         }
         // ---- epilogue
         if (ok) {
@@ -427,8 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             tc_fence_after();
             const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
-            const int h = tg.g * G + row % G;
-            uint16_t* dst = a.out + (((size_t)tg.b * a.T + tok_r) * a.Hq + h) * D;
+            const int h = pg.g * G + row % G;
+            uint16_t* dst = a.out + (((size_t)pg.b * a.T + tok_r) * a.Hq + h) * D;
             for (int c = 0; c < D / 16; ++c) {
                 float o[16];
                 tmem_ld16(tm_o + c * 16 + lane_off, o);
@@ -442,17 +453,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (row_valid && a.lse)
-                a.lse[((size_t)tg.b * a.Hq + h) * a.T + tok_r] =
+                a.lse[((size_t)pg.b * a.Hq + h) * a.T + tok_r] =
                     l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
         }
     }
 
     // -------------------------------------------------------------------- teardown
-    tc_fence_before();
+    // A CTA that gave up tells its peer, so the peer's waits end promptly too.
     __syncthreads();
+    if (*abort && threadIdx.x == 0) st_shared_remote_u32((const void*)&sm.abort, rank ^ 1u, 1u);
+    tc_fence_before();
+    cluster_sync();
+    if (leader && warp == 1 && lane == 0) {
+        // every MMA of the pair must be complete before either CTA frees its columns
+        mma_commit_pair(&sm.drain);
+        mbar_wait_drain(&sm.drain, 0, a.wait_limit);
+    }
+    tc_fence_before();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc_pair(tmem, kTmemCols);
     }
 }
 
@@ -464,8 +485,21 @@ cudaError_t run_prefill(const PrefillArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     const int tpt = kBM / a.G;
     const int mt_count = (a.T + tpt - 1) / tpt;
-    const long long grid = (long long)mt_count * a.B * a.Hkv;
-    prefill_kernel<D><<<(unsigned)grid, kThreads, smem, stream>>>(a);
+    const int pairs = (mt_count + 1) / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2LL * pairs * a.B * a.Hkv), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, prefill_kernel<D>, a);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
