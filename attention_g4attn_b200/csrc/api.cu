@@ -99,7 +99,7 @@ int check_cfg(const g4attn_layer_cfg* c, bool tensor_core_path) {
     if (!(c->rope_p >= 0.f && c->rope_p <= 1.f)) return G4ATTN_ERR_INVALID_ARG;
     if (!(c->rope_base > 0.0) || !std::isfinite(c->rope_base)) return G4ATTN_ERR_INVALID_ARG;
     if (c->window < 0) return G4ATTN_ERR_INVALID_ARG;
-    if (!std::isfinite(c->scale)) return G4ATTN_ERR_INVALID_ARG;
+    if (!std::isfinite(c->scale) || !(c->scale > 0.f)) return G4ATTN_ERR_INVALID_ARG;
     if (c->kv_is_k < 0 || c->kv_is_k > 2) return G4ATTN_ERR_INVALID_ARG;
     if (c->qk_norm != 0 && c->qk_norm != 1) return G4ATTN_ERR_INVALID_ARG;
     if (c->qk_norm && !(c->qk_norm_eps >= 0.f)) return G4ATTN_ERR_INVALID_ARG;

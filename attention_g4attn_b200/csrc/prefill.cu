@@ -101,7 +101,7 @@ __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs& a, uint32_t ran
     return g;
 }
 
-template <int D>
+template <int D, bool PF16>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillArgs a) {
     using C = PrefillCfg<D>;
@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ MMA issuer (leader CTA only)
         if (lane == 0 && leader) {
             const uint32_t idesc_s = idesc_f16kind_f32(256, kBN, false, false, false);
-            const uint32_t idesc_o = idesc_f16kind_f32(256, 256, false, true, a.kv_is_k == 0);
+            const uint32_t idesc_o = idesc_f16kind_f32(256, 256, false, true, !PF16);
             uint32_t q = 0;
             for (int n = 0; n < ntiles; ++n) {
                 if (!mbar_wait_cluster(&sm.s_free, n & 1, wc, abort)) goto done;
@@ -309,15 +309,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 
         // ---- main loop
-        const bool p_f16 = a.kv_is_k != 0;           // P in the format of V
         const int tok_r = pg.m0 + row / G;          // token of this row
         const bool row_valid = (row / G) < pg.tq;
         const int t_first = pg.m0, t_last = pg.m0 + pg.tq - 1;
-        float m_ref = -INFINITY, l_sum = 0.f;
-        float o1[C::SWAP ? 128 : 1];
+        const float c2 = a.scale_log2;              // > 0 (checked on the host)
+        // rows past the end of the sequence hold zero queries; a finite reference keeps
+        // their (never stored) P finite on the unmasked path
+        float m_ref = row_valid ? -INFINITY : 0.f, l_sum = 0.f;
+        uint32_t o1[C::SWAP ? 128 : 1];
         if constexpr (C::SWAP) {
 #pragma unroll
-            for (int i = 0; i < 128; ++i) o1[i] = 0.f;
+            for (int i = 0; i < 128; ++i) o1[i] = 0u;
         }
         bool ok = true;
         for (int n = 0; n < ntiles && ok; ++n) {
@@ -329,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) tmem_ld16(tm_s + c * 16 + lane_off, o1 + c * 16);
+                    for (int c = 0; c < 4; ++c) tmem_ld32_nowait(tm_s + c * 32 + lane_off, o1 + c * 32);
                     tmem_ld_wait();
                     tc_fence_before();
                     group_sync(kBarWG, 128);
@@ -343,86 +345,127 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
             const bool need_mask = (key0 + kBN - 1 > t_first) ||
                                    (a.window > 0 && key0 <= t_last - a.window);
-            const int lo_r = a.window > 0 ? tok_r - a.window + 1 : 0;
-            // pass 1: row max of the scaled, masked scores
-            float mx = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-                float s[16];
-                tmem_ld16(tm_s + c * 16 + lane_off, s);
+            float psum = 0.f, alpha = 1.f;
+            // fast path: no mask in this tile and a finite reference max in every row of
+            // the warp: one pass over S with the current reference
+            bool slow = need_mask || !__all_sync(0xffffffffu, m_ref != -INFINITY);
+            if (!slow) {
+                uint32_t sa[32], sb[32];
+                float mxr = -INFINITY;
+                const float negm = -m_ref;
+                tmem_ld32_nowait(tm_s + lane_off, sa);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int j = key0 + c * 16 + e;
-                    const bool vis = !need_mask || (j <= tok_r && j >= lo_r);
-                    mx = fmaxf(mx, vis ? s[e] * a.scale_log2 : -INFINITY);
+                for (int b = 0; b < 4; ++b) {
+                    uint32_t* cur = (b & 1) ? sb : sa;
+                    uint32_t* nxt = (b & 1) ? sa : sb;
+                    if (b < 3) tmem_ld32_nowait(tm_s + (b + 1) * 32 + lane_off, nxt);
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const float s0 = __uint_as_float(cur[e]), s1 = __uint_as_float(cur[e + 1]);
+                        mxr = fmaxf(mxr, fmaxf(s0, s1));
+                        const float p0 = ex2_approx(fmaf(s0, c2, negm));
+                        const float p1 = ex2_approx(fmaf(s1, c2, negm));
+                        if constexpr (PF16) {
+                            w[e / 2] = pack_f16x2(p0, p1);
+                            psum += p0 + p1;
+                        } else {
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
+                            const float2 f = __bfloat1622float2(h);
+                            psum += f.x + f.y;
+                            w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+                        }
+                    }
+                    uint8_t* pb = sm.p[b >> 1];
+                    const int col = (b & 1) * 32;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8 * k)) =
+                            make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    if (b < 3) tmem_ld_wait();
                 }
+                // the reference stays unless this tile's max exceeds it by more than 2^8
+                slow = __any_sync(0xffffffffu, mxr * c2 > m_ref + kLazyMax);
+                if (slow) psum = 0.f;
             }
-            if (!row_valid) mx = -INFINITY;
-            float alpha = 1.f;
-            if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
-                alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
-                m_ref = mx;
-            }
-            // pass 2: P = exp2(s * scale_log2 - m_ref), rounded, into the A tile of P.V
-            float psum = 0.f;
+            if (slow) {
+                // two passes with masks: row max, then P with a (lazily) updated reference
+                const int lo_r = a.window > 0 ? tok_r - a.window + 1 : 0;
+                float mx = -INFINITY;
 #pragma unroll 1
-            for (int c = 0; c < 8; ++c) {
-                float s[16];
-                tmem_ld16(tm_s + c * 16 + lane_off, s);
-                tmem_ld_wait();
-                uint32_t w[8];
+                for (int b = 0; b < 4; ++b) {
+                    uint32_t sv[32];
+                    tmem_ld32_nowait(tm_s + b * 32 + lane_off, sv);
+                    tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    float pv[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int j = key0 + c * 16 + e + u;
-                        const bool vis = row_valid && (!need_mask || (j <= tok_r && j >= lo_r));
-                        pv[u] = vis ? exp2f(fmaf(s[e + u], a.scale_log2, -m_ref)) : 0.f;
-                    }
-                    if (p_f16) {
-                        const __half2 h = __floats2half2_rn(pv[0], pv[1]);
-                        const float2 f = __half22float2(h);
-                        psum += f.x + f.y;
-                        w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
-                    } else {
-                        const __nv_bfloat162 h = __floats2bfloat162_rn(pv[0], pv[1]);
-                        const float2 f = __bfloat1622float2(h);
-                        psum += f.x + f.y;
-                        w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+                    for (int e = 0; e < 32; ++e) {
+                        const int j = key0 + b * 32 + e;
+                        const bool vis = !need_mask || (j <= tok_r && j >= lo_r);
+                        mx = fmaxf(mx, vis ? __uint_as_float(sv[e]) * c2 : -INFINITY);
                     }
                 }
-                uint8_t* pb = sm.p[c >> 2];
-                const int col = (c & 3) * 16;
-                *reinterpret_cast<uint4*>(pb + sw128_offset(row, col)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8)) =
-                    make_uint4(w[4], w[5], w[6], w[7]);
+                if (!row_valid) mx = -INFINITY;
+                if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
+                    alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
+                    m_ref = mx;
+                }
+                const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+#pragma unroll 1
+                for (int b = 0; b < 4; ++b) {
+                    uint32_t sv[32];
+                    tmem_ld32_nowait(tm_s + b * 32 + lane_off, sv);
+                    tmem_ld_wait();
+                    uint32_t w[16];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        float pv[2];
+#pragma unroll
+                        for (int u = 0; u < 2; ++u) {
+                            const int j = key0 + b * 32 + e + u;
+                            const bool vis = row_valid && (!need_mask || (j <= tok_r && j >= lo_r));
+                            pv[u] = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, negm)) : 0.f;
+                        }
+                        if constexpr (PF16) {
+                            w[e / 2] = pack_f16x2(pv[0], pv[1]);
+                            psum += pv[0] + pv[1];
+                        } else {
+                            const __nv_bfloat162 h = __floats2bfloat162_rn(pv[0], pv[1]);
+                            const float2 f = __bfloat1622float2(h);
+                            psum += f.x + f.y;
+                            w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+                        }
+                    }
+                    uint8_t* pb = sm.p[b >> 1];
+                    const int col = (b & 1) * 32;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8 * k)) =
+                            make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                }
             }
             l_sum = l_sum * alpha + psum;
             // correction of the accumulator when the reference max moved (rare)
-            const bool warp_rescale = __any_sync(0xffffffffu, alpha != 1.f && n > 0);
-            if constexpr (C::SWAP) {
+            if (__any_sync(0xffffffffu, alpha != 1.f && n > 0)) {
+                if constexpr (C::SWAP) {
 #pragma unroll
-                for (int i = 0; i < 128; ++i) o1[i] *= alpha;
-            }
-            if (warp_rescale) {
-                for (int c = 0; c < D / 16; ++c) {
-                    if (C::SWAP && c >= 8 && c < 16) continue;   // that quarter is in o1
-                    float o[16];
-                    tmem_ld16(tm_o + c * 16 + lane_off, o);
+                    for (int i = 0; i < 128; ++i) o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
+                }
+                for (int c = 0; c < D / 32; ++c) {
+                    if (C::SWAP && c >= 4 && c < 8) continue;   // that quarter is in o1
+                    uint32_t o[32];
+                    tmem_ld32_nowait(tm_o + c * 32 + lane_off, o);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) o[e] *= alpha;
-                    tmem_st16(tm_o + c * 16 + lane_off, o);
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    tmem_st32_nowait(tm_o + c * 32 + lane_off, o);
                 }
                 tmem_st_wait();
             }
             if constexpr (C::SWAP) {
                 // put O[:, 128..255] back for the P.V product
 #pragma unroll
-                for (int c = 0; c < 8; ++c) tmem_st16(tm_s + c * 16 + lane_off, o1 + c * 16);
+                for (int c = 0; c < 4; ++c) tmem_st32_nowait(tm_s + c * 32 + lane_off, o1 + c * 32);
                 tmem_st_wait();
             }
             fence_proxy_async_smem();
@@ -440,16 +483,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
             const int h = pg.g * G + row % G;
             uint16_t* dst = a.out + (((size_t)pg.b * a.T + tok_r) * a.Hq + h) * D;
-            for (int c = 0; c < D / 16; ++c) {
-                float o[16];
-                tmem_ld16(tm_o + c * 16 + lane_off, o);
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32_nowait(tm_o + c * 32 + lane_off, o);
                 tmem_ld_wait();
                 if (row_valid) {
-                    uint32_t w[8];
+                    uint32_t w[16];
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) w[e / 2] = pack_bf16x2(o[e] * inv, o[e + 1] * inv);
-                    *reinterpret_cast<uint4*>(dst + c * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-                    *reinterpret_cast<uint4*>(dst + c * 16 + 8) = make_uint4(w[4], w[5], w[6], w[7]);
+                    for (int e = 0; e < 32; e += 2)
+                        w[e / 2] = pack_bf16x2(__uint_as_float(o[e]) * inv,
+                                               __uint_as_float(o[e + 1]) * inv);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        *reinterpret_cast<uint4*>(dst + c * 32 + 8 * k) =
+                            make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
                 }
             }
             if (row_valid && a.lse)
@@ -477,10 +524,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
-template <int D>
+template <int D, bool PF16>
 cudaError_t run_prefill(const PrefillArgs& a, cudaStream_t stream) {
     const size_t smem = sizeof(PrefillSmem<D>) + 1024;
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, PF16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int tpt = kBM / a.G;
@@ -498,7 +545,7 @@ cudaError_t run_prefill(const PrefillArgs& a, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, prefill_kernel<D>, a);
+    e = cudaLaunchKernelEx(&cfg, prefill_kernel<D, PF16>, a);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
@@ -511,8 +558,11 @@ size_t prefill_smem_bytes(int d) {
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream) {
     if (a.B == 0 || a.T == 0) return cudaSuccess;
-    if (a.d == 512) return run_prefill<512>(a, stream);
-    if (a.d == 256) return run_prefill<256>(a, stream);
+    // P takes the 16-bit format of V: fp16 when V is the normalised key copy, bf16 when V
+    // is the caller's values
+    const bool pf16 = a.kv_is_k != 0;
+    if (a.d == 512) return pf16 ? run_prefill<512, true>(a, stream) : run_prefill<512, false>(a, stream);
+    if (a.d == 256) return pf16 ? run_prefill<256, true>(a, stream) : run_prefill<256, false>(a, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -264,8 +264,64 @@ def oracle_sample(max_seconds=20.0, seed=0):
 
 # --------------------------------------------------------------------------- main
 
+CASES = {
+    # small cases for profiler captures: inputs larger than L2, a few GB on the device
+    "global_prefill_T8192": ("prefill", dict(B=1, T=8192, layer="GLOBAL_8TO1")),
+    "local_prefill_T16384": ("prefill", dict(B=1, T=16384, layer="LOCAL_W1024")),
+    "global_decode_L8192": ("decode", dict(B=16, L=8192, layer="GLOBAL_8TO1")),
+}
+
+
+def run_case(name, steps, warmup):
+    """One named workload alone, `steps` timed calls (used under profilers)."""
+    import torch
+    from attention_g4attn_b200 import binding as b, synth, workloads
+    kind, p = CASES[name]
+    ly = getattr(workloads, p["layer"])
+    dev = torch.device("cuda:0")
+    stream = torch.cuda.Stream(dev)
+    cfg = b.LayerCfg.from_layer(ly)
+    if kind == "prefill":
+        inp = synth.layer_inputs(p["B"], p["T"], ly.n_q_heads, ly.n_kv_heads, ly.head_dim,
+                                 ly.separate_v, seed=3, device=dev)
+        ws = torch.empty(b.g4attn_prefill_workspace_size(p["B"], p["T"], cfg), dtype=torch.uint8,
+                         device=dev)
+        out = torch.empty_like(inp.q)
+
+        def call():
+            b.g4attn_prefill(inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, cfg, out=out,
+                             workspace=ws, stream=stream)
+        work = 4.0 * ly.head_dim * ly.n_q_heads * p["B"] * workloads.visible_pairs(p["T"], ly.window)
+        unit = "TFLOP/s"
+    else:
+        d = synth.decode_inputs(p["B"], p["L"], ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False,
+                                seed=3, device=dev)
+        ws = torch.empty(b.g4attn_decode_workspace_size(p["B"], p["L"], cfg), dtype=torch.uint8,
+                         device=dev)
+        out = torch.empty_like(d.q)
+
+        def call():
+            b.g4attn_decode(d.q, d.k, None, cfg, out=out, workspace=ws, stream=stream)
+        work = float(p["B"] * ly.n_kv_heads * p["L"] * ly.head_dim * 2) * 1e3   # -> GB/s
+        unit = "GB/s"
+    for _ in range(warmup):
+        call()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    e1.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / steps
+    assert b.g4attn_device_status(stream) == 0
+    print(json.dumps({"case": name, "ms": t * 1e3, "value": work / t / 1e12, "unit": unit}))
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--case", choices=sorted(CASES), default=None,
+                    help="time one small workload alone (profiler captures)")
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
@@ -273,6 +329,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case, max(args.steps, 1), max(args.warmup, 0))
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

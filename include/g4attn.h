@@ -66,7 +66,7 @@ typedef struct g4attn_layer_cfg {
     float rope_p;       /* fraction of rotary pairs that turn, 0 <= p <= 1 (0.25 global, 1 local) */
     double rope_base;   /* RoPE base > 0 (1e6 global, 1e4 local) */
     int window;         /* 0 = full causal; W > 0 = sliding window i - W < j <= i */
-    float scale;        /* softmax scale (1/sqrt(d) for the pages' layers) */
+    float scale;        /* softmax scale > 0 (1/sqrt(d) for the pages' layers) */
     int kv_is_k;        /* 0 separate v; 1 v = normed pre-RoPE key; 2 v = normed rotated key */
     int qk_norm;        /* 1 = apply QKNorm (the layers on the pages), 0 = inputs are used as is */
     float qk_norm_eps;  /* eps inside the RMS (1e-6) */

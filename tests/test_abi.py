@@ -83,6 +83,7 @@ def test_invalid_configs_are_rejected(b):
         b.LayerCfg(8, 1, 512, 0.25, 1e6, -3),    # negative window
         b.LayerCfg(8, 1, 512, 0.25, 1e6, 0, None, 3),   # kv_is_k out of range
         b.LayerCfg(256, 1, 512, 0.25, 1e6),      # G = 256 does not divide 128
+        b.LayerCfg(8, 1, 512, 0.25, 1e6, 0, -0.1),   # non-positive softmax scale
     ]
     for cfg in bad:
         assert b.g4attn_prefill_workspace_size(1, 16, cfg) == 0
