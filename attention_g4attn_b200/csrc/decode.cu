@@ -18,6 +18,7 @@
 // The CTA is persistent over work items blockIdx.x, +gridDim.x, ...  Every mbarrier wait
 // is bounded (sm100.cuh); on a timeout all roles drain their in-flight work and exit.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kernels.h"
 #include "rope.cuh"
@@ -35,6 +36,7 @@ constexpr int kMaxRotChunks = 2;     // side buffers when values are the pre-RoP
 constexpr int kN = 16;               // MMA N: query heads of one KV head, zero padded
 constexpr uint32_t kTmemCols = 128;
 constexpr int kBarWG = 1;            // named barrier of the softmax warpgroup
+constexpr float kLazyMax = 8.0f;     // log2 units: headroom of the lazy reference max
 
 struct __align__(1024) DecodeSmem {
     uint8_t ring[kNSlots][kSlotBytes];
@@ -44,6 +46,7 @@ struct __align__(1024) DecodeSmem {
     float theta[256];                // base^(-2i/d) in fp32, i < R
     float2 base_cs[256];             // cos/sin of tile_start * theta_i (fp64-reduced angle)
     float red[4][kN];                // cross-warp reductions
+    float qb[kN][128];               // rotated dims of q (first and second half, R <= 64)
     uint64_t full[kNSlots];
     uint64_t empty[kNSlots];
     uint64_t s_full, p_full, rot_ready, q_ready, o_done, drain;
@@ -77,7 +80,9 @@ __device__ __forceinline__ bool chunk_rotated(int c, int d, int R) {
     return (lo < R) || (lo < h + R && hi > h);
 }
 
-template <int D>
+// D: head dim; NH: query heads per KV head handled by the softmax (8 or 16, >= G);
+// REL: relative rotation (values are not the rotated key and R <= 64).
+template <int D, int NH, bool REL>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a) {
     constexpr int NCH = D / 64;     // 64-dim chunks per key row
@@ -109,9 +114,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
-    if (warp >= 2)
+    if (warp >= 2) {
         for (int i = threadIdx.x - 64; i < R; i += 128)
             sm.theta[i] = (float)exp2(-(2.0 * (double)i / (double)D) * a.rope.log2_base);
+        for (int i = threadIdx.x - 64; i < (int)(sizeof(sm.p) / 16); i += 128)
+            reinterpret_cast<uint4*>(&sm.p[0][0])[i] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -249,6 +258,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int row = quarter * 32 + lane;          // TMEM lane: key row or d-row
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int G = a.G;
+        const float c2 = a.scale_log2;
+        // Relative rotation (REL): key row `row` of every tile sits at angle row*theta_i from
+        // the tile start, so its (cos, sin) are fixed per thread; the tile start angle goes
+        // onto the query instead: q' = R(-key0 theta) q, and q' . R(row theta) k equals
+        // q . R((key0 + row) theta) k.
+        __half2 rcs[REL ? 64 : 1];
+        if constexpr (REL) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+                float sn = 0.f, cn = 1.f;
+                if (i < R) sincosf((float)row * sm.theta[i], &sn, &cn);
+                rcs[i] = __floats2half2_rn(cn, sn);
+            }
+        }
         uint32_t q = 0, tile = 0, item_n = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++item_n) {
@@ -263,13 +286,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                         a.q + ((size_t)w.b * a.Hq + (size_t)w.g * G + h) * D + c8 * 8);
                 *reinterpret_cast<uint4*>(sm.q[c8 / 8] + sw128_offset(h, (c8 % 8) * 8)) = v;
             }
+            if constexpr (REL) {   // the rotated dims of q, to be turned per tile
+                for (int e = t128; e < NH * 2 * R; e += 128) {
+                    const int h = e / (2 * R), k = e % (2 * R);
+                    const int dim = k < R ? k : D / 2 + (k - R);
+                    float v = 0.f;
+                    if (h < G)
+                        v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                            a.q + ((size_t)w.b * a.Hq + (size_t)w.g * G + h) * D + dim));
+                    sm.qb[h][k < R ? k : 64 + (k - R)] = v;
+                }
+            }
             fence_proxy_async_smem();
             group_sync(kBarWG, 128);
             if (t128 == 0) mbar_arrive(&sm.q_ready);
 
-            float m_run[kN], l_part[kN];
+            float m_run[NH], l_part[NH];
 #pragma unroll
-            for (int h = 0; h < kN; ++h) {
+            for (int h = 0; h < NH; ++h) {
                 m_run[h] = -INFINITY;
                 l_part[h] = 0.f;
             }
@@ -277,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int key0 = w.k0 + t * kTileKeys;
                 const uint32_t qk = q;
                 q += slots_per_tile;
-                // ---- turn the rotated pairs of this tile's keys to their positions
+                // ---- turn the rotated pairs of this tile's keys (and, REL, the queries)
                 if (R > 0) {
                     for (int i = t128; i < R; i += 128)
                         sm.base_cs[i] = rope_cos_sin((long long)key0, i, D, a.rope.log2_base);
@@ -288,49 +322,97 @@ __global__ void __launch_bounds__(kThreads, 1)
                                             ((qk + pr) / kNSlots) & 1, wc, abort);
                     ok = group_all(got, kBarWG, 128);   // also orders base_cs writes
                     if (!ok) break;
-                    const float fr = (float)row;
-                    int ri = 0;
-                    for (int c = 0; c < NCH / 2; ++c) {
-                        if (!chunk_rotated(c, D, R)) continue;
-                        const int c2 = c + NCH / 2;   // partner chunk: dims + d/2
-                        uint8_t* src1 = sm.ring[(qk + c / 2) % kNSlots] + (c & 1) * kChunkBytes;
-                        uint8_t* src2 = sm.ring[(qk + c2 / 2) % kNSlots] + (c2 & 1) * kChunkBytes;
-                        uint8_t* dst1 = side_rot ? sm.rot[ri] : src1;
-                        uint8_t* dst2 = side_rot ? sm.rot[ri + 1] : src2;
-                        ri += 2;
+                    if constexpr (REL) {
+                        // q' = R(-key0 theta) q on the rotated dims (chunks 0 and NCH/2)
+                        for (int e = t128; e < G * R; e += 128) {
+                            const int h = e / R, i = e % R;
+                            const float2 cs = sm.base_cs[i];
+                            const float x = sm.qb[h][i], y = sm.qb[h][64 + i];
+                            *reinterpret_cast<__nv_bfloat16*>(sm.q[0] + sw128_offset(h, i)) =
+                                __float2bfloat16_rn(x * cs.x + y * cs.y);
+                            *reinterpret_cast<__nv_bfloat16*>(sm.q[NCH / 2] + sw128_offset(h, i)) =
+                                __float2bfloat16_rn(y * cs.x - x * cs.y);
+                        }
+                        // keys: R(row theta) on the rotated pairs of this thread's row
+                        uint8_t* src1 = sm.ring[qk % kNSlots];
+                        uint8_t* src2 = sm.ring[(qk + NCH / 4) % kNSlots] +
+                                        ((NCH / 2) & 1) * kChunkBytes;
+                        uint8_t* dst1 = side_rot ? sm.rot[0] : src1;
+                        uint8_t* dst2 = side_rot ? sm.rot[1] : src2;
+#pragma unroll
                         for (int g8 = 0; g8 < 8; ++g8) {
+                            if (!side_rot && g8 * 8 >= R) break;
                             const uint32_t off = sw128_offset(row, g8 * 8);
                             uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
                             uint4 x2 = *reinterpret_cast<const uint4*>(src2 + off);
-                            __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&x1);
-                            __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x2);
+                            if (g8 * 8 < R) {
+                                __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&x1);
+                                __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x2);
 #pragma unroll
-                            for (int e2 = 0; e2 < 4; ++e2) {
-                                const float2 u = __bfloat1622float2(h1[e2]);
-                                const float2 v = __bfloat1622float2(h2[e2]);
-                                float uo[2] = {u.x, u.y}, vo[2] = {v.x, v.y};
-#pragma unroll
-                                for (int e = 0; e < 2; ++e) {
-                                    const int i = c * 64 + g8 * 8 + e2 * 2 + e;
-                                    if (i < R) {
-                                        // angle(key0 + row) = angle(key0) + row * theta_i
-                                        float x = fr * sm.theta[i];
-                                        x = fmaf(-6.2831853f, rintf(x * 0.15915494f), x);
-                                        float so, co;
-                                        __sincosf(x, &so, &co);
-                                        const float2 b = sm.base_cs[i];
-                                        const float cc = b.x * co - b.y * so;
-                                        const float ss = b.y * co + b.x * so;
-                                        const float p0 = uo[e], p1 = vo[e];
-                                        uo[e] = p0 * cc - p1 * ss;
-                                        vo[e] = p0 * ss + p1 * cc;
-                                    }
+                                for (int e2 = 0; e2 < 4; ++e2) {
+                                    const float2 u = __bfloat1622float2(h1[e2]);
+                                    const float2 v = __bfloat1622float2(h2[e2]);
+                                    const int i0 = g8 * 8 + 2 * e2;
+                                    const float2 ca = __half22float2(rcs[i0]);
+                                    const float2 cb = __half22float2(rcs[i0 + 1]);
+                                    const bool r0 = i0 < R, r1 = i0 + 1 < R;
+                                    const float u0 = r0 ? u.x * ca.x - v.x * ca.y : u.x;
+                                    const float v0 = r0 ? u.x * ca.y + v.x * ca.x : v.x;
+                                    const float u1 = r1 ? u.y * cb.x - v.y * cb.y : u.y;
+                                    const float v1 = r1 ? u.y * cb.y + v.y * cb.x : v.y;
+                                    h1[e2] = __floats2bfloat162_rn(u0, u1);
+                                    h2[e2] = __floats2bfloat162_rn(v0, v1);
                                 }
-                                h1[e2] = __floats2bfloat162_rn(uo[0], uo[1]);
-                                h2[e2] = __floats2bfloat162_rn(vo[0], vo[1]);
                             }
                             *reinterpret_cast<uint4*>(dst1 + off) = x1;
                             *reinterpret_cast<uint4*>(dst2 + off) = x2;
+                        }
+                    } else {
+                        // absolute angles: angle(key0 + row) = angle(key0) + row * theta_i
+                        const float fr = (float)row;
+                        int ri = 0;
+                        for (int c = 0; c < NCH / 2; ++c) {
+                            if (!chunk_rotated(c, D, R)) continue;
+                            const int c2i = c + NCH / 2;   // partner chunk: dims + d/2
+                            uint8_t* src1 = sm.ring[(qk + c / 2) % kNSlots] + (c & 1) * kChunkBytes;
+                            uint8_t* src2 =
+                                sm.ring[(qk + c2i / 2) % kNSlots] + (c2i & 1) * kChunkBytes;
+                            uint8_t* dst1 = side_rot ? sm.rot[ri] : src1;
+                            uint8_t* dst2 = side_rot ? sm.rot[ri + 1] : src2;
+                            ri += 2;
+                            for (int g8 = 0; g8 < 8; ++g8) {
+                                const uint32_t off = sw128_offset(row, g8 * 8);
+                                uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
+                                uint4 x2 = *reinterpret_cast<const uint4*>(src2 + off);
+                                __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&x1);
+                                __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x2);
+#pragma unroll
+                                for (int e2 = 0; e2 < 4; ++e2) {
+                                    const float2 u = __bfloat1622float2(h1[e2]);
+                                    const float2 v = __bfloat1622float2(h2[e2]);
+                                    float uo[2] = {u.x, u.y}, vo[2] = {v.x, v.y};
+#pragma unroll
+                                    for (int e = 0; e < 2; ++e) {
+                                        const int i = c * 64 + g8 * 8 + e2 * 2 + e;
+                                        if (i < R) {
+                                            float x = fr * sm.theta[i];
+                                            x = fmaf(-6.2831853f, rintf(x * 0.15915494f), x);
+                                            float so, co;
+                                            __sincosf(x, &so, &co);
+                                            const float2 b = sm.base_cs[i];
+                                            const float cc = b.x * co - b.y * so;
+                                            const float ss = b.y * co + b.x * so;
+                                            const float p0 = uo[e], p1 = vo[e];
+                                            uo[e] = p0 * cc - p1 * ss;
+                                            vo[e] = p0 * ss + p1 * cc;
+                                        }
+                                    }
+                                    h1[e2] = __floats2bfloat162_rn(uo[0], uo[1]);
+                                    h2[e2] = __floats2bfloat162_rn(vo[0], vo[1]);
+                                }
+                                *reinterpret_cast<uint4*>(dst1 + off) = x1;
+                                *reinterpret_cast<uint4*>(dst2 + off) = x2;
+                            }
                         }
                     }
                     fence_proxy_async_smem();
@@ -345,58 +427,71 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld16(tm_s + lane_off, s);
                 tmem_ld_wait();
                 const bool valid = key0 + row < w.k1;
-                float mt[kN];
+                float x[NH];
+                bool big = false;
 #pragma unroll
-                for (int h = 0; h < kN; ++h) {
-                    s[h] = (valid && h < G) ? s[h] * a.scale_log2 : -INFINITY;
-                    mt[h] = s[h];
+                for (int h = 0; h < NH; ++h) {
+                    x[h] = (valid && h < G) ? s[h] * c2 : -INFINITY;
+                    big |= x[h] > m_run[h] + kLazyMax;
                 }
+                // lazy reference max: only when some score of the tile exceeds the running
+                // reference by more than 2^8 (and on the first tile) do the warps reduce
+                const bool fast = (t > 0) && group_all(!big, kBarWG, 128);
+                float alpha[NH];
 #pragma unroll
-                for (int h = 0; h < kN; ++h)
+                for (int h = 0; h < NH; ++h) alpha[h] = 1.f;
+                if (!fast) {
+                    float mt[NH];
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1)
-                        mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], o));
-                if (lane == 0)
+                    for (int h = 0; h < NH; ++h) {
+                        mt[h] = x[h];
 #pragma unroll
-                    for (int h = 0; h < kN; ++h) sm.red[quarter][h] = mt[h];
-                group_sync(kBarWG, 128);
-                float alpha[kN];
-                bool rescale = false;
+                        for (int o = 16; o > 0; o >>= 1)
+                            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], o));
+                    }
+                    if (lane == 0)
 #pragma unroll
-                for (int h = 0; h < kN; ++h) {
-                    const float tmax = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]),
-                                             fmaxf(sm.red[2][h], sm.red[3][h]));
-                    const float mn = fmaxf(m_run[h], tmax);
-                    alpha[h] = (m_run[h] == mn) ? 1.f : exp2f(m_run[h] - mn);
-                    rescale |= (t > 0) && (alpha[h] != 1.f);
-                    m_run[h] = mn;
+                        for (int h = 0; h < NH; ++h) sm.red[quarter][h] = mt[h];
+                    group_sync(kBarWG, 128);
+                    bool rescale = false;
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        const float tmax = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]),
+                                                 fmaxf(sm.red[2][h], sm.red[3][h]));
+                        if (tmax > m_run[h] + kLazyMax ||
+                            (m_run[h] == -INFINITY && tmax != -INFINITY)) {
+                            alpha[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - tmax);
+                            m_run[h] = tmax;
+                            rescale |= t > 0;
+                        }
+                    }
+                    group_sync(kBarWG, 128);   // red[] is rewritten below
+                    // rescale O^T (thread = d-row, column = head).  O is idle: the MMA that
+                    // wrote S for this tile ran after the previous O update.
+                    if (rescale) {
+                        for (int pr = 0; pr < NPAIR; ++pr) {
+                            float o[kN];
+                            tmem_ld16(tm_o + pr * 16 + lane_off, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int h = 0; h < NH; ++h) o[h] *= alpha[h];
+                            tmem_st16(tm_o + pr * 16 + lane_off, o);
+                        }
+                        tmem_st_wait();
+                    }
                 }
                 // P^T: row = head, K-major, 64 keys per 128-byte row, two chunks
                 {
                     uint8_t* pb = sm.p[row >> 6];
                     const int kc = row & 63;
 #pragma unroll
-                    for (int h = 0; h < kN; ++h) {
-                        const float p = (s[h] == -INFINITY) ? 0.f : exp2f(s[h] - m_run[h]);
+                    for (int h = 0; h < NH; ++h) {
+                        const float p = (x[h] == -INFINITY) ? 0.f : ex2_approx(x[h] - m_run[h]);
                         const __nv_bfloat16 pr = __float2bfloat16_rn(p);
                         // the running sum uses the rounded weight the MMA sees
                         l_part[h] = l_part[h] * alpha[h] + __bfloat162float(pr);
                         *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(h, kc)) = pr;
                     }
-                }
-                // rescale O^T when a running max moved.  O is idle: the MMA that wrote S for
-                // this tile was issued after the previous tile's O update, and commits track
-                // every earlier MMA.  Thread = d-row, column = head.
-                if (!group_all(!rescale, kBarWG, 128)) {
-                    for (int pr = 0; pr < NPAIR; ++pr) {
-                        float o[kN];
-                        tmem_ld16(tm_o + pr * 16 + lane_off, o);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int h = 0; h < kN; ++h) o[h] *= alpha[h];
-                        tmem_st16(tm_o + pr * 16 + lane_off, o);
-                    }
-                    tmem_st_wait();
                 }
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -413,24 +508,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 float o[kN];
                 tmem_ld16(tm_o + pr * 16 + lane_off, o);
                 tmem_ld_wait();
-                for (int h = 0; h < G; ++h)
-                    a.part_o[(obase + h) * D + pr * 128 + row] = nt > 0 ? o[h] : 0.f;
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    if (h < G) a.part_o[(obase + h) * D + pr * 128 + row] = nt > 0 ? o[h] : 0.f;
             }
 #pragma unroll
-            for (int h = 0; h < kN; ++h)
+            for (int h = 0; h < NH; ++h)
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1)
                     l_part[h] += __shfl_xor_sync(0xffffffffu, l_part[h], o);
             if (lane == 0)
 #pragma unroll
-                for (int h = 0; h < kN; ++h) sm.red[quarter][h] = l_part[h];
+                for (int h = 0; h < NH; ++h) sm.red[quarter][h] = l_part[h];
             group_sync(kBarWG, 128);
             if (t128 < G) {
                 const float l = sm.red[0][t128] + sm.red[1][t128] + sm.red[2][t128] +
                                 sm.red[3][t128];
                 float mv = m_run[0];
 #pragma unroll
-                for (int h = 1; h < kN; ++h) mv = (t128 == h) ? m_run[h] : mv;
+                for (int h = 1; h < NH; ++h) mv = (t128 == h) ? m_run[h] : mv;
                 a.part_ml[(obase + t128) * 2 + 0] = mv;
                 a.part_ml[(obase + t128) * 2 + 1] = l;
             }
@@ -473,13 +569,23 @@ __global__ void decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
         a.lse[bh] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int D>
+template <int D, int NH, bool REL>
 cudaError_t run_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
-    cudaError_t e =
-        cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NH, REL>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_kernel<D><<<grid, kThreads, smem, stream>>>(a);
+    decode_kernel<D, NH, REL><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t dispatch_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
+    const bool rel = a.kv_is_k != 2 && a.rope.R <= 64;
+    if (a.G <= 8)
+        return rel ? run_decode<D, 8, true>(a, grid, smem, stream)
+                   : run_decode<D, 8, false>(a, grid, smem, stream);
+    return rel ? run_decode<D, 16, true>(a, grid, smem, stream)
+               : run_decode<D, 16, false>(a, grid, smem, stream);
 }
 
 }  // namespace
@@ -494,8 +600,8 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const int grid = n_items < sms ? n_items : sms;
-        cudaError_t e = a.d == 512 ? run_decode<512>(a, grid, smem, stream)
-                        : a.d == 256 ? run_decode<256>(a, grid, smem, stream)
+        cudaError_t e = a.d == 512 ? dispatch_decode<512>(a, grid, smem, stream)
+                        : a.d == 256 ? dispatch_decode<256>(a, grid, smem, stream)
                                      : cudaErrorInvalidValue;
         if (e != cudaSuccess) return e;
     }
