@@ -10,8 +10,10 @@
 // the first product and, read MN-major, the V operand of the second (keys reused as
 // values, report section 2 / explainer "K=V": one cache read serves both).  The cache
 // holds pre-RoPE keys; the rotated pairs (i, i + d/2), i < R, of every key are turned to
-// the key's position on the fly (report section 2, p-RoPE) by the softmax warps, into a
-// side buffer when the values are the pre-RoPE keys, in place otherwise.
+// the key's position on the fly (report section 2, p-RoPE) by the softmax warps, in place.
+// When the values are the pre-RoPE keys, the value operand is a second TMA pass over the
+// same rows (served from L2: the score pass has just read them), so the score copy can be
+// turned in place and released as soon as S^T has read it; HBM still reads the cache once.
 //
 // Warp roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
 // warps 2..5 rotation / softmax / epilogue (thread = TMEM lane = key row or d-row).
@@ -29,10 +31,9 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kTileKeys = 128;
-constexpr int kNSlots = 5;           // ring of 32 KB slots: 128 keys x 128 dims (2 chunks)
+constexpr int kNSlots = 6;           // ring of 32 KB slots: 128 keys x 128 dims (2 chunks)
 constexpr int kSlotBytes = 32768;
 constexpr int kChunkBytes = 16384;   // 128 keys x 64 dims, 128-byte swizzled rows
-constexpr int kMaxRotChunks = 2;     // side buffers when values are the pre-RoPE keys
 constexpr int kN = 16;               // MMA N: query heads of one KV head, zero padded
 constexpr uint32_t kTmemCols = 128;
 constexpr int kBarWG = 1;            // named barrier of the softmax warpgroup
@@ -40,7 +41,6 @@ constexpr float kLazyMax = 8.0f;     // log2 units: headroom of the lazy referen
 
 struct __align__(1024) DecodeSmem {
     uint8_t ring[kNSlots][kSlotBytes];
-    uint8_t rot[kMaxRotChunks][kChunkBytes];
     uint8_t q[8][kN * 128];          // B operand of S^T: per 64-dim chunk, 16 rows x 128 B
     uint8_t p[2][kN * 128];          // B operand of O^T: P^T, K-major, 2 chunks of 64 keys
     float theta[256];                // base^(-2i/d) in fp32, i < R
@@ -94,8 +94,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const WaitCtl wc{a.wait_limit, a.status};
     volatile int* abort = &sm.abort;
     const int R = a.rope.R;
-    const bool sep_v = a.kv_is_k == 0;
-    const bool side_rot = a.kv_is_k == 1;
+    // Values come from a second pass over the cache (from L2: the score pass has just read
+    // the same rows) unless they are the rotated keys; the score copy is then free to be
+    // turned in place and released right after S^T.
+    const bool sep_v = a.kv_is_k != 2;
     const int n_items = a.splits * a.Hkv * a.B;
     const int slots_per_tile = sep_v ? 2 * NPAIR : NPAIR;
 
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (t + 2 < nt)
                         for (int c = 0; c < NCH; ++c) {
                             tma_prefetch_l2_4d(&a.tm_k, c * 64, w.g, key + 2 * kTileKeys, w.b);
-                            if (sep_v)
+                            if (a.kv_is_k == 0)   // a separate value cache
                                 tma_prefetch_l2_4d(&a.tm_v, c * 64, w.g, key + 2 * kTileKeys, w.b);
                         }
                     for (int pass = 0; pass < (sep_v ? 2 : 1) && !*abort; ++pass) {
@@ -204,12 +206,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (R > 0) {
                         if (!mbar_wait(&sm.rot_ready, tile & 1, wc, abort)) goto done;
                         tc_fence_after();
-                        int ri = 0;
                         for (int c = 0; c < NCH; ++c) {
                             if (!chunk_rotated(c, D, R)) continue;
                             const uint32_t slot = (qk + c / 2) % kNSlots;
-                            const uint8_t* src = side_rot ? sm.rot[ri++]
-                                                          : sm.ring[slot] + (c & 1) * kChunkBytes;
+                            const uint8_t* src = sm.ring[slot] + (c & 1) * kChunkBytes;
                             const uint32_t ab = smem_u32(src);
                             const uint32_t bb = smem_u32(sm.q[c]);
                             for (int kk = 0; kk < 4; ++kk) {
@@ -337,11 +337,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         uint8_t* src1 = sm.ring[qk % kNSlots];
                         uint8_t* src2 = sm.ring[(qk + NCH / 4) % kNSlots] +
                                         ((NCH / 2) & 1) * kChunkBytes;
-                        uint8_t* dst1 = side_rot ? sm.rot[0] : src1;
-                        uint8_t* dst2 = side_rot ? sm.rot[1] : src2;
+                        uint8_t* dst1 = src1;
+                        uint8_t* dst2 = src2;
 #pragma unroll
                         for (int g8 = 0; g8 < 8; ++g8) {
-                            if (!side_rot && g8 * 8 >= R) break;
+                            if (g8 * 8 >= R) break;
                             const uint32_t off = sw128_offset(row, g8 * 8);
                             uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
                             uint4 x2 = *reinterpret_cast<const uint4*>(src2 + off);
@@ -370,16 +370,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     } else {
                         // absolute angles: angle(key0 + row) = angle(key0) + row * theta_i
                         const float fr = (float)row;
-                        int ri = 0;
                         for (int c = 0; c < NCH / 2; ++c) {
                             if (!chunk_rotated(c, D, R)) continue;
                             const int c2i = c + NCH / 2;   // partner chunk: dims + d/2
                             uint8_t* src1 = sm.ring[(qk + c / 2) % kNSlots] + (c & 1) * kChunkBytes;
                             uint8_t* src2 =
                                 sm.ring[(qk + c2i / 2) % kNSlots] + (c2i & 1) * kChunkBytes;
-                            uint8_t* dst1 = side_rot ? sm.rot[ri] : src1;
-                            uint8_t* dst2 = side_rot ? sm.rot[ri + 1] : src2;
-                            ri += 2;
+                            uint8_t* dst1 = src1;
+                            uint8_t* dst2 = src2;
                             for (int g8 = 0; g8 < 8; ++g8) {
                                 const uint32_t off = sw128_offset(row, g8 * 8);
                                 uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
