@@ -38,6 +38,7 @@ constexpr int kN = 16;               // MMA N: query heads of one KV head, zero 
 constexpr uint32_t kTmemCols = 128;
 constexpr int kBarWG = 1;            // named barrier of the softmax warpgroup
 constexpr float kLazyMax = 8.0f;     // log2 units: headroom of the lazy reference max
+constexpr int kPrefetchTiles = 3;    // L2 prefetch distance, in tiles
 
 struct __align__(1024) DecodeSmem {
     uint8_t ring[kNSlots][kSlotBytes];
@@ -82,6 +83,14 @@ __device__ __forceinline__ bool chunk_rotated(int c, int d, int R) {
 
 // D: head dim; NH: query heads per KV head handled by the softmax (8 or 16, >= G);
 // REL: relative rotation (values are not the rotated key and R <= 64).
+// Chunk (64 dims) held by half h of the k-th slot of a tile.  Score slots of the two-pass
+// mode pair each chunk with its rotation partner (chunks k and k + NCH/2), so turning a
+// key needs one slot; value slots, and the slots of the one-pass mode (values = rotated
+// keys), hold consecutive chunks (2k, 2k+1), the 128 value rows of one O^T block.
+__device__ __forceinline__ int slot_chunk(int k, int h, bool partner_pairs, int nch) {
+    return partner_pairs ? k + h * (nch / 2) : 2 * k + h;
+}
+
 template <int D, int NH, bool REL>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a) {
@@ -135,29 +144,44 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&a.tm_k);
             if (sep_v) prefetch_tmap(&a.tm_v);
+            // L2 prefetch cursor: runs kPrefetchTiles tiles ahead of the loads, across the
+            // items of this CTA, so HBM keeps streaming while the ring slots are busy
+            int pf_it = blockIdx.x, pf_t = 0;
+            long long pf_count = 0, load_count = 0;
             uint32_t q = 0;   // ring slots filled so far
             for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
                 const Item w = item_of(a, it);
                 const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
-                for (int t = 0; t < nt && !*abort; ++t) {
+                for (int t = 0; t < nt && !*abort; ++t, ++load_count) {
                     const int key = w.k0 + t * kTileKeys;
-                    // keep HBM busy beyond the ring: pull the tile two steps ahead into L2
-                    if (t + 2 < nt)
-                        for (int c = 0; c < NCH; ++c) {
-                            tma_prefetch_l2_4d(&a.tm_k, c * 64, w.g, key + 2 * kTileKeys, w.b);
-                            if (a.kv_is_k == 0)   // a separate value cache
-                                tma_prefetch_l2_4d(&a.tm_v, c * 64, w.g, key + 2 * kTileKeys, w.b);
+                    while (pf_count <= load_count + kPrefetchTiles && pf_it < n_items) {
+                        const Item pw = item_of(a, pf_it);
+                        const int pnt = ceil_div(pw.k1 - pw.k0, kTileKeys);
+                        if (pf_t < pnt) {
+                            const int pk = pw.k0 + pf_t * kTileKeys;
+                            for (int c = 0; c < NCH; ++c) {
+                                tma_prefetch_l2_4d(&a.tm_k, c * 64, pw.g, pk, pw.b);
+                                if (a.kv_is_k == 0)   // a separate value cache
+                                    tma_prefetch_l2_4d(&a.tm_v, c * 64, pw.g, pk, pw.b);
+                            }
+                            ++pf_count;
                         }
+                        if (++pf_t >= pnt) {
+                            pf_t = 0;
+                            pf_it += gridDim.x;
+                        }
+                    }
                     for (int pass = 0; pass < (sep_v ? 2 : 1) && !*abort; ++pass) {
                         const CUtensorMap* map = pass ? &a.tm_v : &a.tm_k;
-                        for (int pr = 0; pr < NPAIR; ++pr) {
+                        const bool partner = sep_v && pass == 0;
+                        for (int k = 0; k < NPAIR; ++k) {
                             const int slot = q % kNSlots;
                             if (!mbar_wait(&sm.empty[slot], ((q / kNSlots) & 1) ^ 1, wc, abort))
                                 break;
                             mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes);
-                            tma_load_4d(sm.ring[slot], map, &sm.full[slot], pr * 128, w.g, key, w.b);
-                            tma_load_4d(sm.ring[slot] + kChunkBytes, map, &sm.full[slot],
-                                        pr * 128 + 64, w.g, key, w.b);
+                            for (int h = 0; h < 2; ++h)
+                                tma_load_4d(sm.ring[slot] + h * kChunkBytes, map, &sm.full[slot],
+                                            slot_chunk(k, h, partner, NCH) * 64, w.g, key, w.b);
                             ++q;
                         }
                     }
@@ -184,14 +208,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t qk = q;
                     const uint32_t qv = sep_v ? q + NPAIR : q;
                     bool first = true;
-                    // S^T over the chunks that need no rotation, as soon as they land
-                    for (int pr = 0; pr < NPAIR; ++pr) {
-                        const uint32_t k = qk + pr, slot = k % kNSlots;
-                        if (!mbar_wait(&sm.full[slot], (k / kNSlots) & 1, wc, abort)) goto done;
+                    // S^T over the chunks that need no rotation, as soon as they land; in the
+                    // two-pass mode each score slot is released right after its last MMA
+                    for (int k = 0; k < NPAIR; ++k) {
+                        const uint32_t qq = qk + k, slot = qq % kNSlots;
+                        if (!mbar_wait(&sm.full[slot], (qq / kNSlots) & 1, wc, abort)) goto done;
                         tc_fence_after();
+                        bool has_rot = false;
                         for (int h = 0; h < 2; ++h) {
-                            const int c = pr * 2 + h;
-                            if (chunk_rotated(c, D, R)) continue;
+                            const int c = slot_chunk(k, h, sep_v, NCH);
+                            if (chunk_rotated(c, D, R)) { has_rot = true; continue; }
                             const uint32_t ab = smem_u32(sm.ring[slot] + h * kChunkBytes);
                             const uint32_t bb = smem_u32(sm.q[c]);
                             for (int kk = 0; kk < 4; ++kk) {
@@ -201,28 +227,32 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 first = false;
                             }
                         }
+                        if (sep_v && !has_rot) mma_commit(&sm.empty[slot]);
                     }
                     // then the rotated chunks, once the softmax warps have turned them
                     if (R > 0) {
                         if (!mbar_wait(&sm.rot_ready, tile & 1, wc, abort)) goto done;
                         tc_fence_after();
-                        for (int c = 0; c < NCH; ++c) {
-                            if (!chunk_rotated(c, D, R)) continue;
-                            const uint32_t slot = (qk + c / 2) % kNSlots;
-                            const uint8_t* src = sm.ring[slot] + (c & 1) * kChunkBytes;
-                            const uint32_t ab = smem_u32(src);
-                            const uint32_t bb = smem_u32(sm.q[c]);
-                            for (int kk = 0; kk < 4; ++kk) {
-                                mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
-                                            sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
-                                            first ? 0u : 1u);
-                                first = false;
+                        for (int k = 0; k < NPAIR; ++k) {
+                            const uint32_t slot = (qk + k) % kNSlots;
+                            bool has_rot = false;
+                            for (int h = 0; h < 2; ++h) {
+                                const int c = slot_chunk(k, h, sep_v, NCH);
+                                if (!chunk_rotated(c, D, R)) continue;
+                                has_rot = true;
+                                const uint32_t ab = smem_u32(sm.ring[slot] + h * kChunkBytes);
+                                const uint32_t bb = smem_u32(sm.q[c]);
+                                for (int kk = 0; kk < 4; ++kk) {
+                                    mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
+                                                sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
+                                                first ? 0u : 1u);
+                                    first = false;
+                                }
                             }
+                            if (sep_v && has_rot) mma_commit(&sm.empty[slot]);
                         }
                     }
                     mma_commit(&sm.s_full);
-                    if (sep_v)   // key slots are free once S^T has read them
-                        for (int pr = 0; pr < NPAIR; ++pr) mma_commit(&sm.empty[(qk + pr) % kNSlots]);
                     // O^T += V^T . P^T once the softmax warps have written P
                     if (!mbar_wait(&sm.p_full, tile & 1, wc, abort)) goto done;
                     tc_fence_after();
@@ -240,8 +270,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mma_bf16_ss(tm_o + pr * 16, ad, sdesc_sw128(pb, 16, 1024), idesc_o,
                                         (t > 0 || kk > 0) ? 1u : 0u);
                         }
+                        if (sep_v) mma_commit(&sm.empty[slot]);
                     }
-                    for (int pr = 0; pr < NPAIR; ++pr) mma_commit(&sm.empty[(qv + pr) % kNSlots]);
+                    if (!sep_v)
+                        for (int pr = 0; pr < NPAIR; ++pr) mma_commit(&sm.empty[(qv + pr) % kNSlots]);
                     q += slots_per_tile;
                 }
                 mma_commit(&sm.o_done);
@@ -316,10 +348,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int i = t128; i < R; i += 128)
                         sm.base_cs[i] = rope_cos_sin((long long)key0, i, D, a.rope.log2_base);
                     bool got = true;
-                    for (int pr = 0; pr < NPAIR && got; ++pr)
-                        if (chunk_rotated(2 * pr, D, R) || chunk_rotated(2 * pr + 1, D, R))
-                            got = mbar_wait(&sm.full[(qk + pr) % kNSlots],
-                                            ((qk + pr) / kNSlots) & 1, wc, abort);
+                    for (int k = 0; k < NPAIR && got; ++k)
+                        if (chunk_rotated(slot_chunk(k, 0, sep_v, NCH), D, R) ||
+                            chunk_rotated(slot_chunk(k, 1, sep_v, NCH), D, R))
+                            got = mbar_wait(&sm.full[(qk + k) % kNSlots],
+                                            ((qk + k) / kNSlots) & 1, wc, abort);
                     ok = group_all(got, kBarWG, 128);   // also orders base_cs writes
                     if (!ok) break;
                     if constexpr (REL) {
@@ -334,9 +367,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 __float2bfloat16_rn(y * cs.x - x * cs.y);
                         }
                         // keys: R(row theta) on the rotated pairs of this thread's row
+                        // REL implies the two-pass mode: chunks 0 and NCH/2 share slot 0
                         uint8_t* src1 = sm.ring[qk % kNSlots];
-                        uint8_t* src2 = sm.ring[(qk + NCH / 4) % kNSlots] +
-                                        ((NCH / 2) & 1) * kChunkBytes;
+                        uint8_t* src2 = sm.ring[qk % kNSlots] + kChunkBytes;
                         uint8_t* dst1 = src1;
                         uint8_t* dst2 = src2;
 #pragma unroll
@@ -373,9 +406,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int c = 0; c < NCH / 2; ++c) {
                             if (!chunk_rotated(c, D, R)) continue;
                             const int c2i = c + NCH / 2;   // partner chunk: dims + d/2
-                            uint8_t* src1 = sm.ring[(qk + c / 2) % kNSlots] + (c & 1) * kChunkBytes;
-                            uint8_t* src2 =
-                                sm.ring[(qk + c2i / 2) % kNSlots] + (c2i & 1) * kChunkBytes;
+                            uint8_t* src1;
+                            uint8_t* src2;
+                            if (sep_v) {   // partner pairs share a slot
+                                src1 = sm.ring[(qk + c) % kNSlots];
+                                src2 = src1 + kChunkBytes;
+                            } else {
+                                src1 = sm.ring[(qk + c / 2) % kNSlots] + (c & 1) * kChunkBytes;
+                                src2 = sm.ring[(qk + c2i / 2) % kNSlots] + (c2i & 1) * kChunkBytes;
+                            }
                             uint8_t* dst1 = src1;
                             uint8_t* dst2 = src2;
                             for (int g8 = 0; g8 < 8; ++g8) {
