@@ -357,6 +357,12 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
     if ((cfg->kv_is_k == 0) != (vcache != nullptr)) return G4ATTN_ERR_INVALID_ARG;
     const int G = cfg->n_q_heads / cfg->n_kv_heads;
     if (G > 16) return G4ATTN_ERR_UNSUPPORTED;
+    if (cfg->kv_is_k == 1) {   // two side buffers hold the turned chunks
+        const int R = rope_pairs(cfg);
+        int n = 0;
+        for (int c = 0; c < cfg->head_dim / 64; ++c) n += chunk_rotated(c, cfg->head_dim, R);
+        if (n > 2) return G4ATTN_ERR_UNSUPPORTED;
+    }
     const void* ptrs[] = {q, kcache, vcache, out, lse};
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;

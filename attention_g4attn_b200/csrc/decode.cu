@@ -31,7 +31,8 @@ namespace {
 
 constexpr int kThreads = 192;
 constexpr int kTileKeys = 128;
-constexpr int kNSlots = 6;           // ring of 32 KB slots: 128 keys x 128 dims (2 chunks)
+constexpr int kNSlots = 5;           // ring of 32 KB slots: 128 keys x 128 dims (2 chunks)
+constexpr int kMaxRotChunks = 2;     // side buffers for the turned chunks (values = pre-RoPE)
 constexpr int kSlotBytes = 32768;
 constexpr int kChunkBytes = 16384;   // 128 keys x 64 dims, 128-byte swizzled rows
 constexpr int kN = 16;               // MMA N: query heads of one KV head, zero padded
@@ -42,6 +43,7 @@ constexpr int kPrefetchTiles = 3;    // L2 prefetch distance, in tiles
 
 struct __align__(1024) DecodeSmem {
     uint8_t ring[kNSlots][kSlotBytes];
+    uint8_t rot[kMaxRotChunks][kChunkBytes];
     uint8_t q[8][kN * 128];          // B operand of S^T: per 64-dim chunk, 16 rows x 128 B
     uint8_t p[2][kN * 128];          // B operand of O^T: P^T, K-major, 2 chunks of 64 keys
     float theta[256];                // base^(-2i/d) in fp32, i < R
@@ -87,8 +89,24 @@ __device__ __forceinline__ bool chunk_rotated(int c, int d, int R) {
 // mode pair each chunk with its rotation partner (chunks k and k + NCH/2), so turning a
 // key needs one slot; value slots, and the slots of the one-pass mode (values = rotated
 // keys), hold consecutive chunks (2k, 2k+1), the 128 value rows of one O^T block.
+// One-pass slots hold chunk pairs (2m, 2m+1) in the order m = 0, npair/2, 1, npair/2+1, ...
+// so the two rotation partners (chunks 0 and nch/2) arrive in the first two slots.
+__device__ __forceinline__ int slot_pair(int k, int npair) {
+    return (k & 1) ? (npair / 2 + k / 2) : (k / 2);
+}
 __device__ __forceinline__ int slot_chunk(int k, int h, bool partner_pairs, int nch) {
-    return partner_pairs ? k + h * (nch / 2) : 2 * k + h;
+    return partner_pairs ? k + h * (nch / 2) : 2 * slot_pair(k, nch / 2) + h;
+}
+// Slot index and half of chunk c within a tile.
+__device__ __forceinline__ void chunk_slot(int c, bool partner_pairs, int nch, int& k, int& h) {
+    if (partner_pairs) {
+        k = c % (nch / 2);
+        h = c / (nch / 2);
+    } else {
+        const int m = c / 2, np = nch / 2;
+        h = c & 1;
+        k = (m < np / 2) ? 2 * m : 2 * (m - np / 2) + 1;
+    }
 }
 
 template <int D, int NH, bool REL>
@@ -103,10 +121,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const WaitCtl wc{a.wait_limit, a.status};
     volatile int* abort = &sm.abort;
     const int R = a.rope.R;
-    // Values come from a second pass over the cache (from L2: the score pass has just read
-    // the same rows) unless they are the rotated keys; the score copy is then free to be
-    // turned in place and released right after S^T.
-    const bool sep_v = a.kv_is_k != 2;
+    // One pass over the cache: a tile in shared memory is the K operand of S^T and the V
+    // operand of O^T.  Turned chunks go to side buffers when the values are the pre-RoPE
+    // keys, in place when they are the rotated keys.  Separate values take a second pass.
+    const bool sep_v = a.kv_is_k == 0;
+    const bool side_rot = a.kv_is_k == 1;
     const int n_items = a.splits * a.Hkv * a.B;
     const int slots_per_tile = sep_v ? 2 * NPAIR : NPAIR;
 
@@ -179,9 +198,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             if (!mbar_wait(&sm.empty[slot], ((q / kNSlots) & 1) ^ 1, wc, abort))
                                 break;
                             mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes);
-                            for (int h = 0; h < 2; ++h)
+                            for (int h = 0; h < 2; ++h) {
+                                const int c = pass ? 2 * k + h : slot_chunk(k, h, partner, NCH);
                                 tma_load_4d(sm.ring[slot] + h * kChunkBytes, map, &sm.full[slot],
-                                            slot_chunk(k, h, partner, NCH) * 64, w.g, key, w.b);
+                                            c * 64, w.g, key, w.b);
+                            }
                             ++q;
                         }
                     }
@@ -240,7 +261,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 const int c = slot_chunk(k, h, sep_v, NCH);
                                 if (!chunk_rotated(c, D, R)) continue;
                                 has_rot = true;
-                                const uint32_t ab = smem_u32(sm.ring[slot] + h * kChunkBytes);
+                                const uint32_t ab =
+                                    side_rot ? smem_u32(sm.rot[c == 0 ? 0 : 1])
+                                             : smem_u32(sm.ring[slot] + h * kChunkBytes);
                                 const uint32_t bb = smem_u32(sm.q[c]);
                                 for (int kk = 0; kk < 4; ++kk) {
                                     mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
@@ -261,19 +284,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (sep_v && !mbar_wait(&sm.full[slot], (k / kNSlots) & 1, wc, abort))
                             goto done;
                         tc_fence_after();
+                        const int blk = sep_v ? pr : slot_pair(pr, NPAIR);   // O^T block
                         const uint32_t ab = smem_u32(sm.ring[slot]);
                         for (int kk = 0; kk < 8; ++kk) {
                             // 16 keys per step = two 8-row groups of 1024 B; the slot's second
                             // 64-dim chunk is the next 64-element MN block (LBO)
                             const uint64_t ad = sdesc_sw128(ab + kk * 2048, kChunkBytes, 1024);
                             const uint32_t pb = smem_u32(sm.p[kk >> 2]) + (kk & 3) * 32;
-                            mma_bf16_ss(tm_o + pr * 16, ad, sdesc_sw128(pb, 16, 1024), idesc_o,
+                            mma_bf16_ss(tm_o + blk * 16, ad, sdesc_sw128(pb, 16, 1024), idesc_o,
                                         (t > 0 || kk > 0) ? 1u : 0u);
                         }
-                        if (sep_v) mma_commit(&sm.empty[slot]);
+                        mma_commit(&sm.empty[slot]);   // each slot as soon as its MMAs finish
                     }
-                    if (!sep_v)
-                        for (int pr = 0; pr < NPAIR; ++pr) mma_commit(&sm.empty[(qv + pr) % kNSlots]);
                     q += slots_per_tile;
                 }
                 mma_commit(&sm.o_done);
@@ -367,18 +389,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 __float2bfloat16_rn(y * cs.x - x * cs.y);
                         }
                         // keys: R(row theta) on the rotated pairs of this thread's row
-                        // REL implies the two-pass mode: chunks 0 and NCH/2 share slot 0
-                        uint8_t* src1 = sm.ring[qk % kNSlots];
-                        uint8_t* src2 = sm.ring[qk % kNSlots] + kChunkBytes;
-                        uint8_t* dst1 = src1;
-                        uint8_t* dst2 = src2;
+                        int k1, h1s, k2, h2s;
+                        chunk_slot(0, sep_v, NCH, k1, h1s);
+                        chunk_slot(NCH / 2, sep_v, NCH, k2, h2s);
+                        uint8_t* src1 = sm.ring[(qk + k1) % kNSlots] + h1s * kChunkBytes;
+                        uint8_t* src2 = sm.ring[(qk + k2) % kNSlots] + h2s * kChunkBytes;
+                        uint8_t* dst1 = side_rot ? sm.rot[0] : src1;
+                        uint8_t* dst2 = side_rot ? sm.rot[1] : src2;
 #pragma unroll
                         for (int g8 = 0; g8 < 8; ++g8) {
-                            if (g8 * 8 >= R) break;
+                            const bool rotg = g8 * 8 < R;
+                            if (!side_rot && !rotg) continue;   // in place: nothing to copy
                             const uint32_t off = sw128_offset(row, g8 * 8);
                             uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
                             uint4 x2 = *reinterpret_cast<const uint4*>(src2 + off);
-                            if (g8 * 8 < R) {
+                            if (rotg) {
                                 __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&x1);
                                 __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x2);
 #pragma unroll
@@ -408,15 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int c2i = c + NCH / 2;   // partner chunk: dims + d/2
                             uint8_t* src1;
                             uint8_t* src2;
-                            if (sep_v) {   // partner pairs share a slot
-                                src1 = sm.ring[(qk + c) % kNSlots];
-                                src2 = src1 + kChunkBytes;
-                            } else {
-                                src1 = sm.ring[(qk + c / 2) % kNSlots] + (c & 1) * kChunkBytes;
-                                src2 = sm.ring[(qk + c2i / 2) % kNSlots] + (c2i & 1) * kChunkBytes;
-                            }
-                            uint8_t* dst1 = src1;
-                            uint8_t* dst2 = src2;
+                            int k1, h1s, k2, h2s;
+                            chunk_slot(c, sep_v, NCH, k1, h1s);
+                            chunk_slot(c2i, sep_v, NCH, k2, h2s);
+                            src1 = sm.ring[(qk + k1) % kNSlots] + h1s * kChunkBytes;
+                            src2 = sm.ring[(qk + k2) % kNSlots] + h2s * kChunkBytes;
+                            uint8_t* dst1 = side_rot ? sm.rot[0] : src1;
+                            uint8_t* dst2 = side_rot ? sm.rot[1] : src2;
                             for (int g8 = 0; g8 < 8; ++g8) {
                                 const uint32_t off = sw128_offset(row, g8 * 8);
                                 uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
