@@ -22,6 +22,7 @@ G4ATTN_ERR_MISALIGNED = -3
 G4ATTN_ERR_WORKSPACE = -4
 G4ATTN_ERR_CUDA = -5
 G4ATTN_ERR_TIMEOUT = -6
+G4ATTN_ERR_TOO_LARGE = -7
 
 
 class G4AttnError(RuntimeError):
@@ -90,6 +91,7 @@ def _load():
         "g4attn_prefill": (I, [P, P, P, P, P, P, P, P, SZ, I, I, CFG, P]),
         "g4attn_decode_workspace_size": (SZ, [I, I, CFG]),
         "g4attn_decode": (I, [P, P, P, I, P, P, P, SZ, I, CFG, P]),
+        "g4attn_decode_noalloc": (I, [P, P, P, I, P, P, I, CFG, P]),
         "g4attn_status_string": (ctypes.c_char_p, [I]),
         "g4attn_device_status": (I, [P]),
         "g4attn_set_wait_limit": (LL, [LL]),
@@ -230,4 +232,27 @@ def g4attn_decode(q, kcache, vcache, cfg: LayerCfg, out=None, lse=None, want_lse
                             _ptr(workspace), workspace.numel(), B, ctypes.byref(c),
                             _stream(stream))
     _check(rc, "g4attn_decode")
+    return out, lse
+
+
+def g4attn_decode_noalloc(q, kcache, vcache, cfg: LayerCfg, out=None, lse=None, want_lse=False,
+                          stream=None):
+    """Decode one token without a workspace: for callers that cannot allocate device memory
+    (a plugin whose host framework owns all device memory and hands it only input and
+    output buffers, a service that reserves the whole device up front).  The split
+    partials go to a fixed 8 MiB scratch inside the library; problems that do not fit are
+    refused with G4ATTN_ERR_TOO_LARGE.  Calls share that scratch, so calls that overlap on
+    the GPU race; keep them on one stream.  `out` and `lse` are allocated here only when
+    not given."""
+    for t, n in ((q, "q"), (kcache, "kcache"), (vcache, "vcache")):
+        _bf16(t, n)
+    B, L = kcache.shape[0], kcache.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.n_q_heads), dtype=torch.float32, device=q.device)
+    c = cfg.c()
+    rc = _lib.g4attn_decode_noalloc(_ptr(q), _ptr(kcache), _ptr(vcache), L, _ptr(out), _ptr(lse),
+                                    B, ctypes.byref(c), _stream(stream))
+    _check(rc, "g4attn_decode_noalloc")
     return out, lse

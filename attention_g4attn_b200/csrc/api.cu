@@ -207,6 +207,8 @@ const char* g4attn_status_string(int s) {
         case G4ATTN_ERR_WORKSPACE: return "workspace missing or too small";
         case G4ATTN_ERR_CUDA: return "CUDA error";
         case G4ATTN_ERR_TIMEOUT: return "device wait timed out";
+        case G4ATTN_ERR_TOO_LARGE:
+            return "problem needs more than the fixed 8 MiB scratch of g4attn_decode_noalloc";
         default: return "unknown status";
     }
 }
@@ -372,6 +374,74 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
     if (!workspace || ws_bytes < plan.total) return G4ATTN_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
     uint8_t* w = static_cast<uint8_t*>(workspace);
+    g4::DecodeArgs a{};
+    const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
+    if (L > 0) {
+        if ((rc = encode_rows(&a.tm_k, kcache, B, L, Hkv, d))) return rc;
+        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, L, Hkv, d))) return rc;
+    }
+    a.q = q;
+    a.part_o = reinterpret_cast<float*>(w + plan.o_off);
+    a.part_ml = reinterpret_cast<float*>(w + plan.ml_off);
+    a.out = out;
+    a.lse = lse;
+    a.B = B; a.L = L; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d; a.G = G;
+    a.key_lo = plan.key_lo;
+    a.splits = plan.splits;
+    a.keys_per_split = plan.keys_per_split;
+    a.rope = make_rope(cfg);
+    a.scale_log2 = cfg->scale * 1.4426950408889634f;
+    a.kv_is_k = cfg->kv_is_k;
+    a.wait_limit = g_wait_limit.load();
+    a.status = dev->status;
+    return cuda_status(g4::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// Decode with no workspace argument and no allocation: the split partials go to the
+// library's fixed device scratch.  The split count is lowered until the partials fit; a
+// problem whose single-split partials (B * Hq * (d + 2) fp32) exceed the scratch is refused.
+int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
+                          const g4attn_bf16* vcache, int L, g4attn_bf16* out, float* lse, int B,
+                          const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
+    int rc = check_cfg(cfg, true);
+    if (rc) return rc;
+    if (B < 0 || L < 0) return G4ATTN_ERR_INVALID_ARG;
+    if (B == 0) return G4ATTN_OK;
+    if (!q || !out || (L > 0 && !kcache)) return G4ATTN_ERR_INVALID_ARG;
+    if ((cfg->kv_is_k == 0) != (vcache != nullptr)) return G4ATTN_ERR_INVALID_ARG;
+    const int G = cfg->n_q_heads / cfg->n_kv_heads;
+    if (G > 16) return G4ATTN_ERR_UNSUPPORTED;
+    if (cfg->kv_is_k == 1) {
+        const int R = rope_pairs(cfg);
+        int n = 0;
+        for (int c = 0; c < cfg->head_dim / 64; ++c) n += chunk_rotated(c, cfg->head_dim, R);
+        if (n > 2) return G4ATTN_ERR_UNSUPPORTED;
+    }
+    const void* ptrs[] = {q, kcache, vcache, out, lse};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    const size_t cap = g4::decode_scratch_bytes();
+    const size_t per_split = (size_t)B * cfg->n_q_heads;
+    if (align256(per_split * cfg->head_dim * sizeof(float)) + align256(per_split * 2 * sizeof(float)) >
+        cap)
+        return G4ATTN_ERR_TOO_LARGE;
+    DecodePlan plan = decode_plan(B, L, cfg, dev->sms);
+    while (plan.total > cap && plan.splits > 1) {   // fewer, longer splits until they fit
+        const int len = L - plan.key_lo;
+        const int tiles = (len + 127) / 128;
+        const int S = plan.splits - 1;
+        plan.keys_per_split = ((tiles + S - 1) / S) * 128;
+        plan.splits = (len + plan.keys_per_split - 1) / plan.keys_per_split;
+        const size_t n = (size_t)plan.splits * per_split;
+        plan.ml_off = align256(n * cfg->head_dim * sizeof(float));
+        plan.total = plan.ml_off + align256(n * 2 * sizeof(float));
+    }
+    if (plan.total > cap) return G4ATTN_ERR_TOO_LARGE;
+    void* scratch = nullptr;
+    if (g4::decode_scratch_ptr(&scratch) != cudaSuccess) return cuda_status(cudaErrorUnknown);
+    uint8_t* w = static_cast<uint8_t*>(scratch);
     g4::DecodeArgs a{};
     const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
     if (L > 0) {

@@ -22,6 +22,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <mutex>
+
 #include "kernels.h"
 #include "rope.cuh"
 #include "sm100.cuh"
@@ -651,6 +653,39 @@ cudaError_t dispatch_decode(const DecodeArgs& a, int grid, size_t smem, cudaStre
 }  // namespace
 
 size_t decode_smem_bytes() { return sizeof(DecodeSmem) + 1024; }
+
+// ------------------------------------------------------------------------------------
+// Fixed scratch for g4attn_decode_noalloc: the split partials live in this file-scope
+// device array instead of a caller workspace.  Every device that loads the library holds
+// it until the process exits.  In host code the array's name is only a stand-in, so its
+// device address is fetched with cudaGetSymbolAddress, once per device, with that device
+// current, and passed to the kernels.
+// ------------------------------------------------------------------------------------
+constexpr size_t kDecodeScratchBytes = size_t(8) << 20;   // 8 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+size_t decode_scratch_bytes() { return kDecodeScratchBytes; }
+
+cudaError_t decode_scratch_ptr(void** out) {
+    constexpr int kMaxDev = 64;
+    static void* ptr[kMaxDev] = {};
+    static bool ready[kMaxDev] = {};
+    static std::mutex mu;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(mu);
+    if (!ready[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess) return e;
+        ptr[dev] = p;
+        ready[dev] = true;
+    }
+    *out = ptr[dev];
+    return cudaSuccess;
+}
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     const size_t smem = decode_smem_bytes();

@@ -55,6 +55,9 @@ struct DecodeArgs {
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
 size_t decode_smem_bytes();
+// Fixed device scratch of g4attn_decode_noalloc (defined in decode.cu).
+size_t decode_scratch_bytes();
+cudaError_t decode_scratch_ptr(void** out);
 
 // Flash-attention prefill.
 struct PrefillArgs {

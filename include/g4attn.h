@@ -55,7 +55,8 @@ enum {
     G4ATTN_ERR_MISALIGNED = -3,    /* a pointer is not 16-byte aligned */
     G4ATTN_ERR_WORKSPACE = -4,     /* workspace missing or smaller than *_workspace_size */
     G4ATTN_ERR_CUDA = -5,          /* a CUDA runtime / driver call or launch failed */
-    G4ATTN_ERR_TIMEOUT = -6        /* a device wait gave up (see g4attn_device_status) */
+    G4ATTN_ERR_TIMEOUT = -6,       /* a device wait gave up (see g4attn_device_status) */
+    G4ATTN_ERR_TOO_LARGE = -7      /* g4attn_decode_noalloc: partials exceed its fixed scratch */
 };
 
 /* Layer configuration (one attention layer). */
@@ -137,6 +138,29 @@ G4ATTN_API size_t g4attn_decode_workspace_size(int B, int L, const g4attn_layer_
 G4ATTN_API int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_bf16* vcache,
                   int L, g4attn_bf16* out, float* lse, void* workspace, size_t ws_bytes,
                   int B, const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/*
+ * Decode without a workspace and without allocating (the papers describe no such call;
+ * it exists for callers that cannot allocate device memory: plugins whose host framework
+ * owns every device allocation and hands them only input and output buffers, and services
+ * that reserve the whole device up front).  Same operation, arguments and layouts as
+ * g4attn_decode minus the workspace: the split-KV partials live in a fixed 8 MiB device
+ * array inside the library, which every device that loads the library holds until the
+ * process exits.  The call allocates nothing.
+ *   - The split count is lowered until the partials fit; if even one split needs more
+ *     than 8 MiB (B * Hq * (head_dim + 2) * 4 bytes > 8 MiB), the call returns
+ *     G4ATTN_ERR_TOO_LARGE and launches nothing.
+ *   - The first call on a device looks up the array's device address (once per device,
+ *     with that device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's partials.  Nothing in it
+ *     needs to start at zero (every partial is written before it is read), but calls that
+ *     overlap on the GPU (different streams, or several host threads) race on it: order
+ *     them on one stream or synchronise between them.
+ */
+G4ATTN_API int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
+                                     const g4attn_bf16* vcache, int L, g4attn_bf16* out,
+                                     float* lse, int B, const g4attn_layer_cfg* cfg,
+                                     g4attn_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
 G4ATTN_API const char* g4attn_status_string(int status);

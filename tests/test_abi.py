@@ -45,7 +45,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings(b):
     assert b.g4attn_status_string(0) == "ok"
-    for code in range(-6, 0):
+    for code in range(-7, 0):
         s = b.g4attn_status_string(code)
         assert s and s != "unknown status"
     assert b.g4attn_status_string(-99) == "unknown status"
