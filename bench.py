@@ -267,6 +267,7 @@ def oracle_sample(max_seconds=20.0, seed=0):
 CASES = {
     # small cases for profiler captures: inputs larger than L2, a few GB on the device
     "global_prefill_T8192": ("prefill", dict(B=1, T=8192, layer="GLOBAL_8TO1")),
+    "global_prefill_T65536": ("prefill", dict(B=1, T=65536, layer="GLOBAL_8TO1")),
     "local_prefill_T16384": ("prefill", dict(B=1, T=16384, layer="LOCAL_W1024")),
     "global_decode_L8192": ("decode", dict(B=16, L=8192, layer="GLOBAL_8TO1")),
 }
