@@ -49,7 +49,8 @@ struct __align__(1024) DecodeSmem {
     uint8_t q[8][kN * 128];          // B operand of S^T: per 64-dim chunk, 16 rows x 128 B
     uint8_t p[2][kN * 128];          // B operand of O^T: P^T, K-major, 2 chunks of 64 keys
     float theta[256];                // base^(-2i/d) in fp32, i < R
-    float2 base_cs[256];             // cos/sin of tile_start * theta_i (fp64-reduced angle)
+    float2 base_cs[256];             // cos/sin of tile_start * theta_i
+    float2 step_cs[256];             // cos/sin of 128 * theta_i: one tile further
     float red[4][kN];                // cross-warp reductions
     float qb[kN][128];               // rotated dims of q (first and second half, R <= 64)
     uint64_t full[kNSlots];
@@ -147,8 +148,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
     if (warp >= 2) {
-        for (int i = threadIdx.x - 64; i < R; i += 128)
+        for (int i = threadIdx.x - 64; i < R; i += 128) {
             sm.theta[i] = (float)exp2(-(2.0 * (double)i / (double)D) * a.rope.log2_base);
+            sm.step_cs[i] = rope_cos_sin((long long)kTileKeys, i, D, a.rope.log2_base);
+        }
         for (int i = threadIdx.x - 64; i < (int)(sizeof(sm.p) / 16); i += 128)
             reinterpret_cast<uint4*>(&sm.p[0][0])[i] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
@@ -369,8 +372,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 q += slots_per_tile;
                 // ---- turn the rotated pairs of this tile's keys (and, REL, the queries)
                 if (R > 0) {
-                    for (int i = t128; i < R; i += 128)
-                        sm.base_cs[i] = rope_cos_sin((long long)key0, i, D, a.rope.log2_base);
+                    // start angle of the tile: exact (fp64-reduced) at the first tile of an
+                    // item, then advanced by one tile (128 keys) per step
+                    for (int i = t128; i < R; i += 128) {
+                        if (t == 0) {
+                            sm.base_cs[i] = rope_cos_sin((long long)key0, i, D, a.rope.log2_base);
+                        } else {
+                            const float2 b0 = sm.base_cs[i], st = sm.step_cs[i];
+                            sm.base_cs[i] = make_float2(b0.x * st.x - b0.y * st.y,
+                                                        b0.x * st.y + b0.y * st.x);
+                        }
+                    }
                     bool got = true;
                     for (int k = 0; k < NPAIR && got; ++k)
                         if (chunk_rotated(slot_chunk(k, 0, sep_v, NCH), D, R) ||
