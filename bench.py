@@ -357,11 +357,8 @@ def main():
         return
 
     import torch
-    dist = None
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from attention_g4attn_b200 import replicas
+    dist, rank, world, local_rank = replicas.init_from_env("nccl")
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     from attention_g4attn_b200 import binding as b  # noqa: F401  (fails loudly without the .so)
@@ -394,15 +391,12 @@ def main():
     total_s = t_start.elapsed_time(t_end) / 1e3
     pre_s = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
     dec_s = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
-    if dist:
-        t = torch.tensor([total_s, pre_s, dec_s], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_s, pre_s, dec_s = t.tolist()
+    total_s, pre_s, dec_s = replicas.max_over_ranks([total_s, pre_s, dec_s], dist, device)
 
     blk, dec = S["blk"], S["dec"]
     flops_step = blk.flops()
-    value = world * flops_step * args.steps / pre_s / 1e12
-    dec_gbs = world * dec.cache_bytes() * args.steps / dec_s / 1e9
+    value = replicas.job_rate(flops_step * args.steps, pre_s, world, 1e12)
+    dec_gbs = replicas.job_rate(dec.cache_bytes() * args.steps, dec_s, world, 1e9)
     peaks, peak_src = load_peaks()
     tf_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
@@ -447,11 +441,8 @@ def main():
         except RuntimeError as exc:   # pinned host memory refused
             e2e = {"error": str(exc)[:200]}
     if e2e is not None and "error" not in e2e:
-        if dist:
-            t = torch.tensor([e2e["seconds"]], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e["seconds"] = t.item()
-        e2e = {"value": world * flops_step * e2e["steps"] / e2e["seconds"] / 1e12,
+        e2e["seconds"] = replicas.max_over_ranks([e2e["seconds"]], dist, device)[0]
+        e2e = {"value": replicas.job_rate(flops_step * e2e["steps"], e2e["seconds"], world, 1e12),
                "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
                "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"]}
 

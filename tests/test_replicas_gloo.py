@@ -1,0 +1,54 @@
+"""The N > 1 path of the benchmark on CPU: two gloo ranks, each an independent replica, reduce
+their timings with MAX and report the whole-job rate (no data-path collective)."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    from attention_g4attn_b200 import replicas
+    dist, r, w, lr = replicas.init_from_env("gloo", timeout_s=30)
+    try:
+        # rank-dependent device times: rank 1 is the slowest on the first value only
+        local = [1.0 + r, 5.0 - r, 0.25]
+        got = replicas.max_over_ranks(local, dist)
+        rate = replicas.job_rate(100.0, got[0], w)
+        q.put((r, w, got, rate))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_replicas_reduce_timings_with_max():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    for r, w, got, rate in res:
+        assert w == 2
+        assert got == [2.0, 5.0, 0.25]          # max over ranks, element-wise
+        assert rate == pytest.approx(2 * 100.0 / 2.0)   # all ranks' units over the slowest time
+
+
+def test_single_process_is_a_no_op():
+    from attention_g4attn_b200 import replicas
+    assert replicas.max_over_ranks([1.5, 2.5]) == [1.5, 2.5]
+    assert replicas.job_rate(10.0, 2.0, 1) == 5.0
+    with pytest.raises(ValueError):
+        replicas.job_rate(1.0, 0.0, 1)
