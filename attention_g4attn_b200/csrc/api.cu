@@ -148,6 +148,8 @@ PrefillWs prefill_ws(int B, int T, const g4attn_layer_cfg* c) {
     return w;
 }
 
+constexpr int kDecodeTile = 64;   // keys per decode tile: splits are whole tiles
+
 struct DecodePlan {
     int key_lo, splits, keys_per_split;
     size_t o_off, ml_off, total;
@@ -157,7 +159,7 @@ DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms) {
     DecodePlan p{};
     p.key_lo = (c->window > 0 && L > c->window) ? L - c->window : 0;
     const int len = L - p.key_lo;
-    const int tiles = (len + 127) / 128;
+    const int tiles = (len + kDecodeTile - 1) / kDecodeTile;
     const int nbg = B * c->n_kv_heads;
     int S = 1;
     if (tiles > 0 && nbg > 0) {
@@ -170,7 +172,7 @@ DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms) {
         if (S < 1) S = 1;
     }
     const int tps = tiles > 0 ? (tiles + S - 1) / S : 1;
-    p.keys_per_split = tps * 128;
+    p.keys_per_split = tps * kDecodeTile;
     p.splits = len > 0 ? (len + p.keys_per_split - 1) / p.keys_per_split : 0;
     const size_t n = (size_t)(p.splits > 0 ? p.splits : 1) * B * c->n_q_heads;
     p.o_off = 0;
@@ -377,8 +379,8 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
     g4::DecodeArgs a{};
     const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
     if (L > 0) {
-        if ((rc = encode_rows(&a.tm_k, kcache, B, L, Hkv, d))) return rc;
-        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, L, Hkv, d))) return rc;
+        if ((rc = encode_rows(&a.tm_k, kcache, B, L, Hkv, d, false, 64))) return rc;
+        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, L, Hkv, d, false, 64))) return rc;
     }
     a.q = q;
     a.part_o = reinterpret_cast<float*>(w + plan.o_off);
@@ -430,9 +432,9 @@ int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
     DecodePlan plan = decode_plan(B, L, cfg, dev->sms);
     while (plan.total > cap && plan.splits > 1) {   // fewer, longer splits until they fit
         const int len = L - plan.key_lo;
-        const int tiles = (len + 127) / 128;
+        const int tiles = (len + kDecodeTile - 1) / kDecodeTile;
         const int S = plan.splits - 1;
-        plan.keys_per_split = ((tiles + S - 1) / S) * 128;
+        plan.keys_per_split = ((tiles + S - 1) / S) * kDecodeTile;
         plan.splits = (len + plan.keys_per_split - 1) / plan.keys_per_split;
         const size_t n = (size_t)plan.splits * per_split;
         plan.ml_off = align256(n * cfg->head_dim * sizeof(float));
@@ -445,8 +447,8 @@ int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
     g4::DecodeArgs a{};
     const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
     if (L > 0) {
-        if ((rc = encode_rows(&a.tm_k, kcache, B, L, Hkv, d))) return rc;
-        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, L, Hkv, d))) return rc;
+        if ((rc = encode_rows(&a.tm_k, kcache, B, L, Hkv, d, false, 64))) return rc;
+        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, L, Hkv, d, false, 64))) return rc;
     }
     a.q = q;
     a.part_o = reinterpret_cast<float*>(w + plan.o_off);

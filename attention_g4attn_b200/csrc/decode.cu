@@ -3,22 +3,33 @@
 //
 // Work item = (split s, kv head g, batch b): keys [k0, k1) of one sequence and all G query
 // heads that share kv head g (GQA; explainer "GQA": 8 query heads per KV head in global
-// layers).  Per tile of 128 keys:
-//   S^T[key, head]  = K_tile . Q^T         M = 128 keys, N = 16 (heads, zero padded), K = d
-//   O^T[d, head]   += K_tile^T . P^T        M = 128 d-rows per chunk, N = 16, K = 128 keys
-// Keys sit on the MMA's M side, so one 128-key tile in shared memory is the K operand of
-// the first product and, read MN-major, the V operand of the second (keys reused as
-// values, report section 2 / explainer "K=V": one cache read serves both).  The cache
-// holds pre-RoPE keys; the rotated pairs (i, i + d/2), i < R, of every key are turned to
-// the key's position on the fly (report section 2, p-RoPE) by the softmax warps, in place.
-// When the values are the pre-RoPE keys, the value operand is a second TMA pass over the
-// same rows (served from L2: the score pass has just read them), so the score copy can be
-// turned in place and released as soon as S^T has read it; HBM still reads the cache once.
+// layers).  Keys stream through in tiles of 64.  A tile sits in shared memory as D/128
+// slots of 128 rows x 64 dims: in slot j, row r < 64 holds dims [64j, 64j + 64) of key r
+// and row 64 + r holds dims [d/2 + 64j, d/2 + 64j + 64) of the same key, so the two
+// halves of every key row are stacked on the MMA's M = 128 side:
+//   S^T[half*64 + key, n] = sum over the slot's 64 dims of K . Q^T   N = 2 NH
+// with columns n < NH holding the queries' first-half dims and n >= NH their second-half
+// dims; the two useful quarters (rows < 64 with n < NH, rows >= 64 with n >= NH) are the
+// two halves of the score and are added by the softmax threads.  The same slot, read
+// MN-major, is the value operand of
+//   O^T[dim, head] += V^T . P^T                                       M = 128 dims, N = 16
+// (keys reused as values, report section 2 / explainer "K=V": one cache read serves both).
+// RoPE pairs dims (i, i + d/2), i < R (report section 2, p-RoPE): both members of a pair
+// sit in the same slot, rows r and 64 + r, so the softmax warps turn a key's rotated
+// pairs inside one slot.  With pre-RoPE values the turned slot goes to a side buffer and
+// the original stays as the value operand.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
-// warps 2..5 rotation / softmax / epilogue (thread = TMEM lane = key row or d-row).
-// The CTA is persistent over work items blockIdx.x, +gridDim.x, ...  Every mbarrier wait
-// is bounded (sm100.cuh); on a timeout all roles drain their in-flight work and exit.
+// Pipeline: one warpgroup turns the rotated pairs of tile t + 1 (and stages the queries)
+// while another runs the softmax of tile t, and the MMA warp issues S^T of tile t + 1
+// before O^T of tile t, so loads, rotation, scores, softmax and the value product of
+// neighbouring tiles overlap.  A 64-key tile holds 64 KB (d = 512), so the ring keeps
+// two and a half tiles.
+//
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// warps 2..5 softmax / epilogue (thread = TMEM lane), warps 6..9 query staging and key
+// rotation.  The CTA is persistent over work items blockIdx.x, +gridDim.x, ...  Every
+// mbarrier wait is bounded (sm100.cuh); on a timeout all roles drain their in-flight work
+// and exit.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -31,31 +42,46 @@
 namespace g4 {
 namespace {
 
-constexpr int kThreads = 192;
-constexpr int kTileKeys = 128;
-constexpr int kNSlots = 5;           // ring of 32 KB slots: 128 keys x 128 dims (2 chunks)
-constexpr int kMaxRotChunks = 2;     // side buffers for the turned chunks (values = pre-RoPE)
-constexpr int kSlotBytes = 32768;
-constexpr int kChunkBytes = 16384;   // 128 keys x 64 dims, 128-byte swizzled rows
-constexpr int kN = 16;               // MMA N: query heads of one KV head, zero padded
-constexpr uint32_t kTmemCols = 128;
-constexpr int kBarWG = 1;            // named barrier of the softmax warpgroup
+constexpr int kThreads = 320;
+constexpr int kTileKeys = 64;
+constexpr int kSlotBytes = 16384;    // 128 rows x 128 B: 64 keys x 64 dims of each half
+constexpr int kBoxBytes = 8192;      // one TMA box: 64 keys x 64 dims
+constexpr int kNO = 16;              // N of the value product: query heads, zero padded
+constexpr uint32_t kTmemCols = 128;  // S^T double buffer (2 x 32) + O^T (4 x 16)
+constexpr int kBarSM = 1;            // named barrier of the softmax warpgroup
+constexpr int kBarRot = 2;           // named barrier of the rotation warpgroup
 constexpr float kLazyMax = 8.0f;     // log2 units: headroom of the lazy reference max
-constexpr int kPrefetchTiles = 3;    // L2 prefetch distance, in tiles
 
+template <int NH>
+struct DecodeCfg {
+    static constexpr int NS = 2 * NH;                // N of S^T
+    static constexpr int HH = NH / 2;                // heads finished by each half of the rows
+    static constexpr int NSLOT = NH == 8 ? 10 : 9;   // ring slots of 16 KB
+};
+
+template <int NH>
 struct __align__(1024) DecodeSmem {
-    uint8_t ring[kNSlots][kSlotBytes];
-    uint8_t rot[kMaxRotChunks][kChunkBytes];
-    uint8_t q[8][kN * 128];          // B operand of S^T: per 64-dim chunk, 16 rows x 128 B
-    uint8_t p[2][kN * 128];          // B operand of O^T: P^T, K-major, 2 chunks of 64 keys
-    float theta[256];                // base^(-2i/d) in fp32, i < R
-    float2 base_cs[256];             // cos/sin of tile_start * theta_i
-    float2 step_cs[256];             // cos/sin of 128 * theta_i: one tile further
-    float red[4][kN];                // cross-warp reductions
-    float qb[kN][128];               // rotated dims of q (first and second half, R <= 64)
-    uint64_t full[kNSlots];
-    uint64_t empty[kNSlots];
-    uint64_t s_full, p_full, rot_ready, q_ready, o_done, drain;
+    using C = DecodeCfg<NH>;
+    uint8_t ring[C::NSLOT][kSlotBytes];
+    uint8_t side[2][kSlotBytes];       // turned slot 0 of tiles j & 1 (values = pre-RoPE keys)
+    // B operand of S^T per slot, K-major, swizzled; q[4] is the second copy of slot 0's
+    // operand, which the relative rotation rewrites for every tile (tile j uses copy j & 1)
+    uint8_t q[5][C::NS * 128];
+    uint8_t p[2][kNO * 128];           // B operand of O^T: P^T, K-major, 64 keys per row
+    float xs[2][64][C::HH];            // score halves handed to the other half's threads
+    float theta[256];                  // base^(-2i/d) in fp32
+    float2 base_cs[256];               // cos/sin of tile_start * theta_i
+    float2 step_cs[256];               // cos/sin of 64 * theta_i: one tile further
+    float red[4][C::HH];               // cross-warp reductions
+    float alpha[NH];                   // rescale factors of O^T
+    float mfin[NH];                    // running max per head at the end of an item
+    float qb[NH][128];                 // rotated dims of q (first and second half, R <= 64)
+    uint64_t full[C::NSLOT];
+    uint64_t empty[C::NSLOT];
+    // per-tile barriers come in pairs (tile j uses [j & 1], phase (j >> 1) & 1): a waiter is
+    // never more than one phase of a barrier behind
+    uint64_t s_full[2], p_full[2], pv_done[2], rot_ready[2];
+    uint64_t q_ready, q_free, drain;   // once per item: q staged / all its scores done
     uint32_t tmem_base;
     int abort;
 };
@@ -80,79 +106,85 @@ __device__ __forceinline__ Item item_of(const DecodeArgs& a, int it) {
     return r;
 }
 
-// Does 64-dim chunk c hold rotated dims?  Rotated dims: [0, R) and [d/2, d/2 + R).
-__device__ __forceinline__ bool chunk_rotated(int c, int d, int R) {
-    const int lo = c * 64, hi = lo + 64, h = d / 2;
-    return (lo < R) || (lo < h + R && hi > h);
+// O^T += V^T . P^T for one tile: the value slots at ring position qv, P^T in p[j & 1].
+// Releases every slot once its MMAs finish, then signals pv_done.
+template <int D, int NH>
+__device__ __forceinline__ bool issue_pv(DecodeSmem<NH>& sm, uint32_t tm_o, uint32_t j,
+                                         uint32_t qv, bool first, bool sep_v,
+                                         const WaitCtl& wc, volatile int* abort) {
+    using C = DecodeCfg<NH>;
+    constexpr int NSB = D / 128;
+    const uint32_t idesc_o = idesc_bf16_f32(128, kNO, true, false);  // A = V^T, MN-major
+    if (!mbar_wait(&sm.p_full[j & 1], (j >> 1) & 1, wc, abort)) return false;
+    tc_fence_after();
+    const uint32_t pb = smem_u32(sm.p[j & 1]);
+    for (int sb = 0; sb < NSB; ++sb) {
+        const uint32_t k = qv + sb, slot = k % C::NSLOT;
+        if (sep_v && !mbar_wait(&sm.full[slot], (k / C::NSLOT) & 1, wc, abort)) return false;
+        tc_fence_after();
+        const uint32_t ab = smem_u32(sm.ring[slot]);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            // 16 keys per step = two 8-row groups of 1024 B; the second half's dims are the
+            // next 64-element MN block, one TMA box (8 KB) further
+            mma_bf16_ss(tm_o + sb * 16, sdesc_sw128(ab + kk * 2048, kBoxBytes, 1024),
+                        sdesc_sw128(pb + kk * 32, 16, 1024), idesc_o,
+                        (first && kk == 0) ? 0u : 1u);
+        }
+        mma_commit(&sm.empty[slot]);
+    }
+    mma_commit(&sm.pv_done[j & 1]);
+    return true;
 }
 
 // D: head dim; NH: query heads per KV head handled by the softmax (8 or 16, >= G);
 // REL: relative rotation (values are not the rotated key and R <= 64).
-// Chunk (64 dims) held by half h of the k-th slot of a tile.  Score slots of the two-pass
-// mode pair each chunk with its rotation partner (chunks k and k + NCH/2), so turning a
-// key needs one slot; value slots, and the slots of the one-pass mode (values = rotated
-// keys), hold consecutive chunks (2k, 2k+1), the 128 value rows of one O^T block.
-// One-pass slots hold chunk pairs (2m, 2m+1) in the order m = 0, npair/2, 1, npair/2+1, ...
-// so the two rotation partners (chunks 0 and nch/2) arrive in the first two slots.
-__device__ __forceinline__ int slot_pair(int k, int npair) {
-    return (k & 1) ? (npair / 2 + k / 2) : (k / 2);
-}
-__device__ __forceinline__ int slot_chunk(int k, int h, bool partner_pairs, int nch) {
-    return partner_pairs ? k + h * (nch / 2) : 2 * slot_pair(k, nch / 2) + h;
-}
-// Slot index and half of chunk c within a tile.
-__device__ __forceinline__ void chunk_slot(int c, bool partner_pairs, int nch, int& k, int& h) {
-    if (partner_pairs) {
-        k = c % (nch / 2);
-        h = c / (nch / 2);
-    } else {
-        const int m = c / 2, np = nch / 2;
-        h = c & 1;
-        k = (m < np / 2) ? 2 * m : 2 * (m - np / 2) + 1;
-    }
-}
-
 template <int D, int NH, bool REL>
 __global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a) {
-    constexpr int NCH = D / 64;     // 64-dim chunks per key row
-    constexpr int NPAIR = D / 128;  // 32 KB ring slots per tile and tensor
+    using C = DecodeCfg<NH>;
+    constexpr int NSB = D / 128;    // slots per tile and tensor
+    constexpr int NS = C::NS, HH = C::HH, NSLOT = C::NSLOT;
     extern __shared__ uint8_t smem_raw[];
-    DecodeSmem& sm = *reinterpret_cast<DecodeSmem*>(
+    DecodeSmem<NH>& sm = *reinterpret_cast<DecodeSmem<NH>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const WaitCtl wc{a.wait_limit, a.status};
     volatile int* abort = &sm.abort;
     const int R = a.rope.R;
-    // One pass over the cache: a tile in shared memory is the K operand of S^T and the V
-    // operand of O^T.  Turned chunks go to side buffers when the values are the pre-RoPE
-    // keys, in place when they are the rotated keys.  Separate values take a second pass.
+    const int nrot = (R + 63) / 64;   // slots holding rotated pairs: 0 .. nrot-1
+    // K and V share the ring slots unless the values are a separate tensor (second pass).
+    // Turned slots go to the side buffer when the values are the pre-RoPE keys.
     const bool sep_v = a.kv_is_k == 0;
     const bool side_rot = a.kv_is_k == 1;
     const int n_items = a.splits * a.Hkv * a.B;
-    const int slots_per_tile = sep_v ? 2 * NPAIR : NPAIR;
+    const int slots_per_tile = sep_v ? 2 * NSB : NSB;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kNSlots; ++i) {
+        for (int i = 0; i < NSLOT; ++i) {
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], 1);
         }
-        mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.p_full, 1);
-        mbar_init(&sm.rot_ready, 1);
         mbar_init(&sm.q_ready, 1);
-        mbar_init(&sm.o_done, 1);
+        mbar_init(&sm.q_free, 1);
+        mbar_init(&sm.rot_ready[0], 1);
+        mbar_init(&sm.rot_ready[1], 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.s_full[i], 1);
+            mbar_init(&sm.p_full[i], 1);
+            mbar_init(&sm.pv_done[i], 1);
+        }
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
     if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
     if (warp >= 2) {
-        for (int i = threadIdx.x - 64; i < R; i += 128) {
+        for (int i = threadIdx.x - 64; i < R; i += 256) {
             sm.theta[i] = (float)exp2(-(2.0 * (double)i / (double)D) * a.rope.log2_base);
             sm.step_cs[i] = rope_cos_sin((long long)kTileKeys, i, D, a.rope.log2_base);
         }
-        for (int i = threadIdx.x - 64; i < (int)(sizeof(sm.p) / 16); i += 128)
+        for (int i = threadIdx.x - 64; i < (int)(sizeof(sm.p) / 16); i += 256)
             reinterpret_cast<uint4*>(&sm.p[0][0])[i] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
@@ -160,54 +192,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t tm_s = tmem;          // S^T: 16 columns
-    const uint32_t tm_o = tmem + 16;     // O^T: NPAIR blocks of 16 columns
+    const uint32_t tm_o = tmem + 64;     // O^T: NSB blocks of 16 columns
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
             prefetch_tmap(&a.tm_k);
             if (sep_v) prefetch_tmap(&a.tm_v);
-            // L2 prefetch cursor: runs kPrefetchTiles tiles ahead of the loads, across the
-            // items of this CTA, so HBM keeps streaming while the ring slots are busy
-            int pf_it = blockIdx.x, pf_t = 0;
-            long long pf_count = 0, load_count = 0;
             uint32_t q = 0;   // ring slots filled so far
             for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
                 const Item w = item_of(a, it);
                 const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
-                for (int t = 0; t < nt && !*abort; ++t, ++load_count) {
+                for (int t = 0; t < nt && !*abort; ++t) {
                     const int key = w.k0 + t * kTileKeys;
-                    while (pf_count <= load_count + kPrefetchTiles && pf_it < n_items) {
-                        const Item pw = item_of(a, pf_it);
-                        const int pnt = ceil_div(pw.k1 - pw.k0, kTileKeys);
-                        if (pf_t < pnt) {
-                            const int pk = pw.k0 + pf_t * kTileKeys;
-                            for (int c = 0; c < NCH; ++c) {
-                                tma_prefetch_l2_4d(&a.tm_k, c * 64, pw.g, pk, pw.b);
-                                if (a.kv_is_k == 0)   // a separate value cache
-                                    tma_prefetch_l2_4d(&a.tm_v, c * 64, pw.g, pk, pw.b);
-                            }
-                            ++pf_count;
-                        }
-                        if (++pf_t >= pnt) {
-                            pf_t = 0;
-                            pf_it += gridDim.x;
-                        }
-                    }
                     for (int pass = 0; pass < (sep_v ? 2 : 1) && !*abort; ++pass) {
                         const CUtensorMap* map = pass ? &a.tm_v : &a.tm_k;
-                        const bool partner = sep_v && pass == 0;
-                        for (int k = 0; k < NPAIR; ++k) {
-                            const int slot = q % kNSlots;
-                            if (!mbar_wait(&sm.empty[slot], ((q / kNSlots) & 1) ^ 1, wc, abort))
+                        for (int sb = 0; sb < NSB; ++sb) {
+                            const int slot = q % NSLOT;
+                            if (!mbar_wait(&sm.empty[slot], ((q / NSLOT) & 1) ^ 1, wc, abort))
                                 break;
                             mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes);
-                            for (int h = 0; h < 2; ++h) {
-                                const int c = pass ? 2 * k + h : slot_chunk(k, h, partner, NCH);
-                                tma_load_4d(sm.ring[slot] + h * kChunkBytes, map, &sm.full[slot],
-                                            c * 64, w.g, key, w.b);
-                            }
+                            tma_load_4d(sm.ring[slot], map, &sm.full[slot], sb * 64, w.g, key, w.b);
+                            tma_load_4d(sm.ring[slot] + kBoxBytes, map, &sm.full[slot],
+                                        D / 2 + sb * 64, w.g, key, w.b);
                             ++q;
                         }
                     }
@@ -215,165 +222,333 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             // before the CTA exits, every copy it started must have landed
             if (*abort) {
-                const uint32_t first = q > (uint32_t)kNSlots ? q - kNSlots : 0;
+                const uint32_t first = q > (uint32_t)NSLOT ? q - NSLOT : 0;
                 for (uint32_t k = first; k < q; ++k)
-                    mbar_wait_drain(&sm.full[k % kNSlots], (k / kNSlots) & 1, a.wait_limit);
+                    mbar_wait_drain(&sm.full[k % NSLOT], (k / NSLOT) & 1, a.wait_limit);
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16_f32(128, kN, false, false);
-            const uint32_t idesc_o = idesc_bf16_f32(128, kN, true, false);  // A = V^T, MN-major
-            uint32_t q = 0, tile = 0, item_n = 0;
+            const uint32_t idesc_s = idesc_bf16_f32(128, NS, false, false);
+            uint32_t q = 0, gt = 0, item_n = 0;
+            // the value product of a tile goes out as soon as its P is ready, between the
+            // score MMAs of the next tile, which are issued slot by slot as the slots land
+            bool pv_pending = false, pv_first = false;
+            uint32_t pv_tile = 0, pv_q = 0;
             for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++item_n) {
                 const Item w = item_of(a, it);
                 const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
-                if (!mbar_wait(&sm.q_ready, item_n & 1, wc, abort)) goto done;
-                for (int t = 0; t < nt; ++t, ++tile) {
+                for (int t = 0; t < nt; ++t, ++gt) {
                     const uint32_t qk = q;
-                    const uint32_t qv = sep_v ? q + NPAIR : q;
+                    const uint32_t qv = sep_v ? q + NSB : q;
+                    q += slots_per_tile;
+                    const uint32_t tm_s = tmem + (gt & 1) * 32;
                     bool first = true;
-                    // S^T over the chunks that need no rotation, as soon as they land; in the
-                    // two-pass mode each score slot is released right after its last MMA
-                    for (int k = 0; k < NPAIR; ++k) {
-                        const uint32_t qq = qk + k, slot = qq % kNSlots;
-                        if (!mbar_wait(&sm.full[slot], (qq / kNSlots) & 1, wc, abort)) goto done;
-                        tc_fence_after();
-                        bool has_rot = false;
-                        for (int h = 0; h < 2; ++h) {
-                            const int c = slot_chunk(k, h, sep_v, NCH);
-                            if (chunk_rotated(c, D, R)) { has_rot = true; continue; }
-                            const uint32_t ab = smem_u32(sm.ring[slot] + h * kChunkBytes);
-                            const uint32_t bb = smem_u32(sm.q[c]);
+                    bool q_ok = t > 0;               // the item's queries are staged
+                    int next_sb = nrot;              // next unrotated slot
+                    bool rot_done = nrot == 0;
+                    const unsigned long long t_start = global_ns();
+                    long long polls = 0;
+                    while (next_sb < NSB || !rot_done) {
+                        if (pv_pending &&
+                            mbar_test_wait(&sm.p_full[pv_tile & 1], (pv_tile >> 1) & 1)) {
+                            if (!issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v, wc,
+                                                 abort))
+                                goto done;
+                            pv_pending = false;
+                            continue;
+                        }
+                        if (!q_ok) {
+                            q_ok = mbar_test_wait(&sm.q_ready, item_n & 1);
+                            if (q_ok) continue;
+                        } else if (next_sb < NSB &&
+                                   mbar_test_wait(&sm.full[(qk + next_sb) % NSLOT],
+                                                  ((qk + next_sb) / NSLOT) & 1)) {
+                            tc_fence_after();
+                            const uint32_t slot = (qk + next_sb) % NSLOT;
+                            const uint32_t ab = smem_u32(sm.ring[slot]);
+                            const uint32_t bb = smem_u32(sm.q[next_sb]);
+#pragma unroll
                             for (int kk = 0; kk < 4; ++kk) {
                                 mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
                                             sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
                                             first ? 0u : 1u);
                                 first = false;
                             }
-                        }
-                        if (sep_v && !has_rot) mma_commit(&sm.empty[slot]);
-                    }
-                    // then the rotated chunks, once the softmax warps have turned them
-                    if (R > 0) {
-                        if (!mbar_wait(&sm.rot_ready, tile & 1, wc, abort)) goto done;
-                        tc_fence_after();
-                        for (int k = 0; k < NPAIR; ++k) {
-                            const uint32_t slot = (qk + k) % kNSlots;
-                            bool has_rot = false;
-                            for (int h = 0; h < 2; ++h) {
-                                const int c = slot_chunk(k, h, sep_v, NCH);
-                                if (!chunk_rotated(c, D, R)) continue;
-                                has_rot = true;
-                                const uint32_t ab =
-                                    side_rot ? smem_u32(sm.rot[c == 0 ? 0 : 1])
-                                             : smem_u32(sm.ring[slot] + h * kChunkBytes);
-                                const uint32_t bb = smem_u32(sm.q[c]);
+                            // score slots of a separate-value layer go back right away
+                            if (sep_v) mma_commit(&sm.empty[slot]);
+                            ++next_sb;
+                            continue;
+                        } else if (!rot_done &&
+                                   mbar_test_wait(&sm.rot_ready[gt & 1], (gt >> 1) & 1)) {
+                            // the rotated slots, once the rotation warps have turned them
+                            tc_fence_after();
+                            for (int sb = 0; sb < nrot; ++sb) {
+                                const uint32_t slot = (qk + sb) % NSLOT;
+                                const uint32_t ab = side_rot ? smem_u32(sm.side[gt & 1])
+                                                             : smem_u32(sm.ring[slot]);
+                                const uint32_t bb =
+                                    smem_u32(sm.q[(REL && sb == 0 && (gt & 1)) ? 4 : sb]);
+#pragma unroll
                                 for (int kk = 0; kk < 4; ++kk) {
                                     mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
                                                 sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
                                                 first ? 0u : 1u);
                                     first = false;
                                 }
+                                if (sep_v) mma_commit(&sm.empty[slot]);
                             }
-                            if (sep_v && has_rot) mma_commit(&sm.empty[slot]);
+                            rot_done = true;
+                            continue;
                         }
-                    }
-                    mma_commit(&sm.s_full);
-                    // O^T += V^T . P^T once the softmax warps have written P
-                    if (!mbar_wait(&sm.p_full, tile & 1, wc, abort)) goto done;
-                    tc_fence_after();
-                    for (int pr = 0; pr < NPAIR; ++pr) {
-                        const uint32_t k = qv + pr, slot = k % kNSlots;
-                        if (sep_v && !mbar_wait(&sm.full[slot], (k / kNSlots) & 1, wc, abort))
+                        // nothing ready: bounded polling, like every other wait
+                        if (*abort) goto done;
+                        if ((++polls & 63) == 0 &&
+                            (polls >= a.wait_limit || global_ns() - t_start > kWaitTimeoutNs)) {
+                            atomicExch(a.status, (int)G4ATTN_ERR_TIMEOUT);
+                            *abort = 1;
                             goto done;
-                        tc_fence_after();
-                        const int blk = sep_v ? pr : slot_pair(pr, NPAIR);   // O^T block
-                        const uint32_t ab = smem_u32(sm.ring[slot]);
-                        for (int kk = 0; kk < 8; ++kk) {
-                            // 16 keys per step = two 8-row groups of 1024 B; the slot's second
-                            // 64-dim chunk is the next 64-element MN block (LBO)
-                            const uint64_t ad = sdesc_sw128(ab + kk * 2048, kChunkBytes, 1024);
-                            const uint32_t pb = smem_u32(sm.p[kk >> 2]) + (kk & 3) * 32;
-                            mma_bf16_ss(tm_o + blk * 16, ad, sdesc_sw128(pb, 16, 1024), idesc_o,
-                                        (t > 0 || kk > 0) ? 1u : 0u);
                         }
-                        mma_commit(&sm.empty[slot]);   // each slot as soon as its MMAs finish
                     }
-                    q += slots_per_tile;
+                    mma_commit(&sm.s_full[gt & 1]);
+                    if (t == nt - 1) mma_commit(&sm.q_free);   // q may be restaged
+                    if (pv_pending &&
+                        !issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v, wc, abort))
+                        goto done;
+                    pv_pending = true;
+                    pv_tile = gt;
+                    pv_q = qv;
+                    pv_first = t == 0;
                 }
-                mma_commit(&sm.o_done);
             }
+            if (pv_pending) issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v, wc, abort);
         done:
             // all issued MMAs must finish before the tensor memory is released
             mma_commit(&sm.drain);
             mbar_wait_drain(&sm.drain, 0, a.wait_limit);
         }
-    } else {
-        // ---------------------------------------------- rotation / softmax / epilogue
+    } else if (warp < 6) {
+        // ------------------------------------------------- softmax / epilogue (warps 2..5)
         const int t128 = threadIdx.x - 64;            // 0..127
         const int quarter = warp & 3;                 // TMEM lane quarter of this warp
-        const int row = quarter * 32 + lane;          // TMEM lane: key row or d-row
+        const int row = quarter * 32 + lane;          // TMEM lane: (half, key) or O^T dim row
+        const int hf = row >> 6;                      // half of d whose score rows this is
+        const int key = row & 63;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int G = a.G;
         const float c2 = a.scale_log2;
-        // Relative rotation (REL): key row `row` of every tile sits at angle row*theta_i from
+        uint32_t gt = 0;
+        bool ok = true;
+        // the value product of tile j is complete (a no-op for j < 0)
+        auto wait_pv = [&](int j) -> bool {
+            const bool good = j < 0 || mbar_wait(&sm.pv_done[j & 1], (j >> 1) & 1, wc, abort);
+            return group_all(good, kBarSM, 128);
+        };
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const Item w = item_of(a, it);
+            const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+            float m_run[HH], l_part[HH];
+#pragma unroll
+            for (int j = 0; j < HH; ++j) {
+                m_run[j] = -INFINITY;
+                l_part[j] = 0.f;
+            }
+            for (int t = 0; t < nt; ++t, ++gt) {
+                ok = group_all(mbar_wait(&sm.s_full[gt & 1], (gt >> 1) & 1, wc, abort), kBarSM,
+                               128);
+                if (!ok) break;
+                tc_fence_after();
+                const int key0 = w.k0 + t * kTileKeys;
+                float sp[NH];
+                if constexpr (NH == 8) tmem_ld8(tmem + (gt & 1) * 32 + hf * NH + lane_off, sp);
+                else tmem_ld16(tmem + (gt & 1) * 32 + hf * NH + lane_off, sp);
+                tmem_ld_wait();
+                // hand the heads the other half finishes to it, take ours from it
+#pragma unroll
+                for (int j = 0; j < HH; ++j) sm.xs[hf ^ 1][key][j] = hf ? sp[j] : sp[HH + j];
+                group_sync(kBarSM, 128);
+                const bool valid = key0 + key < w.k1;
+                float x[HH];
+                bool big = false;
+#pragma unroll
+                for (int j = 0; j < HH; ++j) {
+                    const int h = hf * HH + j;
+                    const float sc = (hf ? sp[HH + j] : sp[j]) + sm.xs[hf][key][j];
+                    x[j] = (valid && h < G) ? sc * c2 : -INFINITY;
+                    big |= x[j] > m_run[j] + kLazyMax;
+                }
+                // lazy reference max: only when some score of the tile exceeds the running
+                // reference by more than 2^8 (and on the first tile) do the warps reduce
+                const bool fast = (t > 0) && group_all(!big, kBarSM, 128);
+                float alpha[HH];
+#pragma unroll
+                for (int j = 0; j < HH; ++j) alpha[j] = 1.f;
+                if (!fast) {
+#pragma unroll
+                    for (int j = 0; j < HH; ++j) {
+                        float mt = x[j];
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1)
+                            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+                        if (lane == 0) sm.red[quarter][j] = mt;
+                    }
+                    group_sync(kBarSM, 128);
+                    bool resc = false;
+#pragma unroll
+                    for (int j = 0; j < HH; ++j) {
+                        const float tmax = fmaxf(sm.red[2 * hf][j], sm.red[2 * hf + 1][j]);
+                        if (tmax > m_run[j] + kLazyMax ||
+                            (m_run[j] == -INFINITY && tmax != -INFINITY)) {
+                            alpha[j] = (m_run[j] == -INFINITY) ? 0.f : exp2f(m_run[j] - tmax);
+                            m_run[j] = tmax;
+                            resc |= t > 0;
+                        }
+                    }
+                    if (lane == 0 && (quarter & 1) == 0)
+#pragma unroll
+                        for (int j = 0; j < HH; ++j) sm.alpha[hf * HH + j] = alpha[j];
+                    const bool rescale = !group_all(!resc, kBarSM, 128);  // also orders alpha
+                    // rescale O^T (thread = dim row, column = head) once the value product
+                    // of the tile before is complete; the next one waits for this tile's P
+                    if (rescale) {
+                        ok = wait_pv((int)gt - 1);
+                        if (!ok) break;
+                        tc_fence_after();
+                        for (int sb = 0; sb < NSB; ++sb) {
+                            float o[kNO];
+                            tmem_ld16(tm_o + sb * 16 + lane_off, o);
+                            tmem_ld_wait();
+#pragma unroll
+                            for (int h = 0; h < NH; ++h) o[h] *= sm.alpha[h];
+                            tmem_st16(tm_o + sb * 16 + lane_off, o);
+                        }
+                        tmem_st_wait();
+                    }
+                }
+                // P^T into p[gt & 1] once the value product that last read it is complete
+                ok = wait_pv((int)gt - 2);
+                if (!ok) break;
+                {
+                    uint8_t* pb = sm.p[gt & 1];
+#pragma unroll
+                    for (int j = 0; j < HH; ++j) {
+                        const float p = (x[j] == -INFINITY) ? 0.f : ex2_approx(x[j] - m_run[j]);
+                        const __nv_bfloat16 pr = __float2bfloat16_rn(p);
+                        // the running sum uses the rounded weight the MMA sees
+                        l_part[j] = l_part[j] * alpha[j] + __bfloat162float(pr);
+                        *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(hf * HH + j, key)) = pr;
+                    }
+                }
+                fence_proxy_async_smem();
+                tc_fence_before();
+                group_sync(kBarSM, 128);
+                if (t128 == 0) mbar_arrive(&sm.p_full[gt & 1]);
+            }
+            if (!ok) break;
+            // ---- item epilogue: partial O^T, running max and sum
+            ok = wait_pv((int)gt - 1);
+            if (!ok) break;
+            tc_fence_after();
+            const size_t obase = ((size_t)w.s * a.B + w.b) * a.Hq + (size_t)w.g * G;
+            const int dim0 = (row < 64) ? row : D / 2 + (row - 64);
+            for (int sb = 0; sb < NSB; ++sb) {
+                float o[kNO];
+                tmem_ld16(tm_o + sb * 16 + lane_off, o);
+                tmem_ld_wait();
+#pragma unroll
+                for (int h = 0; h < NH; ++h)
+                    if (h < G) a.part_o[(obase + h) * D + sb * 64 + dim0] = o[h];
+            }
+#pragma unroll
+            for (int j = 0; j < HH; ++j) {
+                float l = l_part[j];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+                if (lane == 0) sm.red[quarter][j] = l;
+                if (lane == 0 && (quarter & 1) == 0) sm.mfin[hf * HH + j] = m_run[j];
+            }
+            group_sync(kBarSM, 128);
+            if (t128 < G) {
+                const int h = t128, hh = h / HH, j = h % HH;
+                a.part_ml[(obase + h) * 2 + 0] = sm.mfin[h];
+                a.part_ml[(obase + h) * 2 + 1] = sm.red[2 * hh][j] + sm.red[2 * hh + 1][j];
+            }
+            tc_fence_before();
+            group_sync(kBarSM, 128);   // red[] and O^T are reused by the next item
+        }
+    } else {
+        // ---------------------------------------- query staging / key rotation (warps 6..9)
+        const int t128 = threadIdx.x - 192;           // 0..127
+        const int rk = t128 & 63;                     // key row of this thread
+        const int cp = t128 >> 6;                     // columns [32 cp, 32 cp + 32)
+        const int G = a.G;
+        // Relative rotation (REL): key row rk of every tile sits at angle rk*theta_i from
         // the tile start, so its (cos, sin) are fixed per thread; the tile start angle goes
-        // onto the query instead: q' = R(-key0 theta) q, and q' . R(row theta) k equals
-        // q . R((key0 + row) theta) k.
-        __half2 rcs[REL ? 64 : 1];
+        // onto the query instead: q' = R(-key0 theta) q, and q' . R(rk theta) k equals
+        // q . R((key0 + rk) theta) k.
+        __half2 rcs[REL ? 32 : 1];
         if constexpr (REL) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) {
+            for (int c = 0; c < 32; ++c) {
+                const int i = 32 * cp + c;
                 float sn = 0.f, cn = 1.f;
-                if (i < R) sincosf((float)row * sm.theta[i], &sn, &cn);
-                rcs[i] = __floats2half2_rn(cn, sn);
+                if (i < R) sincosf((float)rk * sm.theta[i], &sn, &cn);
+                rcs[c] = __floats2half2_rn(cn, sn);
             }
         }
-        uint32_t q = 0, tile = 0, item_n = 0;
+        uint32_t q = 0, gt = 0, item_n = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++item_n) {
             const Item w = item_of(a, it);
             const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
-            // stage the G queries of (b, g) as the B operand of S^T (K-major, swizzled)
-            for (int e = t128; e < kN * (D / 8); e += 128) {
-                const int h = e / (D / 8), c8 = e % (D / 8);
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (h < G)
-                    v = *reinterpret_cast<const uint4*>(
-                        a.q + ((size_t)w.b * a.Hq + (size_t)w.g * G + h) * D + c8 * 8);
-                *reinterpret_cast<uint4*>(sm.q[c8 / 8] + sw128_offset(h, (c8 % 8) * 8)) = v;
-            }
-            if constexpr (REL) {   // the rotated dims of q, to be turned per tile
-                for (int e = t128; e < NH * 2 * R; e += 128) {
-                    const int h = e / (2 * R), k = e % (2 * R);
-                    const int dim = k < R ? k : D / 2 + (k - R);
-                    float v = 0.f;
-                    if (h < G)
-                        v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                            a.q + ((size_t)w.b * a.Hq + (size_t)w.g * G + h) * D + dim));
-                    sm.qb[h][k < R ? k : 64 + (k - R)] = v;
-                }
-            }
-            fence_proxy_async_smem();
-            group_sync(kBarWG, 128);
-            if (t128 == 0) mbar_arrive(&sm.q_ready);
-
-            float m_run[NH], l_part[NH];
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                m_run[h] = -INFINITY;
-                l_part[h] = 0.f;
-            }
-            for (int t = 0; t < nt; ++t, ++tile) {
-                const int key0 = w.k0 + t * kTileKeys;
+            for (int t = 0; t < nt; ++t, ++gt) {
                 const uint32_t qk = q;
                 q += slots_per_tile;
-                // ---- turn the rotated pairs of this tile's keys (and, REL, the queries)
+                const int key0 = w.k0 + t * kTileKeys;
+                // before rewriting the B operands: the first tile of an item needs every
+                // score product of the previous item complete (it restages all of q), a
+                // later tile only the one that last read its side buffer and q copy (gt - 2)
+                if (t == 0 && item_n > 0) {
+                    ok = group_all(mbar_wait(&sm.q_free, (item_n - 1) & 1, wc, abort), kBarRot,
+                                   128);
+                } else if (t > 0 && R > 0 && gt > 1) {
+                    ok = group_all(mbar_wait(&sm.s_full[gt & 1], ((gt - 2) >> 1) & 1, wc, abort),
+                                   kBarRot, 128);
+                }
+                if (!ok) break;
+                if (t == 0) {
+                    // stage the G queries of (b, g) as the B operand of S^T: row n < NH is
+                    // head n over the slot's first-half dims, row NH + n the second half;
+                    // slot 0's operand goes to both of its copies
+                    const uint16_t* qg = a.q + ((size_t)w.b * a.Hq + (size_t)w.g * G) * D;
+                    for (int e = t128; e < NS * NSB * 8; e += 128) {
+                        const int n = e / (NSB * 8), sb = (e / 8) % NSB, c8 = e % 8;
+                        const int h = n % NH, half = n / NH;
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (h < G)
+                            v = *reinterpret_cast<const uint4*>(
+                                qg + (size_t)h * D + half * (D / 2) + sb * 64 + c8 * 8);
+                        *reinterpret_cast<uint4*>(sm.q[sb] + sw128_offset(n, c8 * 8)) = v;
+                        if (sb == 0) *reinterpret_cast<uint4*>(sm.q[4] + sw128_offset(n, c8 * 8)) = v;
+                    }
+                    if constexpr (REL) {   // the rotated dims of q, to be turned per tile
+                        for (int e = t128; e < NH * 128; e += 128) {
+                            const int h = e >> 7, k = e & 127, i = k & 63;
+                            float v = 0.f;
+                            if (h < G && i < R)
+                                v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                    qg + (size_t)h * D + (k < 64 ? i : D / 2 + i)));
+                            sm.qb[h][k] = v;
+                        }
+                    }
+                    fence_proxy_async_smem();
+                    group_sync(kBarRot, 128);
+                    if (t128 == 0) mbar_arrive(&sm.q_ready);
+                }
                 if (R > 0) {
                     // start angle of the tile: exact (fp64-reduced) at the first tile of an
-                    // item, then advanced by one tile (128 keys) per step
+                    // item, then advanced by one tile (64 keys) per step
                     for (int i = t128; i < R; i += 128) {
                         if (t == 0) {
                             sm.base_cs[i] = rope_cos_sin((long long)key0, i, D, a.rope.log2_base);
@@ -384,39 +559,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                     bool got = true;
-                    for (int k = 0; k < NPAIR && got; ++k)
-                        if (chunk_rotated(slot_chunk(k, 0, sep_v, NCH), D, R) ||
-                            chunk_rotated(slot_chunk(k, 1, sep_v, NCH), D, R))
-                            got = mbar_wait(&sm.full[(qk + k) % kNSlots],
-                                            ((qk + k) / kNSlots) & 1, wc, abort);
-                    ok = group_all(got, kBarWG, 128);   // also orders base_cs writes
+                    for (int sb = 0; sb < nrot && got; ++sb)
+                        got = mbar_wait(&sm.full[(qk + sb) % NSLOT], ((qk + sb) / NSLOT) & 1,
+                                        wc, abort);
+                    ok = group_all(got, kBarRot, 128);   // also orders base_cs writes
                     if (!ok) break;
                     if constexpr (REL) {
-                        // q' = R(-key0 theta) q on the rotated dims (chunks 0 and NCH/2)
-                        for (int e = t128; e < G * R; e += 128) {
-                            const int h = e / R, i = e % R;
-                            const float2 cs = sm.base_cs[i];
-                            const float x = sm.qb[h][i], y = sm.qb[h][64 + i];
-                            *reinterpret_cast<__nv_bfloat16*>(sm.q[0] + sw128_offset(h, i)) =
-                                __float2bfloat16_rn(x * cs.x + y * cs.y);
-                            *reinterpret_cast<__nv_bfloat16*>(sm.q[NCH / 2] + sw128_offset(h, i)) =
-                                __float2bfloat16_rn(y * cs.x - x * cs.y);
+                        // q' = R(-key0 theta) q on the rotated dims, into copy gt & 1 of slot
+                        // 0's operand (R <= 64: all rotated dims sit in slot 0)
+                        uint8_t* qd = sm.q[(gt & 1) ? 4 : 0];
+                        for (int e = t128; e < NH * 64; e += 128) {
+                            const int h = e >> 6, i = e & 63;
+                            if (h < G && i < R) {
+                                const float2 cs = sm.base_cs[i];
+                                const float x = sm.qb[h][i], y = sm.qb[h][64 + i];
+                                *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(h, i)) =
+                                    __float2bfloat16_rn(x * cs.x + y * cs.y);
+                                *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(NH + h, i)) =
+                                    __float2bfloat16_rn(y * cs.x - x * cs.y);
+                            }
                         }
-                        // keys: R(row theta) on the rotated pairs of this thread's row
-                        int k1, h1s, k2, h2s;
-                        chunk_slot(0, sep_v, NCH, k1, h1s);
-                        chunk_slot(NCH / 2, sep_v, NCH, k2, h2s);
-                        uint8_t* src1 = sm.ring[(qk + k1) % kNSlots] + h1s * kChunkBytes;
-                        uint8_t* src2 = sm.ring[(qk + k2) % kNSlots] + h2s * kChunkBytes;
-                        uint8_t* dst1 = side_rot ? sm.rot[0] : src1;
-                        uint8_t* dst2 = side_rot ? sm.rot[1] : src2;
+                        // keys: R(rk theta) on the rotated pairs of row rk (dims in row rk,
+                        // their partners in row 64 + rk of slot 0)
+                        uint8_t* src = sm.ring[qk % NSLOT];
+                        uint8_t* dst = side_rot ? sm.side[gt & 1] : src;
 #pragma unroll
-                        for (int g8 = 0; g8 < 8; ++g8) {
-                            const bool rotg = g8 * 8 < R;
+                        for (int g8 = 0; g8 < 4; ++g8) {
+                            const int col = 32 * cp + 8 * g8;
+                            const bool rotg = col < R;
                             if (!side_rot && !rotg) continue;   // in place: nothing to copy
-                            const uint32_t off = sw128_offset(row, g8 * 8);
-                            uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
-                            uint4 x2 = *reinterpret_cast<const uint4*>(src2 + off);
+                            const uint32_t o1 = sw128_offset(rk, col);
+                            const uint32_t o2 = sw128_offset(64 + rk, col);
+                            uint4 x1 = *reinterpret_cast<const uint4*>(src + o1);
+                            uint4 x2 = *reinterpret_cast<const uint4*>(src + o2);
                             if (rotg) {
                                 __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&x1);
                                 __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x2);
@@ -424,10 +599,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 for (int e2 = 0; e2 < 4; ++e2) {
                                     const float2 u = __bfloat1622float2(h1[e2]);
                                     const float2 v = __bfloat1622float2(h2[e2]);
-                                    const int i0 = g8 * 8 + 2 * e2;
-                                    const float2 ca = __half22float2(rcs[i0]);
-                                    const float2 cb = __half22float2(rcs[i0 + 1]);
-                                    const bool r0 = i0 < R, r1 = i0 + 1 < R;
+                                    const int c0 = 8 * g8 + 2 * e2;
+                                    const float2 ca = __half22float2(rcs[c0]);
+                                    const float2 cb = __half22float2(rcs[c0 + 1]);
+                                    const bool r0 = col + 2 * e2 < R, r1 = col + 2 * e2 + 1 < R;
                                     const float u0 = r0 ? u.x * ca.x - v.x * ca.y : u.x;
                                     const float v0 = r0 ? u.x * ca.y + v.x * ca.x : v.x;
                                     const float u1 = r1 ? u.y * cb.x - v.y * cb.y : u.y;
@@ -436,28 +611,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     h2[e2] = __floats2bfloat162_rn(v0, v1);
                                 }
                             }
-                            *reinterpret_cast<uint4*>(dst1 + off) = x1;
-                            *reinterpret_cast<uint4*>(dst2 + off) = x2;
+                            *reinterpret_cast<uint4*>(dst + o1) = x1;
+                            *reinterpret_cast<uint4*>(dst + o2) = x2;
                         }
                     } else {
-                        // absolute angles: angle(key0 + row) = angle(key0) + row * theta_i
-                        const float fr = (float)row;
-                        for (int c = 0; c < NCH / 2; ++c) {
-                            if (!chunk_rotated(c, D, R)) continue;
-                            const int c2i = c + NCH / 2;   // partner chunk: dims + d/2
-                            uint8_t* src1;
-                            uint8_t* src2;
-                            int k1, h1s, k2, h2s;
-                            chunk_slot(c, sep_v, NCH, k1, h1s);
-                            chunk_slot(c2i, sep_v, NCH, k2, h2s);
-                            src1 = sm.ring[(qk + k1) % kNSlots] + h1s * kChunkBytes;
-                            src2 = sm.ring[(qk + k2) % kNSlots] + h2s * kChunkBytes;
-                            uint8_t* dst1 = side_rot ? sm.rot[0] : src1;
-                            uint8_t* dst2 = side_rot ? sm.rot[1] : src2;
-                            for (int g8 = 0; g8 < 8; ++g8) {
-                                const uint32_t off = sw128_offset(row, g8 * 8);
-                                uint4 x1 = *reinterpret_cast<const uint4*>(src1 + off);
-                                uint4 x2 = *reinterpret_cast<const uint4*>(src2 + off);
+                        // absolute angles: angle(key0 + rk) = angle(key0) + rk * theta_i
+                        const float fr = (float)rk;
+                        for (int sb = 0; sb < nrot; ++sb) {
+                            uint8_t* src = sm.ring[(qk + sb) % NSLOT];
+                            uint8_t* dst = side_rot ? sm.side[gt & 1] : src;
+                            for (int g8 = 0; g8 < 4; ++g8) {
+                                const int col = 32 * cp + 8 * g8;
+                                const uint32_t o1 = sw128_offset(rk, col);
+                                const uint32_t o2 = sw128_offset(64 + rk, col);
+                                uint4 x1 = *reinterpret_cast<const uint4*>(src + o1);
+                                uint4 x2 = *reinterpret_cast<const uint4*>(src + o2);
                                 __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&x1);
                                 __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x2);
 #pragma unroll
@@ -467,7 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     float uo[2] = {u.x, u.y}, vo[2] = {v.x, v.y};
 #pragma unroll
                                     for (int e = 0; e < 2; ++e) {
-                                        const int i = c * 64 + g8 * 8 + e2 * 2 + e;
+                                        const int i = sb * 64 + col + e2 * 2 + e;
                                         if (i < R) {
                                             float x = fr * sm.theta[i];
                                             x = fmaf(-6.2831853f, rintf(x * 0.15915494f), x);
@@ -484,128 +652,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     h1[e2] = __floats2bfloat162_rn(uo[0], uo[1]);
                                     h2[e2] = __floats2bfloat162_rn(vo[0], vo[1]);
                                 }
-                                *reinterpret_cast<uint4*>(dst1 + off) = x1;
-                                *reinterpret_cast<uint4*>(dst2 + off) = x2;
+                                *reinterpret_cast<uint4*>(dst + o1) = x1;
+                                *reinterpret_cast<uint4*>(dst + o2) = x2;
                             }
                         }
                     }
                     fence_proxy_async_smem();
-                    group_sync(kBarWG, 128);
-                    if (t128 == 0) mbar_arrive(&sm.rot_ready);
+                    group_sync(kBarRot, 128);
+                    if (t128 == 0) mbar_arrive(&sm.rot_ready[gt & 1]);
                 }
-                // ---- softmax over the 128 keys of the tile (thread = key)
-                ok = group_all(mbar_wait(&sm.s_full, tile & 1, wc, abort), kBarWG, 128);
-                if (!ok) break;
-                tc_fence_after();
-                float s[kN];
-                tmem_ld16(tm_s + lane_off, s);
-                tmem_ld_wait();
-                const bool valid = key0 + row < w.k1;
-                float x[NH];
-                bool big = false;
-#pragma unroll
-                for (int h = 0; h < NH; ++h) {
-                    x[h] = (valid && h < G) ? s[h] * c2 : -INFINITY;
-                    big |= x[h] > m_run[h] + kLazyMax;
-                }
-                // lazy reference max: only when some score of the tile exceeds the running
-                // reference by more than 2^8 (and on the first tile) do the warps reduce
-                const bool fast = (t > 0) && group_all(!big, kBarWG, 128);
-                float alpha[NH];
-#pragma unroll
-                for (int h = 0; h < NH; ++h) alpha[h] = 1.f;
-                if (!fast) {
-                    float mt[NH];
-#pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        mt[h] = x[h];
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1)
-                            mt[h] = fmaxf(mt[h], __shfl_xor_sync(0xffffffffu, mt[h], o));
-                    }
-                    if (lane == 0)
-#pragma unroll
-                        for (int h = 0; h < NH; ++h) sm.red[quarter][h] = mt[h];
-                    group_sync(kBarWG, 128);
-                    bool rescale = false;
-#pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        const float tmax = fmaxf(fmaxf(sm.red[0][h], sm.red[1][h]),
-                                                 fmaxf(sm.red[2][h], sm.red[3][h]));
-                        if (tmax > m_run[h] + kLazyMax ||
-                            (m_run[h] == -INFINITY && tmax != -INFINITY)) {
-                            alpha[h] = (m_run[h] == -INFINITY) ? 0.f : exp2f(m_run[h] - tmax);
-                            m_run[h] = tmax;
-                            rescale |= t > 0;
-                        }
-                    }
-                    group_sync(kBarWG, 128);   // red[] is rewritten below
-                    // rescale O^T (thread = d-row, column = head).  O is idle: the MMA that
-                    // wrote S for this tile ran after the previous O update.
-                    if (rescale) {
-                        for (int pr = 0; pr < NPAIR; ++pr) {
-                            float o[kN];
-                            tmem_ld16(tm_o + pr * 16 + lane_off, o);
-                            tmem_ld_wait();
-#pragma unroll
-                            for (int h = 0; h < NH; ++h) o[h] *= alpha[h];
-                            tmem_st16(tm_o + pr * 16 + lane_off, o);
-                        }
-                        tmem_st_wait();
-                    }
-                }
-                // P^T: row = head, K-major, 64 keys per 128-byte row, two chunks
-                {
-                    uint8_t* pb = sm.p[row >> 6];
-                    const int kc = row & 63;
-#pragma unroll
-                    for (int h = 0; h < NH; ++h) {
-                        const float p = (x[h] == -INFINITY) ? 0.f : ex2_approx(x[h] - m_run[h]);
-                        const __nv_bfloat16 pr = __float2bfloat16_rn(p);
-                        // the running sum uses the rounded weight the MMA sees
-                        l_part[h] = l_part[h] * alpha[h] + __bfloat162float(pr);
-                        *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(h, kc)) = pr;
-                    }
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
-                group_sync(kBarWG, 128);
-                if (t128 == 0) mbar_arrive(&sm.p_full);
             }
-            if (!ok) break;
-            // ---- item epilogue: partial O^T, running max and sum
-            ok = group_all(mbar_wait(&sm.o_done, item_n & 1, wc, abort), kBarWG, 128);
-            if (!ok) break;
-            tc_fence_after();
-            const size_t obase = ((size_t)w.s * a.B + w.b) * a.Hq + (size_t)w.g * G;
-            for (int pr = 0; pr < NPAIR; ++pr) {
-                float o[kN];
-                tmem_ld16(tm_o + pr * 16 + lane_off, o);
-                tmem_ld_wait();
-#pragma unroll
-                for (int h = 0; h < NH; ++h)
-                    if (h < G) a.part_o[(obase + h) * D + pr * 128 + row] = nt > 0 ? o[h] : 0.f;
-            }
-#pragma unroll
-            for (int h = 0; h < NH; ++h)
-#pragma unroll
-                for (int o = 16; o > 0; o >>= 1)
-                    l_part[h] += __shfl_xor_sync(0xffffffffu, l_part[h], o);
-            if (lane == 0)
-#pragma unroll
-                for (int h = 0; h < NH; ++h) sm.red[quarter][h] = l_part[h];
-            group_sync(kBarWG, 128);
-            if (t128 < G) {
-                const float l = sm.red[0][t128] + sm.red[1][t128] + sm.red[2][t128] +
-                                sm.red[3][t128];
-                float mv = m_run[0];
-#pragma unroll
-                for (int h = 1; h < NH; ++h) mv = (t128 == h) ? m_run[h] : mv;
-                a.part_ml[(obase + t128) * 2 + 0] = mv;
-                a.part_ml[(obase + t128) * 2 + 1] = l;
-            }
-            tc_fence_before();
-            group_sync(kBarWG, 128);   // red[] and O^T are reused by the next item
         }
     }
 
@@ -644,7 +700,9 @@ __global__ void decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
 }
 
 template <int D, int NH, bool REL>
-cudaError_t run_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
+cudaError_t run_decode(const DecodeArgs& a, int grid, cudaStream_t stream) {
+    const size_t smem = sizeof(DecodeSmem<NH>) + 1024;
+    static_assert(sizeof(DecodeSmem<NH>) + 1024 <= 227 * 1024, "decode shared memory");
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NH, REL>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -653,18 +711,16 @@ cudaError_t run_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t 
 }
 
 template <int D>
-cudaError_t dispatch_decode(const DecodeArgs& a, int grid, size_t smem, cudaStream_t stream) {
+cudaError_t dispatch_decode(const DecodeArgs& a, int grid, cudaStream_t stream) {
     const bool rel = a.kv_is_k != 2 && a.rope.R <= 64;
     if (a.G <= 8)
-        return rel ? run_decode<D, 8, true>(a, grid, smem, stream)
-                   : run_decode<D, 8, false>(a, grid, smem, stream);
-    return rel ? run_decode<D, 16, true>(a, grid, smem, stream)
-               : run_decode<D, 16, false>(a, grid, smem, stream);
+        return rel ? run_decode<D, 8, true>(a, grid, stream)
+                   : run_decode<D, 8, false>(a, grid, stream);
+    return rel ? run_decode<D, 16, true>(a, grid, stream)
+               : run_decode<D, 16, false>(a, grid, stream);
 }
 
 }  // namespace
-
-size_t decode_smem_bytes() { return sizeof(DecodeSmem) + 1024; }
 
 // ------------------------------------------------------------------------------------
 // Fixed scratch for g4attn_decode_noalloc: the split partials live in this file-scope
@@ -700,15 +756,14 @@ cudaError_t decode_scratch_ptr(void** out) {
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-    const size_t smem = decode_smem_bytes();
     const int n_items = a.splits * a.Hkv * a.B;
     if (n_items > 0) {
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
         const int grid = n_items < sms ? n_items : sms;
-        cudaError_t e = a.d == 512 ? dispatch_decode<512>(a, grid, smem, stream)
-                        : a.d == 256 ? dispatch_decode<256>(a, grid, smem, stream)
+        cudaError_t e = a.d == 512 ? dispatch_decode<512>(a, grid, stream)
+                        : a.d == 256 ? dispatch_decode<256>(a, grid, stream)
                                      : cudaErrorInvalidValue;
         if (e != cudaSuccess) return e;
     }

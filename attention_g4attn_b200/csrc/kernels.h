@@ -36,7 +36,7 @@ cudaError_t launch_qknorm_rope(const QkNormRopeArgs& a, cudaStream_t stream);
 
 // Split-KV decode (one query per (b, h) at position L-1) and its combine pass.
 struct DecodeArgs {
-    CUtensorMap tm_k;       // kcache [B, L, Hkv, d] as a 4-D map (d, Hkv, L, B), box (64, 1, 128, 1)
+    CUtensorMap tm_k;       // kcache [B, L, Hkv, d] as a 4-D map (d, Hkv, L, B), box (64, 1, 64, 1)
     CUtensorMap tm_v;       // vcache, same geometry (kv_is_k == 0), else a copy of tm_k
     const uint16_t* q;      // [B, Hq, d], normalised and rotated
     float* part_o;          // [S, B, Hq, d]
@@ -45,7 +45,7 @@ struct DecodeArgs {
     float* lse;             // [B, Hq] or null
     int B, L, Hq, Hkv, d, G;
     int key_lo;             // first visible key (window), 0 for full attention
-    int splits, keys_per_split;  // multiples of 128
+    int splits, keys_per_split;  // multiples of 64
     Rope rope;
     float scale_log2;       // scale * log2(e)
     int kv_is_k;
@@ -54,7 +54,6 @@ struct DecodeArgs {
 };
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream);
-size_t decode_smem_bytes();
 // Fixed device scratch of g4attn_decode_noalloc (defined in decode.cu).
 size_t decode_scratch_bytes();
 cudaError_t decode_scratch_ptr(void** out);
