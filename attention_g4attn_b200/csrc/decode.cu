@@ -106,31 +106,40 @@ __device__ __forceinline__ Item item_of(const DecodeArgs& a, int it) {
     return r;
 }
 
+// Four K-steps of one slot (64 dims of S^T, or 64 keys of O^T): the matrix descriptors
+// advance by a fixed amount of their start-address field (16-byte units) per step.
+__device__ __forceinline__ void mma4(uint32_t d, uint64_t a, uint32_t a_step, uint64_t b,
+                                     uint32_t b_step, uint32_t idesc, uint32_t acc0) {
+    mma_bf16_ss(d, a, b, idesc, acc0);
+    mma_bf16_ss(d, a + a_step, b + b_step, idesc, 1u);
+    mma_bf16_ss(d, a + 2 * a_step, b + 2 * b_step, idesc, 1u);
+    mma_bf16_ss(d, a + 3 * a_step, b + 3 * b_step, idesc, 1u);
+}
+
+constexpr uint32_t kSlotDesc = kSlotBytes >> 4;   // one ring slot, in descriptor units
+
 // O^T += V^T . P^T for one tile: the value slots at ring position qv, P^T in p[j & 1].
-// Releases every slot once its MMAs finish, then signals pv_done.
+// Releases every slot once its MMAs finish, then signals pv_done.  d_ring_mn: descriptor
+// of ring slot 0 read MN-major (the second half's dims are the next 64-element MN block,
+// one TMA box further); d_p: descriptor of p[0].
 template <int D, int NH>
 __device__ __forceinline__ bool issue_pv(DecodeSmem<NH>& sm, uint32_t tm_o, uint32_t j,
-                                         uint32_t qv, bool first, bool sep_v,
-                                         const WaitCtl& wc, volatile int* abort) {
+                                         uint32_t qv, bool first, bool sep_v, uint64_t d_ring_mn,
+                                         uint64_t d_p, const WaitCtl& wc, volatile int* abort) {
     using C = DecodeCfg<NH>;
     constexpr int NSB = D / 128;
-    const uint32_t idesc_o = idesc_bf16_f32(128, kNO, true, false);  // A = V^T, MN-major
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, kNO, true, false);  // A = V^T, MN-major
     if (!mbar_wait(&sm.p_full[j & 1], (j >> 1) & 1, wc, abort)) return false;
     tc_fence_after();
-    const uint32_t pb = smem_u32(sm.p[j & 1]);
+    const uint64_t pb = d_p + (j & 1) * ((kNO * 128) >> 4);
+#pragma unroll
     for (int sb = 0; sb < NSB; ++sb) {
         const uint32_t k = qv + sb, slot = k % C::NSLOT;
         if (sep_v && !mbar_wait(&sm.full[slot], (k / C::NSLOT) & 1, wc, abort)) return false;
         tc_fence_after();
-        const uint32_t ab = smem_u32(sm.ring[slot]);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            // 16 keys per step = two 8-row groups of 1024 B; the second half's dims are the
-            // next 64-element MN block, one TMA box (8 KB) further
-            mma_bf16_ss(tm_o + sb * 16, sdesc_sw128(ab + kk * 2048, kBoxBytes, 1024),
-                        sdesc_sw128(pb + kk * 32, 16, 1024), idesc_o,
-                        (first && kk == 0) ? 0u : 1u);
-        }
+        // 16 keys per step = two 8-row groups of 1024 B
+        mma4(tm_o + sb * 16, d_ring_mn + slot * kSlotDesc, 2048 >> 4, pb, 32 >> 4, idesc_o,
+             first ? 0u : 1u);
         mma_commit(&sm.empty[slot]);
     }
     mma_commit(&sm.pv_done[j & 1]);
@@ -230,7 +239,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc_s = idesc_bf16_f32(128, NS, false, false);
+            constexpr uint32_t idesc_s = idesc_bf16_f32(128, NS, false, false);
+            constexpr uint32_t kQDesc = (NS * 128) >> 4;
+            const uint64_t d_ring_k = sdesc_sw128(smem_u32(sm.ring[0]), 16, 1024);
+            const uint64_t d_ring_mn = sdesc_sw128(smem_u32(sm.ring[0]), kBoxBytes, 1024);
+            const uint64_t d_side = sdesc_sw128(smem_u32(sm.side[0]), 16, 1024);
+            const uint64_t d_q = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+            const uint64_t d_p = sdesc_sw128(smem_u32(sm.p[0]), 16, 1024);
             uint32_t q = 0, gt = 0, item_n = 0;
             // the value product of a tile goes out as soon as its P is ready, between the
             // score MMAs of the next tile, which are issued slot by slot as the slots land
@@ -253,8 +268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     while (next_sb < NSB || !rot_done) {
                         if (pv_pending &&
                             mbar_test_wait(&sm.p_full[pv_tile & 1], (pv_tile >> 1) & 1)) {
-                            if (!issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v, wc,
-                                                 abort))
+                            if (!issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v,
+                                                 d_ring_mn, d_p, wc, abort))
                                 goto done;
                             pv_pending = false;
                             continue;
@@ -267,15 +282,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                   ((qk + next_sb) / NSLOT) & 1)) {
                             tc_fence_after();
                             const uint32_t slot = (qk + next_sb) % NSLOT;
-                            const uint32_t ab = smem_u32(sm.ring[slot]);
-                            const uint32_t bb = smem_u32(sm.q[next_sb]);
-#pragma unroll
-                            for (int kk = 0; kk < 4; ++kk) {
-                                mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
-                                            sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
-                                            first ? 0u : 1u);
-                                first = false;
-                            }
+                            mma4(tm_s, d_ring_k + slot * kSlotDesc, 32 >> 4,
+                                 d_q + next_sb * kQDesc, 32 >> 4, idesc_s, first ? 0u : 1u);
+                            first = false;
                             // score slots of a separate-value layer go back right away
                             if (sep_v) mma_commit(&sm.empty[slot]);
                             ++next_sb;
@@ -286,17 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                             tc_fence_after();
                             for (int sb = 0; sb < nrot; ++sb) {
                                 const uint32_t slot = (qk + sb) % NSLOT;
-                                const uint32_t ab = side_rot ? smem_u32(sm.side[gt & 1])
-                                                             : smem_u32(sm.ring[slot]);
-                                const uint32_t bb =
-                                    smem_u32(sm.q[(REL && sb == 0 && (gt & 1)) ? 4 : sb]);
-#pragma unroll
-                                for (int kk = 0; kk < 4; ++kk) {
-                                    mma_bf16_ss(tm_s, sdesc_sw128(ab + kk * 32, 16, 1024),
-                                                sdesc_sw128(bb + kk * 32, 16, 1024), idesc_s,
-                                                first ? 0u : 1u);
-                                    first = false;
-                                }
+                                const uint64_t ad = side_rot ? d_side + (gt & 1) * kSlotDesc
+                                                             : d_ring_k + slot * kSlotDesc;
+                                const uint64_t bd =
+                                    d_q + ((REL && sb == 0 && (gt & 1)) ? 4 : sb) * kQDesc;
+                                mma4(tm_s, ad, 32 >> 4, bd, 32 >> 4, idesc_s, first ? 0u : 1u);
+                                first = false;
                                 if (sep_v) mma_commit(&sm.empty[slot]);
                             }
                             rot_done = true;
@@ -313,8 +317,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     mma_commit(&sm.s_full[gt & 1]);
                     if (t == nt - 1) mma_commit(&sm.q_free);   // q may be restaged
-                    if (pv_pending &&
-                        !issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v, wc, abort))
+                    if (pv_pending && !issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v,
+                                                       d_ring_mn, d_p, wc, abort))
                         goto done;
                     pv_pending = true;
                     pv_tile = gt;
@@ -322,7 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     pv_first = t == 0;
                 }
             }
-            if (pv_pending) issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v, wc, abort);
+            if (pv_pending)
+                issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v, d_ring_mn, d_p, wc, abort);
         done:
             // all issued MMAs must finish before the tensor memory is released
             mma_commit(&sm.drain);
