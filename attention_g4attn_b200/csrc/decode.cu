@@ -20,14 +20,14 @@
 // the original stays as the value operand.
 //
 // Pipeline: one warpgroup turns the rotated pairs of tile t + 1 (and stages the queries)
-// while another runs the softmax of tile t, and the MMA warp issues S^T of tile t + 1
-// before O^T of tile t, so loads, rotation, scores, softmax and the value product of
-// neighbouring tiles overlap.  A 64-key tile holds 64 KB (d = 512), so the ring keeps
-// two and a half tiles.
+// while another runs the softmax of tile t; one thread issues the score MMAs as slots land
+// and another the value MMAs as P becomes ready, so loads, rotation, scores, softmax and
+// the value product of neighbouring tiles overlap.  A 64-key tile holds 64 KB (d = 512),
+// so the ring keeps two and a half tiles.
 //
-// Warp roles (320 threads): warp 0 TMA producer, warp 1 MMA issuer and TMEM owner,
+// Warp roles (352 threads): warp 0 TMA producer, warp 1 score-MMA issuer and TMEM owner,
 // warps 2..5 softmax / epilogue (thread = TMEM lane), warps 6..9 query staging and key
-// rotation.  The CTA is persistent over work items blockIdx.x, +gridDim.x, ...  Every
+// rotation, warp 10 value-MMA issuer.  The CTA is persistent over work items blockIdx.x, +gridDim.x, ...  Every
 // mbarrier wait is bounded (sm100.cuh); on a timeout all roles drain their in-flight work
 // and exit.
 #include <cuda_bf16.h>
@@ -42,7 +42,7 @@
 namespace g4 {
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 constexpr int kTileKeys = 64;
 constexpr int kSlotBytes = 16384;    // 128 rows x 128 B: 64 keys x 64 dims of each half
 constexpr int kBoxBytes = 8192;      // one TMA box: 64 keys x 64 dims
@@ -183,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.p_full[i], 1);
             mbar_init(&sm.pv_done[i], 1);
         }
-        mbar_init(&sm.drain, 1);
+        mbar_init(&sm.drain, 2);   // one commit from each MMA-issuing thread
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -237,99 +237,80 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
+        // ---------------------------------------------------- score-MMA issuer (warp 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = idesc_bf16_f32(128, NS, false, false);
             constexpr uint32_t kQDesc = (NS * 128) >> 4;
             const uint64_t d_ring_k = sdesc_sw128(smem_u32(sm.ring[0]), 16, 1024);
-            const uint64_t d_ring_mn = sdesc_sw128(smem_u32(sm.ring[0]), kBoxBytes, 1024);
             const uint64_t d_side = sdesc_sw128(smem_u32(sm.side[0]), 16, 1024);
             const uint64_t d_q = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
-            const uint64_t d_p = sdesc_sw128(smem_u32(sm.p[0]), 16, 1024);
             uint32_t q = 0, gt = 0, item_n = 0;
-            // the value product of a tile goes out as soon as its P is ready, between the
-            // score MMAs of the next tile, which are issued slot by slot as the slots land
-            bool pv_pending = false, pv_first = false;
-            uint32_t pv_tile = 0, pv_q = 0;
             for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++item_n) {
                 const Item w = item_of(a, it);
                 const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+                if (!mbar_wait(&sm.q_ready, item_n & 1, wc, abort)) goto s_done;
                 for (int t = 0; t < nt; ++t, ++gt) {
                     const uint32_t qk = q;
-                    const uint32_t qv = sep_v ? q + NSB : q;
                     q += slots_per_tile;
+                    // S^T buffer gt & 1 is free once the softmax of tile gt - 2 has read it
+                    if (gt >= 2 && !mbar_wait(&sm.p_full[gt & 1], ((gt - 2) >> 1) & 1, wc, abort))
+                        goto s_done;
                     const uint32_t tm_s = tmem + (gt & 1) * 32;
-                    bool first = true;
-                    bool q_ok = t > 0;               // the item's queries are staged
-                    int next_sb = nrot;              // next unrotated slot
-                    bool rot_done = nrot == 0;
-                    const unsigned long long t_start = global_ns();
-                    long long polls = 0;
-                    while (next_sb < NSB || !rot_done) {
-                        if (pv_pending &&
-                            mbar_test_wait(&sm.p_full[pv_tile & 1], (pv_tile >> 1) & 1)) {
-                            if (!issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v,
-                                                 d_ring_mn, d_p, wc, abort))
-                                goto done;
-                            pv_pending = false;
-                            continue;
-                        }
-                        if (!q_ok) {
-                            q_ok = mbar_test_wait(&sm.q_ready, item_n & 1);
-                            if (q_ok) continue;
-                        } else if (next_sb < NSB &&
-                                   mbar_test_wait(&sm.full[(qk + next_sb) % NSLOT],
-                                                  ((qk + next_sb) / NSLOT) & 1)) {
-                            tc_fence_after();
-                            const uint32_t slot = (qk + next_sb) % NSLOT;
-                            mma4(tm_s, d_ring_k + slot * kSlotDesc, 32 >> 4,
-                                 d_q + next_sb * kQDesc, 32 >> 4, idesc_s, first ? 0u : 1u);
-                            first = false;
-                            // score slots of a separate-value layer go back right away
+                    uint32_t acc = 0;
+                    // the slots that need no rotation, as they land; score slots of a
+                    // separate-value layer go back right after their MMAs
+                    for (int sb = nrot; sb < NSB; ++sb) {
+                        const uint32_t k = qk + sb, slot = k % NSLOT;
+                        if (!mbar_wait(&sm.full[slot], (k / NSLOT) & 1, wc, abort)) goto s_done;
+                        tc_fence_after();
+                        mma4(tm_s, d_ring_k + slot * kSlotDesc, 32 >> 4, d_q + sb * kQDesc, 32 >> 4,
+                             idesc_s, acc);
+                        acc = 1;
+                        if (sep_v) mma_commit(&sm.empty[slot]);
+                    }
+                    // then the rotated slots, once the rotation warps have turned them
+                    if (nrot > 0) {
+                        if (!mbar_wait(&sm.rot_ready[gt & 1], (gt >> 1) & 1, wc, abort))
+                            goto s_done;
+                        tc_fence_after();
+                        for (int sb = 0; sb < nrot; ++sb) {
+                            const uint32_t slot = (qk + sb) % NSLOT;
+                            const uint64_t ad = side_rot ? d_side + (gt & 1) * kSlotDesc
+                                                         : d_ring_k + slot * kSlotDesc;
+                            const uint64_t bd =
+                                d_q + ((REL && sb == 0 && (gt & 1)) ? 4 : sb) * kQDesc;
+                            mma4(tm_s, ad, 32 >> 4, bd, 32 >> 4, idesc_s, acc);
+                            acc = 1;
                             if (sep_v) mma_commit(&sm.empty[slot]);
-                            ++next_sb;
-                            continue;
-                        } else if (!rot_done &&
-                                   mbar_test_wait(&sm.rot_ready[gt & 1], (gt >> 1) & 1)) {
-                            // the rotated slots, once the rotation warps have turned them
-                            tc_fence_after();
-                            for (int sb = 0; sb < nrot; ++sb) {
-                                const uint32_t slot = (qk + sb) % NSLOT;
-                                const uint64_t ad = side_rot ? d_side + (gt & 1) * kSlotDesc
-                                                             : d_ring_k + slot * kSlotDesc;
-                                const uint64_t bd =
-                                    d_q + ((REL && sb == 0 && (gt & 1)) ? 4 : sb) * kQDesc;
-                                mma4(tm_s, ad, 32 >> 4, bd, 32 >> 4, idesc_s, first ? 0u : 1u);
-                                first = false;
-                                if (sep_v) mma_commit(&sm.empty[slot]);
-                            }
-                            rot_done = true;
-                            continue;
-                        }
-                        // nothing ready: bounded polling, like every other wait
-                        if (*abort) goto done;
-                        if ((++polls & 63) == 0 &&
-                            (polls >= a.wait_limit || global_ns() - t_start > kWaitTimeoutNs)) {
-                            atomicExch(a.status, (int)G4ATTN_ERR_TIMEOUT);
-                            *abort = 1;
-                            goto done;
                         }
                     }
                     mma_commit(&sm.s_full[gt & 1]);
                     if (t == nt - 1) mma_commit(&sm.q_free);   // q may be restaged
-                    if (pv_pending && !issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v,
-                                                       d_ring_mn, d_p, wc, abort))
-                        goto done;
-                    pv_pending = true;
-                    pv_tile = gt;
-                    pv_q = qv;
-                    pv_first = t == 0;
                 }
             }
-            if (pv_pending)
-                issue_pv<D, NH>(sm, tm_o, pv_tile, pv_q, pv_first, sep_v, d_ring_mn, d_p, wc, abort);
-        done:
+        s_done:
             // all issued MMAs must finish before the tensor memory is released
+            mma_commit(&sm.drain);
+            mbar_wait_drain(&sm.drain, 0, a.wait_limit);
+        }
+    } else if (warp == 10) {
+        // ---------------------------------------------------- value-MMA issuer (warp 10)
+        if (lane == 0) {
+            const uint64_t d_ring_mn = sdesc_sw128(smem_u32(sm.ring[0]), kBoxBytes, 1024);
+            const uint64_t d_p = sdesc_sw128(smem_u32(sm.p[0]), 16, 1024);
+            uint32_t q = 0, gt = 0;
+            for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+                const Item w = item_of(a, it);
+                const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+                for (int t = 0; t < nt; ++t, ++gt) {
+                    const uint32_t qv = sep_v ? q + NSB : q;
+                    q += slots_per_tile;
+                    if (!issue_pv<D, NH>(sm, tm_o, gt, qv, t == 0, sep_v, d_ring_mn, d_p, wc,
+                                         abort))
+                        goto v_done;
+                }
+            }
+        v_done:
             mma_commit(&sm.drain);
             mbar_wait_drain(&sm.drain, 0, a.wait_limit);
         }
