@@ -469,20 +469,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rk = t128 & 63;                     // key row of this thread
         const int cp = t128 >> 6;                     // columns [32 cp, 32 cp + 32)
         const int G = a.G;
+        constexpr int QV = NS * NSB * 8 / 128;        // 16-byte pieces of q staged per thread
+        constexpr int QH = NH / 2;                    // REL: heads cp, cp + 2, ... of pair rk
         // Relative rotation (REL): key row rk of every tile sits at angle rk*theta_i from
         // the tile start, so its (cos, sin) are fixed per thread; the tile start angle goes
         // onto the query instead: q' = R(-key0 theta) q, and q' . R(rk theta) k equals
-        // q . R((key0 + rk) theta) k.
-        __half2 rcs[REL ? 32 : 1];
+        // q . R((key0 + rk) theta) k.  rc / rs hold (cos, cos) / (sin, sin) of the column
+        // pairs (2m, 2m + 1) of this thread, as packed fp32 pairs.
+        float2 rc[REL ? 16 : 1], rs[REL ? 16 : 1];
+        float qx[REL ? QH : 1], qy[REL ? QH : 1];    // REL: pair rk of q, heads cp + 2j
+        float2 bcs = make_float2(1.f, 0.f);          // REL: cos/sin of key0 * theta_rk
+        float2 stp = make_float2(1.f, 0.f);          // REL: cos/sin of 64 * theta_rk
         if constexpr (REL) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const int i = 32 * cp + c;
-                float sn = 0.f, cn = 1.f;
-                if (i < R) sincosf((float)rk * sm.theta[i], &sn, &cn);
-                rcs[c] = __floats2half2_rn(cn, sn);
+            for (int m = 0; m < 16; ++m) {
+                const int i0 = 32 * cp + 2 * m;
+                float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
+                if (i0 < R) sincosf((float)rk * sm.theta[i0], &s0, &c0);
+                if (i0 + 1 < R) sincosf((float)rk * sm.theta[i0 + 1], &s1, &c1);
+                rc[m] = make_float2(c0, c1);
+                rs[m] = make_float2(s0, s1);
             }
+            if (rk < R) stp = sm.step_cs[rk];
         }
+        // the next item's queries and start angles, fetched one tile ahead of their use
+        uint4 qpre[QV];
+        float qxp[REL ? QH : 1], qyp[REL ? QH : 1];
+        float2 bpre[2];
+        auto prefetch = [&](int it2) {
+            const Item w2 = item_of(a, it2);
+            const uint16_t* qg = a.q + ((size_t)w2.b * a.Hq + (size_t)w2.g * G) * D;
+#pragma unroll
+            for (int j = 0; j < QV; ++j) {
+                const int e = t128 + 128 * j;
+                const int n = e / (NSB * 8), sb = (e / 8) % NSB, c8 = e % 8;
+                const int h = n % NH, half = n / NH;
+                qpre[j] = make_uint4(0, 0, 0, 0);
+                if (h < G)
+                    qpre[j] = *reinterpret_cast<const uint4*>(qg + (size_t)h * D + half * (D / 2) +
+                                                              sb * 64 + c8 * 8);
+            }
+            if constexpr (REL) {
+#pragma unroll
+                for (int j = 0; j < QH; ++j) {
+                    const int h = cp + 2 * j;
+                    const bool on = h < G && rk < R;
+                    qxp[j] = on ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                      qg + (size_t)h * D + rk))
+                                : 0.f;
+                    qyp[j] = on ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                                      qg + (size_t)h * D + D / 2 + rk))
+                                : 0.f;
+                }
+                bpre[0] = rk < R ? rope_cos_sin((long long)w2.k0, rk, D, a.rope.log2_base)
+                                 : make_float2(1.f, 0.f);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int i = t128 + 128 * j;
+                    bpre[j] = i < R ? rope_cos_sin((long long)w2.k0, i, D, a.rope.log2_base)
+                                    : make_float2(1.f, 0.f);
+                }
+            }
+        };
+        if (blockIdx.x < n_items) prefetch(blockIdx.x);
         uint32_t q = 0, gt = 0, item_n = 0;
         bool ok = true;
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++item_n) {
@@ -491,7 +541,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = 0; t < nt; ++t, ++gt) {
                 const uint32_t qk = q;
                 q += slots_per_tile;
-                const int key0 = w.k0 + t * kTileKeys;
                 // before rewriting the B operands: the first tile of an item needs every
                 // score product of the previous item complete (it restages all of q), a
                 // later tile only the one that last read its side buffer and q copy (gt - 2)
@@ -507,38 +556,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // stage the G queries of (b, g) as the B operand of S^T: row n < NH is
                     // head n over the slot's first-half dims, row NH + n the second half;
                     // slot 0's operand goes to both of its copies
-                    const uint16_t* qg = a.q + ((size_t)w.b * a.Hq + (size_t)w.g * G) * D;
-                    for (int e = t128; e < NS * NSB * 8; e += 128) {
+#pragma unroll
+                    for (int j = 0; j < QV; ++j) {
+                        const int e = t128 + 128 * j;
                         const int n = e / (NSB * 8), sb = (e / 8) % NSB, c8 = e % 8;
-                        const int h = n % NH, half = n / NH;
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (h < G)
-                            v = *reinterpret_cast<const uint4*>(
-                                qg + (size_t)h * D + half * (D / 2) + sb * 64 + c8 * 8);
-                        *reinterpret_cast<uint4*>(sm.q[sb] + sw128_offset(n, c8 * 8)) = v;
-                        if (sb == 0) *reinterpret_cast<uint4*>(sm.q[4] + sw128_offset(n, c8 * 8)) = v;
+                        *reinterpret_cast<uint4*>(sm.q[sb] + sw128_offset(n, c8 * 8)) = qpre[j];
+                        if (sb == 0)
+                            *reinterpret_cast<uint4*>(sm.q[4] + sw128_offset(n, c8 * 8)) = qpre[j];
                     }
-                    if constexpr (REL) {   // the rotated dims of q, to be turned per tile
-                        for (int e = t128; e < NH * 128; e += 128) {
-                            const int h = e >> 7, k = e & 127, i = k & 63;
-                            float v = 0.f;
-                            if (h < G && i < R)
-                                v = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                    qg + (size_t)h * D + (k < 64 ? i : D / 2 + i)));
-                            sm.qb[h][k] = v;
+                    if constexpr (REL) {
+#pragma unroll
+                        for (int j = 0; j < QH; ++j) {
+                            qx[j] = qxp[j];
+                            qy[j] = qyp[j];
                         }
+                        bcs = bpre[0];
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 2; ++j)
+                            if (t128 + 128 * j < R) sm.base_cs[t128 + 128 * j] = bpre[j];
                     }
                     fence_proxy_async_smem();
                     group_sync(kBarRot, 128);
                     if (t128 == 0) mbar_arrive(&sm.q_ready);
                 }
+                // fetch the next item's queries now: the loads fly during this tile's work
+                if (t == nt - 1 && it + (int)gridDim.x < n_items) prefetch(it + gridDim.x);
                 if (R > 0) {
                     // start angle of the tile: exact (fp64-reduced) at the first tile of an
                     // item, then advanced by one tile (64 keys) per step
-                    for (int i = t128; i < R; i += 128) {
-                        if (t == 0) {
-                            sm.base_cs[i] = rope_cos_sin((long long)key0, i, D, a.rope.log2_base);
-                        } else {
+                    if constexpr (REL) {
+                        if (t > 0)
+                            bcs = make_float2(bcs.x * stp.x - bcs.y * stp.y,
+                                              bcs.x * stp.y + bcs.y * stp.x);
+                    } else if (t > 0) {
+                        for (int i = t128; i < R; i += 128) {
                             const float2 b0 = sm.base_cs[i], st = sm.step_cs[i];
                             sm.base_cs[i] = make_float2(b0.x * st.x - b0.y * st.y,
                                                         b0.x * st.y + b0.y * st.x);
@@ -551,18 +603,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ok = group_all(got, kBarRot, 128);   // also orders base_cs writes
                     if (!ok) break;
                     if constexpr (REL) {
-                        // q' = R(-key0 theta) q on the rotated dims, into copy gt & 1 of slot
-                        // 0's operand (R <= 64: all rotated dims sit in slot 0)
+                        // q' = R(-key0 theta) q on pair rk, into copy gt & 1 of slot 0's
+                        // operand (R <= 64: all rotated dims sit in slot 0)
                         uint8_t* qd = sm.q[(gt & 1) ? 4 : 0];
-                        for (int e = t128; e < NH * 64; e += 128) {
-                            const int h = e >> 6, i = e & 63;
-                            if (h < G && i < R) {
-                                const float2 cs = sm.base_cs[i];
-                                const float x = sm.qb[h][i], y = sm.qb[h][64 + i];
-                                *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(h, i)) =
-                                    __float2bfloat16_rn(x * cs.x + y * cs.y);
-                                *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(NH + h, i)) =
-                                    __float2bfloat16_rn(y * cs.x - x * cs.y);
+                        if (rk < R) {
+#pragma unroll
+                            for (int j = 0; j < QH; ++j) {
+                                const int h = cp + 2 * j;
+                                if (h < G) {
+                                    *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(h, rk)) =
+                                        __float2bfloat16_rn(qx[j] * bcs.x + qy[j] * bcs.y);
+                                    *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(NH + h, rk)) =
+                                        __float2bfloat16_rn(qy[j] * bcs.x - qx[j] * bcs.y);
+                                }
                             }
                         }
                         // keys: R(rk theta) on the rotated pairs of row rk (dims in row rk,
@@ -579,22 +632,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                             uint4 x1 = *reinterpret_cast<const uint4*>(src + o1);
                             uint4 x2 = *reinterpret_cast<const uint4*>(src + o2);
                             if (rotg) {
-                                __nv_bfloat162* h1 = reinterpret_cast<__nv_bfloat162*>(&x1);
-                                __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&x2);
+                                // pairs whose cos/sin are (1, 0) turn into themselves, so the
+                                // columns at or past R need no special case
+                                uint32_t* w1 = &x1.x;
+                                uint32_t* w2 = &x2.x;
 #pragma unroll
-                                for (int e2 = 0; e2 < 4; ++e2) {
-                                    const float2 u = __bfloat1622float2(h1[e2]);
-                                    const float2 v = __bfloat1622float2(h2[e2]);
-                                    const int c0 = 8 * g8 + 2 * e2;
-                                    const float2 ca = __half22float2(rcs[c0]);
-                                    const float2 cb = __half22float2(rcs[c0 + 1]);
-                                    const bool r0 = col + 2 * e2 < R, r1 = col + 2 * e2 + 1 < R;
-                                    const float u0 = r0 ? u.x * ca.x - v.x * ca.y : u.x;
-                                    const float v0 = r0 ? u.x * ca.y + v.x * ca.x : v.x;
-                                    const float u1 = r1 ? u.y * cb.x - v.y * cb.y : u.y;
-                                    const float v1 = r1 ? u.y * cb.y + v.y * cb.x : v.y;
-                                    h1[e2] = __floats2bfloat162_rn(u0, u1);
-                                    h2[e2] = __floats2bfloat162_rn(v0, v1);
+                                for (int m = 0; m < 4; ++m) {
+                                    const float2 u = bf16x2_to_f2(w1[m]);
+                                    const float2 v = bf16x2_to_f2(w2[m]);
+                                    const float2 c = rc[4 * g8 + m], sn = rs[4 * g8 + m];
+                                    const float2 u2 = sub_f2(mul_f2(u, c), mul_f2(v, sn));
+                                    const float2 v2 = fma_f2(u, sn, mul_f2(v, c));
+                                    w1[m] = pack_bf16x2(u2.x, u2.y);
+                                    w2[m] = pack_bf16x2(v2.x, v2.y);
                                 }
                             }
                             *reinterpret_cast<uint4*>(dst + o1) = x1;

@@ -436,6 +436,34 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
     return row * 128u + chunk16 * 16u + (col & 7u) * 2u;
 }
 
+// Packed fp32 pairs (two lanes of one 64-bit register pair, each op rounds per lane).
+__device__ __forceinline__ unsigned long long f2_to_u64(float2 v) {
+    return ((unsigned long long)__float_as_uint(v.y) << 32) | __float_as_uint(v.x);
+}
+__device__ __forceinline__ float2 u64_to_f2(unsigned long long r) {
+    return make_float2(__uint_as_float((uint32_t)r), __uint_as_float((uint32_t)(r >> 32)));
+}
+__device__ __forceinline__ float2 mul_f2(float2 a, float2 b) {
+    unsigned long long r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_to_u64(a)), "l"(f2_to_u64(b)));
+    return u64_to_f2(r);
+}
+__device__ __forceinline__ float2 fma_f2(float2 a, float2 b, float2 c) {
+    unsigned long long r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(f2_to_u64(a)), "l"(f2_to_u64(b)),
+        "l"(f2_to_u64(c)));
+    return u64_to_f2(r);
+}
+__device__ __forceinline__ float2 sub_f2(float2 a, float2 b) {
+    unsigned long long r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(f2_to_u64(a)), "l"(f2_to_u64(b)));
+    return u64_to_f2(r);
+}
+// The two bf16 of a 32-bit word as fp32 (exact: bf16 is the top half of an fp32).
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
