@@ -148,7 +148,7 @@ PrefillWs prefill_ws(int B, int T, const g4attn_layer_cfg* c) {
     return w;
 }
 
-constexpr int kDecodeTile = 64;   // keys per decode tile: splits are whole tiles
+constexpr int kDecodeTile = 128;   // keys per decode pair-tile: splits are whole tiles
 
 struct DecodePlan {
     int key_lo, splits, keys_per_split;
@@ -162,11 +162,12 @@ DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms) {
     const int tiles = (len + kDecodeTile - 1) / kDecodeTile;
     const int nbg = B * c->n_kv_heads;
     int S = 1;
+    const int pairs = (sms > 1 ? sms : 148) / 2;   // the decode kernel runs on CTA pairs
     if (tiles > 0 && nbg > 0) {
-        // enough items that every SM holds the same number of them
-        int a = nbg, b = sms > 0 ? sms : 148;
+        // enough items that every pair holds the same number of them
+        int a = nbg, b = pairs;
         while (b) { int t = a % b; a = b; b = t; }
-        const int base = (sms > 0 ? sms : 148) / a;
+        const int base = pairs / a;
         S = base;
         while (S > tiles) S = (S + 1) / 2;
         if (S < 1) S = 1;
@@ -174,7 +175,8 @@ DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms) {
     const int tps = tiles > 0 ? (tiles + S - 1) / S : 1;
     p.keys_per_split = tps * kDecodeTile;
     p.splits = len > 0 ? (len + p.keys_per_split - 1) / p.keys_per_split : 0;
-    const size_t n = (size_t)(p.splits > 0 ? p.splits : 1) * B * c->n_q_heads;
+    // two partials per split: one from each CTA of the pair that runs it
+    const size_t n = 2 * (size_t)(p.splits > 0 ? p.splits : 1) * B * c->n_q_heads;
     p.o_off = 0;
     p.ml_off = align256(n * c->head_dim * sizeof(float));
     p.total = p.ml_off + align256(n * 2 * sizeof(float));
@@ -401,7 +403,8 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
 
 // Decode with no workspace argument and no allocation: the split partials go to the
 // library's fixed device scratch.  The split count is lowered until the partials fit; a
-// problem whose single-split partials (B * Hq * (d + 2) fp32) exceed the scratch is refused.
+// problem whose single-split partials (2 * B * Hq * (d + 2) fp32: one set per CTA of the
+// pair) exceed the scratch is refused.
 int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
                           const g4attn_bf16* vcache, int L, g4attn_bf16* out, float* lse, int B,
                           const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
@@ -425,7 +428,7 @@ int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
     DeviceInfo* dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
     const size_t cap = g4::decode_scratch_bytes();
-    const size_t per_split = (size_t)B * cfg->n_q_heads;
+    const size_t per_split = 2 * (size_t)B * cfg->n_q_heads;   // two partials per split
     if (align256(per_split * cfg->head_dim * sizeof(float)) + align256(per_split * 2 * sizeof(float)) >
         cap)
         return G4ATTN_ERR_TOO_LARGE;

@@ -3,33 +3,36 @@
 //
 // Work item = (split s, kv head g, batch b): keys [k0, k1) of one sequence and all G query
 // heads that share kv head g (GQA; explainer "GQA": 8 query heads per KV head in global
-// layers).  Keys stream through in tiles of 64.  A tile sits in shared memory as D/128
-// slots of 128 rows x 64 dims: in slot j, row r < 64 holds dims [64j, 64j + 64) of key r
-// and row 64 + r holds dims [d/2 + 64j, d/2 + 64j + 64) of the same key, so the two
-// halves of every key row are stacked on the MMA's M = 128 side:
-//   S^T[half*64 + key, n] = sum over the slot's 64 dims of K . Q^T   N = 2 NH
-// with columns n < NH holding the queries' first-half dims and n >= NH their second-half
-// dims; the two useful quarters (rows < 64 with n < NH, rows >= 64 with n >= NH) are the
-// two halves of the score and are added by the softmax threads.  The same slot, read
-// MN-major, is the value operand of
-//   O^T[dim, head] += V^T . P^T                                       M = 128 dims, N = 16
-// (keys reused as values, report section 2 / explainer "K=V": one cache read serves both).
-// RoPE pairs dims (i, i + d/2), i < R (report section 2, p-RoPE): both members of a pair
-// sit in the same slot, rows r and 64 + r, so the softmax warps turn a key's rotated
-// pairs inside one slot.  With pre-RoPE values the turned slot goes to a side buffer and
-// the original stays as the value operand.
+// layers).  Two CTAs of a cluster share an item and stream it in pair-tiles of 128 keys:
+// CTA r takes keys [64 r, 64 r + 64) of each pair-tile and keeps its own running softmax,
+// so each CTA's result is one partial of the split-KV combine.  A CTA's 64 keys sit in
+// shared memory as D/128 slots of 128 rows x 64 dims: in slot j, row k < 64 holds dims
+// [64j, 64j + 64) of key k and row 64 + k holds dims [d/2 + 64j, d/2 + 64j + 64) of the
+// same key, so the two halves of every key row are stacked on the MMA's M side.  One
+// 2-CTA MMA (cta_group::2, M = 256: 128 rows from each CTA) serves the pair:
+//   S^T[half*64 + key, n] = K . Q^T over the slot's 64 dims        N = 2 NH
+// where B rows n < NH (queries over the first-half dims) come from CTA 0 and rows n >= NH
+// (second-half dims) from CTA 1; the two useful quarters of each CTA's S^T (rows < 64 with
+// n < NH, rows >= 64 with n >= NH) are the two halves of its scores and are added by its
+// softmax threads.  The same slot, read MN-major, is the value operand of
+//   O^T[dim, n] += V^T . P^T                                        M = 128 dims per CTA
+// with B rows n < NH holding CTA 0's P and rows n >= NH CTA 1's P: columns [r NH, r NH + NH)
+// of CTA r's O^T are its own partial (keys reused as values, report section 2 / explainer
+// "K=V": one cache read serves both).  RoPE pairs dims (i, i + d/2), i < R (report
+// section 2, p-RoPE): both members of a pair sit in the same slot, rows k and 64 + k, so
+// the rotation warps turn a key's rotated pairs inside one slot.  With pre-RoPE values the
+// turned slot goes to a side buffer and the original stays as the value operand.
 //
-// Pipeline: one warpgroup turns the rotated pairs of tile t + 1 (and stages the queries)
-// while another runs the softmax of tile t; one thread issues the score MMAs as slots land
-// and another the value MMAs as P becomes ready, so loads, rotation, scores, softmax and
-// the value product of neighbouring tiles overlap.  A 64-key tile holds 64 KB (d = 512),
-// so the ring keeps two and a half tiles.
+// Pipeline: per CTA, a rotation warpgroup waits for a pair-tile's slots, stages the queries
+// of a new item and turns the rotated pairs, while a softmax warpgroup works on the tile
+// before; one thread of the first CTA issues every MMA of the pair (a single issuing thread
+// keeps the tensor pipe fed best), the value product of a tile as soon as both CTAs' P are
+// ready and the score product of the next tile once both CTAs have it turned.
 //
-// Warp roles (352 threads): warp 0 TMA producer, warp 1 score-MMA issuer and TMEM owner,
-// warps 2..5 softmax / epilogue (thread = TMEM lane), warps 6..9 query staging and key
-// rotation, warp 10 value-MMA issuer.  The CTA is persistent over work items blockIdx.x, +gridDim.x, ...  Every
-// mbarrier wait is bounded (sm100.cuh); on a timeout all roles drain their in-flight work
-// and exit.
+// Warp roles (320 threads per CTA): warp 0 TMA producer, warp 1 TMEM owner and (first CTA)
+// MMA issuer, warps 2..5 softmax / epilogue (thread = TMEM lane), warps 6..9 query staging
+// and key rotation.  Every mbarrier wait is bounded (sm100.cuh); on a timeout all roles
+// drain their in-flight work and exit.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -42,21 +45,21 @@
 namespace g4 {
 namespace {
 
-constexpr int kThreads = 352;
-constexpr int kTileKeys = 64;
+constexpr int kThreads = 320;
+constexpr int kTileKeys = 64;        // keys per CTA per pair-tile
+constexpr int kPairKeys = 128;       // keys per pair-tile
 constexpr int kSlotBytes = 16384;    // 128 rows x 128 B: 64 keys x 64 dims of each half
 constexpr int kBoxBytes = 8192;      // one TMA box: 64 keys x 64 dims
-constexpr int kNO = 16;              // N of the value product: query heads, zero padded
-constexpr uint32_t kTmemCols = 128;  // S^T double buffer (2 x 32) + O^T (4 x 16)
 constexpr int kBarSM = 1;            // named barrier of the softmax warpgroup
 constexpr int kBarRot = 2;           // named barrier of the rotation warpgroup
 constexpr float kLazyMax = 8.0f;     // log2 units: headroom of the lazy reference max
 
 template <int NH>
 struct DecodeCfg {
-    static constexpr int NS = 2 * NH;                // N of S^T
+    static constexpr int NS = 2 * NH;                // N of both MMAs (the pair's B rows)
     static constexpr int HH = NH / 2;                // heads finished by each half of the rows
-    static constexpr int NSLOT = NH == 8 ? 10 : 9;   // ring slots of 16 KB
+    static constexpr int NSLOT = NH == 8 ? 11 : 10;  // ring slots of 16 KB
+    static constexpr uint32_t TMEM_COLS = NH == 8 ? 128 : 256;   // 2 S^T + D/128 O^T blocks
 };
 
 template <int NH>
@@ -64,24 +67,26 @@ struct __align__(1024) DecodeSmem {
     using C = DecodeCfg<NH>;
     uint8_t ring[C::NSLOT][kSlotBytes];
     uint8_t side[2][kSlotBytes];       // turned slot 0 of tiles j & 1 (values = pre-RoPE keys)
-    // B operand of S^T per slot, K-major, swizzled; q[4] is the second copy of slot 0's
-    // operand, which the relative rotation rewrites for every tile (tile j uses copy j & 1)
-    uint8_t q[5][C::NS * 128];
-    uint8_t p[2][kNO * 128];           // B operand of O^T: P^T, K-major, 64 keys per row
+    // this CTA's half of the B operand of S^T per slot (NH rows: queries over the first
+    // half of d in CTA 0, the second half in CTA 1), K-major, swizzled; q[4] is the second
+    // copy of slot 0's operand, which the relative rotation rewrites per tile (tile j uses
+    // copy j & 1)
+    uint8_t q[5][NH * 128];
+    uint8_t p[2][NH * 128];            // this CTA's half of the B operand of O^T: its P^T
     float xs[2][64][C::HH];            // score halves handed to the other half's threads
     float theta[256];                  // base^(-2i/d) in fp32
     float2 base_cs[256];               // cos/sin of tile_start * theta_i
-    float2 step_cs[256];               // cos/sin of 64 * theta_i: one tile further
+    float2 step_cs[256];               // cos/sin of 128 * theta_i: one pair-tile further
     float red[4][C::HH];               // cross-warp reductions
     float alpha[NH];                   // rescale factors of O^T
     float mfin[NH];                    // running max per head at the end of an item
-    float qb[NH][128];                 // rotated dims of q (first and second half, R <= 64)
-    uint64_t full[C::NSLOT];
-    uint64_t empty[C::NSLOT];
+    uint64_t full[C::NSLOT];           // this CTA's loads landed
+    uint64_t empty[C::NSLOT];          // the pair's MMAs are done with the slot
     // per-tile barriers come in pairs (tile j uses [j & 1], phase (j >> 1) & 1): a waiter is
-    // never more than one phase of a barrier behind
+    // never more than one phase of a barrier behind.  rot_ready and p_full live in the first
+    // CTA and count one arrival from each CTA.
     uint64_t s_full[2], p_full[2], pv_done[2], rot_ready[2];
-    uint64_t q_ready, q_free, drain;   // once per item: q staged / all its scores done
+    uint64_t q_free, drain;            // once per item: all its scores done / teardown
     uint32_t tmem_base;
     int abort;
 };
@@ -92,7 +97,7 @@ struct Item {
     int s, g, b, k0, k1;
 };
 
-// Splits of one sequence are consecutive items, so concurrent CTAs stream neighbouring
+// Splits of one sequence are consecutive items, so concurrent pairs stream neighbouring
 // key ranges of the same (b, g).
 __device__ __forceinline__ Item item_of(const DecodeArgs& a, int it) {
     Item r;
@@ -106,50 +111,22 @@ __device__ __forceinline__ Item item_of(const DecodeArgs& a, int it) {
     return r;
 }
 
-// Four K-steps of one slot (64 dims of S^T, or 64 keys of O^T): the matrix descriptors
-// advance by a fixed amount of their start-address field (16-byte units) per step.
-__device__ __forceinline__ void mma4(uint32_t d, uint64_t a, uint32_t a_step, uint64_t b,
-                                     uint32_t b_step, uint32_t idesc, uint32_t acc0) {
-    mma_bf16_ss(d, a, b, idesc, acc0);
-    mma_bf16_ss(d, a + a_step, b + b_step, idesc, 1u);
-    mma_bf16_ss(d, a + 2 * a_step, b + 2 * b_step, idesc, 1u);
-    mma_bf16_ss(d, a + 3 * a_step, b + 3 * b_step, idesc, 1u);
+// Four K-steps of one slot (64 dims of S^T, or 64 keys of O^T) as pair MMAs: the matrix
+// descriptors advance by a fixed amount of their start-address field (16-byte units).
+__device__ __forceinline__ void mma4_pair(uint32_t d, uint64_t a, uint32_t a_step, uint64_t b,
+                                          uint32_t b_step, uint32_t idesc, uint32_t acc0) {
+    mma_pair_f16(d, a, b, idesc, acc0);
+    mma_pair_f16(d, a + a_step, b + b_step, idesc, 1u);
+    mma_pair_f16(d, a + 2 * a_step, b + 2 * b_step, idesc, 1u);
+    mma_pair_f16(d, a + 3 * a_step, b + 3 * b_step, idesc, 1u);
 }
 
 constexpr uint32_t kSlotDesc = kSlotBytes >> 4;   // one ring slot, in descriptor units
 
-// O^T += V^T . P^T for one tile: the value slots at ring position qv, P^T in p[j & 1].
-// Releases every slot once its MMAs finish, then signals pv_done.  d_ring_mn: descriptor
-// of ring slot 0 read MN-major (the second half's dims are the next 64-element MN block,
-// one TMA box further); d_p: descriptor of p[0].
-template <int D, int NH>
-__device__ __forceinline__ bool issue_pv(DecodeSmem<NH>& sm, uint32_t tm_o, uint32_t j,
-                                         uint32_t qv, bool first, bool sep_v, uint64_t d_ring_mn,
-                                         uint64_t d_p, const WaitCtl& wc, volatile int* abort) {
-    using C = DecodeCfg<NH>;
-    constexpr int NSB = D / 128;
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, kNO, true, false);  // A = V^T, MN-major
-    if (!mbar_wait(&sm.p_full[j & 1], (j >> 1) & 1, wc, abort)) return false;
-    tc_fence_after();
-    const uint64_t pb = d_p + (j & 1) * ((kNO * 128) >> 4);
-#pragma unroll
-    for (int sb = 0; sb < NSB; ++sb) {
-        const uint32_t k = qv + sb, slot = k % C::NSLOT;
-        if (sep_v && !mbar_wait(&sm.full[slot], (k / C::NSLOT) & 1, wc, abort)) return false;
-        tc_fence_after();
-        // 16 keys per step = two 8-row groups of 1024 B
-        mma4(tm_o + sb * 16, d_ring_mn + slot * kSlotDesc, 2048 >> 4, pb, 32 >> 4, idesc_o,
-             first ? 0u : 1u);
-        mma_commit(&sm.empty[slot]);
-    }
-    mma_commit(&sm.pv_done[j & 1]);
-    return true;
-}
-
 // D: head dim; NH: query heads per KV head handled by the softmax (8 or 16, >= G);
 // REL: relative rotation (values are not the rotated key and R <= 64).
 template <int D, int NH, bool REL>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a) {
     using C = DecodeCfg<NH>;
     constexpr int NSB = D / 128;    // slots per tile and tensor
@@ -166,6 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Turned slots go to the side buffer when the values are the pre-RoPE keys.
     const bool sep_v = a.kv_is_k == 0;
     const bool side_rot = a.kv_is_k == 1;
+    const uint32_t rank = cluster_rank();
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
     const int n_items = a.splits * a.Hkv * a.B;
     const int slots_per_tile = sep_v ? 2 * NSB : NSB;
 
@@ -174,34 +153,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], 1);
         }
-        mbar_init(&sm.q_ready, 1);
-        mbar_init(&sm.q_free, 1);
-        mbar_init(&sm.rot_ready[0], 1);
-        mbar_init(&sm.rot_ready[1], 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&sm.s_full[i], 1);
-            mbar_init(&sm.p_full[i], 1);
+            mbar_init(&sm.p_full[i], 2);
             mbar_init(&sm.pv_done[i], 1);
+            mbar_init(&sm.rot_ready[i], 2);
         }
-        mbar_init(&sm.drain, 2);   // one commit from each MMA-issuing thread
+        mbar_init(&sm.q_free, 1);
+        mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
-    if (warp == 1) tmem_alloc(&sm.tmem_base, kTmemCols);
-    if (warp >= 2) {
-        for (int i = threadIdx.x - 64; i < R; i += 256) {
+    if (warp == 1) tmem_alloc_pair(&sm.tmem_base, C::TMEM_COLS);
+    if (warp >= 2 && warp < 6) {
+        for (int i = threadIdx.x - 64; i < R; i += 128) {
             sm.theta[i] = (float)exp2(-(2.0 * (double)i / (double)D) * a.rope.log2_base);
-            sm.step_cs[i] = rope_cos_sin((long long)kTileKeys, i, D, a.rope.log2_base);
+            sm.step_cs[i] = rope_cos_sin((long long)kPairKeys, i, D, a.rope.log2_base);
         }
-        for (int i = threadIdx.x - 64; i < (int)(sizeof(sm.p) / 16); i += 256)
+        for (int i = threadIdx.x - 64; i < (int)(sizeof(sm.p) / 16); i += 128)
             reinterpret_cast<uint4*>(&sm.p[0][0])[i] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();   // barriers of both CTAs initialised before any remote arrival
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const uint32_t tm_o = tmem + 64;     // O^T: NSB blocks of 16 columns
+    const uint32_t tm_o = tmem + 64;     // O^T: NSB blocks of NS columns
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
@@ -209,11 +186,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&a.tm_k);
             if (sep_v) prefetch_tmap(&a.tm_v);
             uint32_t q = 0;   // ring slots filled so far
-            for (int it = blockIdx.x; it < n_items && !*abort; it += gridDim.x) {
+            for (int it = pair; it < n_items && !*abort; it += npairs) {
                 const Item w = item_of(a, it);
-                const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+                const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
                 for (int t = 0; t < nt && !*abort; ++t) {
-                    const int key = w.k0 + t * kTileKeys;
+                    const int key = w.k0 + t * kPairKeys + (int)rank * kTileKeys;
                     for (int pass = 0; pass < (sep_v ? 2 : 1) && !*abort; ++pass) {
                         const CUtensorMap* map = pass ? &a.tm_v : &a.tm_k;
                         for (int sb = 0; sb < NSB; ++sb) {
@@ -237,81 +214,102 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp == 1) {
-        // ---------------------------------------------------- score-MMA issuer (warp 1)
-        if (lane == 0) {
-            constexpr uint32_t idesc_s = idesc_bf16_f32(128, NS, false, false);
-            constexpr uint32_t kQDesc = (NS * 128) >> 4;
+        // ------------------------------------------------- MMA issuer (first CTA only)
+        if (lane == 0 && rank == 0) {
+            constexpr uint32_t idesc_s = idesc_bf16_f32(256, NS, false, false);
+            constexpr uint32_t idesc_o = idesc_bf16_f32(256, NS, true, false);  // A = V^T
+            constexpr uint32_t kQDesc = (NH * 128) >> 4;
+            constexpr uint32_t kPDesc = (NH * 128) >> 4;
             const uint64_t d_ring_k = sdesc_sw128(smem_u32(sm.ring[0]), 16, 1024);
+            const uint64_t d_ring_mn = sdesc_sw128(smem_u32(sm.ring[0]), kBoxBytes, 1024);
             const uint64_t d_side = sdesc_sw128(smem_u32(sm.side[0]), 16, 1024);
             const uint64_t d_q = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
-            uint32_t q = 0, gt = 0, item_n = 0;
-            for (int it = blockIdx.x; it < n_items; it += gridDim.x, ++item_n) {
-                const Item w = item_of(a, it);
-                const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
-                if (!mbar_wait(&sm.q_ready, item_n & 1, wc, abort)) goto s_done;
-                for (int t = 0; t < nt; ++t, ++gt) {
-                    const uint32_t qk = q;
-                    q += slots_per_tile;
-                    // S^T buffer gt & 1 is free once the softmax of tile gt - 2 has read it
-                    if (gt >= 2 && !mbar_wait(&sm.p_full[gt & 1], ((gt - 2) >> 1) & 1, wc, abort))
-                        goto s_done;
-                    const uint32_t tm_s = tmem + (gt & 1) * 32;
-                    uint32_t acc = 0;
-                    // the slots that need no rotation, as they land; score slots of a
-                    // separate-value layer go back right after their MMAs
-                    for (int sb = nrot; sb < NSB; ++sb) {
-                        const uint32_t k = qk + sb, slot = k % NSLOT;
-                        if (!mbar_wait(&sm.full[slot], (k / NSLOT) & 1, wc, abort)) goto s_done;
-                        tc_fence_after();
-                        mma4(tm_s, d_ring_k + slot * kSlotDesc, 32 >> 4, d_q + sb * kQDesc, 32 >> 4,
-                             idesc_s, acc);
-                        acc = 1;
-                        if (sep_v) mma_commit(&sm.empty[slot]);
-                    }
-                    // then the rotated slots, once the rotation warps have turned them
-                    if (nrot > 0) {
-                        if (!mbar_wait(&sm.rot_ready[gt & 1], (gt >> 1) & 1, wc, abort))
-                            goto s_done;
-                        tc_fence_after();
-                        for (int sb = 0; sb < nrot; ++sb) {
-                            const uint32_t slot = (qk + sb) % NSLOT;
-                            const uint64_t ad = side_rot ? d_side + (gt & 1) * kSlotDesc
-                                                         : d_ring_k + slot * kSlotDesc;
-                            const uint64_t bd =
-                                d_q + ((REL && sb == 0 && (gt & 1)) ? 4 : sb) * kQDesc;
-                            mma4(tm_s, ad, 32 >> 4, bd, 32 >> 4, idesc_s, acc);
-                            acc = 1;
-                            if (sep_v) mma_commit(&sm.empty[slot]);
-                        }
-                    }
-                    mma_commit(&sm.s_full[gt & 1]);
-                    if (t == nt - 1) mma_commit(&sm.q_free);   // q may be restaged
-                }
-            }
-        s_done:
-            // all issued MMAs must finish before the tensor memory is released
-            mma_commit(&sm.drain);
-            mbar_wait_drain(&sm.drain, 0, a.wait_limit);
-        }
-    } else if (warp == 10) {
-        // ---------------------------------------------------- value-MMA issuer (warp 10)
-        if (lane == 0) {
-            const uint64_t d_ring_mn = sdesc_sw128(smem_u32(sm.ring[0]), kBoxBytes, 1024);
             const uint64_t d_p = sdesc_sw128(smem_u32(sm.p[0]), 16, 1024);
-            uint32_t q = 0, gt = 0;
-            for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+            // cursors of the score product (sc) and the value product (pc): item, tile
+            // within it, global tile index and ring position
+            struct Cursor {
+                int it, t, nt;
+                uint32_t g, q;
+            };
+            auto tiles_of = [&](int it) {
+                if (it >= n_items) return 0;
                 const Item w = item_of(a, it);
-                const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
-                for (int t = 0; t < nt; ++t, ++gt) {
-                    const uint32_t qv = sep_v ? q + NSB : q;
-                    q += slots_per_tile;
-                    if (!issue_pv<D, NH>(sm, tm_o, gt, qv, t == 0, sep_v, d_ring_mn, d_p, wc,
-                                         abort))
-                        goto v_done;
+                return ceil_div(w.k1 - w.k0, kPairKeys);
+            };
+            auto advance = [&](Cursor& c) {
+                c.q += slots_per_tile;
+                ++c.g;
+                if (++c.t >= c.nt) {
+                    c.t = 0;
+                    c.it += npairs;
+                    c.nt = tiles_of(c.it);
+                }
+            };
+            Cursor sc{pair, 0, tiles_of(pair), 0u, 0u};
+            Cursor pc = sc;
+            unsigned long long t_idle = 0;
+            long long polls = 0;
+            while (pc.it < n_items) {
+                bool did = false;
+                if (pc.g < sc.g && mbar_test_wait_cluster(&sm.p_full[pc.g & 1], (pc.g >> 1) & 1)) {
+                    // O^T += V^T . P^T for tile pc.g: both CTAs' P are ready
+                    tc_fence_after();
+                    const uint64_t pb = d_p + (pc.g & 1) * kPDesc;
+                    const uint32_t qv = sep_v ? pc.q + NSB : pc.q;
+#pragma unroll
+                    for (int sb = 0; sb < NSB; ++sb) {
+                        const uint32_t slot = (qv + sb) % NSLOT;
+                        // 16 keys per step = two 8-row groups of 1024 B
+                        mma4_pair(tm_o + sb * NS, d_ring_mn + slot * kSlotDesc, 2048 >> 4, pb,
+                                  32 >> 4, idesc_o, pc.t == 0 ? 0u : 1u);
+                        mma_commit_pair(&sm.empty[slot]);
+                    }
+                    mma_commit_pair(&sm.pv_done[pc.g & 1]);
+                    advance(pc);
+                    did = true;
+                } else if (sc.it < n_items && sc.g < pc.g + 2 &&
+                           mbar_test_wait_cluster(&sm.rot_ready[sc.g & 1], (sc.g >> 1) & 1)) {
+                    // S^T for tile sc.g: both CTAs have its slots (turned) and, at the
+                    // start of an item, its queries; its S^T buffer was read by the softmax
+                    // of tile sc.g - 2, whose value product has been issued
+                    tc_fence_after();
+                    const uint32_t tm_s = tmem + (sc.g & 1) * 32;
+                    uint32_t acc = 0;
+#pragma unroll
+                    for (int sb = 0; sb < NSB; ++sb) {
+                        const uint32_t slot = (sc.q + sb) % NSLOT;
+                        const bool rot = sb < nrot;
+                        const uint64_t ad = (rot && side_rot) ? d_side + (sc.g & 1) * kSlotDesc
+                                                              : d_ring_k + slot * kSlotDesc;
+                        const uint64_t bd = d_q + ((REL && sb == 0 && (sc.g & 1)) ? 4 : sb) * kQDesc;
+                        mma4_pair(tm_s, ad, 32 >> 4, bd, 32 >> 4, idesc_s, acc);
+                        acc = 1;
+                        // score slots of a separate-value layer go back right away
+                        if (sep_v) mma_commit_pair(&sm.empty[slot]);
+                    }
+                    mma_commit_pair(&sm.s_full[sc.g & 1]);
+                    if (sc.t == sc.nt - 1) mma_commit_pair(&sm.q_free);   // q may be restaged
+                    advance(sc);
+                    did = true;
+                }
+                if (did) {
+                    polls = 0;
+                    continue;
+                }
+                // nothing ready: bounded polling, like every other wait
+                if (*abort) break;
+                if ((++polls & 63) == 0) {
+                    const unsigned long long now = global_ns();
+                    if (polls == 64) t_idle = now;
+                    if (polls >= a.wait_limit || now - t_idle > kWaitTimeoutNs) {
+                        atomicExch(a.status, (int)G4ATTN_ERR_TIMEOUT);
+                        *abort = 1;
+                        break;
+                    }
                 }
             }
-        v_done:
-            mma_commit(&sm.drain);
+            // all issued MMAs must finish before either CTA frees its tensor memory
+            mma_commit_pair(&sm.drain);
             mbar_wait_drain(&sm.drain, 0, a.wait_limit);
         }
     } else if (warp < 6) {
@@ -324,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int G = a.G;
         const float c2 = a.scale_log2;
+        const uint32_t ocol = rank * NH;              // this CTA's columns of O^T
         uint32_t gt = 0;
         bool ok = true;
         // the value product of tile j is complete (a no-op for j < 0)
@@ -331,9 +330,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool good = j < 0 || mbar_wait(&sm.pv_done[j & 1], (j >> 1) & 1, wc, abort);
             return group_all(good, kBarSM, 128);
         };
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        for (int it = pair; it < n_items && ok; it += npairs) {
             const Item w = item_of(a, it);
-            const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+            const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
             float m_run[HH], l_part[HH];
 #pragma unroll
             for (int j = 0; j < HH; ++j) {
@@ -345,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                128);
                 if (!ok) break;
                 tc_fence_after();
-                const int key0 = w.k0 + t * kTileKeys;
+                const int key0 = w.k0 + t * kPairKeys + (int)rank * kTileKeys;
                 float sp[NH];
                 if constexpr (NH == 8) tmem_ld8(tmem + (gt & 1) * 32 + hf * NH + lane_off, sp);
                 else tmem_ld16(tmem + (gt & 1) * 32 + hf * NH + lane_off, sp);
@@ -395,19 +394,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int j = 0; j < HH; ++j) sm.alpha[hf * HH + j] = alpha[j];
                     const bool rescale = !group_all(!resc, kBarSM, 128);  // also orders alpha
-                    // rescale O^T (thread = dim row, column = head) once the value product
-                    // of the tile before is complete; the next one waits for this tile's P
+                    // rescale this CTA's O^T columns (thread = dim row, column = head) once
+                    // the value product of the tile before is complete; the next one waits
+                    // for this tile's P
                     if (rescale) {
                         ok = wait_pv((int)gt - 1);
                         if (!ok) break;
                         tc_fence_after();
                         for (int sb = 0; sb < NSB; ++sb) {
-                            float o[kNO];
-                            tmem_ld16(tm_o + sb * 16 + lane_off, o);
+                            float o[NH];
+                            if constexpr (NH == 8) tmem_ld8(tm_o + sb * NS + ocol + lane_off, o);
+                            else tmem_ld16(tm_o + sb * NS + ocol + lane_off, o);
                             tmem_ld_wait();
 #pragma unroll
                             for (int h = 0; h < NH; ++h) o[h] *= sm.alpha[h];
-                            tmem_st16(tm_o + sb * 16 + lane_off, o);
+                            if constexpr (NH == 8) tmem_st8(tm_o + sb * NS + ocol + lane_off, o);
+                            else tmem_st16(tm_o + sb * NS + ocol + lane_off, o);
                         }
                         tmem_st_wait();
                     }
@@ -429,18 +431,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                 fence_proxy_async_smem();
                 tc_fence_before();
                 group_sync(kBarSM, 128);
-                if (t128 == 0) mbar_arrive(&sm.p_full[gt & 1]);
+                if (t128 == 0) {
+                    if (rank == 0) mbar_arrive(&sm.p_full[gt & 1]);
+                    else mbar_arrive_peer(&sm.p_full[gt & 1], 0);
+                }
             }
             if (!ok) break;
-            // ---- item epilogue: partial O^T, running max and sum
+            // ---- item epilogue: this CTA's partial O^T, running max and sum
             ok = wait_pv((int)gt - 1);
             if (!ok) break;
             tc_fence_after();
-            const size_t obase = ((size_t)w.s * a.B + w.b) * a.Hq + (size_t)w.g * G;
+            const size_t obase =
+                ((size_t)(2 * w.s + (int)rank) * a.B + w.b) * a.Hq + (size_t)w.g * G;
             const int dim0 = (row < 64) ? row : D / 2 + (row - 64);
             for (int sb = 0; sb < NSB; ++sb) {
-                float o[kNO];
-                tmem_ld16(tm_o + sb * 16 + lane_off, o);
+                float o[NH];
+                if constexpr (NH == 8) tmem_ld8(tm_o + sb * NS + ocol + lane_off, o);
+                else tmem_ld16(tm_o + sb * NS + ocol + lane_off, o);
                 tmem_ld_wait();
 #pragma unroll
                 for (int h = 0; h < NH; ++h)
@@ -469,24 +476,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rk = t128 & 63;                     // key row of this thread
         const int cp = t128 >> 6;                     // columns [32 cp, 32 cp + 32)
         const int G = a.G;
-        constexpr int QV = NS * NSB * 8 / 128;        // 16-byte pieces of q staged per thread
+        constexpr int QV = NH * NSB * 8 / 128;        // 16-byte pieces of q staged per thread
         constexpr int QH = NH / 2;                    // REL: heads cp, cp + 2, ... of pair rk
-        // Relative rotation (REL): key row rk of every tile sits at angle rk*theta_i from
-        // the tile start, so its (cos, sin) are fixed per thread; the tile start angle goes
-        // onto the query instead: q' = R(-key0 theta) q, and q' . R(rk theta) k equals
-        // q . R((key0 + rk) theta) k.  rc / rs hold (cos, cos) / (sin, sin) of the column
-        // pairs (2m, 2m + 1) of this thread, as packed fp32 pairs.
+        // Relative rotation (REL): key row rk of this CTA sits at angle (64 rank + rk) theta_i
+        // from the start of the pair-tile, so its (cos, sin) are fixed per thread; the start
+        // angle goes onto the query, which both CTAs' keys share in the pair MMA:
+        // q' = R(-key0 theta) q, and q' . R((64 rank + rk) theta) k equals
+        // q . R((key0 + 64 rank + rk) theta) k.  rc / rs hold (cos, cos) / (sin, sin) of the
+        // column pairs (2m, 2m + 1) of this thread, as packed fp32 pairs.
         float2 rc[REL ? 16 : 1], rs[REL ? 16 : 1];
         float qx[REL ? QH : 1], qy[REL ? QH : 1];    // REL: pair rk of q, heads cp + 2j
-        float2 bcs = make_float2(1.f, 0.f);          // REL: cos/sin of key0 * theta_rk
-        float2 stp = make_float2(1.f, 0.f);          // REL: cos/sin of 64 * theta_rk
+        float2 bcs = make_float2(1.f, 0.f);          // REL: cos/sin of pair start * theta_rk
+        float2 stp = make_float2(1.f, 0.f);          // REL: cos/sin of 128 * theta_rk
         if constexpr (REL) {
+            const float pos = (float)((int)rank * kTileKeys + rk);
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
                 const int i0 = 32 * cp + 2 * m;
                 float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
-                if (i0 < R) sincosf((float)rk * sm.theta[i0], &s0, &c0);
-                if (i0 + 1 < R) sincosf((float)rk * sm.theta[i0 + 1], &s1, &c1);
+                if (i0 < R) sincosf(pos * sm.theta[i0], &s0, &c0);
+                if (i0 + 1 < R) sincosf(pos * sm.theta[i0 + 1], &s1, &c1);
                 rc[m] = make_float2(c0, c1);
                 rs[m] = make_float2(s0, s1);
             }
@@ -498,16 +507,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         float2 bpre[2];
         auto prefetch = [&](int it2) {
             const Item w2 = item_of(a, it2);
+            const long long k0r = (long long)w2.k0 + (long long)rank * kTileKeys;
             const uint16_t* qg = a.q + ((size_t)w2.b * a.Hq + (size_t)w2.g * G) * D;
 #pragma unroll
             for (int j = 0; j < QV; ++j) {
+                // this CTA's B rows: head h over dims (rank * d/2 + 64 sb + [0, 64))
                 const int e = t128 + 128 * j;
-                const int n = e / (NSB * 8), sb = (e / 8) % NSB, c8 = e % 8;
-                const int h = n % NH, half = n / NH;
+                const int h = e / (NSB * 8), sb = (e / 8) % NSB, c8 = e % 8;
                 qpre[j] = make_uint4(0, 0, 0, 0);
                 if (h < G)
-                    qpre[j] = *reinterpret_cast<const uint4*>(qg + (size_t)h * D + half * (D / 2) +
-                                                              sb * 64 + c8 * 8);
+                    qpre[j] = *reinterpret_cast<const uint4*>(
+                        qg + (size_t)h * D + rank * (D / 2) + sb * 64 + c8 * 8);
             }
             if constexpr (REL) {
 #pragma unroll
@@ -521,23 +531,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       qg + (size_t)h * D + D / 2 + rk))
                                 : 0.f;
                 }
+                // q' turns by the start of the pair-tile (shared by both CTAs)
                 bpre[0] = rk < R ? rope_cos_sin((long long)w2.k0, rk, D, a.rope.log2_base)
                                  : make_float2(1.f, 0.f);
             } else {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int i = t128 + 128 * j;
-                    bpre[j] = i < R ? rope_cos_sin((long long)w2.k0, i, D, a.rope.log2_base)
+                    bpre[j] = i < R ? rope_cos_sin(k0r, i, D, a.rope.log2_base)
                                     : make_float2(1.f, 0.f);
                 }
             }
         };
-        if (blockIdx.x < n_items) prefetch(blockIdx.x);
+        if (pair < n_items) prefetch(pair);
         uint32_t q = 0, gt = 0, item_n = 0;
         bool ok = true;
-        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++item_n) {
+        for (int it = pair; it < n_items && ok; it += npairs, ++item_n) {
             const Item w = item_of(a, it);
-            const int nt = ceil_div(w.k1 - w.k0, kTileKeys);
+            const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
             for (int t = 0; t < nt; ++t, ++gt) {
                 const uint32_t qk = q;
                 q += slots_per_tile;
@@ -553,16 +564,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 if (t == 0) {
-                    // stage the G queries of (b, g) as the B operand of S^T: row n < NH is
-                    // head n over the slot's first-half dims, row NH + n the second half;
-                    // slot 0's operand goes to both of its copies
+                    // stage this CTA's half of the queries' B operand; slot 0's operand goes
+                    // to both of its copies
 #pragma unroll
                     for (int j = 0; j < QV; ++j) {
                         const int e = t128 + 128 * j;
-                        const int n = e / (NSB * 8), sb = (e / 8) % NSB, c8 = e % 8;
-                        *reinterpret_cast<uint4*>(sm.q[sb] + sw128_offset(n, c8 * 8)) = qpre[j];
+                        const int h = e / (NSB * 8), sb = (e / 8) % NSB, c8 = e % 8;
+                        *reinterpret_cast<uint4*>(sm.q[sb] + sw128_offset(h, c8 * 8)) = qpre[j];
                         if (sb == 0)
-                            *reinterpret_cast<uint4*>(sm.q[4] + sw128_offset(n, c8 * 8)) = qpre[j];
+                            *reinterpret_cast<uint4*>(sm.q[4] + sw128_offset(h, c8 * 8)) = qpre[j];
                     }
                     if constexpr (REL) {
 #pragma unroll
@@ -576,15 +586,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int j = 0; j < 2; ++j)
                             if (t128 + 128 * j < R) sm.base_cs[t128 + 128 * j] = bpre[j];
                     }
-                    fence_proxy_async_smem();
-                    group_sync(kBarRot, 128);
-                    if (t128 == 0) mbar_arrive(&sm.q_ready);
                 }
                 // fetch the next item's queries now: the loads fly during this tile's work
-                if (t == nt - 1 && it + (int)gridDim.x < n_items) prefetch(it + gridDim.x);
+                if (t == nt - 1 && it + npairs < n_items) prefetch(it + npairs);
+                // every slot of the tile has landed (the MMA issuer relies on this barrier)
+                bool got = true;
+                for (int k = 0; k < slots_per_tile && got; ++k)
+                    got = mbar_wait(&sm.full[(qk + k) % NSLOT], ((qk + k) / NSLOT) & 1, wc, abort);
                 if (R > 0) {
-                    // start angle of the tile: exact (fp64-reduced) at the first tile of an
-                    // item, then advanced by one tile (64 keys) per step
+                    // start angle of this CTA's tile: exact (fp64-reduced) at the first tile
+                    // of an item, then advanced by one pair-tile (128 keys) per step
                     if constexpr (REL) {
                         if (t > 0)
                             bcs = make_float2(bcs.x * stp.x - bcs.y * stp.y,
@@ -596,25 +607,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                         b0.x * st.y + b0.y * st.x);
                         }
                     }
-                    bool got = true;
-                    for (int sb = 0; sb < nrot && got; ++sb)
-                        got = mbar_wait(&sm.full[(qk + sb) % NSLOT], ((qk + sb) / NSLOT) & 1,
-                                        wc, abort);
-                    ok = group_all(got, kBarRot, 128);   // also orders base_cs writes
-                    if (!ok) break;
+                }
+                ok = group_all(got, kBarRot, 128);   // also orders base_cs writes
+                if (!ok) break;
+                if (R > 0) {
                     if constexpr (REL) {
-                        // q' = R(-key0 theta) q on pair rk, into copy gt & 1 of slot 0's
-                        // operand (R <= 64: all rotated dims sit in slot 0)
+                        // this CTA's half of q' = R(-key0 theta) q on pair rk, key0 the start
+                        // of the pair-tile (first-half dim in CTA 0, second-half dim in CTA 1),
+                        // into copy gt & 1 of slot 0's operand (R <= 64: all rotated dims sit
+                        // in slot 0)
                         uint8_t* qd = sm.q[(gt & 1) ? 4 : 0];
                         if (rk < R) {
 #pragma unroll
                             for (int j = 0; j < QH; ++j) {
                                 const int h = cp + 2 * j;
                                 if (h < G) {
+                                    const float v = rank == 0 ? qx[j] * bcs.x + qy[j] * bcs.y
+                                                              : qy[j] * bcs.x - qx[j] * bcs.y;
                                     *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(h, rk)) =
-                                        __float2bfloat16_rn(qx[j] * bcs.x + qy[j] * bcs.y);
-                                    *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(NH + h, rk)) =
-                                        __float2bfloat16_rn(qy[j] * bcs.x - qx[j] * bcs.y);
+                                        __float2bfloat16_rn(v);
                                 }
                             }
                         }
@@ -693,39 +704,47 @@ __global__ void __launch_bounds__(kThreads, 1)
                             }
                         }
                     }
-                    fence_proxy_async_smem();
-                    group_sync(kBarRot, 128);
-                    if (t128 == 0) mbar_arrive(&sm.rot_ready[gt & 1]);
+                }
+                // the tile's operands are in place: one arrival per CTA on the first CTA
+                fence_proxy_async_smem();
+                group_sync(kBarRot, 128);
+                if (t128 == 0) {
+                    if (rank == 0) mbar_arrive(&sm.rot_ready[gt & 1]);
+                    else mbar_arrive_peer(&sm.rot_ready[gt & 1], 0);
                 }
             }
         }
     }
 
     // -------------------------------------------------------------------- teardown
-    tc_fence_before();
     __syncthreads();
+    // the first CTA's MMAs read both CTAs' shared memory: neither leaves before they are
+    // done (the issuer waited for its drain commit above)
+    tc_fence_before();
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, kTmemCols);
+        tmem_dealloc_pair(tmem, C::TMEM_COLS);
     }
 }
 
-// Merge the split partials of one (b, h):
-//   out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,   M = max_s m_s (log2 units).
+// Merge the partials of one (b, h): two per split, one from each CTA of the pair,
+//   out = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p,   M = max_p m_p (log2 units).
 __global__ void decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
     const int bh = blockIdx.x;   // b * Hq + h
     const size_t stride = (size_t)a.B * a.Hq;
+    const int parts = 2 * a.splits;
     float M = -INFINITY;
-    for (int s = 0; s < a.splits; ++s) M = fmaxf(M, a.part_ml[(s * stride + bh) * 2]);
+    for (int s = 0; s < parts; ++s) M = fmaxf(M, a.part_ml[(s * stride + bh) * 2]);
     float den = 0.f;
-    for (int s = 0; s < a.splits; ++s) {
+    for (int s = 0; s < parts; ++s) {
         const float m = a.part_ml[(s * stride + bh) * 2];
         if (m != -INFINITY) den += exp2f(m - M) * a.part_ml[(s * stride + bh) * 2 + 1];
     }
     const float inv = den > 0.f ? 1.f / den : 0.f;
     for (int c = threadIdx.x; c < a.d; c += blockDim.x) {
         float acc = 0.f;
-        for (int s = 0; s < a.splits; ++s) {
+        for (int s = 0; s < parts; ++s) {
             const float m = a.part_ml[(s * stride + bh) * 2];
             if (m != -INFINITY) acc += exp2f(m - M) * a.part_o[(s * stride + bh) * a.d + c];
         }
@@ -797,7 +816,9 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         int dev = 0, sms = 148;
         cudaGetDevice(&dev);
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        const int grid = n_items < sms ? n_items : sms;
+        // CTA pairs: one cluster of two per work item in flight
+        const int pairs = n_items < sms / 2 ? n_items : sms / 2;
+        const int grid = 2 * (pairs > 0 ? pairs : 1);
         cudaError_t e = a.d == 512 ? dispatch_decode<512>(a, grid, stream)
                         : a.d == 256 ? dispatch_decode<256>(a, grid, stream)
                                      : cudaErrorInvalidValue;

@@ -39,13 +39,14 @@ struct DecodeArgs {
     CUtensorMap tm_k;       // kcache [B, L, Hkv, d] as a 4-D map (d, Hkv, L, B), box (64, 1, 64, 1)
     CUtensorMap tm_v;       // vcache, same geometry (kv_is_k == 0), else a copy of tm_k
     const uint16_t* q;      // [B, Hq, d], normalised and rotated
-    float* part_o;          // [S, B, Hq, d]
-    float* part_ml;         // [S, B, Hq, 2]  (running max in log2 units, sum)
+    float* part_o;          // [2S, B, Hq, d]
+    float* part_ml;         // [2S, B, Hq, 2]  (running max in log2 units, sum)
     uint16_t* out;          // [B, Hq, d]
     float* lse;             // [B, Hq] or null
     int B, L, Hq, Hkv, d, G;
     int key_lo;             // first visible key (window), 0 for full attention
-    int splits, keys_per_split;  // multiples of 64
+    int splits, keys_per_split;  // keys_per_split: a multiple of 128 (pair-tiles)
+    // part_o / part_ml hold two partials per split (one per CTA of the pair)
     Rope rope;
     float scale_log2;       // scale * log2(e)
     int kv_is_k;

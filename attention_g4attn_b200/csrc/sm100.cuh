@@ -81,6 +81,20 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Non-blocking test with cluster-scope acquire: for barriers the other CTA of a pair
+// arrives on (its shared-memory writes become visible with the phase).
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -275,6 +289,18 @@ __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank)
                  : "memory");
 }
 
+// Arrive on the mbarrier at this offset in CTA `rank` of the cluster with CTA-scope release
+// ordering.  A cluster-scope release costs a fence of several hundred cycles per signal (more
+// under load); the per-tile hand-off from the second CTA of a pair uses this form, which is
+// how cluster pipelines signal a peer CTA's barrier: the arriving thread's shared-memory
+// writes (made visible to the tensor core by fence.proxy.async first) reach the peer in
+// order ahead of the arrival.
+__device__ __forceinline__ void mbar_arrive_peer(uint64_t* bar, uint32_t rank) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(
+                     mapa_shared(bar, rank))
+                 : "memory");
+}
+
 __device__ __forceinline__ void st_shared_remote_u32(const void* p, uint32_t rank, uint32_t v) {
     asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(mapa_shared(p, rank)), "r"(v)
                  : "memory");
@@ -422,6 +448,16 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
         "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
         "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
         "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+
+// registers -> TMEM: 32 lanes x 32 bit, 8 consecutive columns per thread.
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float* v) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+        "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7]))
         : "memory");
 }
 

@@ -148,7 +148,8 @@ G4ATTN_API int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, co
  * array inside the library, which every device that loads the library holds until the
  * process exits.  The call allocates nothing.
  *   - The split count is lowered until the partials fit; if even one split needs more
- *     than 8 MiB (B * Hq * (head_dim + 2) * 4 bytes > 8 MiB), the call returns
+ *     than 8 MiB (2 * B * Hq * (head_dim + 2) * 4 bytes > 8 MiB: the kernel keeps two
+ *     partials per split), the call returns
  *     G4ATTN_ERR_TOO_LARGE and launches nothing.
  *   - The first call on a device looks up the array's device address (once per device,
  *     with that device current); make that first call before any stream capture.
