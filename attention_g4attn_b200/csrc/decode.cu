@@ -730,28 +730,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
 // Merge the partials of one (b, h): two per split, one from each CTA of the pair,
 //   out = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p,   M = max_p m_p (log2 units).
-__global__ void decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
+// Block (b h, 128-dim chunk), thread = one dim: the per-part weights are computed once per
+// block into shared memory, then every thread streams its dim of all the partials.
+constexpr int kCombineThreads = 128;
+constexpr int kMaxParts = 1024;
+
+__global__ void __launch_bounds__(kCombineThreads)
+    decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
+    __shared__ float wgt[kMaxParts];
+    __shared__ float red[kCombineThreads / 32];
+    __shared__ float bM, bDen;
     const int bh = blockIdx.x;   // b * Hq + h
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
     const size_t stride = (size_t)a.B * a.Hq;
     const int parts = 2 * a.splits;
-    float M = -INFINITY;
-    for (int s = 0; s < parts; ++s) M = fmaxf(M, a.part_ml[(s * stride + bh) * 2]);
-    float den = 0.f;
-    for (int s = 0; s < parts; ++s) {
+    // running maxima of the parts, and their largest
+    float mx = -INFINITY;
+    for (int s = tid; s < parts; s += kCombineThreads) {
         const float m = a.part_ml[(s * stride + bh) * 2];
-        if (m != -INFINITY) den += exp2f(m - M) * a.part_ml[(s * stride + bh) * 2 + 1];
+        wgt[s] = m;
+        mx = fmaxf(mx, m);
     }
-    const float inv = den > 0.f ? 1.f / den : 0.f;
-    for (int c = threadIdx.x; c < a.d; c += blockDim.x) {
-        float acc = 0.f;
-        for (int s = 0; s < parts; ++s) {
-            const float m = a.part_ml[(s * stride + bh) * 2];
-            if (m != -INFINITY) acc += exp2f(m - M) * a.part_o[(s * stride + bh) * a.d + c];
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    if (lane == 0) red[wp] = mx;
+    __syncthreads();
+    if (tid == 0) {
+        float M = red[0];
+        for (int i = 1; i < kCombineThreads / 32; ++i) M = fmaxf(M, red[i]);
+        bM = M;
+    }
+    __syncthreads();
+    const float M = bM;
+    // weights 2^(m_p - M) and their sum with the running sums
+    float den = 0.f;
+    for (int s = tid; s < parts; s += kCombineThreads) {
+        const float m = wgt[s];
+        const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
+        wgt[s] = w;
+        den += w * a.part_ml[(s * stride + bh) * 2 + 1];
+    }
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    __syncthreads();   // red[] reuse
+    if (lane == 0) red[wp] = den;
+    __syncthreads();
+    if (tid == 0) {
+        float t = 0.f;
+        for (int i = 0; i < kCombineThreads / 32; ++i) t += red[i];
+        bDen = t;
+    }
+    __syncthreads();
+    const float dsum = bDen;
+    const float inv = dsum > 0.f ? 1.f / dsum : 0.f;
+    const int c = blockIdx.y * kCombineThreads + tid;
+    if (c < a.d) {
+        const float* po = a.part_o + (size_t)bh * a.d + c;
+        const size_t ps = stride * a.d;
+        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+        int s = 0;
+        for (; s + 4 <= parts; s += 4) {
+            acc0 += wgt[s] * po[s * ps];
+            acc1 += wgt[s + 1] * po[(s + 1) * ps];
+            acc2 += wgt[s + 2] * po[(s + 2) * ps];
+            acc3 += wgt[s + 3] * po[(s + 3) * ps];
         }
+        for (; s < parts; ++s) acc0 += wgt[s] * po[s * ps];
+        const float acc = (acc0 + acc1) + (acc2 + acc3);
         a.out[(size_t)bh * a.d + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc * inv));
     }
-    if (threadIdx.x == 0 && a.lse)
-        a.lse[bh] = den > 0.f ? (M + log2f(den)) * 0.6931471805599453f : -INFINITY;
+    if (tid == 0 && blockIdx.y == 0 && a.lse)
+        a.lse[bh] = dsum > 0.f ? (M + log2f(dsum)) * 0.6931471805599453f : -INFINITY;
 }
 
 template <int D, int NH, bool REL>
@@ -824,7 +871,11 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
                                      : cudaErrorInvalidValue;
         if (e != cudaSuccess) return e;
     }
-    if (a.B * a.Hq > 0) decode_combine_kernel<<<a.B * a.Hq, 128, 0, stream>>>(a);
+    if (2 * a.splits > kMaxParts) return cudaErrorInvalidValue;
+    if (a.B * a.Hq > 0) {
+        const dim3 grid(a.B * a.Hq, (a.d + kCombineThreads - 1) / kCombineThreads);
+        decode_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(a);
+    }
     return cudaGetLastError();
 }
 

@@ -270,6 +270,7 @@ CASES = {
     "global_prefill_T65536": ("prefill", dict(B=1, T=65536, layer="GLOBAL_8TO1")),
     "local_prefill_T16384": ("prefill", dict(B=1, T=16384, layer="LOCAL_W1024")),
     "global_decode_L8192": ("decode", dict(B=16, L=8192, layer="GLOBAL_8TO1")),
+    "global_decode_L32768": ("decode", dict(B=16, L=32768, layer="GLOBAL_8TO1")),
 }
 
 
