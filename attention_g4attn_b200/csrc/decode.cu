@@ -433,7 +433,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 group_sync(kBarSM, 128);
                 if (t128 == 0) {
                     if (rank == 0) mbar_arrive(&sm.p_full[gt & 1]);
-                    else mbar_arrive_peer(&sm.p_full[gt & 1], 0);
+                    else mbar_arrive_remote(&sm.p_full[gt & 1], 0);
                 }
             }
             if (!ok) break;
@@ -710,7 +710,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 group_sync(kBarRot, 128);
                 if (t128 == 0) {
                     if (rank == 0) mbar_arrive(&sm.rot_ready[gt & 1]);
-                    else mbar_arrive_peer(&sm.rot_ready[gt & 1], 0);
+                    else mbar_arrive_remote(&sm.rot_ready[gt & 1], 0);
                 }
             }
         }

@@ -49,8 +49,11 @@ template <int D>
 struct PrefillCfg {
     static constexpr int NCH = D / 64;
     static constexpr bool SWAP = (D == 512);
-    static constexpr int NSLOT = (D == 512) ? 4 : 8;
+    static constexpr int NSLOT = (D == 512) ? 4 : 6;
     static constexpr uint32_t S_COL = (D == 512) ? 128 : 256;
+    // head_dim 256: two S buffers (columns 256 and 384) and two P buffers, so the scores of
+    // tile n + 1 are computed while the softmax works on tile n
+    static constexpr int NBUF = (D == 512) ? 1 : 2;
     static constexpr int NS = D / 128;     // S stages per tile (128 dims each)
     static constexpr int NV = D / 256;     // P.V blocks per tile (2 slots each)
 };
@@ -58,11 +61,13 @@ struct PrefillCfg {
 template <int D>
 struct __align__(1024) PrefillSmem {
     uint8_t q[PrefillCfg<D>::NCH][16384];  // 128 rows x 64 dims per chunk
-    uint8_t p[2][16384];                   // P: 128 rows x 64 keys per chunk
+    uint8_t p[PrefillCfg<D>::NBUF][2][16384];   // P: 128 rows x 64 keys per chunk
     uint8_t ring[PrefillCfg<D>::NSLOT][kSlot];
     uint64_t full[PrefillCfg<D>::NSLOT];   // used in the leader: both CTAs' bytes land here
     uint64_t empty[PrefillCfg<D>::NSLOT];  // per CTA, released by the leader's MMA commits
-    uint64_t s_free, s_full, p_full, o_done, drain;
+    // per buffer (tile n uses [n % NBUF]); s_free / p_full / q_ready count one arrival per CTA
+    uint64_t s_free[2], s_full[2], p_full[2], pv_done[2];
+    uint64_t q_ready, o_done, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -124,9 +129,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.full[i], 1);
             mbar_init(&sm.empty[i], 1);
         }
-        mbar_init(&sm.s_free, 2);   // one arrival per CTA of the pair
-        mbar_init(&sm.s_full, 1);
-        mbar_init(&sm.p_full, 2);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&sm.s_free[i], 2);   // one arrival per CTA of the pair
+            mbar_init(&sm.s_full[i], 1);
+            mbar_init(&sm.p_full[i], 2);
+            mbar_init(&sm.pv_done[i], 1);
+        }
+        mbar_init(&sm.q_ready, 2);
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
@@ -138,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const uint32_t tm_o = tmem;
-    const uint32_t tm_s = tmem + C::S_COL;
+    const uint32_t tm_s = tmem + C::S_COL;   // S buffer b at tm_s + 128 b
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -188,45 +197,102 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && leader) {
             const uint32_t idesc_s = idesc_f16kind_f32(256, kBN, false, false, false);
             const uint32_t idesc_o = idesc_f16kind_f32(256, 256, false, true, !PF16);
-            uint32_t q = 0;
-            for (int n = 0; n < ntiles; ++n) {
-                if (!mbar_wait_cluster(&sm.s_free, n & 1, wc, abort)) goto done;
-                tc_fence_after();
-                for (int s = 0; s < C::NS; ++s, ++q) {
-                    const uint32_t slot = q % NSLOT;
-                    if (!mbar_wait_cluster(&sm.full[slot], (q / NSLOT) & 1, wc, abort)) goto done;
+            if constexpr (C::SWAP) {
+                uint32_t q = 0;
+                for (int n = 0; n < ntiles; ++n) {
+                    if (!mbar_wait_cluster(&sm.s_free[0], n & 1, wc, abort)) goto done;
                     tc_fence_after();
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t ab = smem_u32(sm.q[2 * s + (kk >> 2)]) + (kk & 3) * 32;
-                        const uint32_t bb =
-                            smem_u32(sm.ring[slot]) + (kk >> 2) * (kSlot / 2) + (kk & 3) * 32;
-                        mma_pair_f16(tm_s, sdesc_sw128(ab, 16, 1024), sdesc_sw128(bb, 16, 1024),
-                                     idesc_s, (s | kk) != 0 ? 1u : 0u);
+                    for (int s = 0; s < C::NS; ++s, ++q) {
+                        const uint32_t slot = q % NSLOT;
+                        if (!mbar_wait_cluster(&sm.full[slot], (q / NSLOT) & 1, wc, abort)) goto done;
+                        tc_fence_after();
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t ab = smem_u32(sm.q[2 * s + (kk >> 2)]) + (kk & 3) * 32;
+                            const uint32_t bb =
+                                smem_u32(sm.ring[slot]) + (kk >> 2) * (kSlot / 2) + (kk & 3) * 32;
+                            mma_pair_f16(tm_s, sdesc_sw128(ab, 16, 1024), sdesc_sw128(bb, 16, 1024),
+                                         idesc_s, (s | kk) != 0 ? 1u : 0u);
+                        }
+                        mma_commit_pair(&sm.empty[slot]);
                     }
-                    mma_commit_pair(&sm.empty[slot]);
-                }
-                mma_commit_pair(&sm.s_full);
-                if (!mbar_wait_cluster(&sm.p_full, n & 1, wc, abort)) goto done;
-                tc_fence_after();
-                for (int v = 0; v < C::NV; ++v, q += 2) {
-                    const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
-                    if (!mbar_wait_cluster(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
-                    if (!mbar_wait_cluster(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
-                        goto done;
+                    mma_commit_pair(&sm.s_full[0]);
+                    if (!mbar_wait_cluster(&sm.p_full[0], n & 1, wc, abort)) goto done;
                     tc_fence_after();
-                    const uint32_t vb = smem_u32(sm.ring[s0]);
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint32_t pa = smem_u32(sm.p[kk >> 2]) + (kk & 3) * 32;
-                        // V: 16 keys per step (two 8-row groups of 1024 B); the CTA's second
-                        // 64-dim chunk sits in the next slot (LBO)
-                        mma_pair_f16(tm_o + v * 256, sdesc_sw128(pa, 16, 1024),
-                                     sdesc_sw128(vb + kk * 2048, kSlot, 1024), idesc_o,
-                                     (n > 0 || kk > 0) ? 1u : 0u);
+                    for (int v = 0; v < C::NV; ++v, q += 2) {
+                        const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
+                        if (!mbar_wait_cluster(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
+                        if (!mbar_wait_cluster(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
+                            goto done;
+                        tc_fence_after();
+                        const uint32_t vb = smem_u32(sm.ring[s0]);
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const uint32_t pa = smem_u32(sm.p[0][kk >> 2]) + (kk & 3) * 32;
+                            // V: 16 keys per step (two 8-row groups of 1024 B); the CTA's second
+                            // 64-dim chunk sits in the next slot (LBO)
+                            mma_pair_f16(tm_o + v * 256, sdesc_sw128(pa, 16, 1024),
+                                         sdesc_sw128(vb + kk * 2048, kSlot, 1024), idesc_o,
+                                         (n > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit_pair(&sm.empty[s0]);
+                        mma_commit_pair(&sm.empty[s1]);
                     }
-                    mma_commit_pair(&sm.empty[s0]);
-                    mma_commit_pair(&sm.empty[s1]);
+                    if (C::SWAP || n == ntiles - 1) mma_commit_pair(&sm.o_done);
                 }
-                if (C::SWAP || n == ntiles - 1) mma_commit_pair(&sm.o_done);
+            } else {
+                // tile n's slots sit at ring positions 4n .. 4n + 3 (S stages, then V); the
+                // MMAs take S(n) before O += P(n-1) V(n-1)
+                if (!mbar_wait_cluster(&sm.q_ready, 0, wc, abort)) goto done;
+                constexpr int SPT = C::NS + 2 * C::NV;   // slots per tile
+                for (int n = 0; n <= ntiles; ++n) {
+                    if (n < ntiles) {
+                        const uint32_t b = n & 1;
+                        // S buffer b was last read by the softmax of tile n - 2
+                        if (n >= 2 && !mbar_wait_cluster(&sm.s_free[b], ((n - 2) >> 1) & 1, wc, abort))
+                            goto done;
+                        tc_fence_after();
+                        for (int s = 0; s < C::NS; ++s) {
+                            const uint32_t q = (uint32_t)(n * SPT + s), slot = q % NSLOT;
+                            if (!mbar_wait_cluster(&sm.full[slot], (q / NSLOT) & 1, wc, abort))
+                                goto done;
+                            tc_fence_after();
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t ab = smem_u32(sm.q[2 * s + (kk >> 2)]) + (kk & 3) * 32;
+                                const uint32_t bb = smem_u32(sm.ring[slot]) + (kk >> 2) * (kSlot / 2) +
+                                                    (kk & 3) * 32;
+                                mma_pair_f16(tm_s + 128 * b, sdesc_sw128(ab, 16, 1024),
+                                             sdesc_sw128(bb, 16, 1024), idesc_s,
+                                             (s | kk) != 0 ? 1u : 0u);
+                            }
+                            mma_commit_pair(&sm.empty[slot]);
+                        }
+                        mma_commit_pair(&sm.s_full[b]);
+                    }
+                    if (n >= 1) {
+                        const int j = n - 1;
+                        const uint32_t pb = j & 1;
+                        if (!mbar_wait_cluster(&sm.p_full[pb], (j >> 1) & 1, wc, abort)) goto done;
+                        tc_fence_after();
+                        for (int v = 0; v < C::NV; ++v) {
+                            const uint32_t q = (uint32_t)(j * SPT + C::NS + 2 * v);
+                            const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
+                            if (!mbar_wait_cluster(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
+                            if (!mbar_wait_cluster(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
+                                goto done;
+                            tc_fence_after();
+                            const uint32_t vb = smem_u32(sm.ring[s0]);
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint32_t pa = smem_u32(sm.p[pb][kk >> 2]) + (kk & 3) * 32;
+                                mma_pair_f16(tm_o + v * 256, sdesc_sw128(pa, 16, 1024),
+                                             sdesc_sw128(vb + kk * 2048, kSlot, 1024), idesc_o,
+                                             (j > 0 || kk > 0) ? 1u : 0u);
+                            }
+                            mma_commit_pair(&sm.empty[s0]);
+                            mma_commit_pair(&sm.empty[s1]);
+                        }
+                        mma_commit_pair(&sm.pv_done[pb]);
+                        if (j == ntiles - 1) mma_commit_pair(&sm.o_done);
+                    }
+                }
             }
         done:;
         }
@@ -305,7 +371,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             group_sync(kBarWG, 128);
-            if (t128 == 0) mbar_arrive_remote(&sm.s_free, 0);   // Q ready, S free for tile 0
+            if (t128 == 0)   // Q ready (and, head_dim 512, S free for tile 0)
+                mbar_arrive_remote(C::SWAP ? &sm.s_free[0] : &sm.q_ready, 0);
         }
 
         // ---- main loop
@@ -335,13 +402,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_wait();
                     tc_fence_before();
                     group_sync(kBarWG, 128);
-                    if (t128 == 0) mbar_arrive_remote(&sm.s_free, 0);
+                    if (t128 == 0) mbar_arrive_remote(&sm.s_free[0], 0);
                 }
-            } else {
-                if (n > 0 && t128 == 0) mbar_arrive_remote(&sm.s_free, 0);
             }
-            ok = group_all(mbar_wait(&sm.s_full, n & 1, wc, abort), kBarWG, 128);
+            const uint32_t sbuf = C::SWAP ? 0u : (uint32_t)(n & 1);
+            const uint32_t tm_sn = tm_s + 128 * sbuf;   // this tile's S
+            ok = group_all(C::SWAP ? mbar_wait(&sm.s_full[0], n & 1, wc, abort)
+                                   : mbar_wait(&sm.s_full[sbuf], (n >> 1) & 1, wc, abort),
+                           kBarWG, 128);
             if (!ok) break;
+            if (!C::SWAP && n >= 2) {
+                // P buffer sbuf was last read by the value product of tile n - 2 (issued before
+                // this tile's scores, so already complete)
+                ok = group_all(mbar_wait(&sm.pv_done[sbuf], ((n - 2) >> 1) & 1, wc, abort),
+                               kBarWG, 128);
+                if (!ok) break;
+            }
             tc_fence_after();
             const bool need_mask = (key0 + kBN - 1 > t_first) ||
                                    (a.window > 0 && key0 <= t_last - a.window);
@@ -353,13 +429,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 uint32_t sa[32], sb[32];
                 float mxr = -INFINITY;
                 const float negm = -m_ref;
-                tmem_ld32_nowait(tm_s + lane_off, sa);
+                tmem_ld32_nowait(tm_sn + lane_off, sa);
                 tmem_ld_wait();
 #pragma unroll
                 for (int b = 0; b < 4; ++b) {
                     uint32_t* cur = (b & 1) ? sb : sa;
                     uint32_t* nxt = (b & 1) ? sa : sb;
-                    if (b < 3) tmem_ld32_nowait(tm_s + (b + 1) * 32 + lane_off, nxt);
+                    if (b < 3) tmem_ld32_nowait(tm_sn + (b + 1) * 32 + lane_off, nxt);
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
@@ -377,7 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
                         }
                     }
-                    uint8_t* pb = sm.p[b >> 1];
+                    uint8_t* pb = sm.p[sbuf][b >> 1];
                     const int col = (b & 1) * 32;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
@@ -396,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int b = 0; b < 4; ++b) {
                     uint32_t sv[32];
-                    tmem_ld32_nowait(tm_s + b * 32 + lane_off, sv);
+                    tmem_ld32_nowait(tm_sn + b * 32 + lane_off, sv);
                     tmem_ld_wait();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
@@ -414,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int b = 0; b < 4; ++b) {
                     uint32_t sv[32];
-                    tmem_ld32_nowait(tm_s + b * 32 + lane_off, sv);
+                    tmem_ld32_nowait(tm_sn + b * 32 + lane_off, sv);
                     tmem_ld_wait();
                     uint32_t w[16];
 #pragma unroll
@@ -436,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
                         }
                     }
-                    uint8_t* pb = sm.p[b >> 1];
+                    uint8_t* pb = sm.p[sbuf][b >> 1];
                     const int col = (b & 1) * 32;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
@@ -445,8 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             l_sum = l_sum * alpha + psum;
-            // correction of the accumulator when the reference max moved (rare)
+            // correction of the accumulator when the reference max moved (rare); with two S
+            // buffers the value product of the tile before may still be running
             if (__any_sync(0xffffffffu, alpha != 1.f && n > 0)) {
+                if (!C::SWAP && !mbar_wait(&sm.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, abort))
+                    *abort = 1;
                 if constexpr (C::SWAP) {
 #pragma unroll
                     for (int i = 0; i < 128; ++i) o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
@@ -471,7 +550,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             tc_fence_before();
             group_sync(kBarWG, 128);
-            if (t128 == 0) mbar_arrive_remote(&sm.p_full, 0);
+            if (t128 == 0) {
+                if constexpr (C::SWAP) {
+                    mbar_arrive_remote(&sm.p_full[0], 0);
+                } else {
+                    mbar_arrive_remote(&sm.s_free[sbuf], 0);   // S read: buffer reusable
+                    mbar_arrive_remote(&sm.p_full[sbuf], 0);
+                }
+            }
         }
         // ---- epilogue
         if (ok) {

@@ -282,20 +282,14 @@ __device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank) {
     return r;
 }
 
-// Arrive on the mbarrier at the same offset in CTA `rank` of the cluster.
+// Arrive on the mbarrier at the same offset in CTA `rank` of the cluster, with CTA-scope
+// release ordering.  A cluster-scope release costs a fence of several hundred cycles per
+// signal (more under load) and sits on the per-tile chain of both kernels; the pair
+// hand-offs use this form, which is how cluster pipelines signal a peer CTA's barrier: the
+// arriving thread's shared-memory writes (made visible to the tensor core by
+// fence.proxy.async first) reach the peer in order ahead of the arrival, and the waiting side
+// acquires at cluster scope.
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
-    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
-                     mapa_shared(bar, rank))
-                 : "memory");
-}
-
-// Arrive on the mbarrier at this offset in CTA `rank` of the cluster with CTA-scope release
-// ordering.  A cluster-scope release costs a fence of several hundred cycles per signal (more
-// under load); the per-tile hand-off from the second CTA of a pair uses this form, which is
-// how cluster pipelines signal a peer CTA's barrier: the arriving thread's shared-memory
-// writes (made visible to the tensor core by fence.proxy.async first) reach the peer in
-// order ahead of the arrival.
-__device__ __forceinline__ void mbar_arrive_peer(uint64_t* bar, uint32_t rank) {
     asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(
                      mapa_shared(bar, rank))
                  : "memory");
