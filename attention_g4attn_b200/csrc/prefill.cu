@@ -305,68 +305,91 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int G = a.G;
 
-        // ---- prologue: QKNorm + RoPE of the 128 packed rows (one warp per row at a time)
+        // ---- prologue: QKNorm + RoPE of the 128 packed rows.  A warp takes four rows at a
+        // time (rows wq, wq + 4, ...) and issues all their global loads before the math, so
+        // the load latency is paid once per four rows instead of once per row.
         {
             constexpr int E = D / 64;             // elements per lane in each half
+            constexpr int RB = 4;                 // rows in flight per warp
             const int half = D / 2;
-            for (int r = wq; r < kBM; r += 4) {
-                const int tl = r / G, hl = r % G;
-                const int tok = pg.m0 + tl;
-                float x0[E], x1[E];
-                if (tl < pg.tq) {
-                    const uint16_t* src =
-                        a.q + (((size_t)pg.b * a.T + tok) * a.Hq + (size_t)pg.g * G + hl) * D;
+            float g0[E], g1[E];
 #pragma unroll
-                    for (int e = 0; e < E; e += 2) {
-                        const float2 f0 = __bfloat1622float2(
-                            *reinterpret_cast<const __nv_bfloat162*>(src + lane * E + e));
-                        const float2 f1 = __bfloat1622float2(
-                            *reinterpret_cast<const __nv_bfloat162*>(src + half + lane * E + e));
-                        x0[e] = f0.x; x0[e + 1] = f0.y;
-                        x1[e] = f1.x; x1[e + 1] = f1.y;
+            for (int e = 0; e < E; ++e) {
+                g0[e] = a.gamma_q[lane * E + e];
+                g1[e] = a.gamma_q[half + lane * E + e];
+            }
+            for (int r0 = wq; r0 < kBM; r0 += 4 * RB) {
+                float x0[RB][E], x1[RB][E];
+                float2 cs[RB][E];
+#pragma unroll
+                for (int k = 0; k < RB; ++k) {
+                    const int r = r0 + 4 * k;
+                    const int tl = r / G, hl = r % G;
+                    const int tok = pg.m0 + tl;
+                    if (tl < pg.tq) {
+                        const uint16_t* src =
+                            a.q + (((size_t)pg.b * a.T + tok) * a.Hq + (size_t)pg.g * G + hl) * D;
+#pragma unroll
+                        for (int e = 0; e < E; e += 2) {
+                            const float2 f0 = __bfloat1622float2(
+                                *reinterpret_cast<const __nv_bfloat162*>(src + lane * E + e));
+                            const float2 f1 = __bfloat1622float2(
+                                *reinterpret_cast<const __nv_bfloat162*>(src + half + lane * E + e));
+                            x0[k][e] = f0.x; x0[k][e + 1] = f0.y;
+                            x1[k][e] = f1.x; x1[k][e + 1] = f1.y;
+                        }
+#pragma unroll
+                        for (int e = 0; e < E; ++e) {
+                            const int i = lane * E + e;
+                            cs[k][e] = i < R ? a.rope_cs[(size_t)tok * R + i] : make_float2(1.f, 0.f);
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < E; ++e) {
+                            x0[k][e] = x1[k][e] = 0.f;
+                            cs[k][e] = make_float2(1.f, 0.f);
+                        }
                     }
+                }
+#pragma unroll
+                for (int k = 0; k < RB; ++k) {
+                    const int r = r0 + 4 * k;
                     if (a.qk_norm) {
                         float ss = 0.f;
 #pragma unroll
-                        for (int e = 0; e < E; ++e) ss += x0[e] * x0[e] + x1[e] * x1[e];
+                        for (int e = 0; e < E; ++e) ss += x0[k][e] * x0[k][e] + x1[k][e] * x1[k][e];
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
                         const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
 #pragma unroll
                         for (int e = 0; e < E; ++e) {
-                            x0[e] = x0[e] * inv * a.gamma_q[lane * E + e];
-                            x1[e] = x1[e] * inv * a.gamma_q[half + lane * E + e];
+                            x0[k][e] = x0[k][e] * inv * g0[e];
+                            x1[k][e] = x1[k][e] * inv * g1[e];
                         }
                     }
 #pragma unroll
                     for (int e = 0; e < E; ++e) {
-                        const int i = lane * E + e;
-                        if (i < R) {
-                            const float2 cs = a.rope_cs[(size_t)tok * R + i];
-                            const float u = x0[e], v = x1[e];
-                            x0[e] = u * cs.x - v * cs.y;
-                            x1[e] = u * cs.y + v * cs.x;
-                        }
+                        // pairs at or past R carry (cos, sin) = (1, 0): unchanged
+                        const float u = x0[k][e], v = x1[k][e];
+                        x0[k][e] = u * cs[k][e].x - v * cs[k][e].y;
+                        x1[k][e] = u * cs[k][e].y + v * cs[k][e].x;
                     }
-                } else {
 #pragma unroll
-                    for (int e = 0; e < E; ++e) x0[e] = x1[e] = 0.f;
-                }
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const float* x = hh ? x1[k] : x0[k];
+                        const int col = hh * half + lane * E;
+                        uint32_t w[E / 2];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const float* x = hh ? x1 : x0;
-                    const int col = hh * half + lane * E;
-                    uint32_t w[E / 2];
-#pragma unroll
-                    for (int e = 0; e < E; e += 2) w[e / 2] = pack_f16x2(x[e], x[e + 1]);
-                    uint8_t* base = sm.q[col / 64];
-                    const uint32_t off = sw128_offset(r, col % 64);
-                    if constexpr (E == 8)
-                        *reinterpret_cast<uint4*>(base + off) = make_uint4(w[0], w[1], w[2], w[3]);
-                    else if constexpr (E == 4)
-                        *reinterpret_cast<uint2*>(base + off) = make_uint2(w[0], w[1]);
-                    else
-                        *reinterpret_cast<uint32_t*>(base + off) = w[0];
+                        for (int e = 0; e < E; e += 2) w[e / 2] = pack_f16x2(x[e], x[e + 1]);
+                        uint8_t* base = sm.q[col / 64];
+                        const uint32_t off = sw128_offset(r, col % 64);
+                        if constexpr (E == 8)
+                            *reinterpret_cast<uint4*>(base + off) = make_uint4(w[0], w[1], w[2], w[3]);
+                        else if constexpr (E == 4)
+                            *reinterpret_cast<uint2*>(base + off) = make_uint2(w[0], w[1]);
+                        else
+                            *reinterpret_cast<uint32_t*>(base + off) = w[0];
+                    }
                 }
             }
             fence_proxy_async_smem();
