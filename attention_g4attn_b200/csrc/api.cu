@@ -129,6 +129,31 @@ int encode_rows(CUtensorMap* m, const void* base, int B, int T, int H, int d, bo
     return r == CUDA_SUCCESS ? G4ATTN_OK : G4ATTN_ERR_CUDA;
 }
 
+// 4-D map over the raw queries [B, T, Hq, d] as (d, Hq, T, B) with box (64, G, 128 / G, 1):
+// one box is a 64-dim chunk of a packed row tile (row = token * G + head), 128-byte swizzle.
+int encode_q_tile(CUtensorMap* m, const void* q, int B, int T, int Hq, int d, int G) {
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)Hq, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)Hq * d * 2, (cuuint64_t)T * Hq * d * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)(128 / G), 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides,
+                          box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? G4ATTN_OK : G4ATTN_ERR_CUDA;
+}
+
+// 2-D map over the [T, R] (cos, sin) table as fp32 (2R, T), box (2R, rows).
+int encode_cs_rows(CUtensorMap* m, const float2* cs, int T, int R, int rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)(2 * R), (cuuint64_t)T};
+    cuuint64_t strides[1] = {(cuuint64_t)R * 8};
+    cuuint32_t box[2] = {(cuuint32_t)(2 * R), (cuuint32_t)rows};
+    cuuint32_t es[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float2*>(cs), dims, strides,
+                          box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                          CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? G4ATTN_OK : G4ATTN_ERR_CUDA;
+}
+
 struct PrefillWs {
     size_t kn_off, kr_off, cs_off, total;
     bool need_kn;
@@ -325,6 +350,17 @@ int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16
     if (v) rc = encode_rows(&a.tm_v, v, B, T, Hkv, d, false, 128);
     else rc = encode_rows(&a.tm_v, kn_or_kr, B, T, Hkv, d, true, 128);
     if (rc) return rc;
+    const int G = cfg->n_q_heads / Hkv;
+    if ((rc = encode_q_tile(&a.tm_q, q, B, T, cfg->n_q_heads, d, G))) return rc;
+    {
+        // the (cos, sin) rows of a row tile go to shared memory by TMA when they fit the
+        // P buffers (free during the prologue) and the row pitch suits TMA
+        const int R = rope_pairs(cfg), rows = 128 / G;
+        const size_t bytes = (size_t)rows * R * 8;
+        a.cs_tma = R > 0 && R % 2 == 0 && 2 * R <= 256 && rows <= 256 &&
+                   bytes <= g4::prefill_p_bytes(d);
+        if (a.cs_tma && (rc = encode_cs_rows(&a.tm_cs, cs, T, R, rows))) return rc;
+    }
     a.q = q;
     a.gamma_q = gamma_q;
     a.rope_cs = cs;

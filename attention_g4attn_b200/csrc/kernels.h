@@ -69,6 +69,9 @@ struct PrefillArgs {
     CUtensorMap tm_kn_v;
     CUtensorMap tm_kr_v;
     CUtensorMap tm_v;       // separate values (bf16, kv_is_k == 0), else a copy of tm_kn_v
+    CUtensorMap tm_q;       // raw queries as (d, Hq, T, B), box (64, G, 128 / G, 1): one row tile
+    CUtensorMap tm_cs;      // rope_cs as fp32 (2R, T), box (2R, 128 / G); valid when cs_tma
+    int cs_tma;             // the (cos, sin) rows of a row tile are loaded by TMA
     const uint16_t* q;      // raw queries [B, T, Hq, d]
     const float* gamma_q;
     const float2* rope_cs;  // [T, R] (cos, sin) of position t, pair i
@@ -87,5 +90,6 @@ struct PrefillArgs {
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 size_t prefill_smem_bytes(int d);
+size_t prefill_p_bytes(int d);   // bytes of the P buffers (staging room during the prologue)
 
 }  // namespace g4

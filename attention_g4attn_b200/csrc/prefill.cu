@@ -67,7 +67,7 @@ struct __align__(1024) PrefillSmem {
     uint64_t empty[PrefillCfg<D>::NSLOT];  // per CTA, released by the leader's MMA commits
     // per buffer (tile n uses [n % NBUF]); s_free / p_full / q_ready count one arrival per CTA
     uint64_t s_free[2], s_full[2], p_full[2], pv_done[2];
-    uint64_t q_ready, o_done, drain;
+    uint64_t q_full, q_ready, o_done, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&sm.p_full[i], 2);
             mbar_init(&sm.pv_done[i], 1);
         }
+        mbar_init(&sm.q_full, 1);   // this CTA's raw query tile (and cos/sin rows) landed
         mbar_init(&sm.q_ready, 2);
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.drain, 1);
@@ -157,6 +158,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&a.tm_kn_v);
             prefetch_tmap(&a.tm_kr_v);
             prefetch_tmap(&a.tm_v);
+            {
+                // the raw query tile (one box per 64-dim chunk, rows = token * G + head) and
+                // the (cos, sin) rows of its tokens; the P buffers hold the latter until the
+                // prologue is done
+                const int tpt = kBM / a.G;
+                const uint32_t cs_bytes = a.cs_tma ? (uint32_t)(tpt * R * 8) : 0u;
+                mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(NCH * 16384) + cs_bytes);
+                for (int c = 0; c < NCH; ++c)
+                    tma_load_4d(sm.q[c], &a.tm_q, &sm.q_full, c * 64, pg.g * a.G, pg.m0, pg.b);
+                if (a.cs_tma) tma_load_2d(&sm.p[0][0][0], &a.tm_cs, &sm.q_full, 0, pg.m0);
+            }
             uint32_t q = 0;
             for (int n = 0; n < ntiles && !*abort; ++n) {
                 const int key0 = (pg.j_lo + n) * kBN;
@@ -305,90 +317,74 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const int G = a.G;
 
-        // ---- prologue: QKNorm + RoPE of the 128 packed rows.  A warp takes four rows at a
-        // time (rows wq, wq + 4, ...) and issues all their global loads before the math, so
-        // the load latency is paid once per four rows instead of once per row.
+        bool ok_pro = true;
+        // ---- prologue: QKNorm + RoPE of the 128 packed rows, in place in shared memory.
+        // The raw bf16 tile arrived by TMA (row r = token r / G, head r % G, the layout the
+        // MMAs read); thread r turns its row into the normalised, rotated fp16 row.
         {
-            constexpr int E = D / 64;             // elements per lane in each half
-            constexpr int RB = 4;                 // rows in flight per warp
             const int half = D / 2;
-            float g0[E], g1[E];
+            const int r = t128;
+            const int tl = r / G;
+            const int tok = pg.m0 + tl;
+            const float2* cs_row = a.cs_tma ? reinterpret_cast<const float2*>(&sm.p[0][0][0]) + tl * R
+                                            : a.rope_cs + (size_t)tok * R;
+            ok_pro = group_all(mbar_wait(&sm.q_full, 0, wc, abort), kBarWG, 128);
+            if (ok_pro) {
+                float inv = 1.f;
+                if (a.qk_norm) {
+                    float ss = 0.f;
+                    for (int c = 0; c < NCH; ++c) {
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                g0[e] = a.gamma_q[lane * E + e];
-                g1[e] = a.gamma_q[half + lane * E + e];
-            }
-            for (int r0 = wq; r0 < kBM; r0 += 4 * RB) {
-                float x0[RB][E], x1[RB][E];
-                float2 cs[RB][E];
+                        for (int k = 0; k < 8; ++k) {
+                            const uint4 w = *reinterpret_cast<const uint4*>(sm.q[c] + sw128_offset(r, 8 * k));
+                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int k = 0; k < RB; ++k) {
-                    const int r = r0 + 4 * k;
-                    const int tl = r / G, hl = r % G;
-                    const int tok = pg.m0 + tl;
-                    if (tl < pg.tq) {
-                        const uint16_t* src =
-                            a.q + (((size_t)pg.b * a.T + tok) * a.Hq + (size_t)pg.g * G + hl) * D;
-#pragma unroll
-                        for (int e = 0; e < E; e += 2) {
-                            const float2 f0 = __bfloat1622float2(
-                                *reinterpret_cast<const __nv_bfloat162*>(src + lane * E + e));
-                            const float2 f1 = __bfloat1622float2(
-                                *reinterpret_cast<const __nv_bfloat162*>(src + half + lane * E + e));
-                            x0[k][e] = f0.x; x0[k][e + 1] = f0.y;
-                            x1[k][e] = f1.x; x1[k][e + 1] = f1.y;
-                        }
-#pragma unroll
-                        for (int e = 0; e < E; ++e) {
-                            const int i = lane * E + e;
-                            cs[k][e] = i < R ? a.rope_cs[(size_t)tok * R + i] : make_float2(1.f, 0.f);
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < E; ++e) {
-                            x0[k][e] = x1[k][e] = 0.f;
-                            cs[k][e] = make_float2(1.f, 0.f);
+                            for (int m = 0; m < 4; ++m) {
+                                const float2 f = bf16x2_to_f2(ww[m]);
+                                ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                            }
                         }
                     }
+                    inv = 1.0f / sqrtf(ss / (float)D + a.eps);
                 }
+                for (int c = 0; c < NCH / 2; ++c) {
+                    const int c2i = c + NCH / 2;   // partner chunk: dims + d/2
+#pragma unroll 2
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = sw128_offset(r, 8 * k);
+                        const uint4 wu = *reinterpret_cast<const uint4*>(sm.q[c] + off);
+                        const uint4 wv = *reinterpret_cast<const uint4*>(sm.q[c2i] + off);
+                        const uint32_t uu[4] = {wu.x, wu.y, wu.z, wu.w};
+                        const uint32_t vv[4] = {wv.x, wv.y, wv.z, wv.w};
+                        uint32_t ou[4], ov[4];
 #pragma unroll
-                for (int k = 0; k < RB; ++k) {
-                    const int r = r0 + 4 * k;
-                    if (a.qk_norm) {
-                        float ss = 0.f;
+                        for (int m = 0; m < 4; ++m) {
+                            const float2 u = bf16x2_to_f2(uu[m]);
+                            const float2 v = bf16x2_to_f2(vv[m]);
+                            float xo[2], yo[2];
+                            const float ux[2] = {u.x, u.y}, vx[2] = {v.x, v.y};
 #pragma unroll
-                        for (int e = 0; e < E; ++e) ss += x0[k][e] * x0[k][e] + x1[k][e] * x1[k][e];
-#pragma unroll
-                        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-                        const float inv = 1.0f / sqrtf(ss / (float)D + a.eps);
-#pragma unroll
-                        for (int e = 0; e < E; ++e) {
-                            x0[k][e] = x0[k][e] * inv * g0[e];
-                            x1[k][e] = x1[k][e] * inv * g1[e];
+                            for (int e = 0; e < 2; ++e) {
+                                const int i = c * 64 + 8 * k + 2 * m + e;
+                                float x = ux[e], y = vx[e];
+                                if (a.qk_norm) {
+                                    x = x * inv * a.gamma_q[i];
+                                    y = y * inv * a.gamma_q[half + i];
+                                }
+                                if (i < R) {
+                                    const float2 cs = cs_row[i];
+                                    const float x2 = x * cs.x - y * cs.y;
+                                    y = x * cs.y + y * cs.x;
+                                    x = x2;
+                                }
+                                xo[e] = x;
+                                yo[e] = y;
+                            }
+                            ou[m] = pack_f16x2(xo[0], xo[1]);
+                            ov[m] = pack_f16x2(yo[0], yo[1]);
                         }
-                    }
-#pragma unroll
-                    for (int e = 0; e < E; ++e) {
-                        // pairs at or past R carry (cos, sin) = (1, 0): unchanged
-                        const float u = x0[k][e], v = x1[k][e];
-                        x0[k][e] = u * cs[k][e].x - v * cs[k][e].y;
-                        x1[k][e] = u * cs[k][e].y + v * cs[k][e].x;
-                    }
-#pragma unroll
-                    for (int hh = 0; hh < 2; ++hh) {
-                        const float* x = hh ? x1[k] : x0[k];
-                        const int col = hh * half + lane * E;
-                        uint32_t w[E / 2];
-#pragma unroll
-                        for (int e = 0; e < E; e += 2) w[e / 2] = pack_f16x2(x[e], x[e + 1]);
-                        uint8_t* base = sm.q[col / 64];
-                        const uint32_t off = sw128_offset(r, col % 64);
-                        if constexpr (E == 8)
-                            *reinterpret_cast<uint4*>(base + off) = make_uint4(w[0], w[1], w[2], w[3]);
-                        else if constexpr (E == 4)
-                            *reinterpret_cast<uint2*>(base + off) = make_uint2(w[0], w[1]);
-                        else
-                            *reinterpret_cast<uint32_t*>(base + off) = w[0];
+                        *reinterpret_cast<uint4*>(sm.q[c] + off) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
+                        *reinterpret_cast<uint4*>(sm.q[c2i] + off) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
                     }
                 }
             }
@@ -411,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 128; ++i) o1[i] = 0u;
         }
-        bool ok = true;
+        bool ok = ok_pro;
         for (int n = 0; n < ntiles && ok; ++n) {
             const int key0 = (pg.j_lo + n) * kBN;
             if constexpr (C::SWAP) {
@@ -445,9 +441,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool need_mask = (key0 + kBN - 1 > t_first) ||
                                    (a.window > 0 && key0 <= t_last - a.window);
             float psum = 0.f, alpha = 1.f;
-            // fast path: no mask in this tile and a finite reference max in every row of
-            // the warp: one pass over S with the current reference
-            bool slow = need_mask || !__all_sync(0xffffffffu, m_ref != -INFINITY);
+            const int lo_r = a.window > 0 ? tok_r - a.window + 1 : 0;
+            // fast path: a finite reference max in every row of the warp: one pass over S
+            // with the current reference; for head_dim 256 masked keys (outside the causal
+            // band or the window) are dropped element by element, head_dim 512 (registers
+            // full with the O quarter) takes masked tiles on the two-pass path
+            bool slow = (C::SWAP && need_mask) || !__all_sync(0xffffffffu, m_ref != -INFINITY);
             if (!slow) {
                 uint32_t sa[32], sb[32];
                 float mxr = -INFINITY;
@@ -462,7 +461,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        const float s0 = __uint_as_float(cur[e]), s1 = __uint_as_float(cur[e + 1]);
+                        float s0 = __uint_as_float(cur[e]), s1 = __uint_as_float(cur[e + 1]);
+                        if (!C::SWAP && need_mask) {
+                            const int j = key0 + b * 32 + e;
+                            if (!(j <= tok_r && j >= lo_r)) s0 = -INFINITY;
+                            if (!(j + 1 <= tok_r && j + 1 >= lo_r)) s1 = -INFINITY;
+                        }
                         mxr = fmaxf(mxr, fmaxf(s0, s1));
                         const float p0 = ex2_approx(fmaf(s0, c2, negm));
                         const float p1 = ex2_approx(fmaf(s1, c2, negm));
@@ -490,7 +494,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (slow) {
                 // two passes with masks: row max, then P with a (lazily) updated reference
-                const int lo_r = a.window > 0 ? tok_r - a.window + 1 : 0;
                 float mx = -INFINITY;
 #pragma unroll 1
                 for (int b = 0; b < 4; ++b) {
@@ -544,9 +547,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             l_sum = l_sum * alpha + psum;
-            // correction of the accumulator when the reference max moved (rare); with two S
+            // correction of the accumulator when a finite reference max moved (rare: a row
+            // whose reference was still -inf has an all-zero accumulator); with two S
             // buffers the value product of the tile before may still be running
-            if (__any_sync(0xffffffffu, alpha != 1.f && n > 0)) {
+            if (__any_sync(0xffffffffu, alpha != 1.f && alpha != 0.f && n > 0)) {
                 if (!C::SWAP && !mbar_wait(&sm.pv_done[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, abort))
                     *abort = 1;
                 if constexpr (C::SWAP) {
@@ -660,6 +664,10 @@ cudaError_t run_prefill(const PrefillArgs& a, cudaStream_t stream) {
 }
 
 }  // namespace
+
+size_t prefill_p_bytes(int d) {
+    return d == 512 ? sizeof(PrefillSmem<512>::p) : sizeof(PrefillSmem<256>::p);
+}
 
 size_t prefill_smem_bytes(int d) {
     return d == 512 ? sizeof(PrefillSmem<512>) + 1024 : sizeof(PrefillSmem<256>) + 1024;
