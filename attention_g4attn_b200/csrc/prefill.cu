@@ -67,7 +67,7 @@ struct __align__(1024) PrefillSmem {
     uint64_t empty[PrefillCfg<D>::NSLOT];  // per CTA, released by the leader's MMA commits
     // per buffer (tile n uses [n % NBUF]); s_free / p_full / q_ready count one arrival per CTA
     uint64_t s_free[2], s_full[2], p_full[2], pv_done[2];
-    uint64_t q_full, q_ready, o_done, drain;
+    uint64_t q_full, q_ready, o_done, o1_done, drain;
     uint32_t tmem_base;
     int abort;
 };
@@ -138,6 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sm.q_full, 1);   // this CTA's raw query tile (and cos/sin rows) landed
         mbar_init(&sm.q_ready, 2);
         mbar_init(&sm.o_done, 1);
+        mbar_init(&sm.o1_done, 1);   // head_dim 512: the first 256-dim block of P.V is done
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -247,8 +248,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                         mma_commit_pair(&sm.empty[s0]);
                         mma_commit_pair(&sm.empty[s1]);
+                        // the O quarter that S borrows lies in block 0: the softmax warps can
+                        // move it out while block 1 runs
+                        if (v == 0) mma_commit_pair(&sm.o1_done);
                     }
-                    if (C::SWAP || n == ntiles - 1) mma_commit_pair(&sm.o_done);
+                    if (n == ntiles - 1) mma_commit_pair(&sm.o_done);
                 }
             } else {
                 // tile n's slots sit at ring positions 4n .. 4n + 3 (S stages, then V); the
@@ -412,8 +416,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int key0 = (pg.j_lo + n) * kBN;
             if constexpr (C::SWAP) {
                 if (n > 0) {
-                    // O[:, 128..255] leaves TMEM so S(n) can use those columns
-                    ok = group_all(mbar_wait(&sm.o_done, (n - 1) & 1, wc, abort), kBarWG, 128);
+                    // O[:, 128..255] leaves TMEM so S(n) can use those columns (block 0 of the
+                    // previous P.V is done; block 1 may still run, it does not touch them)
+                    ok = group_all(mbar_wait(&sm.o1_done, (n - 1) & 1, wc, abort), kBarWG, 128);
                     if (!ok) break;
                     tc_fence_after();
 #pragma unroll
@@ -588,8 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // ---- epilogue
         if (ok) {
-            const uint32_t last = C::SWAP ? (uint32_t)(ntiles - 1) : 0u;
-            ok = group_all(mbar_wait(&sm.o_done, last & 1, wc, abort), kBarWG, 128);
+            ok = group_all(mbar_wait(&sm.o_done, 0, wc, abort), kBarWG, 128);   // once per CTA
         }
         if (ok) {
             tc_fence_after();
