@@ -251,7 +251,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             long long polls = 0;
             while (pc.it < n_items) {
                 bool did = false;
-                if (pc.g < sc.g && mbar_test_wait_cluster(&sm.p_full[pc.g & 1], (pc.g >> 1) & 1)) {
+                if (pc.g < sc.g && mbar_test_wait(&sm.p_full[pc.g & 1], (pc.g >> 1) & 1)) {
                     // O^T += V^T . P^T for tile pc.g: both CTAs' P are ready
                     tc_fence_after();
                     const uint64_t pb = d_p + (pc.g & 1) * kPDesc;
@@ -268,7 +268,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     advance(pc);
                     did = true;
                 } else if (sc.it < n_items && sc.g < pc.g + 2 &&
-                           mbar_test_wait_cluster(&sm.rot_ready[sc.g & 1], (sc.g >> 1) & 1)) {
+                           mbar_test_wait(&sm.rot_ready[sc.g & 1], (sc.g >> 1) & 1)) {
                     // S^T for tile sc.g: both CTAs have its slots (turned) and, at the
                     // start of an item, its queries; its S^T buffer was read by the softmax
                     // of tile sc.g - 2, whose value product has been issued

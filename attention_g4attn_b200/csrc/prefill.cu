@@ -31,6 +31,8 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "kernels.h"
 #include "sm100.cuh"
 
@@ -213,11 +215,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (C::SWAP) {
                 uint32_t q = 0;
                 for (int n = 0; n < ntiles; ++n) {
-                    if (!mbar_wait_cluster(&sm.s_free[0], n & 1, wc, abort)) goto done;
+                    if (!mbar_wait(&sm.s_free[0], n & 1, wc, abort)) goto done;
                     tc_fence_after();
                     for (int s = 0; s < C::NS; ++s, ++q) {
                         const uint32_t slot = q % NSLOT;
-                        if (!mbar_wait_cluster(&sm.full[slot], (q / NSLOT) & 1, wc, abort)) goto done;
+                        if (!mbar_wait(&sm.full[slot], (q / NSLOT) & 1, wc, abort)) goto done;
                         tc_fence_after();
                         for (int kk = 0; kk < 8; ++kk) {
                             const uint32_t ab = smem_u32(sm.q[2 * s + (kk >> 2)]) + (kk & 3) * 32;
@@ -229,12 +231,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mma_commit_pair(&sm.empty[slot]);
                     }
                     mma_commit_pair(&sm.s_full[0]);
-                    if (!mbar_wait_cluster(&sm.p_full[0], n & 1, wc, abort)) goto done;
+                    if (!mbar_wait(&sm.p_full[0], n & 1, wc, abort)) goto done;
                     tc_fence_after();
                     for (int v = 0; v < C::NV; ++v, q += 2) {
                         const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
-                        if (!mbar_wait_cluster(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
-                        if (!mbar_wait_cluster(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
+                        if (!mbar_wait(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
+                        if (!mbar_wait(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
                             goto done;
                         tc_fence_after();
                         const uint32_t vb = smem_u32(sm.ring[s0]);
@@ -257,18 +259,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 // tile n's slots sit at ring positions 4n .. 4n + 3 (S stages, then V); the
                 // MMAs take S(n) before O += P(n-1) V(n-1)
-                if (!mbar_wait_cluster(&sm.q_ready, 0, wc, abort)) goto done;
+                if (!mbar_wait(&sm.q_ready, 0, wc, abort)) goto done;
                 constexpr int SPT = C::NS + 2 * C::NV;   // slots per tile
                 for (int n = 0; n <= ntiles; ++n) {
                     if (n < ntiles) {
                         const uint32_t b = n & 1;
                         // S buffer b was last read by the softmax of tile n - 2
-                        if (n >= 2 && !mbar_wait_cluster(&sm.s_free[b], ((n - 2) >> 1) & 1, wc, abort))
+                        if (n >= 2 && !mbar_wait(&sm.s_free[b], ((n - 2) >> 1) & 1, wc, abort))
                             goto done;
                         tc_fence_after();
                         for (int s = 0; s < C::NS; ++s) {
                             const uint32_t q = (uint32_t)(n * SPT + s), slot = q % NSLOT;
-                            if (!mbar_wait_cluster(&sm.full[slot], (q / NSLOT) & 1, wc, abort))
+                            if (!mbar_wait(&sm.full[slot], (q / NSLOT) & 1, wc, abort))
                                 goto done;
                             tc_fence_after();
                             for (int kk = 0; kk < 8; ++kk) {
@@ -286,13 +288,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (n >= 1) {
                         const int j = n - 1;
                         const uint32_t pb = j & 1;
-                        if (!mbar_wait_cluster(&sm.p_full[pb], (j >> 1) & 1, wc, abort)) goto done;
+                        if (!mbar_wait(&sm.p_full[pb], (j >> 1) & 1, wc, abort)) goto done;
                         tc_fence_after();
                         for (int v = 0; v < C::NV; ++v) {
                             const uint32_t q = (uint32_t)(j * SPT + C::NS + 2 * v);
                             const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
-                            if (!mbar_wait_cluster(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
-                            if (!mbar_wait_cluster(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
+                            if (!mbar_wait(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
+                            if (!mbar_wait(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
                                 goto done;
                             tc_fence_after();
                             const uint32_t vb = smem_u32(sm.ring[s0]);
@@ -452,9 +454,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             // band or the window) are dropped element by element, head_dim 512 (registers
             // full with the O quarter) takes masked tiles on the two-pass path
             bool slow = (C::SWAP && need_mask) || !__all_sync(0xffffffffu, m_ref != -INFINITY);
-            if (!slow) {
+            // one pass over S with the current reference; MASK: drop keys outside the causal
+            // band or the window element by element (a separate copy of the loop, so unmasked
+            // tiles carry no per-element test)
+            auto one_pass = [&](auto mask_tag, float& mxr) {
+                constexpr bool MASK = decltype(mask_tag)::value;
                 uint32_t sa[32], sb[32];
-                float mxr = -INFINITY;
                 const float negm = -m_ref;
                 tmem_ld32_nowait(tm_sn + lane_off, sa);
                 tmem_ld_wait();
@@ -467,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         float s0 = __uint_as_float(cur[e]), s1 = __uint_as_float(cur[e + 1]);
-                        if (!C::SWAP && need_mask) {
+                        if constexpr (MASK) {
                             const int j = key0 + b * 32 + e;
                             if (!(j <= tok_r && j >= lo_r)) s0 = -INFINITY;
                             if (!(j + 1 <= tok_r && j + 1 >= lo_r)) s1 = -INFINITY;
@@ -493,6 +498,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
                     if (b < 3) tmem_ld_wait();
                 }
+            };
+            if (!slow) {
+                float mxr = -INFINITY;
+                if (!C::SWAP && need_mask) one_pass(std::true_type{}, mxr);
+                else one_pass(std::false_type{}, mxr);
                 // the reference stays unless this tile's max exceeds it by more than 2^8
                 slow = __any_sync(0xffffffffu, mxr * c2 > m_ref + kLazyMax);
                 if (slow) psum = 0.f;

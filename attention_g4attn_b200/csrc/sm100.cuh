@@ -81,56 +81,21 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Non-blocking test with cluster-scope acquire: for barriers the other CTA of a pair
-// arrives on (its shared-memory writes become visible with the phase).
-__device__ __forceinline__ bool mbar_test_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-
 // Wait for the phase with the given parity to complete.  Gives up after `limit` polls or
 // kWaitTimeoutNs, whichever comes first, recording G4ATTN_ERR_TIMEOUT and raising the
 // CTA's abort flag; returns false at once when another thread has raised `abort`.
+// The waits and tests use the default CTA-scope acquire also on barriers that the other
+// CTA of a pair arrives on: there the waiting thread only issues tensor-core work that
+// reads the other CTA's shared memory, whose writers made their stores visible to the
+// async proxy (fence.proxy.async) before arriving, and the MMA thread orders its issue
+// after the wait with tcgen05.fence::after_thread_sync.  A cluster-scope acquire cost
+// 300-600 cycles per poll on the MMA thread, a third of a decode tile.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const WaitCtl& w,
                                           volatile int* abort) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     for (long long i = 1; i < w.limit; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*abort) return false;
-        if ((i & 63) == 0 && global_ns() - t0 > kWaitTimeoutNs) break;
-    }
-    atomicExch(w.status, (int)G4ATTN_ERR_TIMEOUT);
-    *abort = 1;
-    return false;
-}
-
-// Same, for barriers that receive arrivals from the other CTA of a cluster.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, const WaitCtl& w,
-                                                  volatile int* abort) {
-    if (mbar_try_wait_cluster(bar, parity)) return true;
-    const unsigned long long t0 = global_ns();
-    for (long long i = 1; i < w.limit; ++i) {
-        if (mbar_try_wait_cluster(bar, parity)) return true;
         if (*abort) return false;
         if ((i & 63) == 0 && global_ns() - t0 > kWaitTimeoutNs) break;
     }
@@ -297,8 +262,8 @@ __device__ __forceinline__ uint32_t mapa_shared(const void* p, uint32_t rank) {
 // signal (more under load) and sits on the per-tile chain of both kernels; the pair
 // hand-offs use this form, which is how cluster pipelines signal a peer CTA's barrier: the
 // arriving thread's shared-memory writes (made visible to the tensor core by
-// fence.proxy.async first) reach the peer in order ahead of the arrival, and the waiting side
-// acquires at cluster scope.
+// fence.proxy.async first) reach the peer in order ahead of the arrival, and the waiting
+// side's tensor-core reads are ordered after its wait (see mbar_wait).
 __device__ __forceinline__ void mbar_arrive_remote(uint64_t* bar, uint32_t rank) {
     asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(
                      mapa_shared(bar, rank))
