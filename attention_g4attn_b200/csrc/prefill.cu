@@ -326,71 +326,112 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok_pro = true;
         // ---- prologue: QKNorm + RoPE of the 128 packed rows, in place in shared memory.
         // The raw bf16 tile arrived by TMA (row r = token r / G, head r % G, the layout the
-        // MMAs read); thread r turns its row into the normalised, rotated fp16 row.
+        // MMAs read).  Warp wq turns rows [32 wq, 32 wq + 32) into normalised, rotated fp16
+        // rows, one row at a time across the warp: lane l holds dims [H l, H l + H) and their
+        // RoPE partners d/2 + [H l, H l + H), so both members of every rotated pair, their
+        // gammas (in registers for the whole tile) and a contiguous run of the row's
+        // (cos, sin) entries are the lane's own; the row's sum of squares is a warp sum.
         {
-            const int half = D / 2;
-            const int r = t128;
-            const int tl = r / G;
-            const int tok = pg.m0 + tl;
-            const float2* cs_row = a.cs_tma ? reinterpret_cast<const float2*>(&sm.p[0][0][0]) + tl * R
-                                            : a.rope_cs + (size_t)tok * R;
+            constexpr int H = D / 64;              // dims per lane in each half of the row
+            constexpr int half = D / 2;
+            const int i0 = lane * H;               // first pair index of this lane
+            const int col = i0 % 64;               // column within the 64-dim chunk
+            uint8_t* const qu = sm.q[i0 / 64];
+            uint8_t* const qv = sm.q[(half + i0) / 64];
+            float gu[H], gv[H];
+#pragma unroll
+            for (int k = 0; k < H; ++k) {
+                gu[k] = a.qk_norm ? a.gamma_q[i0 + k] : 1.f;
+                gv[k] = a.qk_norm ? a.gamma_q[half + i0 + k] : 1.f;
+            }
+            const float2* const cs_base =
+                a.cs_tma ? reinterpret_cast<const float2*>(&sm.p[0][0][0]) : a.rope_cs + (size_t)pg.m0 * R;
+            const bool rot_lane = i0 < R;
             ok_pro = group_all(mbar_wait(&sm.q_full, 0, wc, abort), kBarWG, 128);
             if (ok_pro) {
-                float inv = 1.f;
-                if (a.qk_norm) {
-                    float ss = 0.f;
-                    for (int c = 0; c < NCH; ++c) {
+                // NB rows per step, each stage over all of them, so the rows' load, warp-sum
+                // and square-root latencies overlap
+                constexpr int NB = H == 4 ? 8 : 4;
+#pragma unroll 1
+                for (int r0 = wq * 32; r0 < wq * 32 + 32; r0 += NB) {
+                    float u[NB][H], v[NB][H];
 #pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const uint4 w = *reinterpret_cast<const uint4*>(sm.q[c] + sw128_offset(r, 8 * k));
-                            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                    for (int j = 0; j < NB; ++j) {
+                        const uint32_t off = sw128_offset(r0 + j, col);
+                        if constexpr (H == 4) {
+                            const uint2 wu = *reinterpret_cast<const uint2*>(qu + off);
+                            const uint2 wv = *reinterpret_cast<const uint2*>(qv + off);
+                            const float2 u0 = bf16x2_to_f2(wu.x), u1 = bf16x2_to_f2(wu.y);
+                            const float2 v0 = bf16x2_to_f2(wv.x), v1 = bf16x2_to_f2(wv.y);
+                            u[j][0] = u0.x; u[j][1] = u0.y; u[j][2] = u1.x; u[j][3] = u1.y;
+                            v[j][0] = v0.x; v[j][1] = v0.y; v[j][2] = v1.x; v[j][3] = v1.y;
+                        } else {
+                            const uint4 wu = *reinterpret_cast<const uint4*>(qu + off);
+                            const uint4 wv = *reinterpret_cast<const uint4*>(qv + off);
+                            const uint32_t au[4] = {wu.x, wu.y, wu.z, wu.w};
+                            const uint32_t av[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
                             for (int m = 0; m < 4; ++m) {
-                                const float2 f = bf16x2_to_f2(ww[m]);
-                                ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                                const float2 fu = bf16x2_to_f2(au[m]), fv = bf16x2_to_f2(av[m]);
+                                u[j][2 * m] = fu.x; u[j][2 * m + 1] = fu.y;
+                                v[j][2 * m] = fv.x; v[j][2 * m + 1] = fv.y;
                             }
                         }
                     }
-                    inv = 1.0f / sqrtf(ss / (float)D + a.eps);
-                }
-                for (int c = 0; c < NCH / 2; ++c) {
-                    const int c2i = c + NCH / 2;   // partner chunk: dims + d/2
-#pragma unroll 2
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = sw128_offset(r, 8 * k);
-                        const uint4 wu = *reinterpret_cast<const uint4*>(sm.q[c] + off);
-                        const uint4 wv = *reinterpret_cast<const uint4*>(sm.q[c2i] + off);
-                        const uint32_t uu[4] = {wu.x, wu.y, wu.z, wu.w};
-                        const uint32_t vv[4] = {wv.x, wv.y, wv.z, wv.w};
-                        uint32_t ou[4], ov[4];
+                    if (a.qk_norm) {
+                        float ss[NB];
 #pragma unroll
-                        for (int m = 0; m < 4; ++m) {
-                            const float2 u = bf16x2_to_f2(uu[m]);
-                            const float2 v = bf16x2_to_f2(vv[m]);
-                            float xo[2], yo[2];
-                            const float ux[2] = {u.x, u.y}, vx[2] = {v.x, v.y};
+                        for (int j = 0; j < NB; ++j) {
+                            ss[j] = 0.f;
 #pragma unroll
-                            for (int e = 0; e < 2; ++e) {
-                                const int i = c * 64 + 8 * k + 2 * m + e;
-                                float x = ux[e], y = vx[e];
-                                if (a.qk_norm) {
-                                    x = x * inv * a.gamma_q[i];
-                                    y = y * inv * a.gamma_q[half + i];
-                                }
-                                if (i < R) {
-                                    const float2 cs = cs_row[i];
-                                    const float x2 = x * cs.x - y * cs.y;
-                                    y = x * cs.y + y * cs.x;
-                                    x = x2;
-                                }
-                                xo[e] = x;
-                                yo[e] = y;
-                            }
-                            ou[m] = pack_f16x2(xo[0], xo[1]);
-                            ov[m] = pack_f16x2(yo[0], yo[1]);
+                            for (int k = 0; k < H; ++k)
+                                ss[j] = fmaf(u[j][k], u[j][k], fmaf(v[j][k], v[j][k], ss[j]));
                         }
-                        *reinterpret_cast<uint4*>(sm.q[c] + off) = make_uint4(ou[0], ou[1], ou[2], ou[3]);
-                        *reinterpret_cast<uint4*>(sm.q[c2i] + off) = make_uint4(ov[0], ov[1], ov[2], ov[3]);
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                            for (int j = 0; j < NB; ++j) ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], o);
+#pragma unroll
+                        for (int j = 0; j < NB; ++j) {
+                            const float inv = 1.0f / sqrtf(ss[j] / (float)D + a.eps);
+#pragma unroll
+                            for (int k = 0; k < H; ++k) {
+                                u[j][k] = u[j][k] * inv * gu[k];
+                                v[j][k] = v[j][k] * inv * gv[k];
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < NB; ++j) {
+                        const int r = r0 + j;
+                        // rows past the end of the sequence hold zeros (TMA fill) and have no
+                        // (cos, sin) row in the table: they skip the rotation
+                        if (rot_lane && r / G < pg.tq) {
+                            const float2* cs = cs_base + (size_t)(r / G) * R + i0;
+#pragma unroll
+                            for (int k = 0; k < H; ++k) {
+                                if (i0 + k < R) {
+                                    const float2 c = cs[k];
+                                    const float x = u[j][k] * c.x - v[j][k] * c.y;
+                                    v[j][k] = u[j][k] * c.y + v[j][k] * c.x;
+                                    u[j][k] = x;
+                                }
+                            }
+                        }
+                        const uint32_t off = sw128_offset(r, col);
+                        if constexpr (H == 4) {
+                            *reinterpret_cast<uint2*>(qu + off) =
+                                make_uint2(pack_f16x2(u[j][0], u[j][1]), pack_f16x2(u[j][2], u[j][3]));
+                            *reinterpret_cast<uint2*>(qv + off) =
+                                make_uint2(pack_f16x2(v[j][0], v[j][1]), pack_f16x2(v[j][2], v[j][3]));
+                        } else {
+                            *reinterpret_cast<uint4*>(qu + off) =
+                                make_uint4(pack_f16x2(u[j][0], u[j][1]), pack_f16x2(u[j][2], u[j][3]),
+                                           pack_f16x2(u[j][4], u[j][5]), pack_f16x2(u[j][6], u[j][7]));
+                            *reinterpret_cast<uint4*>(qv + off) =
+                                make_uint4(pack_f16x2(v[j][0], v[j][1]), pack_f16x2(v[j][2], v[j][3]),
+                                           pack_f16x2(v[j][4], v[j][5]), pack_f16x2(v[j][6], v[j][7]));
+                        }
                     }
                 }
             }
@@ -454,13 +495,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // band or the window) are dropped element by element, head_dim 512 (registers
             // full with the O quarter) takes masked tiles on the two-pass path
             bool slow = (C::SWAP && need_mask) || !__all_sync(0xffffffffu, m_ref != -INFINITY);
+            bool fresh = false;   // the reference was set from this tile's row max
             // one pass over S with the current reference; MASK: drop keys outside the causal
             // band or the window element by element (a separate copy of the loop, so unmasked
             // tiles carry no per-element test)
-            auto one_pass = [&](auto mask_tag, float& mxr) {
+            auto one_pass = [&](auto mask_tag, float negm, float& mxr) {
                 constexpr bool MASK = decltype(mask_tag)::value;
                 uint32_t sa[32], sb[32];
-                const float negm = -m_ref;
                 tmem_ld32_nowait(tm_sn + lane_off, sa);
                 tmem_ld_wait();
 #pragma unroll
@@ -499,13 +540,55 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (b < 3) tmem_ld_wait();
                 }
             };
+            if (slow && !(C::SWAP && need_mask)) {
+                // first tile of a row: the row max of the visible scores sets the reference,
+                // then the one-pass loop below runs with it.  A row with no visible key here
+                // keeps a -inf reference; its masked scores give P = 0 whatever the stand-in.
+                auto max_pass = [&](auto mask_tag) -> float {
+                    constexpr bool MASK = decltype(mask_tag)::value;
+                    uint32_t sa[32], sb[32];
+                    float mx = -INFINITY;
+                    tmem_ld32_nowait(tm_sn + lane_off, sa);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int b = 0; b < 4; ++b) {
+                        uint32_t* cur = (b & 1) ? sb : sa;
+                        uint32_t* nxt = (b & 1) ? sa : sb;
+                        if (b < 3) tmem_ld32_nowait(tm_sn + (b + 1) * 32 + lane_off, nxt);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            float sv = __uint_as_float(cur[e]);
+                            if constexpr (MASK) {
+                                const int j = key0 + b * 32 + e;
+                                if (!(j <= tok_r && j >= lo_r)) sv = -INFINITY;
+                            }
+                            mx = fmaxf(mx, sv);
+                        }
+                        if (b < 3) tmem_ld_wait();
+                    }
+                    return mx * c2;
+                };
+                float mx;
+                if constexpr (C::SWAP) mx = max_pass(std::false_type{});   // unmasked here
+                else mx = need_mask ? max_pass(std::true_type{}) : max_pass(std::false_type{});
+                if (!row_valid) mx = -INFINITY;
+                if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
+                    alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
+                    m_ref = mx;
+                }
+                slow = false;
+                fresh = true;
+            }
             if (!slow) {
                 float mxr = -INFINITY;
-                if (!C::SWAP && need_mask) one_pass(std::true_type{}, mxr);
-                else one_pass(std::false_type{}, mxr);
+                const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+                if (!C::SWAP && need_mask) one_pass(std::true_type{}, negm, mxr);
+                else one_pass(std::false_type{}, negm, mxr);
                 // the reference stays unless this tile's max exceeds it by more than 2^8
-                slow = __any_sync(0xffffffffu, mxr * c2 > m_ref + kLazyMax);
-                if (slow) psum = 0.f;
+                if (!fresh) {
+                    slow = __any_sync(0xffffffffu, mxr * c2 > m_ref + kLazyMax);
+                    if (slow) psum = 0.f;
+                }
             }
             if (slow) {
                 // two passes with masks: row max, then P with a (lazily) updated reference

@@ -43,6 +43,25 @@ def test_global_prefill_separate_values():
     check_prefill(_inp(1, 140, ly, 5), ly, what="global separate v")
 
 
+def test_global_prefill_full_rope_cos_sin_from_table():
+    # full RoPE at head_dim 512: the (cos, sin) rows are too wide for the TMA staging, so the
+    # prologue reads them from the workspace table; T = 37 leaves a ragged last row tile
+    ly = workloads.with_layer(TINY, rope_p=1.0)
+    check_prefill(_inp(1, 37, ly, 8), ly, what="global full RoPE T=37")
+
+
+def test_local_prefill_one_query_head_per_kv_head():
+    # G = 1: 128 tokens per row tile, whose (cos, sin) rows also come from the table
+    ly = workloads.with_layer(LOCAL, n_q_heads=8, n_kv_heads=8, window=100)
+    check_prefill(_inp(1, 201, ly, 9), ly, what="local G=1 T=201 W=100")
+
+
+def test_prefill_without_qknorm():
+    check_prefill(_inp(1, 150, TINY, 10), TINY, what="global no QKNorm", qk_norm=0)
+    ly = workloads.with_layer(LOCAL, window=64)
+    check_prefill(_inp(1, 150, ly, 11), ly, what="local no QKNorm", qk_norm=0)
+
+
 @pytest.mark.parametrize("T,W", [(700, 512), (333, 100), (130, 1)])
 def test_local_prefill_window(T, W):
     ly = workloads.with_layer(LOCAL, window=W)
