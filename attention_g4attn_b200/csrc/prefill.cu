@@ -257,22 +257,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (n == ntiles - 1) mma_commit_pair(&sm.o_done);
                 }
             } else {
-                // tile n's slots sit at ring positions 4n .. 4n + 3 (S stages, then V); the
-                // MMAs take S(n) before O += P(n-1) V(n-1)
+                // tile n's slots sit at ring positions 4n .. 4n + 3 (S stages, then V).  The
+                // thread issues whichever product is ready, the scores of the next tile first:
+                // a value product never waits behind the key loads of a later score product,
+                // and its slots go back to the producer as early as possible.
                 if (!mbar_wait(&sm.q_ready, 0, wc, abort)) goto done;
                 constexpr int SPT = C::NS + 2 * C::NV;   // slots per tile
-                for (int n = 0; n <= ntiles; ++n) {
-                    if (n < ntiles) {
-                        const uint32_t b = n & 1;
-                        // S buffer b was last read by the softmax of tile n - 2
-                        if (n >= 2 && !mbar_wait(&sm.s_free[b], ((n - 2) >> 1) & 1, wc, abort))
-                            goto done;
+                auto slots_full = [&](uint32_t q0, int cnt) {
+                    for (int k = 0; k < cnt; ++k) {
+                        const uint32_t q = q0 + (uint32_t)k;
+                        if (!mbar_test_wait(&sm.full[q % NSLOT], (q / NSLOT) & 1)) return false;
+                    }
+                    return true;
+                };
+                int sc = 0, pc = 0;   // next tile of the score product / of the value product
+                long long polls = 0;
+                unsigned long long t_idle = 0;
+                while (pc < ntiles) {
+                    // S(sc) into buffer sc & 1, last read by the softmax of tile sc - 2
+                    if (sc < ntiles &&
+                        (sc < 2 || mbar_test_wait(&sm.s_free[sc & 1], ((sc - 2) >> 1) & 1)) &&
+                        slots_full((uint32_t)(sc * SPT), C::NS)) {
+                        const uint32_t b = sc & 1;
                         tc_fence_after();
                         for (int s = 0; s < C::NS; ++s) {
-                            const uint32_t q = (uint32_t)(n * SPT + s), slot = q % NSLOT;
-                            if (!mbar_wait(&sm.full[slot], (q / NSLOT) & 1, wc, abort))
-                                goto done;
-                            tc_fence_after();
+                            const uint32_t slot = (uint32_t)(sc * SPT + s) % NSLOT;
                             for (int kk = 0; kk < 8; ++kk) {
                                 const uint32_t ab = smem_u32(sm.q[2 * s + (kk >> 2)]) + (kk & 3) * 32;
                                 const uint32_t bb = smem_u32(sm.ring[slot]) + (kk >> 2) * (kSlot / 2) +
@@ -284,31 +293,44 @@ __global__ void __launch_bounds__(kThreads, 1)
                             mma_commit_pair(&sm.empty[slot]);
                         }
                         mma_commit_pair(&sm.s_full[b]);
+                        ++sc;
+                        polls = 0;
+                        continue;
                     }
-                    if (n >= 1) {
-                        const int j = n - 1;
-                        const uint32_t pb = j & 1;
-                        if (!mbar_wait(&sm.p_full[pb], (j >> 1) & 1, wc, abort)) goto done;
+                    // O += P(pc) V(pc) once both CTAs wrote P(pc) and its value slots landed
+                    if (pc < sc && mbar_test_wait(&sm.p_full[pc & 1], (pc >> 1) & 1) &&
+                        slots_full((uint32_t)(pc * SPT + C::NS), 2 * C::NV)) {
+                        const uint32_t pb = pc & 1;
                         tc_fence_after();
                         for (int v = 0; v < C::NV; ++v) {
-                            const uint32_t q = (uint32_t)(j * SPT + C::NS + 2 * v);
+                            const uint32_t q = (uint32_t)(pc * SPT + C::NS + 2 * v);
                             const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
-                            if (!mbar_wait(&sm.full[s0], (q / NSLOT) & 1, wc, abort)) goto done;
-                            if (!mbar_wait(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
-                                goto done;
-                            tc_fence_after();
                             const uint32_t vb = smem_u32(sm.ring[s0]);
                             for (int kk = 0; kk < 8; ++kk) {
                                 const uint32_t pa = smem_u32(sm.p[pb][kk >> 2]) + (kk & 3) * 32;
                                 mma_pair_f16(tm_o + v * 256, sdesc_sw128(pa, 16, 1024),
                                              sdesc_sw128(vb + kk * 2048, kSlot, 1024), idesc_o,
-                                             (j > 0 || kk > 0) ? 1u : 0u);
+                                             (pc > 0 || kk > 0) ? 1u : 0u);
                             }
                             mma_commit_pair(&sm.empty[s0]);
                             mma_commit_pair(&sm.empty[s1]);
                         }
                         mma_commit_pair(&sm.pv_done[pb]);
-                        if (j == ntiles - 1) mma_commit_pair(&sm.o_done);
+                        if (pc == ntiles - 1) mma_commit_pair(&sm.o_done);
+                        ++pc;
+                        polls = 0;
+                        continue;
+                    }
+                    // nothing ready: bounded polling, like every other wait
+                    if (*abort) goto done;
+                    if ((++polls & 63) == 0) {
+                        const unsigned long long now = global_ns();
+                        if (polls == 64) t_idle = now;
+                        if (polls >= a.wait_limit || now - t_idle > kWaitTimeoutNs) {
+                            atomicExch(a.status, (int)G4ATTN_ERR_TIMEOUT);
+                            *abort = 1;
+                            goto done;
+                        }
                     }
                 }
             }
@@ -344,9 +366,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 gu[k] = a.qk_norm ? a.gamma_q[i0 + k] : 1.f;
                 gv[k] = a.qk_norm ? a.gamma_q[half + i0 + k] : 1.f;
             }
-            const float2* const cs_base =
-                a.cs_tma ? reinterpret_cast<const float2*>(&sm.p[0][0][0]) : a.rope_cs + (size_t)pg.m0 * R;
+            const float2* const cs_smem = reinterpret_cast<const float2*>(&sm.p[0][0][0]);
+            const float2* const cs_glob = a.rope_cs + (size_t)pg.m0 * R;
             const bool rot_lane = i0 < R;
+            const int lgG = __ffs(G) - 1;          // G divides 128 (host check): a power of two
             ok_pro = group_all(mbar_wait(&sm.q_full, 0, wc, abort), kBarWG, 128);
             if (ok_pro) {
                 // NB rows per step, each stage over all of them, so the rows' load, warp-sum
@@ -393,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             for (int j = 0; j < NB; ++j) ss[j] += __shfl_xor_sync(0xffffffffu, ss[j], o);
 #pragma unroll
                         for (int j = 0; j < NB; ++j) {
-                            const float inv = 1.0f / sqrtf(ss[j] / (float)D + a.eps);
+                            const float inv = rsqrtf(ss[j] / (float)D + a.eps);
 #pragma unroll
                             for (int k = 0; k < H; ++k) {
                                 u[j][k] = u[j][k] * inv * gu[k];
@@ -406,12 +429,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int r = r0 + j;
                         // rows past the end of the sequence hold zeros (TMA fill) and have no
                         // (cos, sin) row in the table: they skip the rotation
-                        if (rot_lane && r / G < pg.tq) {
-                            const float2* cs = cs_base + (size_t)(r / G) * R + i0;
+                        if (rot_lane && (r >> lgG) < pg.tq) {
+                            const size_t cso = (size_t)(r >> lgG) * R + i0;
 #pragma unroll
                             for (int k = 0; k < H; ++k) {
                                 if (i0 + k < R) {
-                                    const float2 c = cs[k];
+                                    // shared-memory rows (TMA) or the workspace table
+                                    const float2 c = a.cs_tma ? cs_smem[cso + k] : cs_glob[cso + k];
                                     const float x = u[j][k] * c.x - v[j][k] * c.y;
                                     v[j][k] = u[j][k] * c.y + v[j][k] * c.x;
                                     u[j][k] = x;
