@@ -92,8 +92,14 @@ __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs& a, uint32_t ran
     const int pairs = (mt_count + 1) / 2;
     const int c = blockIdx.x >> 1;                      // cluster index
     const int bgn = a.B * a.Hkv;
-    const int pr = pairs - 1 - c / bgn;                 // heavy (late) row tiles first
-    const int bg = c % bgn;
+    // Causal layers: all row tiles of one (batch, kv head) in a row, heavy (late) tiles first,
+    // so the pairs in flight stream the keys of one head (about 80 MB at T = 65536, inside
+    // L2) instead of all heads at staggered positions: DRAM reads of a T = 65536 launch fell
+    // from 269 GB to 6.3 GB and its time from 164 to 141 ms.  Sliding-window layers read a
+    // short band per pair; there interleaving the heads measured faster.
+    const bool head_major = a.window <= 0;
+    const int pr = head_major ? pairs - 1 - c % pairs : pairs - 1 - c / bgn;
+    const int bg = head_major ? c / pairs : c % bgn;
     g.b = bg / a.Hkv;
     g.g = bg % a.Hkv;
     const int mt = 2 * pr + (int)rank;
