@@ -218,6 +218,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0 && leader) {
             const uint32_t idesc_s = idesc_f16kind_f32(256, kBN, false, false, false);
             const uint32_t idesc_o = idesc_f16kind_f32(256, 256, false, true, !PF16);
+            // shared-memory descriptors of the first buffer of each kind; an operand's start
+            // address field (16-byte units) is advanced by adding to the descriptor
+            const uint64_t dq0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
+            const uint64_t dr0 = sdesc_sw128(smem_u32(sm.ring[0]), 16, 1024);
+            const uint64_t dp0 = sdesc_sw128(smem_u32(sm.p[0][0]), 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(smem_u32(sm.ring[0]), kSlot, 1024);   // V: MN-major
+            constexpr uint32_t kChunkD = 16384 >> 4, kSlotD = kSlot >> 4, kHalfD = (kSlot / 2) >> 4;
             if constexpr (C::SWAP) {
                 uint32_t q = 0;
                 for (int n = 0; n < ntiles; ++n) {
@@ -227,13 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const uint32_t slot = q % NSLOT;
                         if (!mbar_wait(&sm.full[slot], (q / NSLOT) & 1, wc, abort)) goto done;
                         tc_fence_after();
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t ab = smem_u32(sm.q[2 * s + (kk >> 2)]) + (kk & 3) * 32;
-                            const uint32_t bb =
-                                smem_u32(sm.ring[slot]) + (kk >> 2) * (kSlot / 2) + (kk & 3) * 32;
-                            mma_pair_f16(tm_s, sdesc_sw128(ab, 16, 1024), sdesc_sw128(bb, 16, 1024),
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_pair_f16(tm_s, dq0 + (2 * s + (kk >> 2)) * kChunkD + (kk & 3) * 2,
+                                         dr0 + slot * kSlotD + (kk >> 2) * kHalfD + (kk & 3) * 2,
                                          idesc_s, (s | kk) != 0 ? 1u : 0u);
-                        }
                         mma_commit_pair(&sm.empty[slot]);
                     }
                     mma_commit_pair(&sm.s_full[0]);
@@ -245,15 +250,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                         if (!mbar_wait(&sm.full[s1], ((q + 1) / NSLOT) & 1, wc, abort))
                             goto done;
                         tc_fence_after();
-                        const uint32_t vb = smem_u32(sm.ring[s0]);
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const uint32_t pa = smem_u32(sm.p[0][kk >> 2]) + (kk & 3) * 32;
-                            // V: 16 keys per step (two 8-row groups of 1024 B); the CTA's second
-                            // 64-dim chunk sits in the next slot (LBO)
-                            mma_pair_f16(tm_o + v * 256, sdesc_sw128(pa, 16, 1024),
-                                         sdesc_sw128(vb + kk * 2048, kSlot, 1024), idesc_o,
+                        // V: 16 keys per step (two 8-row groups of 1024 B); the CTA's second
+                        // 64-dim chunk sits in the next slot (LBO)
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            mma_pair_f16(tm_o + v * 256, dp0 + (kk >> 2) * kChunkD + (kk & 3) * 2,
+                                         dv0 + s0 * kSlotD + kk * (2048 >> 4), idesc_o,
                                          (n > 0 || kk > 0) ? 1u : 0u);
-                        }
                         mma_commit_pair(&sm.empty[s0]);
                         mma_commit_pair(&sm.empty[s1]);
                         // the O quarter that S borrows lies in block 0: the softmax warps can
@@ -288,14 +291,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tc_fence_after();
                         for (int s = 0; s < C::NS; ++s) {
                             const uint32_t slot = (uint32_t)(sc * SPT + s) % NSLOT;
-                            for (int kk = 0; kk < 8; ++kk) {
-                                const uint32_t ab = smem_u32(sm.q[2 * s + (kk >> 2)]) + (kk & 3) * 32;
-                                const uint32_t bb = smem_u32(sm.ring[slot]) + (kk >> 2) * (kSlot / 2) +
-                                                    (kk & 3) * 32;
-                                mma_pair_f16(tm_s + 128 * b, sdesc_sw128(ab, 16, 1024),
-                                             sdesc_sw128(bb, 16, 1024), idesc_s,
-                                             (s | kk) != 0 ? 1u : 0u);
-                            }
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_pair_f16(tm_s + 128 * b,
+                                             dq0 + (2 * s + (kk >> 2)) * kChunkD + (kk & 3) * 2,
+                                             dr0 + slot * kSlotD + (kk >> 2) * kHalfD + (kk & 3) * 2,
+                                             idesc_s, (s | kk) != 0 ? 1u : 0u);
                             mma_commit_pair(&sm.empty[slot]);
                         }
                         mma_commit_pair(&sm.s_full[b]);
@@ -311,13 +312,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int v = 0; v < C::NV; ++v) {
                             const uint32_t q = (uint32_t)(pc * SPT + C::NS + 2 * v);
                             const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
-                            const uint32_t vb = smem_u32(sm.ring[s0]);
-                            for (int kk = 0; kk < 8; ++kk) {
-                                const uint32_t pa = smem_u32(sm.p[pb][kk >> 2]) + (kk & 3) * 32;
-                                mma_pair_f16(tm_o + v * 256, sdesc_sw128(pa, 16, 1024),
-                                             sdesc_sw128(vb + kk * 2048, kSlot, 1024), idesc_o,
+#pragma unroll
+                            for (int kk = 0; kk < 8; ++kk)
+                                mma_pair_f16(tm_o + v * 256,
+                                             dp0 + (2 * pb + (kk >> 2)) * kChunkD + (kk & 3) * 2,
+                                             dv0 + s0 * kSlotD + kk * (2048 >> 4), idesc_o,
                                              (pc > 0 || kk > 0) ? 1u : 0u);
-                            }
                             mma_commit_pair(&sm.empty[s0]);
                             mma_commit_pair(&sm.empty[s1]);
                         }
