@@ -354,11 +354,11 @@ int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16
     if ((rc = encode_q_tile(&a.tm_q, q, B, T, cfg->n_q_heads, d, G))) return rc;
     {
         // the (cos, sin) rows of a row tile go to shared memory by TMA when they fit the
-        // P buffers (free during the prologue) and the row pitch suits TMA
+        // staging room (free during the prologue) and the row pitch suits TMA
         const int R = rope_pairs(cfg), rows = 128 / G;
         const size_t bytes = (size_t)rows * R * 8;
         a.cs_tma = R > 0 && R % 2 == 0 && 2 * R <= 256 && rows <= 256 &&
-                   bytes <= g4::prefill_p_bytes(d);
+                   bytes <= g4::prefill_cs_stage_bytes(d);
         if (a.cs_tma && (rc = encode_cs_rows(&a.tm_cs, cs, T, R, rows))) return rc;
     }
     a.q = q;

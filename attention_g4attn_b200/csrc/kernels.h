@@ -90,6 +90,6 @@ struct PrefillArgs {
 
 cudaError_t launch_prefill(const PrefillArgs& a, cudaStream_t stream);
 size_t prefill_smem_bytes(int d);
-size_t prefill_p_bytes(int d);   // bytes of the P buffers (staging room during the prologue)
+size_t prefill_cs_stage_bytes(int d);   // room for the (cos, sin) rows staged in the prologue
 
 }  // namespace g4

@@ -51,25 +51,40 @@ template <int D>
 struct PrefillCfg {
     static constexpr int NCH = D / 64;
     static constexpr bool SWAP = (D == 512);
-    static constexpr int NSLOT = (D == 512) ? 4 : 6;
+    // head_dim 256: P lives in tensor memory over the scores it came from, so the shared
+    // memory of P buffers goes to the ring (10 slots, 2.5 tiles)
+    static constexpr int NSLOT = (D == 512) ? 4 : 10;
     static constexpr uint32_t S_COL = (D == 512) ? 128 : 256;
-    // head_dim 256: two S buffers (columns 256 and 384) and two P buffers, so the scores of
-    // tile n + 1 are computed while the softmax works on tile n
+    // head_dim 256: two S buffers (columns 256 and 384), so the scores of tile n + 1 are
+    // computed while the softmax works on tile n; P(n) overwrites the first 64 columns of
+    // S(n) as packed bf16 / fp16 and is the tensor-memory A operand of P.V
     static constexpr int NBUF = (D == 512) ? 1 : 2;
+    // the (cos, sin) rows of the query tile are staged by TMA during the prologue: in the P
+    // buffer (head_dim 512) or in the last four ring slots (head_dim 256)
+    static constexpr int CS_SLOT0 = NSLOT - 4;
     static constexpr int NS = D / 128;     // S stages per tile (128 dims each)
     static constexpr int NV = D / 256;     // P.V blocks per tile (2 slots each)
 };
 
+// head_dim 512 keeps P in shared memory (128 rows x 64 keys per chunk): its S borrows O
+// columns, and P.V writes all of them
 template <int D>
-struct __align__(1024) PrefillSmem {
+struct PrefillPArea {
+    uint8_t p[1][2][16384];
+};
+template <>
+struct PrefillPArea<256> {};
+
+template <int D>
+struct __align__(1024) PrefillSmem : PrefillPArea<D> {
     uint8_t q[PrefillCfg<D>::NCH][16384];  // 128 rows x 64 dims per chunk
-    uint8_t p[PrefillCfg<D>::NBUF][2][16384];   // P: 128 rows x 64 keys per chunk
     uint8_t ring[PrefillCfg<D>::NSLOT][kSlot];
     uint64_t full[PrefillCfg<D>::NSLOT];   // used in the leader: both CTAs' bytes land here
     uint64_t empty[PrefillCfg<D>::NSLOT];  // per CTA, released by the leader's MMA commits
     // per buffer (tile n uses [n % NBUF]); s_free / p_full / q_ready count one arrival per CTA
     uint64_t s_free[2], s_full[2], p_full[2], pv_done[2];
     uint64_t q_full, q_ready, o_done, o1_done, drain;
+    uint64_t pro_done;                     // this CTA's prologue is done with its staging area
     uint32_t tmem_base;
     int abort;
 };
@@ -148,6 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sm.o_done, 1);
         mbar_init(&sm.o1_done, 1);   // head_dim 512: the first 256-dim block of P.V is done
         mbar_init(&sm.drain, 1);
+        mbar_init(&sm.pro_done, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -158,6 +174,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = sm.tmem_base;
     const uint32_t tm_o = tmem;
     const uint32_t tm_s = tmem + C::S_COL;   // S buffer b at tm_s + 128 b
+    uint8_t* cs_stage;
+    if constexpr (C::SWAP) cs_stage = &sm.p[0][0][0];
+    else cs_stage = &sm.ring[C::CS_SLOT0][0];
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -169,14 +188,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             prefetch_tmap(&a.tm_v);
             {
                 // the raw query tile (one box per 64-dim chunk, rows = token * G + head) and
-                // the (cos, sin) rows of its tokens; the P buffers hold the latter until the
-                // prologue is done
+                // the (cos, sin) rows of its tokens, staged until the prologue is done
                 const int tpt = kBM / a.G;
                 const uint32_t cs_bytes = a.cs_tma ? (uint32_t)(tpt * R * 8) : 0u;
                 mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(NCH * 16384) + cs_bytes);
                 for (int c = 0; c < NCH; ++c)
                     tma_load_4d(sm.q[c], &a.tm_q, &sm.q_full, c * 64, pg.g * a.G, pg.m0, pg.b);
-                if (a.cs_tma) tma_load_2d(&sm.p[0][0][0], &a.tm_cs, &sm.q_full, 0, pg.m0);
+                if (a.cs_tma) tma_load_2d(cs_stage, &a.tm_cs, &sm.q_full, 0, pg.m0);
             }
             uint32_t q = 0;
             for (int n = 0; n < ntiles && !*abort; ++n) {
@@ -189,6 +207,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 for (int s = 0; s < C::NS && !*abort; ++s, ++q) {
                     const int slot = q % NSLOT;
+                    // the staging slots take keys only after this CTA's prologue used them
+                    if (!C::SWAP && a.cs_tma && q == (uint32_t)C::CS_SLOT0 &&
+                        !mbar_wait(&sm.pro_done, 0, wc, abort))
+                        break;
                     if (!mbar_wait(&sm.empty[slot], ((q / NSLOT) & 1) ^ 1, wc, abort)) break;
                     if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlot);
                     for (int h = 0; h < 2; ++h) {
@@ -201,6 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int v = 0; v < C::NV && !*abort; ++v)
                     for (int u = 0; u < 2 && !*abort; ++u, ++q) {
                         const int slot = q % NSLOT;
+                        if (!C::SWAP && a.cs_tma && q == (uint32_t)C::CS_SLOT0 &&
+                            !mbar_wait(&sm.pro_done, 0, wc, abort))
+                            break;
                         if (!mbar_wait(&sm.empty[slot], ((q / NSLOT) & 1) ^ 1, wc, abort)) break;
                         if (leader) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlot);
                         const int c = 4 * v + 2 * (int)rank + u;   // this CTA's half of the block
@@ -222,10 +247,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // address field (16-byte units) is advanced by adding to the descriptor
             const uint64_t dq0 = sdesc_sw128(smem_u32(sm.q[0]), 16, 1024);
             const uint64_t dr0 = sdesc_sw128(smem_u32(sm.ring[0]), 16, 1024);
-            const uint64_t dp0 = sdesc_sw128(smem_u32(sm.p[0][0]), 16, 1024);
             const uint64_t dv0 = sdesc_sw128(smem_u32(sm.ring[0]), kSlot, 1024);   // V: MN-major
             constexpr uint32_t kChunkD = 16384 >> 4, kSlotD = kSlot >> 4, kHalfD = (kSlot / 2) >> 4;
             if constexpr (C::SWAP) {
+                const uint64_t dp0 = sdesc_sw128(smem_u32(sm.p[0][0]), 16, 1024);
                 uint32_t q = 0;
                 for (int n = 0; n < ntiles; ++n) {
                     if (!mbar_wait(&sm.s_free[0], n & 1, wc, abort)) goto done;
@@ -269,7 +294,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // tile n's slots sit at ring positions 4n .. 4n + 3 (S stages, then V).  The
                 // thread issues whichever product is ready, the scores of the next tile first:
                 // a value product never waits behind the key loads of a later score product,
-                // and its slots go back to the producer as early as possible.
+                // and its slots go back to the producer as early as possible.  S(n) and then
+                // P(n) occupy TMEM buffer n & 1 until the value product of tile n is done.
                 if (!mbar_wait(&sm.q_ready, 0, wc, abort)) goto done;
                 constexpr int SPT = C::NS + 2 * C::NV;   // slots per tile
                 auto slots_full = [&](uint32_t q0, int cnt) {
@@ -283,9 +309,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 long long polls = 0;
                 unsigned long long t_idle = 0;
                 while (pc < ntiles) {
-                    // S(sc) into buffer sc & 1, last read by the softmax of tile sc - 2
+                    // S(sc) into buffer sc & 1, whose P(sc - 2) the value product of tile sc - 2
+                    // has read
                     if (sc < ntiles &&
-                        (sc < 2 || mbar_test_wait(&sm.s_free[sc & 1], ((sc - 2) >> 1) & 1)) &&
+                        (sc < 2 || mbar_test_wait(&sm.pv_done[sc & 1], ((sc - 2) >> 1) & 1)) &&
                         slots_full((uint32_t)(sc * SPT), C::NS)) {
                         const uint32_t b = sc & 1;
                         tc_fence_after();
@@ -304,7 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         polls = 0;
                         continue;
                     }
-                    // O += P(pc) V(pc) once both CTAs wrote P(pc) and its value slots landed
+                    // O += P(pc) V(pc) once both CTAs wrote P(pc) (tensor memory, over S(pc)) and
+                    // its value slots landed
                     if (pc < sc && mbar_test_wait(&sm.p_full[pc & 1], (pc >> 1) & 1) &&
                         slots_full((uint32_t)(pc * SPT + C::NS), 2 * C::NV)) {
                         const uint32_t pb = pc & 1;
@@ -313,11 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const uint32_t q = (uint32_t)(pc * SPT + C::NS + 2 * v);
                             const uint32_t s0 = q % NSLOT, s1 = (q + 1) % NSLOT;
 #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk)
-                                mma_pair_f16(tm_o + v * 256,
-                                             dp0 + (2 * pb + (kk >> 2)) * kChunkD + (kk & 3) * 2,
-                                             dv0 + s0 * kSlotD + kk * (2048 >> 4), idesc_o,
-                                             (pc > 0 || kk > 0) ? 1u : 0u);
+                            for (int kk = 0; kk < 8; ++kk)   // 16 keys = 8 packed P columns
+                                mma_pair_f16_ts(tm_o + v * 256, tm_s + 128 * pb + 8 * kk,
+                                                dv0 + s0 * kSlotD + kk * (2048 >> 4), idesc_o,
+                                                (pc > 0 || kk > 0) ? 1u : 0u);
                             mma_commit_pair(&sm.empty[s0]);
                             mma_commit_pair(&sm.empty[s1]);
                         }
@@ -372,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 gu[k] = a.qk_norm ? a.gamma_q[i0 + k] : 1.f;
                 gv[k] = a.qk_norm ? a.gamma_q[half + i0 + k] : 1.f;
             }
-            const float2* const cs_smem = reinterpret_cast<const float2*>(&sm.p[0][0][0]);
+            const float2* const cs_smem = reinterpret_cast<const float2*>(cs_stage);
             const float2* const cs_glob = a.rope_cs + (size_t)pg.m0 * R;
             const bool rot_lane = i0 < R;
             const int lgG = __ffs(G) - 1;          // G divides 128 (host check): a power of two
@@ -467,8 +494,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             fence_proxy_async_smem();
             group_sync(kBarWG, 128);
-            if (t128 == 0)   // Q ready (and, head_dim 512, S free for tile 0)
+            if (t128 == 0) {   // Q ready (and, head_dim 512, S free for tile 0)
                 mbar_arrive_remote(C::SWAP ? &sm.s_free[0] : &sm.q_ready, 0);
+                mbar_arrive(&sm.pro_done);   // the staged (cos, sin) rows are no longer read
+            }
         }
 
         // ---- main loop
@@ -508,13 +537,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                                    : mbar_wait(&sm.s_full[sbuf], (n >> 1) & 1, wc, abort),
                            kBarWG, 128);
             if (!ok) break;
-            if (!C::SWAP && n >= 2) {
-                // P buffer sbuf was last read by the value product of tile n - 2 (issued before
-                // this tile's scores, so already complete)
-                ok = group_all(mbar_wait(&sm.pv_done[sbuf], ((n - 2) >> 1) & 1, wc, abort),
-                               kBarWG, 128);
-                if (!ok) break;
-            }
             tc_fence_after();
             const bool need_mask = (key0 + kBN - 1 > t_first) ||
                                    (a.window > 0 && key0 <= t_last - a.window);
@@ -526,6 +548,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             // full with the O quarter) takes masked tiles on the two-pass path
             bool slow = (C::SWAP && need_mask) || !__all_sync(0xffffffffu, m_ref != -INFINITY);
             bool fresh = false;   // the reference was set from this tile's row max
+            // head_dim 256: P(n) overwrites S(n) in tensor memory, so it waits in registers
+            // (packed pairs) until the pass is known to stand
+            uint32_t pw[C::SWAP ? 1 : 64];
             // one pass over S with the current reference; MASK: drop keys outside the causal
             // band or the window element by element (a separate copy of the loop, so unmasked
             // tiles carry no per-element test)
@@ -561,19 +586,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                             w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
                         }
                     }
-                    uint8_t* pb = sm.p[sbuf][b >> 1];
-                    const int col = (b & 1) * 32;
+                    if constexpr (C::SWAP) {
+                        uint8_t* pb = sm.p[sbuf][b >> 1];
+                        const int col = (b & 1) * 32;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8 * k)) =
-                            make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                        for (int k = 0; k < 4; ++k)
+                            *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8 * k)) =
+                                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) pw[16 * b + k] = w[k];
+                    }
                     if (b < 3) tmem_ld_wait();
                 }
             };
+            for (;;) {
             if (slow && !(C::SWAP && need_mask)) {
-                // first tile of a row: the row max of the visible scores sets the reference,
-                // then the one-pass loop below runs with it.  A row with no visible key here
-                // keeps a -inf reference; its masked scores give P = 0 whatever the stand-in.
+                // first tile of a row (or, head_dim 256, a jump of the max): the row max of
+                // the visible scores sets the reference, then the one-pass loop below runs
+                // with it.  A row with no visible key here keeps a -inf reference; its masked
+                // scores give P = 0 whatever the stand-in.
                 auto max_pass = [&](auto mask_tag) -> float {
                     constexpr bool MASK = decltype(mask_tag)::value;
                     uint32_t sa[32], sb[32];
@@ -618,60 +650,72 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!fresh) {
                     slow = __any_sync(0xffffffffu, mxr * c2 > m_ref + kLazyMax);
                     if (slow) psum = 0.f;
+                    // head_dim 256: S is intact (P still in registers): the max pass again
+                    if constexpr (!C::SWAP)
+                        if (slow) continue;
                 }
             }
-            if (slow) {
-                // two passes with masks: row max, then P with a (lazily) updated reference
-                float mx = -INFINITY;
-#pragma unroll 1
-                for (int b = 0; b < 4; ++b) {
-                    uint32_t sv[32];
-                    tmem_ld32_nowait(tm_sn + b * 32 + lane_off, sv);
-                    tmem_ld_wait();
+            break;
+            }
+            if constexpr (!C::SWAP) {
+                // P(n) over the first 64 columns of S(n): the A operand of the value product
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const int j = key0 + b * 32 + e;
-                        const bool vis = !need_mask || (j <= tok_r && j >= lo_r);
-                        mx = fmaxf(mx, vis ? __uint_as_float(sv[e]) * c2 : -INFINITY);
-                    }
-                }
-                if (!row_valid) mx = -INFINITY;
-                if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
-                    alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
-                    m_ref = mx;
-                }
-                const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
-#pragma unroll 1
-                for (int b = 0; b < 4; ++b) {
-                    uint32_t sv[32];
-                    tmem_ld32_nowait(tm_sn + b * 32 + lane_off, sv);
-                    tmem_ld_wait();
-                    uint32_t w[16];
-#pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        float pv[2];
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const int j = key0 + b * 32 + e + u;
-                            const bool vis = row_valid && (!need_mask || (j <= tok_r && j >= lo_r));
-                            pv[u] = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, negm)) : 0.f;
-                        }
-                        if constexpr (PF16) {
-                            w[e / 2] = pack_f16x2(pv[0], pv[1]);
-                            psum += pv[0] + pv[1];
-                        } else {
-                            const __nv_bfloat162 h = __floats2bfloat162_rn(pv[0], pv[1]);
-                            const float2 f = __bfloat1622float2(h);
-                            psum += f.x + f.y;
-                            w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+                for (int b = 0; b < 4; ++b) tmem_st16_u32(tm_sn + 16 * b + lane_off, pw + 16 * b);
+            }
+            if constexpr (C::SWAP) {   // head_dim 512: masked tiles and jumps of the max
+                if (slow) {
+                    // two passes with masks: row max, then P with a (lazily) updated reference
+                    float mx = -INFINITY;
+    #pragma unroll 1
+                    for (int b = 0; b < 4; ++b) {
+                        uint32_t sv[32];
+                        tmem_ld32_nowait(tm_sn + b * 32 + lane_off, sv);
+                        tmem_ld_wait();
+    #pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int j = key0 + b * 32 + e;
+                            const bool vis = !need_mask || (j <= tok_r && j >= lo_r);
+                            mx = fmaxf(mx, vis ? __uint_as_float(sv[e]) * c2 : -INFINITY);
                         }
                     }
-                    uint8_t* pb = sm.p[sbuf][b >> 1];
-                    const int col = (b & 1) * 32;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8 * k)) =
-                            make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    if (!row_valid) mx = -INFINITY;
+                    if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
+                        alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
+                        m_ref = mx;
+                    }
+                    const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
+    #pragma unroll 1
+                    for (int b = 0; b < 4; ++b) {
+                        uint32_t sv[32];
+                        tmem_ld32_nowait(tm_sn + b * 32 + lane_off, sv);
+                        tmem_ld_wait();
+                        uint32_t w[16];
+    #pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            float pv[2];
+    #pragma unroll
+                            for (int u = 0; u < 2; ++u) {
+                                const int j = key0 + b * 32 + e + u;
+                                const bool vis = row_valid && (!need_mask || (j <= tok_r && j >= lo_r));
+                                pv[u] = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, negm)) : 0.f;
+                            }
+                            if constexpr (PF16) {
+                                w[e / 2] = pack_f16x2(pv[0], pv[1]);
+                                psum += pv[0] + pv[1];
+                            } else {
+                                const __nv_bfloat162 h = __floats2bfloat162_rn(pv[0], pv[1]);
+                                const float2 f = __bfloat1622float2(h);
+                                psum += f.x + f.y;
+                                w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
+                            }
+                        }
+                        uint8_t* pb = sm.p[sbuf][b >> 1];
+                        const int col = (b & 1) * 32;
+    #pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8 * k)) =
+                                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    }
                 }
             }
             l_sum = l_sum * alpha + psum;
@@ -702,17 +746,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int c = 0; c < 4; ++c) tmem_st32_nowait(tm_s + c * 32 + lane_off, o1 + c * 32);
                 tmem_st_wait();
             }
+            if constexpr (!C::SWAP) tmem_st_wait();   // P (and any rescaled O) in TMEM
             fence_proxy_async_smem();
             tc_fence_before();
             group_sync(kBarWG, 128);
-            if (t128 == 0) {
-                if constexpr (C::SWAP) {
-                    mbar_arrive_remote(&sm.p_full[0], 0);
-                } else {
-                    mbar_arrive_remote(&sm.s_free[sbuf], 0);   // S read: buffer reusable
-                    mbar_arrive_remote(&sm.p_full[sbuf], 0);
-                }
-            }
+            if (t128 == 0) mbar_arrive_remote(&sm.p_full[sbuf], 0);
         }
         // ---- epilogue
         if (ok) {
@@ -767,6 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D, bool PF16>
 cudaError_t run_prefill(const PrefillArgs& a, cudaStream_t stream) {
     const size_t smem = sizeof(PrefillSmem<D>) + 1024;
+    static_assert(sizeof(PrefillSmem<D>) + 1024 <= 227 * 1024, "prefill shared memory");
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D, PF16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -792,8 +831,8 @@ cudaError_t run_prefill(const PrefillArgs& a, cudaStream_t stream) {
 
 }  // namespace
 
-size_t prefill_p_bytes(int d) {
-    return d == 512 ? sizeof(PrefillSmem<512>::p) : sizeof(PrefillSmem<256>::p);
+size_t prefill_cs_stage_bytes(int d) {
+    return d == 512 ? sizeof(PrefillPArea<512>::p) : 4 * (size_t)kSlot;
 }
 
 size_t prefill_smem_bytes(int d) {
