@@ -173,34 +173,42 @@ PrefillWs prefill_ws(int B, int T, const g4attn_layer_cfg* c) {
     return w;
 }
 
-constexpr int kDecodeTile = 128;   // keys per decode pair-tile: splits are whole tiles
+constexpr int kDecodeTile = 128;   // keys per decode pair-tile
 
+// Stream-K split of a decode step: the B * Hkv sequences' pair-tiles form one flat range
+// of W tiles, cut evenly over P CTA pairs; a sequence is split into one segment per pair
+// that touches it, and every segment leaves two partials (one per CTA of its pair).
 struct DecodePlan {
-    int key_lo, splits, keys_per_split;
+    int key_lo, splits, tiles_per_seq, n_pairs;
+    long long total_tiles;
     size_t o_off, ml_off, total;
 };
 
-DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms) {
+// Most segments any sequence is cut into when W tiles (nt per sequence) go to P pairs.
+int max_segments(long long W, int nt, int nbg, int P) {
+    if (W <= 0 || P <= 0) return 0;
+    auto pair_of = [&](long long t) { return (int)(((t + 1) * P - 1) / W); };
+    int m = 0;
+    for (int bg = 0; bg < nbg; ++bg) {
+        const long long s0 = (long long)bg * nt;
+        const int n = pair_of(s0 + nt - 1) - pair_of(s0) + 1;
+        m = n > m ? n : m;
+    }
+    return m;
+}
+
+DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms, int max_pairs = 0) {
     DecodePlan p{};
     p.key_lo = (c->window > 0 && L > c->window) ? L - c->window : 0;
     const int len = L - p.key_lo;
-    const int tiles = (len + kDecodeTile - 1) / kDecodeTile;
     const int nbg = B * c->n_kv_heads;
-    int S = 1;
-    const int pairs = (sms > 1 ? sms : 148) / 2;   // the decode kernel runs on CTA pairs
-    if (tiles > 0 && nbg > 0) {
-        // enough items that every pair holds the same number of them
-        int a = nbg, b = pairs;
-        while (b) { int t = a % b; a = b; b = t; }
-        const int base = pairs / a;
-        S = base;
-        while (S > tiles) S = (S + 1) / 2;
-        if (S < 1) S = 1;
-    }
-    const int tps = tiles > 0 ? (tiles + S - 1) / S : 1;
-    p.keys_per_split = tps * kDecodeTile;
-    p.splits = len > 0 ? (len + p.keys_per_split - 1) / p.keys_per_split : 0;
-    // two partials per split: one from each CTA of the pair that runs it
+    p.tiles_per_seq = len > 0 ? (len + kDecodeTile - 1) / kDecodeTile : 0;
+    p.total_tiles = (long long)nbg * p.tiles_per_seq;
+    long long P = (sms > 1 ? sms : 148) / 2;   // the decode kernel runs on CTA pairs
+    if (max_pairs > 0 && P > max_pairs) P = max_pairs;
+    if (P > p.total_tiles) P = p.total_tiles;
+    p.n_pairs = (int)P;
+    p.splits = max_segments(p.total_tiles, p.tiles_per_seq, nbg, p.n_pairs);
     const size_t n = 2 * (size_t)(p.splits > 0 ? p.splits : 1) * B * c->n_q_heads;
     p.o_off = 0;
     p.ml_off = align256(n * c->head_dim * sizeof(float));
@@ -428,7 +436,9 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
     a.B = B; a.L = L; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d; a.G = G;
     a.key_lo = plan.key_lo;
     a.splits = plan.splits;
-    a.keys_per_split = plan.keys_per_split;
+    a.tiles_per_seq = plan.tiles_per_seq;
+    a.n_pairs = plan.n_pairs;
+    a.total_tiles = plan.total_tiles;
     a.rope = make_rope(cfg);
     a.scale_log2 = cfg->scale * 1.4426950408889634f;
     a.kv_is_k = cfg->kv_is_k;
@@ -438,9 +448,9 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
 }
 
 // Decode with no workspace argument and no allocation: the split partials go to the
-// library's fixed device scratch.  The split count is lowered until the partials fit; a
-// problem whose single-split partials (2 * B * Hq * (d + 2) fp32: one set per CTA of the
-// pair) exceed the scratch is refused.
+// library's fixed device scratch.  The number of CTA pairs (and with it the segments per
+// sequence) is lowered until the partials fit; a problem whose single-segment partials
+// (2 * B * Hq * (d + 2) fp32: one set per CTA of the pair) exceed the scratch is refused.
 int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
                           const g4attn_bf16* vcache, int L, g4attn_bf16* out, float* lse, int B,
                           const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
@@ -469,16 +479,8 @@ int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
         cap)
         return G4ATTN_ERR_TOO_LARGE;
     DecodePlan plan = decode_plan(B, L, cfg, dev->sms);
-    while (plan.total > cap && plan.splits > 1) {   // fewer, longer splits until they fit
-        const int len = L - plan.key_lo;
-        const int tiles = (len + kDecodeTile - 1) / kDecodeTile;
-        const int S = plan.splits - 1;
-        plan.keys_per_split = ((tiles + S - 1) / S) * kDecodeTile;
-        plan.splits = (len + plan.keys_per_split - 1) / plan.keys_per_split;
-        const size_t n = (size_t)plan.splits * per_split;
-        plan.ml_off = align256(n * cfg->head_dim * sizeof(float));
-        plan.total = plan.ml_off + align256(n * 2 * sizeof(float));
-    }
+    while (plan.total > cap && plan.n_pairs > 1)   // fewer pairs, fewer segments, until they fit
+        plan = decode_plan(B, L, cfg, dev->sms, plan.n_pairs / 2);
     if (plan.total > cap) return G4ATTN_ERR_TOO_LARGE;
     void* scratch = nullptr;
     if (g4::decode_scratch_ptr(&scratch) != cudaSuccess) return cuda_status(cudaErrorUnknown);
@@ -497,7 +499,9 @@ int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
     a.B = B; a.L = L; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d; a.G = G;
     a.key_lo = plan.key_lo;
     a.splits = plan.splits;
-    a.keys_per_split = plan.keys_per_split;
+    a.tiles_per_seq = plan.tiles_per_seq;
+    a.n_pairs = plan.n_pairs;
+    a.total_tiles = plan.total_tiles;
     a.rope = make_rope(cfg);
     a.scale_log2 = cfg->scale * 1.4426950408889634f;
     a.kv_is_k = cfg->kv_is_k;

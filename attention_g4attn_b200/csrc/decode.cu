@@ -1,9 +1,11 @@
 // decode.cu -- split-KV flash decoding for one new token per sequence against a bf16
 // K(=V) cache, on the 5th-generation tensor core (tcgen05) with TMA-fed shared memory.
 //
-// Work item = (split s, kv head g, batch b): keys [k0, k1) of one sequence and all G query
-// heads that share kv head g (GQA; explainer "GQA": 8 query heads per KV head in global
-// layers).  Two CTAs of a cluster share an item and stream it in pair-tiles of 128 keys:
+// Work item = a run of consecutive pair-tiles of one sequence (batch b, kv head g): keys
+// [k0, k1) and all G query heads that share kv head g (GQA; explainer "GQA": 8 query heads
+// per KV head in global layers).  The sequences' tiles form one flat range split evenly
+// over the CTA pairs (stream-K), so a pair meets one to three items and every pair the same
+// number of tiles; each item's results are one segment's partials of the combine.  Two CTAs of a cluster share an item and stream it in pair-tiles of 128 keys:
 // CTA r takes keys [64 r, 64 r + 64) of each pair-tile and keeps its own running softmax,
 // so each CTA's result is one partial of the split-KV combine.  A CTA's 64 keys sit in
 // shared memory as D/128 slots of 128 rows x 64 dims: in slot j, row k < 64 holds dims
@@ -97,17 +99,38 @@ struct Item {
     int s, g, b, k0, k1;
 };
 
-// Splits of one sequence are consecutive items, so concurrent pairs stream neighbouring
-// key ranges of the same (b, g).
-__device__ __forceinline__ Item item_of(const DecodeArgs& a, int it) {
+// The pair that owns flat tile t: the largest p with p * total / n_pairs <= t.
+__device__ __forceinline__ int pair_of_tile(const DecodeArgs& a, long long t) {
+    return (int)(((t + 1) * a.n_pairs - 1) / a.total_tiles);
+}
+
+// This pair's flat tile range and the sequences it touches.
+struct PairRange {
+    long long t0, t1;
+    int bg0, n_items;
+};
+
+__device__ __forceinline__ PairRange pair_range(const DecodeArgs& a, int pair) {
+    PairRange r;
+    r.t0 = (long long)pair * a.total_tiles / a.n_pairs;
+    r.t1 = (long long)(pair + 1) * a.total_tiles / a.n_pairs;
+    r.bg0 = (int)(r.t0 / a.tiles_per_seq);
+    r.n_items = r.t1 > r.t0 ? (int)((r.t1 - 1) / a.tiles_per_seq) - r.bg0 + 1 : 0;
+    return r;
+}
+
+// Item k of the pair: its part of sequence bg0 + k, and which segment of that sequence it is.
+__device__ __forceinline__ Item item_of(const DecodeArgs& a, int pair, const PairRange& pr, int k) {
     Item r;
-    r.s = it % a.splits;
-    const int bg = it / a.splits;
+    const int bg = pr.bg0 + k;
+    const long long s0 = (long long)bg * a.tiles_per_seq;
+    const long long lo = pr.t0 > s0 ? pr.t0 : s0;
+    const long long hi = pr.t1 < s0 + a.tiles_per_seq ? pr.t1 : s0 + a.tiles_per_seq;
     r.g = bg % a.Hkv;
     r.b = bg / a.Hkv;
-    r.k0 = a.key_lo + r.s * a.keys_per_split;
-    r.k1 = min(a.L, r.k0 + a.keys_per_split);
-    if (r.k1 < r.k0) r.k1 = r.k0;
+    r.s = pair - pair_of_tile(a, s0);
+    r.k0 = a.key_lo + (int)(lo - s0) * kPairKeys;
+    r.k1 = min(a.L, a.key_lo + (int)(hi - s0) * kPairKeys);
     return r;
 }
 
@@ -144,8 +167,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const bool sep_v = a.kv_is_k == 0;
     const bool side_rot = a.kv_is_k == 1;
     const uint32_t rank = cluster_rank();
-    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-    const int n_items = a.splits * a.Hkv * a.B;
+    const int pair = blockIdx.x >> 1;
+    const PairRange pr = pair_range(a, pair);
+    const int n_items = pr.n_items;   // this pair's items
     const int slots_per_tile = sep_v ? 2 * NSB : NSB;
 
     if (threadIdx.x == 0) {
@@ -186,8 +210,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             prefetch_tmap(&a.tm_k);
             if (sep_v) prefetch_tmap(&a.tm_v);
             uint32_t q = 0;   // ring slots filled so far
-            for (int it = pair; it < n_items && !*abort; it += npairs) {
-                const Item w = item_of(a, it);
+            for (int it = 0; it < n_items && !*abort; ++it) {
+                const Item w = item_of(a, pair, pr, it);
                 const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
                 for (int t = 0; t < nt && !*abort; ++t) {
                     const int key = w.k0 + t * kPairKeys + (int)rank * kTileKeys;
@@ -233,7 +257,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             };
             auto tiles_of = [&](int it) {
                 if (it >= n_items) return 0;
-                const Item w = item_of(a, it);
+                const Item w = item_of(a, pair, pr, it);
                 return ceil_div(w.k1 - w.k0, kPairKeys);
             };
             auto advance = [&](Cursor& c) {
@@ -241,11 +265,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 ++c.g;
                 if (++c.t >= c.nt) {
                     c.t = 0;
-                    c.it += npairs;
+                    c.it += 1;
                     c.nt = tiles_of(c.it);
                 }
             };
-            Cursor sc{pair, 0, tiles_of(pair), 0u, 0u};
+            Cursor sc{0, 0, tiles_of(0), 0u, 0u};
             Cursor pc = sc;
             unsigned long long t_idle = 0;
             long long polls = 0;
@@ -330,8 +354,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool good = j < 0 || mbar_wait(&sm.pv_done[j & 1], (j >> 1) & 1, wc, abort);
             return group_all(good, kBarSM, 128);
         };
-        for (int it = pair; it < n_items && ok; it += npairs) {
-            const Item w = item_of(a, it);
+        for (int it = 0; it < n_items && ok; ++it) {
+            const Item w = item_of(a, pair, pr, it);
             const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
             float m_run[HH], l_part[HH];
 #pragma unroll
@@ -506,7 +530,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float qxp[REL ? QH : 1], qyp[REL ? QH : 1];
         float2 bpre[2];
         auto prefetch = [&](int it2) {
-            const Item w2 = item_of(a, it2);
+            const Item w2 = item_of(a, pair, pr, it2);
             const long long k0r = (long long)w2.k0 + (long long)rank * kTileKeys;
             const uint16_t* qg = a.q + ((size_t)w2.b * a.Hq + (size_t)w2.g * G) * D;
 #pragma unroll
@@ -543,11 +567,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
         };
-        if (pair < n_items) prefetch(pair);
+        if (n_items > 0) prefetch(0);
         uint32_t q = 0, gt = 0, item_n = 0;
         bool ok = true;
-        for (int it = pair; it < n_items && ok; it += npairs, ++item_n) {
-            const Item w = item_of(a, it);
+        for (int it = 0; it < n_items && ok; ++it, ++item_n) {
+            const Item w = item_of(a, pair, pr, it);
             const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
             for (int t = 0; t < nt; ++t, ++gt) {
                 const uint32_t qk = q;
@@ -588,7 +612,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
                 // fetch the next item's queries now: the loads fly during this tile's work
-                if (t == nt - 1 && it + npairs < n_items) prefetch(it + npairs);
+                if (t == nt - 1 && it + 1 < n_items) prefetch(it + 1);
                 // every slot of the tile has landed (the MMA issuer relies on this barrier)
                 bool got = true;
                 for (int k = 0; k < slots_per_tile && got; ++k)
@@ -743,7 +767,13 @@ __global__ void __launch_bounds__(kCombineThreads)
     const int bh = blockIdx.x;   // b * Hq + h
     const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
     const size_t stride = (size_t)a.B * a.Hq;
-    const int parts = 2 * a.splits;
+    // the segments of this (b, h)'s sequence: one per pair whose tiles it spans
+    int nseg = 0;
+    if (a.total_tiles > 0) {
+        const long long s0 = (long long)(bh / a.Hq * a.Hkv + (bh % a.Hq) / a.G) * a.tiles_per_seq;
+        nseg = pair_of_tile(a, s0 + a.tiles_per_seq - 1) - pair_of_tile(a, s0) + 1;
+    }
+    const int parts = 2 * nseg;
     // running maxima of the parts, and their largest
     float mx = -INFINITY;
     for (int s = tid; s < parts; s += kCombineThreads) {
@@ -858,20 +888,15 @@ cudaError_t decode_scratch_ptr(void** out) {
 }
 
 cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
-    const int n_items = a.splits * a.Hkv * a.B;
-    if (n_items > 0) {
-        int dev = 0, sms = 148;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        // CTA pairs: one cluster of two per work item in flight
-        const int pairs = n_items < sms / 2 ? n_items : sms / 2;
-        const int grid = 2 * (pairs > 0 ? pairs : 1);
+    if (2 * a.splits > kMaxParts) return cudaErrorInvalidValue;
+    if (a.n_pairs > 0 && a.total_tiles > 0) {
+        // one cluster of two CTAs per pair of the stream-K split
+        const int grid = 2 * a.n_pairs;
         cudaError_t e = a.d == 512 ? dispatch_decode<512>(a, grid, stream)
                         : a.d == 256 ? dispatch_decode<256>(a, grid, stream)
                                      : cudaErrorInvalidValue;
         if (e != cudaSuccess) return e;
     }
-    if (2 * a.splits > kMaxParts) return cudaErrorInvalidValue;
     if (a.B * a.Hq > 0) {
         const dim3 grid(a.B * a.Hq, (a.d + kCombineThreads - 1) / kCombineThreads);
         decode_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(a);

@@ -45,8 +45,14 @@ struct DecodeArgs {
     float* lse;             // [B, Hq] or null
     int B, L, Hq, Hkv, d, G;
     int key_lo;             // first visible key (window), 0 for full attention
-    int splits, keys_per_split;  // keys_per_split: a multiple of 128 (pair-tiles)
-    // part_o / part_ml hold two partials per split (one per CTA of the pair)
+    // Stream-K split: the B * Hkv sequences' pair-tiles of 128 keys, tiles_per_seq each,
+    // are one flat range of total_tiles; CTA pair p takes tiles
+    // [p * total_tiles / n_pairs, (p + 1) * total_tiles / n_pairs), so a sequence is cut
+    // into segments, one per pair that touches it (at most `splits`).  part_o / part_ml
+    // hold two partials per segment (one per CTA of the pair): index 2 * segment + rank.
+    int splits;
+    int tiles_per_seq, n_pairs;
+    long long total_tiles;
     Rope rope;
     float scale_log2;       // scale * log2(e)
     int kv_is_k;
