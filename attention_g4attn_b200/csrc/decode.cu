@@ -613,9 +613,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 // fetch the next item's queries now: the loads fly during this tile's work
                 if (t == nt - 1 && it + 1 < n_items) prefetch(it + 1);
-                // every slot of the tile has landed (the MMA issuer relies on this barrier)
+                // the slots with rotated pairs first: they are turned while the rest land
                 bool got = true;
-                for (int k = 0; k < slots_per_tile && got; ++k)
+                for (int k = 0; k < nrot && got; ++k)
                     got = mbar_wait(&sm.full[(qk + k) % NSLOT], ((qk + k) / NSLOT) & 1, wc, abort);
                 if (R > 0) {
                     // start angle of this CTA's tile: exact (fp64-reduced) at the first tile
@@ -729,9 +729,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+                // every slot of the tile has landed (the MMA issuer relies on this barrier)
+                for (int k = nrot; k < slots_per_tile && got; ++k)
+                    got = mbar_wait(&sm.full[(qk + k) % NSLOT], ((qk + k) / NSLOT) & 1, wc, abort);
                 // the tile's operands are in place: one arrival per CTA on the first CTA
                 fence_proxy_async_smem();
-                group_sync(kBarRot, 128);
+                ok = group_all(got, kBarRot, 128);
+                if (!ok) break;
                 if (t128 == 0) {
                     if (rank == 0) mbar_arrive(&sm.rot_ready[gt & 1]);
                     else mbar_arrive_remote(&sm.rot_ready[gt & 1], 0);
