@@ -513,13 +513,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float2 bcs = make_float2(1.f, 0.f);          // REL: cos/sin of pair start * theta_rk
         float2 stp = make_float2(1.f, 0.f);          // REL: cos/sin of 128 * theta_rk
         if constexpr (REL) {
+            // angles (64 rank + rk) theta_i <= 127 rad: reduced by the nearest multiple of 2 pi,
+            // then the fast intrinsic on [-pi, pi] (the accurate sincosf took 10 us per CTA here)
             const float pos = (float)((int)rank * kTileKeys + rk);
+            auto turn = [&](int i, float& sn, float& cs) {
+                float x = pos * sm.theta[i];
+                x = fmaf(-6.2831853f, rintf(x * 0.15915494f), x);
+                __sincosf(x, &sn, &cs);
+            };
 #pragma unroll
             for (int m = 0; m < 16; ++m) {
                 const int i0 = 32 * cp + 2 * m;
                 float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
-                if (i0 < R) sincosf(pos * sm.theta[i0], &s0, &c0);
-                if (i0 + 1 < R) sincosf(pos * sm.theta[i0 + 1], &s1, &c1);
+                if (i0 < R) turn(i0, s0, c0);
+                if (i0 + 1 < R) turn(i0 + 1, s1, c1);
                 rc[m] = make_float2(c0, c1);
                 rs[m] = make_float2(s0, s1);
             }
