@@ -74,6 +74,36 @@ def test_prefill_workspace_formula(b):
     assert b.g4attn_prefill_workspace_size(2, 4096, loc) == _align(rows) + _align(4096 * 128 * 8)
 
 
+def _decode_segments(B, Hkv, L, window, pairs=74):
+    """Stream-K split of a decode step, by brute force: the sequences' 128-key tiles form one
+    flat range cut evenly over the CTA pairs; returns the most pairs any sequence meets."""
+    key_lo = L - window if (window > 0 and L > window) else 0
+    nt = -(-(L - key_lo) // 128)
+    W = B * Hkv * nt
+    P = min(pairs, W)
+    if W == 0:
+        return 0
+    starts = [p * W // P for p in range(P + 1)]
+    most = 0
+    for bg in range(B * Hkv):
+        lo, hi = bg * nt, (bg + 1) * nt
+        most = max(most, sum(1 for p in range(P) if starts[p] < hi and starts[p + 1] > lo))
+    return most
+
+
+@pytest.mark.parametrize("B,L,layer", [(16, 32768, "g"), (16, 131072, "g"), (2, 1000, "g"),
+                                       (3, 5000, "l"), (1, 1, "g"), (37, 300, "g"), (5, 129, "l"),
+                                       (1, 0, "g")])
+def test_decode_workspace_follows_the_stream_k_split(b, B, L, layer):
+    # two fp32 partials (d outputs + max, sum) per segment and (b, h), 256-byte aligned parts
+    cfg = (b.LayerCfg(32, 4, 512, 0.25, 1e6, 0, None, 1) if layer == "g"
+           else b.LayerCfg(16, 8, 256, 1.0, 1e4, 512, None, 0))
+    Hq, Hkv, d, window = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim, cfg.window
+    S = _decode_segments(B, Hkv, L, window)
+    n = 2 * max(S, 1) * B * Hq
+    assert b.g4attn_decode_workspace_size(B, L, cfg) == _align(n * d * 4) + _align(n * 2 * 4)
+
+
 def test_invalid_configs_are_rejected(b):
     bad = [
         b.LayerCfg(6, 4, 512, 0.25, 1e6),        # Hq % Hkv != 0
