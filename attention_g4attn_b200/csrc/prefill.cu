@@ -464,15 +464,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // (cos, sin) row in the table: they skip the rotation
                         if (rot_lane && (r >> lgG) < pg.tq) {
                             const size_t cso = (size_t)(r >> lgG) * R + i0;
+                            float2 c[H];
+                            if (H == 4 && a.cs_tma && i0 + 4 <= R) {
+                                // the lane's 32 bytes of (cos, sin) as two 16-byte loads; every
+                                // other group of four lanes takes its second half first, so one
+                                // load instruction covers all 32 banks
+                                const float4* p4 = reinterpret_cast<const float4*>(cs_smem + cso);
+                                const int h0 = (lane >> 2) & 1;
+                                const float4 fa = p4[h0], fb = p4[h0 ^ 1];
+                                const float4 lo = h0 ? fb : fa, hi = h0 ? fa : fb;
+                                c[0] = make_float2(lo.x, lo.y);
+                                c[1] = make_float2(lo.z, lo.w);
+                                c[2 % H] = make_float2(hi.x, hi.y);
+                                c[3 % H] = make_float2(hi.z, hi.w);
+                            } else {
+#pragma unroll
+                                for (int k = 0; k < H; ++k)   // shared-memory rows or the table
+                                    c[k] = i0 + k >= R ? make_float2(1.f, 0.f)
+                                           : a.cs_tma ? cs_smem[cso + k] : cs_glob[cso + k];
+                            }
 #pragma unroll
                             for (int k = 0; k < H; ++k) {
-                                if (i0 + k < R) {
-                                    // shared-memory rows (TMA) or the workspace table
-                                    const float2 c = a.cs_tma ? cs_smem[cso + k] : cs_glob[cso + k];
-                                    const float x = u[j][k] * c.x - v[j][k] * c.y;
-                                    v[j][k] = u[j][k] * c.y + v[j][k] * c.x;
-                                    u[j][k] = x;
-                                }
+                                const float x = u[j][k] * c[k].x - v[j][k] * c[k].y;
+                                v[j][k] = u[j][k] * c[k].y + v[j][k] * c[k].x;
+                                u[j][k] = x;
                             }
                         }
                         const uint32_t off = sw128_offset(r, col);
