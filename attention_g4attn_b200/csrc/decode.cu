@@ -512,26 +512,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float qx[REL ? QH : 1], qy[REL ? QH : 1];    // REL: pair rk of q, heads cp + 2j
         float2 bcs = make_float2(1.f, 0.f);          // REL: cos/sin of pair start * theta_rk
         float2 stp = make_float2(1.f, 0.f);          // REL: cos/sin of 128 * theta_rk
-        if constexpr (REL) {
-            // angles (64 rank + rk) theta_i <= 127 rad: reduced by the nearest multiple of 2 pi,
-            // then the fast intrinsic on [-pi, pi] (the accurate sincosf took 10 us per CTA here)
-            const float pos = (float)((int)rank * kTileKeys + rk);
-            auto turn = [&](int i, float& sn, float& cs) {
-                float x = pos * sm.theta[i];
-                x = fmaf(-6.2831853f, rintf(x * 0.15915494f), x);
-                __sincosf(x, &sn, &cs);
-            };
-#pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const int i0 = 32 * cp + 2 * m;
-                float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
-                if (i0 < R) turn(i0, s0, c0);
-                if (i0 + 1 < R) turn(i0 + 1, s1, c1);
-                rc[m] = make_float2(c0, c1);
-                rs[m] = make_float2(s0, s1);
-            }
-            if (rk < R) stp = sm.step_cs[rk];
-        }
         // the next item's queries and start angles, fetched one tile ahead of their use
         uint4 qpre[QV];
         float qxp[REL ? QH : 1], qyp[REL ? QH : 1];
@@ -574,7 +554,27 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             }
         };
-        if (n_items > 0) prefetch(0);
+        if (n_items > 0) prefetch(0);   // the loads fly while the constants below are computed
+        if constexpr (REL) {
+            // angles (64 rank + rk) theta_i <= 127 rad: reduced by the nearest multiple of 2 pi,
+            // then the fast intrinsic on [-pi, pi] (the accurate sincosf took 10 us per CTA here)
+            const float pos = (float)((int)rank * kTileKeys + rk);
+            auto turn = [&](int i, float& sn, float& cs) {
+                float x = pos * sm.theta[i];
+                x = fmaf(-6.2831853f, rintf(x * 0.15915494f), x);
+                __sincosf(x, &sn, &cs);
+            };
+#pragma unroll
+            for (int m = 0; m < 16; ++m) {
+                const int i0 = 32 * cp + 2 * m;
+                float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
+                if (i0 < R) turn(i0, s0, c0);
+                if (i0 + 1 < R) turn(i0 + 1, s1, c1);
+                rc[m] = make_float2(c0, c1);
+                rs[m] = make_float2(s0, s1);
+            }
+            if (rk < R) stp = sm.step_cs[rk];
+        }
         uint32_t q = 0, gt = 0, item_n = 0;
         bool ok = true;
         for (int it = 0; it < n_items && ok; ++it, ++item_n) {
@@ -772,6 +772,10 @@ constexpr int kMaxParts = 1024;
 
 __global__ void __launch_bounds__(kCombineThreads)
     decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
+    // launched as a programmatic dependent of the decode kernel: its blocks may start while
+    // the decode's last CTAs finish; the partials are read only after the decode grid has
+    // completed and its writes are visible
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     __shared__ float wgt[kMaxParts];
     __shared__ float red[kCombineThreads / 32];
     __shared__ float bM, bDen;
@@ -909,8 +913,17 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
         if (e != cudaSuccess) return e;
     }
     if (a.B * a.Hq > 0) {
-        const dim3 grid(a.B * a.Hq, (a.d + kCombineThreads - 1) / kCombineThreads);
-        decode_combine_kernel<<<grid, kCombineThreads, 0, stream>>>(a);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(a.B * a.Hq, (a.d + kCombineThreads - 1) / kCombineThreads);
+        cfg.blockDim = dim3(kCombineThreads);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_combine_kernel, a);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }
