@@ -95,6 +95,7 @@ def _load():
         "g4attn_status_string": (ctypes.c_char_p, [I]),
         "g4attn_device_status": (I, [P]),
         "g4attn_set_wait_limit": (LL, [LL]),
+        "g4attn_wait_selftest": (I, [LL, P]),
         "g4attn_version": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
@@ -158,6 +159,12 @@ def g4attn_set_wait_limit(polls: int) -> int:
 
 def g4attn_device_status(stream=None) -> int:
     return _lib.g4attn_device_status(_stream(stream))
+
+
+def g4attn_wait_selftest(polls: int = 0, stream=None) -> int:
+    """Launch the bounded-wait self-test (a wait that nothing satisfies); read the outcome
+    with g4attn_device_status."""
+    return _lib.g4attn_wait_selftest(int(polls), _stream(stream))
 
 
 def g4attn_prefill_workspace_size(B: int, T: int, cfg: LayerCfg) -> int:

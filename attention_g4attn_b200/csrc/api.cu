@@ -250,6 +250,15 @@ const char* g4attn_status_string(int s) {
     }
 }
 
+int g4attn_wait_selftest(long long polls, g4attn_stream_t stream) {
+    DeviceInfo* dev = nullptr;
+    const int rc = current_device(&dev);
+    if (rc) return rc;
+    const long long limit = polls < 1 ? g_wait_limit.load() : polls;
+    return cuda_status(g4::launch_wait_selftest(dev->status, limit,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 long long g4attn_set_wait_limit(long long polls) {
     return g_wait_limit.exchange(polls < 1 ? kDefaultWaitLimit : polls);
 }

@@ -234,7 +234,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             if (*abort) {
                 const uint32_t first = q > (uint32_t)NSLOT ? q - NSLOT : 0;
                 for (uint32_t k = first; k < q; ++k)
-                    mbar_wait_drain(&sm.full[k % NSLOT], (k / NSLOT) & 1, a.wait_limit);
+                    mbar_wait_drain(&sm.full[k % NSLOT], (k / NSLOT) & 1);
             }
         }
     } else if (warp == 1) {
@@ -334,7 +334,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             // all issued MMAs must finish before either CTA frees its tensor memory
             mma_commit_pair(&sm.drain);
-            mbar_wait_drain(&sm.drain, 0, a.wait_limit);
+            mbar_wait_drain(&sm.drain, 0);
         }
     } else if (warp < 6) {
         // ------------------------------------------------- softmax / epilogue (warps 2..5)

@@ -34,6 +34,10 @@ struct QkNormRopeArgs {
 
 cudaError_t launch_qknorm_rope(const QkNormRopeArgs& a, cudaStream_t stream);
 
+// Self-test of the bounded waits: a wait that nothing satisfies gives up after `limit` polls
+// (or 2 s) and records G4ATTN_ERR_TIMEOUT in *status.
+cudaError_t launch_wait_selftest(int* status, long long limit, cudaStream_t stream);
+
 // Split-KV decode (one query per (b, h) at position L-1) and its combine pass.
 struct DecodeArgs {
     CUtensorMap tm_k;       // kcache [B, L, Hkv, d] as a 4-D map (d, Hkv, L, B), box (64, 1, 64, 1)

@@ -801,13 +801,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     // -------------------------------------------------------------------- teardown
     // A CTA that gave up tells its peer, so the peer's waits end promptly too.
     __syncthreads();
-    if (*abort && threadIdx.x == 0) st_shared_remote_u32((const void*)&sm.abort, rank ^ 1u, 1u);
+    if (*abort && threadIdx.x == 0) {
+        st_shared_remote_u32((const void*)&sm.abort, rank ^ 1u, 1u);
+        // copies this CTA started must land before its shared memory is freed: the query
+        // tile on its own barrier; the key/value slots complete on the pair leader's
+        // barrier, which this CTA cannot observe, so it gives them a settle time (copies
+        // land in microseconds)
+        mbar_wait_drain(&sm.q_full, 0);
+        spin_ns(100000);
+    }
     tc_fence_before();
     cluster_sync();
     if (leader && warp == 1 && lane == 0) {
         // every MMA of the pair must be complete before either CTA frees its columns
         mma_commit_pair(&sm.drain);
-        mbar_wait_drain(&sm.drain, 0, a.wait_limit);
+        mbar_wait_drain(&sm.drain, 0);
     }
     tc_fence_before();
     cluster_sync();

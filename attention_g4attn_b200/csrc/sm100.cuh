@@ -105,14 +105,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 // Wait that ignores the abort flag: used only while draining in-flight copies and MMAs
-// before a CTA frees its tensor memory and exits.
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, long long limit) {
+// before a CTA frees its shared or tensor memory and exits.  Bounded by wall-clock time
+// alone, not by the caller's poll limit: a tiny limit (set to exercise the timeout path)
+// must not let a CTA free memory that a copy or an MMA still writes.
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
     const unsigned long long t0 = global_ns();
-    for (long long i = 0; i < limit; ++i) {
+    for (long long i = 0;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((i & 63) == 63 && global_ns() - t0 > kWaitTimeoutNs) break;
+        if ((i & 63) == 63 && global_ns() - t0 > kWaitTimeoutNs) return false;
     }
-    return false;
+}
+
+// Spin for `ns` nanoseconds of wall-clock time.
+__device__ __forceinline__ void spin_ns(unsigned long long ns) {
+    const unsigned long long t0 = global_ns();
+    while (global_ns() - t0 < ns) {
+    }
 }
 
 // Named barrier over the `nthreads` threads of a warpgroup that returns true only if

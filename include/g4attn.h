@@ -182,6 +182,17 @@ G4ATTN_API int g4attn_device_status(g4attn_stream_t stream);
  */
 G4ATTN_API long long g4attn_set_wait_limit(long long polls);
 
+/*
+ * Self-test of failure detection.  Launches one CTA on `stream` whose thread waits, with the
+ * kernels' bounded wait and at most `polls` polls (polls < 1: the current wait limit), on
+ * an mbarrier that nothing arrives on.  The wait gives up and records G4ATTN_ERR_TIMEOUT in
+ * the device status word, which g4attn_device_status(stream) then returns (and clears).
+ * The CTA holds no copies, MMAs or tensor memory, so the context stays usable.
+ * Returns G4ATTN_OK once launched, G4ATTN_ERR_UNSUPPORTED without an sm_100 device,
+ * G4ATTN_ERR_CUDA if the launch fails.
+ */
+G4ATTN_API int g4attn_wait_selftest(long long polls, g4attn_stream_t stream);
+
 /* Library version string. */
 G4ATTN_API const char* g4attn_version(void);
 

@@ -99,3 +99,17 @@ def test_decode_matches_last_prefill_row():
     torch.cuda.synchronize()
     assert_parity(to_np(dout)[:, 0], to_np(pre)[:, T - 1], "decode vs prefill row")
     assert_parity(to_np(dlse), to_np(pre_lse)[:, :, T - 1], "decode vs prefill lse")
+
+
+def test_bounded_wait_gives_up_and_reports_timeout():
+    # a device wait that nothing satisfies gives up after its poll bound and records
+    # G4ATTN_ERR_TIMEOUT; the status read clears it and the context stays usable
+    b = binding()
+    assert b.g4attn_device_status() == 0
+    assert b.g4attn_wait_selftest(4096) == 0
+    assert b.g4attn_device_status() == b.G4ATTN_ERR_TIMEOUT
+    assert b.g4attn_device_status() == 0
+    # the 2-second wall-clock bound applies with the default (unbounded) poll limit too
+    assert b.g4attn_wait_selftest(0) == 0
+    assert b.g4attn_device_status() == b.G4ATTN_ERR_TIMEOUT
+    test_decode_global_small(300)   # kernels still run and match the oracle afterwards
