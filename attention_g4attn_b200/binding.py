@@ -92,6 +92,8 @@ def _load():
         "g4attn_decode_workspace_size": (SZ, [I, I, CFG]),
         "g4attn_decode": (I, [P, P, P, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_decode_noalloc": (I, [P, P, P, I, P, P, I, CFG, P]),
+        "g4attn_decode_ring_workspace_size": (SZ, [I, I, I, CFG]),
+        "g4attn_decode_ring": (I, [P, P, P, I, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_status_string": (ctypes.c_char_p, [I]),
         "g4attn_device_status": (I, [P]),
         "g4attn_set_wait_limit": (LL, [LL]),
@@ -239,6 +241,33 @@ def g4attn_decode(q, kcache, vcache, cfg: LayerCfg, out=None, lse=None, want_lse
                             _ptr(workspace), workspace.numel(), B, ctypes.byref(c),
                             _stream(stream))
     _check(rc, "g4attn_decode")
+    return out, lse
+
+
+def g4attn_decode_ring_workspace_size(B: int, L: int, C: int, cfg: LayerCfg) -> int:
+    c = cfg.c()
+    return _lib.g4attn_decode_ring_workspace_size(B, L, C, ctypes.byref(c))
+
+
+def g4attn_decode_ring(q, kring, vring, L: int, cfg: LayerCfg, out=None, lse=None,
+                       want_lse=False, workspace=None, stream=None):
+    """Decode one token at position L-1 against ring caches kring/vring [B, C, Hkv, d]
+    (position p in row p % C; window = cfg.window <= C)."""
+    for t, n in ((q, "q"), (kring, "kring"), (vring, "vring")):
+        _bf16(t, n)
+    B, C = kring.shape[0], kring.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.n_q_heads), dtype=torch.float32, device=q.device)
+    c = cfg.c()
+    ws_bytes = _lib.g4attn_decode_ring_workspace_size(B, L, C, ctypes.byref(c))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    rc = _lib.g4attn_decode_ring(_ptr(q), _ptr(kring), _ptr(vring), int(L), C, _ptr(out),
+                                 _ptr(lse), _ptr(workspace), workspace.numel(), B,
+                                 ctypes.byref(c), _stream(stream))
+    _check(rc, "g4attn_decode_ring")
     return out, lse
 
 

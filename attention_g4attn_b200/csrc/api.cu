@@ -115,10 +115,13 @@ int check_cfg(const g4attn_layer_cfg* c, bool tensor_core_path) {
 
 // 4-D map over a [B, T, H, d] 16-bit tensor: dims (d, H, T, B), box (64, 1, box_rows, 1),
 // 128-byte swizzle, zero fill outside the tensor.
+// `T_phys` (default T): rows per batch in memory, when only the first T are exposed (rows
+// from T on read as zero).
 int encode_rows(CUtensorMap* m, const void* base, int B, int T, int H, int d, bool f16 = false,
-                int box_rows = 128) {
+                int box_rows = 128, int T_phys = 0) {
+    const cuuint64_t tp = (cuuint64_t)(T_phys > 0 ? T_phys : T);
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
-    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)T * H * d * 2};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, tp * H * d * 2};
     cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     cuuint32_t es[4] = {1, 1, 1, 1};
     CUresult r = g_encode(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
@@ -179,7 +182,7 @@ constexpr int kDecodeTile = 128;   // keys per decode pair-tile
 // of W tiles, cut evenly over P CTA pairs; a sequence is split into one segment per pair
 // that touches it, and every segment leaves two partials (one per CTA of its pair).
 struct DecodePlan {
-    int key_lo, splits, tiles_per_seq, n_pairs;
+    int key_lo, tile_base, splits, tiles_per_seq, n_pairs;
     long long total_tiles;
     size_t o_off, ml_off, total;
 };
@@ -197,10 +200,14 @@ int max_segments(long long W, int nt, int nbg, int P) {
     return m;
 }
 
-DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms, int max_pairs = 0) {
+// ring > 0: the cache is a ring of `ring` rows (position p in row p % ring); the tiles then
+// start at the 64-aligned position at or below the window start, so no 64-key box wraps.
+DecodePlan decode_plan(int B, int L, const g4attn_layer_cfg* c, int sms, int max_pairs = 0,
+                       int ring = 0) {
     DecodePlan p{};
     p.key_lo = (c->window > 0 && L > c->window) ? L - c->window : 0;
-    const int len = L - p.key_lo;
+    p.tile_base = ring > 0 ? p.key_lo / 64 * 64 : p.key_lo;
+    const int len = L - p.tile_base;
     const int nbg = B * c->n_kv_heads;
     p.tiles_per_seq = len > 0 ? (len + kDecodeTile - 1) / kDecodeTile : 0;
     p.total_tiles = (long long)nbg * p.tiles_per_seq;
@@ -227,6 +234,77 @@ int cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return G4ATTN_OK;
     cudaGetLastError();
     return G4ATTN_ERR_CUDA;
+}
+
+// Argument checks shared by the decode entry points (before any launch).
+int check_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_bf16* vcache,
+                 int L, const g4attn_bf16* out, const float* lse, int B,
+                 const g4attn_layer_cfg* cfg) {
+    int rc = check_cfg(cfg, true);
+    if (rc) return rc;
+    if (B < 0 || L < 0) return G4ATTN_ERR_INVALID_ARG;
+    if (B > 0 && (!q || !out || (L > 0 && !kcache))) return G4ATTN_ERR_INVALID_ARG;
+    if ((cfg->kv_is_k == 0) != (vcache != nullptr)) return G4ATTN_ERR_INVALID_ARG;
+    const int G = cfg->n_q_heads / cfg->n_kv_heads;
+    if (G > 16) return G4ATTN_ERR_UNSUPPORTED;
+    if (cfg->kv_is_k == 1) {   // the turned slot of a tile must be a single slot (R <= 64)
+        const int R = rope_pairs(cfg);
+        int n = 0;
+        for (int c = 0; c < cfg->head_dim / 64; ++c) n += chunk_rotated(c, cfg->head_dim, R);
+        if (n > 2) return G4ATTN_ERR_UNSUPPORTED;
+    }
+    const void* ptrs[] = {q, kcache, vcache, out, lse};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;
+    return G4ATTN_OK;
+}
+
+// Fills the decode arguments for a planned call and launches decode + combine.
+// `rows`: cache rows in memory (L for a linear cache, C for a ring); `ring`: 0 or C.  A ring
+// that is not full yet (L < C) exposes only its first L rows to the copies: the last tile's
+// positions past L then read zeros instead of never-written rows (whose values, times a zero
+// weight, could still be NaN).
+int launch_decode_plan(const g4attn_bf16* q, const g4attn_bf16* kcache,
+                       const g4attn_bf16* vcache, int L, int rows, int ring, g4attn_bf16* out,
+                       float* lse, uint8_t* w, const DecodePlan& plan, int B,
+                       const g4attn_layer_cfg* cfg, const DeviceInfo* dev, g4attn_stream_t stream) {
+    g4::DecodeArgs a{};
+    const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
+    int rc;
+    if (L > 0) {
+        const int seen = L < rows ? L : rows;   // rows that hold positions
+        if ((rc = encode_rows(&a.tm_k, kcache, B, seen, Hkv, d, false, 64, rows))) return rc;
+        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, seen, Hkv, d, false, 64, rows)))
+            return rc;
+    }
+    a.q = q;
+    a.part_o = reinterpret_cast<float*>(w + plan.o_off);
+    a.part_ml = reinterpret_cast<float*>(w + plan.ml_off);
+    a.out = out;
+    a.lse = lse;
+    a.B = B; a.L = L; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d;
+    a.G = cfg->n_q_heads / Hkv;
+    a.key_lo = plan.key_lo;
+    a.tile_base = plan.tile_base;
+    a.ring = ring;
+    a.splits = plan.splits;
+    a.tiles_per_seq = plan.tiles_per_seq;
+    a.n_pairs = plan.n_pairs;
+    a.total_tiles = plan.total_tiles;
+    a.rope = make_rope(cfg);
+    a.scale_log2 = cfg->scale * 1.4426950408889634f;
+    a.kv_is_k = cfg->kv_is_k;
+    a.wait_limit = g_wait_limit.load();
+    a.status = dev->status;
+    return cuda_status(g4::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// A ring cache holds the last C positions, C a positive multiple of 64 (pair-tile halves
+// never wrap), and must hold the whole window.
+int check_ring(int C, const g4attn_layer_cfg* cfg) {
+    if (!cfg || C <= 0 || C % 64 != 0) return G4ATTN_ERR_INVALID_ARG;
+    if (cfg->window <= 0 || cfg->window > C) return G4ATTN_ERR_INVALID_ARG;
+    return G4ATTN_OK;
 }
 
 }  // namespace
@@ -408,52 +486,42 @@ size_t g4attn_decode_workspace_size(int B, int L, const g4attn_layer_cfg* cfg) {
 int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_bf16* vcache,
                   int L, g4attn_bf16* out, float* lse, void* workspace, size_t ws_bytes, int B,
                   const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
-    int rc = check_cfg(cfg, true);
+    int rc = check_decode(q, kcache, vcache, L, out, lse, B, cfg);
     if (rc) return rc;
-    if (B < 0 || L < 0) return G4ATTN_ERR_INVALID_ARG;
     if (B == 0) return G4ATTN_OK;
-    if (!q || !out || (L > 0 && !kcache)) return G4ATTN_ERR_INVALID_ARG;
-    if ((cfg->kv_is_k == 0) != (vcache != nullptr)) return G4ATTN_ERR_INVALID_ARG;
-    const int G = cfg->n_q_heads / cfg->n_kv_heads;
-    if (G > 16) return G4ATTN_ERR_UNSUPPORTED;
-    if (cfg->kv_is_k == 1) {   // two side buffers hold the turned chunks
-        const int R = rope_pairs(cfg);
-        int n = 0;
-        for (int c = 0; c < cfg->head_dim / 64; ++c) n += chunk_rotated(c, cfg->head_dim, R);
-        if (n > 2) return G4ATTN_ERR_UNSUPPORTED;
-    }
-    const void* ptrs[] = {q, kcache, vcache, out, lse};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;
     DeviceInfo* dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
     const DecodePlan plan = decode_plan(B, L, cfg, dev->sms);
     if (!workspace || ws_bytes < plan.total) return G4ATTN_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
-    uint8_t* w = static_cast<uint8_t*>(workspace);
-    g4::DecodeArgs a{};
-    const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
-    if (L > 0) {
-        if ((rc = encode_rows(&a.tm_k, kcache, B, L, Hkv, d, false, 64))) return rc;
-        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, L, Hkv, d, false, 64))) return rc;
-    }
-    a.q = q;
-    a.part_o = reinterpret_cast<float*>(w + plan.o_off);
-    a.part_ml = reinterpret_cast<float*>(w + plan.ml_off);
-    a.out = out;
-    a.lse = lse;
-    a.B = B; a.L = L; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d; a.G = G;
-    a.key_lo = plan.key_lo;
-    a.splits = plan.splits;
-    a.tiles_per_seq = plan.tiles_per_seq;
-    a.n_pairs = plan.n_pairs;
-    a.total_tiles = plan.total_tiles;
-    a.rope = make_rope(cfg);
-    a.scale_log2 = cfg->scale * 1.4426950408889634f;
-    a.kv_is_k = cfg->kv_is_k;
-    a.wait_limit = g_wait_limit.load();
-    a.status = dev->status;
-    return cuda_status(g4::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+    return launch_decode_plan(q, kcache, vcache, L, L, 0, out, lse,
+                              static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream);
+}
+
+size_t g4attn_decode_ring_workspace_size(int B, int L, int C, const g4attn_layer_cfg* cfg) {
+    if (check_cfg(cfg, true) || check_ring(C, cfg) || B < 0 || L < 0) return 0;
+    DeviceInfo* dev = nullptr;
+    int sms = 148;
+    if (current_device(&dev) == G4ATTN_OK) sms = dev->sms;
+    else cudaGetLastError();
+    return decode_plan(B, L, cfg, sms, 0, C).total;
+}
+
+int g4attn_decode_ring(const g4attn_bf16* q, const g4attn_bf16* kring, const g4attn_bf16* vring,
+                       int L, int C, g4attn_bf16* out, float* lse, void* workspace,
+                       size_t ws_bytes, int B, const g4attn_layer_cfg* cfg,
+                       g4attn_stream_t stream) {
+    int rc = check_decode(q, kring, vring, L, out, lse, B, cfg);
+    if (rc) return rc;
+    if ((rc = check_ring(C, cfg))) return rc;
+    if (B == 0) return G4ATTN_OK;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    const DecodePlan plan = decode_plan(B, L, cfg, dev->sms, 0, C);
+    if (!workspace || ws_bytes < plan.total) return G4ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
+    return launch_decode_plan(q, kring, vring, L, C, C, out, lse,
+                              static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream);
 }
 
 // Decode with no workspace argument and no allocation: the split partials go to the
@@ -463,27 +531,13 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
 int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
                           const g4attn_bf16* vcache, int L, g4attn_bf16* out, float* lse, int B,
                           const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
-    int rc = check_cfg(cfg, true);
+    int rc = check_decode(q, kcache, vcache, L, out, lse, B, cfg);
     if (rc) return rc;
-    if (B < 0 || L < 0) return G4ATTN_ERR_INVALID_ARG;
     if (B == 0) return G4ATTN_OK;
-    if (!q || !out || (L > 0 && !kcache)) return G4ATTN_ERR_INVALID_ARG;
-    if ((cfg->kv_is_k == 0) != (vcache != nullptr)) return G4ATTN_ERR_INVALID_ARG;
-    const int G = cfg->n_q_heads / cfg->n_kv_heads;
-    if (G > 16) return G4ATTN_ERR_UNSUPPORTED;
-    if (cfg->kv_is_k == 1) {
-        const int R = rope_pairs(cfg);
-        int n = 0;
-        for (int c = 0; c < cfg->head_dim / 64; ++c) n += chunk_rotated(c, cfg->head_dim, R);
-        if (n > 2) return G4ATTN_ERR_UNSUPPORTED;
-    }
-    const void* ptrs[] = {q, kcache, vcache, out, lse};
-    for (const void* p : ptrs)
-        if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;
     DeviceInfo* dev = nullptr;
     if ((rc = current_device(&dev))) return rc;
     const size_t cap = g4::decode_scratch_bytes();
-    const size_t per_split = 2 * (size_t)B * cfg->n_q_heads;   // two partials per split
+    const size_t per_split = 2 * (size_t)B * cfg->n_q_heads;   // two partials per segment
     if (align256(per_split * cfg->head_dim * sizeof(float)) + align256(per_split * 2 * sizeof(float)) >
         cap)
         return G4ATTN_ERR_TOO_LARGE;
@@ -493,30 +547,8 @@ int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
     if (plan.total > cap) return G4ATTN_ERR_TOO_LARGE;
     void* scratch = nullptr;
     if (g4::decode_scratch_ptr(&scratch) != cudaSuccess) return cuda_status(cudaErrorUnknown);
-    uint8_t* w = static_cast<uint8_t*>(scratch);
-    g4::DecodeArgs a{};
-    const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
-    if (L > 0) {
-        if ((rc = encode_rows(&a.tm_k, kcache, B, L, Hkv, d, false, 64))) return rc;
-        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, L, Hkv, d, false, 64))) return rc;
-    }
-    a.q = q;
-    a.part_o = reinterpret_cast<float*>(w + plan.o_off);
-    a.part_ml = reinterpret_cast<float*>(w + plan.ml_off);
-    a.out = out;
-    a.lse = lse;
-    a.B = B; a.L = L; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d; a.G = G;
-    a.key_lo = plan.key_lo;
-    a.splits = plan.splits;
-    a.tiles_per_seq = plan.tiles_per_seq;
-    a.n_pairs = plan.n_pairs;
-    a.total_tiles = plan.total_tiles;
-    a.rope = make_rope(cfg);
-    a.scale_log2 = cfg->scale * 1.4426950408889634f;
-    a.kv_is_k = cfg->kv_is_k;
-    a.wait_limit = g_wait_limit.load();
-    a.status = dev->status;
-    return cuda_status(g4::launch_decode(a, reinterpret_cast<cudaStream_t>(stream)));
+    return launch_decode_plan(q, kcache, vcache, L, L, 0, out, lse,
+                              static_cast<uint8_t*>(scratch), plan, B, cfg, dev, stream);
 }
 
 }  // extern "C"

@@ -96,7 +96,8 @@ struct __align__(1024) DecodeSmem {
 __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 
 struct Item {
-    int s, g, b, k0, k1;
+    int s, g, b, k0, k1;   // segment, kv head, batch; positions [k0, k1) of the item's tiles
+    int lo;                // first visible position in the item (>= k0)
 };
 
 // The pair that owns flat tile t: the largest p with p * total / n_pairs <= t.
@@ -129,8 +130,9 @@ __device__ __forceinline__ Item item_of(const DecodeArgs& a, int pair, const Pai
     r.g = bg % a.Hkv;
     r.b = bg / a.Hkv;
     r.s = pair - pair_of_tile(a, s0);
-    r.k0 = a.key_lo + (int)(lo - s0) * kPairKeys;
-    r.k1 = min(a.L, a.key_lo + (int)(hi - s0) * kPairKeys);
+    r.k0 = a.tile_base + (int)(lo - s0) * kPairKeys;
+    r.k1 = min(a.L, a.tile_base + (int)(hi - s0) * kPairKeys);
+    r.lo = max(r.k0, a.key_lo);
     return r;
 }
 
@@ -214,7 +216,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const Item w = item_of(a, pair, pr, it);
                 const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
                 for (int t = 0; t < nt && !*abort; ++t) {
-                    const int key = w.k0 + t * kPairKeys + (int)rank * kTileKeys;
+                    const int kpos = w.k0 + t * kPairKeys + (int)rank * kTileKeys;
+                    // cache row of this CTA's 64 keys (a ring holds position p at p % C; the
+                    // tiles are 64-aligned and C a multiple of 64, so a box never wraps)
+                    const int key = a.ring > 0 ? kpos % a.ring : kpos;
                     for (int pass = 0; pass < (sep_v ? 2 : 1) && !*abort; ++pass) {
                         const CUtensorMap* map = pass ? &a.tm_v : &a.tm_k;
                         for (int sb = 0; sb < NSB; ++sb) {
@@ -377,7 +382,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int j = 0; j < HH; ++j) sm.xs[hf ^ 1][key][j] = hf ? sp[j] : sp[HH + j];
                 group_sync(kBarSM, 128);
-                const bool valid = key0 + key < w.k1;
+                const bool valid = key0 + key < w.k1 && key0 + key >= w.lo;
                 float x[HH];
                 bool big = false;
 #pragma unroll

@@ -40,7 +40,7 @@ cudaError_t launch_wait_selftest(int* status, long long limit, cudaStream_t stre
 
 // Split-KV decode (one query per (b, h) at position L-1) and its combine pass.
 struct DecodeArgs {
-    CUtensorMap tm_k;       // kcache [B, L, Hkv, d] as a 4-D map (d, Hkv, L, B), box (64, 1, 64, 1)
+    CUtensorMap tm_k;       // kcache [B, L or C, Hkv, d] as a 4-D map (d, Hkv, rows, B), box (64, 1, 64, 1)
     CUtensorMap tm_v;       // vcache, same geometry (kv_is_k == 0), else a copy of tm_k
     const uint16_t* q;      // [B, Hq, d], normalised and rotated
     float* part_o;          // [2S, B, Hq, d]
@@ -48,7 +48,9 @@ struct DecodeArgs {
     uint16_t* out;          // [B, Hq, d]
     float* lse;             // [B, Hq] or null
     int B, L, Hq, Hkv, d, G;
-    int key_lo;             // first visible key (window), 0 for full attention
+    int key_lo;             // first visible key position (window), 0 for full attention
+    int tile_base;          // position where the pair-tiles start (<= key_lo)
+    int ring;               // 0: cache row = position; C > 0: ring of C rows, row = position % C
     // Stream-K split: the B * Hkv sequences' pair-tiles of 128 keys, tiles_per_seq each,
     // are one flat range of total_tiles; CTA pair p takes tiles
     // [p * total_tiles / n_pairs, (p + 1) * total_tiles / n_pairs), so a sequence is cut

@@ -140,6 +140,27 @@ G4ATTN_API int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, co
                   int B, const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
 
 /*
+ * Decode of a sliding-window layer against a ring-buffer cache (report section 2 and the
+ * explainer's "interleaved layers": local layers attend to the last W tokens, so their cache
+ * only needs the last C >= W positions).  Same operation as g4attn_decode with window W =
+ * cfg->window, but the cache holds position p in row p % C:
+ *   kring   [B, C, Hkv, d] bf16: normalised, NOT rotated keys; row p % C holds position p
+ *           for the last C positions p < L
+ *   vring   [B, C, Hkv, d] bf16 or NULL: separate values, same ring (kv_is_k = 0 only)
+ *   L       tokens so far; the new query sits at position L-1
+ *   C       ring rows: a positive multiple of 64, with 0 < W = cfg->window <= C
+ *   workspace / ws_bytes  >= g4attn_decode_ring_workspace_size(B, L, C, cfg)
+ * Other arguments and results as in g4attn_decode.  C or W out of range returns
+ * G4ATTN_ERR_INVALID_ARG before any launch (and the workspace size function returns 0).
+ */
+G4ATTN_API size_t g4attn_decode_ring_workspace_size(int B, int L, int C,
+                                                    const g4attn_layer_cfg* cfg);
+G4ATTN_API int g4attn_decode_ring(const g4attn_bf16* q, const g4attn_bf16* kring,
+                                  const g4attn_bf16* vring, int L, int C, g4attn_bf16* out,
+                                  float* lse, void* workspace, size_t ws_bytes, int B,
+                                  const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/*
  * Decode without a workspace and without allocating (the papers describe no such call;
  * it exists for callers that cannot allocate device memory: plugins whose host framework
  * owns every device allocation and hands them only input and output buffers, and services
@@ -147,10 +168,10 @@ G4ATTN_API int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, co
  * g4attn_decode minus the workspace: the split-KV partials live in a fixed 8 MiB device
  * array inside the library, which every device that loads the library holds until the
  * process exits.  The call allocates nothing.
- *   - The split count is lowered until the partials fit; if even one split needs more
- *     than 8 MiB (2 * B * Hq * (head_dim + 2) * 4 bytes > 8 MiB: the kernel keeps two
- *     partials per split), the call returns
- *     G4ATTN_ERR_TOO_LARGE and launches nothing.
+ *   - The number of CTA pairs (and with it the segments each sequence is split into) is
+ *     lowered until the partials fit; if even one segment per sequence needs more than
+ *     8 MiB (2 * B * Hq * (head_dim + 2) * 4 bytes > 8 MiB: the kernel keeps two partials
+ *     per segment), the call returns G4ATTN_ERR_TOO_LARGE and launches nothing.
  *   - The first call on a device looks up the array's device address (once per device,
  *     with that device current); make that first call before any stream capture.
  *   - All calls share the one array and it keeps the last call's partials.  Nothing in it

@@ -12,5 +12,6 @@ from .oracle import (  # noqa: F401
     qknorm_rope,
     prefill_rows,
     decode,
+    decode_ring,
     bf16_bits,
 )

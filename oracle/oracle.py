@@ -172,3 +172,26 @@ def decode(q, kcache, vcache, cfg: OracleCfg, items=None, nthreads: int = 0):
     if rc != 0:
         raise ValueError("oracle decode rejected its arguments (%d)" % rc)
     return out, lse
+
+
+def decode_ring(q, kring, vring, L: int, cfg: OracleCfg, nthreads: int = 0):
+    """Decode of a sliding-window layer against ring caches (Gemma 4 report section 2 and the
+    explainer's "interleaved layers": a local layer attends to the last W tokens, so its cache
+    keeps only the last C >= W positions, position p in row p % C).
+
+    Written out as the definition: the ring is unrolled into a linear cache of L positions
+    (row p = ring row p % C for the last C positions; earlier positions, outside the window,
+    are zero) and the linear decode above runs on it with the same window."""
+    kb = bf16_bits(kring)
+    vb = None if vring is None else bf16_bits(vring)
+    B, C = kb.shape[0], kb.shape[1]
+    if not (cfg.window and 0 < cfg.window <= C):
+        raise ValueError("ring decode needs 0 < window <= C")
+    shape = (B, L) + kb.shape[2:]
+    k_lin = np.zeros(shape, np.uint16)
+    v_lin = None if vb is None else np.zeros(shape, np.uint16)
+    for p in range(max(0, L - C), L):
+        k_lin[:, p] = kb[:, p % C]
+        if vb is not None:
+            v_lin[:, p] = vb[:, p % C]
+    return decode(q, k_lin, v_lin, cfg, nthreads=nthreads)

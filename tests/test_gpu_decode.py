@@ -113,3 +113,61 @@ def test_bounded_wait_gives_up_and_reports_timeout():
     assert b.g4attn_wait_selftest(0) == 0
     assert b.g4attn_device_status() == b.G4ATTN_ERR_TIMEOUT
     test_decode_global_small(300)   # kernels still run and match the oracle afterwards
+
+
+# ------------------------------------------------------------ ring-buffer (local) decode
+LOCAL = workloads.LOCAL_W512
+
+
+def _ring(lin, L, C):
+    """Ring of C rows (position p in row p % C) holding the last C positions of a linear
+    [B, L, H, d] bf16 cache; rows never written hold NaN, which must never reach a result."""
+    ring = torch.full((lin.shape[0], C) + tuple(lin.shape[2:]), float("nan"), dtype=torch.bfloat16)
+    for p in range(max(0, L - C), L):
+        ring[:, p % C] = lin[:, p]
+    return ring
+
+
+def check_ring(dec, layer, L, C, what, **kw):
+    b = binding()
+    dev = torch.device("cuda:0")
+    cfg = b.LayerCfg.from_layer(layer, **kw)
+    kr = _ring(dec.k, L, C)
+    vr = None if dec.v is None else _ring(dec.v, L, C)
+    out, lse = b.g4attn_decode_ring(dec.q.to(dev), kr.to(dev), None if vr is None else vr.to(dev),
+                                    L, cfg, want_lse=True)
+    torch.cuda.synchronize()
+    assert b.g4attn_device_status() == 0
+    ro, rl = oracle.decode_ring(dec.q[:, 0], kr, vr, L, ocfg(layer, **kw))
+    go, gl = to_np(out.cpu())[:, 0], to_np(lse.cpu())
+    assert np.all(np.isfinite(go)) and np.all(np.isfinite(gl))
+    assert_parity(go, ro, what + " out")
+    assert_parity(gl, rl, what + " lse")
+
+
+@pytest.mark.parametrize("L,C", [(1, 512), (100, 512), (512, 512), (513, 512), (700, 576),
+                                 (3001, 512), (5000, 1024)])
+def test_decode_ring_local_layer(L, C):
+    # local layer: 16 q / 8 kv heads, d 256, full RoPE base 1e4, window 512, separate values
+    dec = synth.decode_inputs(2, L, LOCAL.n_q_heads, LOCAL.n_kv_heads, LOCAL.head_dim, True,
+                              seed=60 + L)
+    check_ring(dec, LOCAL, L, C, "ring decode L=%d C=%d" % (L, C))
+
+
+def test_decode_ring_keys_as_values_with_window():
+    # a head_dim-512 keys-as-values layer with a window (the turned-slot path) on a ring
+    dec = synth.decode_inputs(2, 1000, 32, 4, 512, False, seed=61)
+    check_ring(dec, GLOBAL, 1000, 384, "ring decode K=V W=300", window=300)
+
+
+def test_decode_ring_rejects_bad_rings():
+    b = binding()
+    dev = torch.device("cuda:0")
+    dec = synth.decode_inputs(1, 10, 16, 8, 256, True, seed=62)
+    q = dec.q.to(dev)
+    kr = torch.zeros(1, 100, 8, 256, dtype=torch.bfloat16, device=dev)   # C not a multiple of 64
+    with pytest.raises(b.G4AttnError):
+        b.g4attn_decode_ring(q, kr, kr.clone(), 10, b.LayerCfg.from_layer(LOCAL))
+    kr = torch.zeros(1, 256, 8, 256, dtype=torch.bfloat16, device=dev)   # window 512 > C
+    with pytest.raises(b.G4AttnError):
+        b.g4attn_decode_ring(q, kr, kr.clone(), 10, b.LayerCfg.from_layer(LOCAL))

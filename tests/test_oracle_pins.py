@@ -332,3 +332,54 @@ def test_invalid_arguments_rejected():
         oracle.prefill_rows(inp.q, inp.k, inp.v, None, None, _cfg(6, 4, 8, kv_is_k=0))
     with pytest.raises(ValueError):   # separate values requested but none given
         oracle.prefill_rows(inp.q, inp.k, None, None, None, _cfg(6, 6, 8, kv_is_k=0))
+
+
+# --------------------------------------------------------------- ring-buffer decode
+def _ring_from_linear(lin_bits, L, C):
+    """Ring of C rows holding positions max(0, L-C) .. L-1 of a linear cache (row p % C);
+    rows never written hold a marker value that must never be read."""
+    ring = np.full((lin_bits.shape[0], C) + lin_bits.shape[2:], 0x7F80, np.uint16)   # +inf
+    for p in range(max(0, L - C), L):
+        ring[:, p % C] = lin_bits[:, p]
+    return ring
+
+
+@pytest.mark.parametrize("L,C,W,kv_is_k", [(5, 64, 16, 0), (40, 64, 64, 0), (100, 64, 48, 0),
+                                           (131, 128, 100, 1), (200, 64, 64, 1)])
+def test_decode_ring_matches_direct_attention(L, C, W, kv_is_k):
+    # direct computation from the ring: visible positions p in (L-1-W, L-1], key and value
+    # in ring row p % C, key turned to angle p
+    B, Hq, Hkv, d = 2, 4, 2, 32
+    dec = synth.decode_inputs(B, L, Hq, Hkv, d, kv_is_k == 0, seed=40 + L)
+    kring = _ring_from_linear(_bits(dec.k), L, C)
+    vring = None if dec.v is None else _ring_from_linear(_bits(dec.v), L, C)
+    cfg = _cfg(Hq, Hkv, d, p=1.0, base=1e4, window=W, kv_is_k=kv_is_k)
+    out, lse = oracle.decode_ring(dec.q[:, 0], kring, vring, L, cfg)
+    R = oracle.rope_pairs(d, 1.0)
+    pos = np.arange(max(0, L - W), L)
+    kf = bf.bf16_to_f64(kring[:, pos % C])
+    kr = bf.rope_complex(kf, pos, R, 1e4)
+    vf = kf if kv_is_k == 1 else bf.bf16_to_f64(vring[:, pos % C])
+    qf = bf.bf16_to_f64(_bits(dec.q))[:, 0]
+    for b in range(B):
+        for h in range(Hq):
+            s = (kr[b, :, h // (Hq // Hkv)] @ qf[b, h]) / math.sqrt(d)
+            w = np.exp(s - s.max())
+            np.testing.assert_allclose(out[b, h], (w / w.sum()) @ vf[b, :, h // (Hq // Hkv)],
+                                       atol=1e-13)
+            assert lse[b, h] == pytest.approx(s.max() + math.log(w.sum()), abs=1e-12)
+
+
+def test_decode_ring_agrees_across_capacities_and_with_the_linear_cache():
+    # the same last positions in rings of different sizes (and in the linear cache with the
+    # window) give bit-identical results
+    B, L, Hq, Hkv, d, W = 1, 150, 4, 1, 64, 60
+    dec = synth.decode_inputs(B, L, Hq, Hkv, d, True, seed=44)
+    kb, vb = _bits(dec.k), _bits(dec.v)
+    cfg = _cfg(Hq, Hkv, d, p=1.0, base=1e4, window=W, kv_is_k=0)
+    ref = oracle.decode(dec.q[:, 0], dec.k, dec.v, cfg)
+    for C in (64, 128, 192):
+        got = oracle.decode_ring(dec.q[:, 0], _ring_from_linear(kb, L, C),
+                                 _ring_from_linear(vb, L, C), L, cfg)
+        np.testing.assert_array_equal(got[0], ref[0])
+        np.testing.assert_array_equal(got[1], ref[1])
