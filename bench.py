@@ -217,6 +217,36 @@ def time_decode_128k(device, stream, reps=5):
     return {"workload": wl.name, "ms": t * 1e3, "gbs": wl.cache_bytes() / t / 1e9}
 
 
+def time_local_ring_decode(device, stream, reps=10):
+    """Decode step of the block's local layer (32 q / 16 kv heads, d 256, window 1024,
+    separate values) for 16 sequences at position 65535, against ring caches of 1024 rows:
+    the keys and values of the window, each read once."""
+    import torch
+    from attention_g4attn_b200 import binding as b, synth, workloads
+    ly = workloads.LOCAL_W1024
+    B, L, C = 16, 65536, 1024
+    d = synth.decode_inputs(B, C, ly.n_q_heads, ly.n_kv_heads, ly.head_dim, True, seed=9,
+                            device=device)   # the ring's rows are random: any ring content works
+    cfg = b.LayerCfg.from_layer(ly)
+    ws = torch.empty(b.g4attn_decode_ring_workspace_size(B, L, C, cfg), dtype=torch.uint8,
+                     device=device)
+    out = torch.empty_like(d.q)
+    for _ in range(3):
+        b.g4attn_decode_ring(d.q, d.k, d.v, L, cfg, out=out, workspace=ws, stream=stream)
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        b.g4attn_decode_ring(d.q, d.k, d.v, L, cfg, out=out, workspace=ws, stream=stream)
+        e1.record(stream)
+        e1.synchronize()
+        ts.append(e0.elapsed_time(e1) / 1e3)
+    t = statistics.median(ts)
+    nbytes = 2.0 * B * ly.n_kv_heads * ly.window * ly.head_dim * 2
+    return {"workload": "local_decode_ring_B16_pos65535_C1024_h32x16_d256_w1024", "ms": t * 1e3,
+            "gbs": nbytes / t / 1e9}
+
+
 # --------------------------------------------------------------------------- CPU oracle
 
 def oracle_sample(max_seconds=20.0, seed=0):
@@ -433,6 +463,8 @@ def main():
         extra["global_decode_L131072"] = time_decode_128k(device, stream)
         extra["global_decode_L131072"]["frac_of_hbm"] = \
             extra["global_decode_L131072"]["gbs"] / hbm_peak
+        extra["local_decode_ring"] = time_local_ring_decode(device, stream)
+        extra["local_decode_ring"]["frac_of_hbm"] = extra["local_decode_ring"]["gbs"] / hbm_peak
 
     # end to end through the public API with host buffers (pinned), copies inside the region
     e2e = None

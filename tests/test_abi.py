@@ -74,11 +74,13 @@ def test_prefill_workspace_formula(b):
     assert b.g4attn_prefill_workspace_size(2, 4096, loc) == _align(rows) + _align(4096 * 128 * 8)
 
 
-def _decode_segments(B, Hkv, L, window, pairs=74):
+def _decode_segments(B, Hkv, L, window, pairs=74, ring=0):
     """Stream-K split of a decode step, by brute force: the sequences' 128-key tiles form one
-    flat range cut evenly over the CTA pairs; returns the most pairs any sequence meets."""
+    flat range cut evenly over the CTA pairs; returns the most pairs any sequence meets.
+    With a ring cache the tiles start at the 64-aligned position at or below the window."""
     key_lo = L - window if (window > 0 and L > window) else 0
-    nt = -(-(L - key_lo) // 128)
+    base = key_lo // 64 * 64 if ring else key_lo
+    nt = -(-(L - base) // 128)
     W = B * Hkv * nt
     P = min(pairs, W)
     if W == 0:
@@ -102,6 +104,24 @@ def test_decode_workspace_follows_the_stream_k_split(b, B, L, layer):
     S = _decode_segments(B, Hkv, L, window)
     n = 2 * max(S, 1) * B * Hq
     assert b.g4attn_decode_workspace_size(B, L, cfg) == _align(n * d * 4) + _align(n * 2 * 4)
+
+
+@pytest.mark.parametrize("B,L,C", [(2, 3001, 512), (16, 1024, 1024), (1, 1, 512), (3, 700, 576),
+                                   (16, 70000, 1024)])
+def test_decode_ring_workspace_follows_the_aligned_split(b, B, L, C):
+    loc = b.LayerCfg(16, 8, 256, 1.0, 1e4, 512, None, 0)
+    S = _decode_segments(B, 8, L, 512, ring=C)
+    n = 2 * max(S, 1) * B * 16
+    assert b.g4attn_decode_ring_workspace_size(B, L, C, loc) == _align(n * 256 * 4) + _align(n * 2 * 4)
+
+
+def test_decode_ring_rejects_bad_rings_without_gpu(b):
+    loc = b.LayerCfg(16, 8, 256, 1.0, 1e4, 512, None, 0)
+    assert b.g4attn_decode_ring_workspace_size(1, 10, 100, loc) == 0   # C not a multiple of 64
+    assert b.g4attn_decode_ring_workspace_size(1, 10, 256, loc) == 0   # window 512 > C
+    assert b.g4attn_decode_ring_workspace_size(1, 10, 0, loc) == 0
+    nowin = b.LayerCfg(16, 8, 256, 1.0, 1e4, 0, None, 0)
+    assert b.g4attn_decode_ring_workspace_size(1, 10, 512, nowin) == 0  # no window: no ring
 
 
 def test_invalid_configs_are_rejected(b):
