@@ -94,6 +94,7 @@ def _load():
         "g4attn_decode_noalloc": (I, [P, P, P, I, P, P, I, CFG, P]),
         "g4attn_decode_ring_workspace_size": (SZ, [I, I, I, CFG]),
         "g4attn_decode_ring": (I, [P, P, P, I, I, P, P, P, SZ, I, CFG, P]),
+        "g4attn_decode_split_cache": (I, [P, P, P, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_status_string": (ctypes.c_char_p, [I]),
         "g4attn_device_status": (I, [P]),
         "g4attn_set_wait_limit": (LL, [LL]),
@@ -268,6 +269,28 @@ def g4attn_decode_ring(q, kring, vring, L: int, cfg: LayerCfg, out=None, lse=Non
                                  _ptr(lse), _ptr(workspace), workspace.numel(), B,
                                  ctypes.byref(c), _stream(stream))
     _check(rc, "g4attn_decode_ring")
+    return out, lse
+
+
+def g4attn_decode_split_cache(q, krot, vside, cfg: LayerCfg, out=None, lse=None, want_lse=False,
+                              workspace=None, stream=None):
+    """Decode one token against the split cache: krot [B,L,Hkv,d] rotated keys and vside
+    [B,L,Hkv,128] pre-RoPE values of the rotated dims."""
+    for t, n in ((q, "q"), (krot, "krot"), (vside, "vside")):
+        _bf16(t, n)
+    B, L = krot.shape[0], krot.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.n_q_heads), dtype=torch.float32, device=q.device)
+    c = cfg.c()
+    ws_bytes = _lib.g4attn_decode_workspace_size(B, L, ctypes.byref(c))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    rc = _lib.g4attn_decode_split_cache(_ptr(q), _ptr(krot), _ptr(vside), L, _ptr(out),
+                                        _ptr(lse), _ptr(workspace), workspace.numel(), B,
+                                        ctypes.byref(c), _stream(stream))
+    _check(rc, "g4attn_decode_split_cache")
     return out, lse
 
 

@@ -267,7 +267,8 @@ int check_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_b
 int launch_decode_plan(const g4attn_bf16* q, const g4attn_bf16* kcache,
                        const g4attn_bf16* vcache, int L, int rows, int ring, g4attn_bf16* out,
                        float* lse, uint8_t* w, const DecodePlan& plan, int B,
-                       const g4attn_layer_cfg* cfg, const DeviceInfo* dev, g4attn_stream_t stream) {
+                       const g4attn_layer_cfg* cfg, const DeviceInfo* dev, g4attn_stream_t stream,
+                       const g4attn_bf16* vside = nullptr) {
     g4::DecodeArgs a{};
     const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
     int rc;
@@ -292,6 +293,17 @@ int launch_decode_plan(const g4attn_bf16* q, const g4attn_bf16* kcache,
     a.n_pairs = plan.n_pairs;
     a.total_tiles = plan.total_tiles;
     a.rope = make_rope(cfg);
+    if (vside) {
+        // split cache: keys arrive rotated, so the kernel turns nothing (R = 0); slot 0's
+        // values come from the side copy of the 2R = 128 rotated dims
+        if (L > 0) {
+            const int seen = L < rows ? L : rows;
+            if ((rc = encode_rows(&a.tm_vside, vside, B, seen, Hkv, 128, false, 64, rows)))
+                return rc;
+        }
+        a.split_cache = 1;
+        a.rope.R = 0;
+    }
     a.scale_log2 = cfg->scale * 1.4426950408889634f;
     a.kv_is_k = cfg->kv_is_k;
     a.wait_limit = g_wait_limit.load();
@@ -496,6 +508,25 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
     return launch_decode_plan(q, kcache, vcache, L, L, 0, out, lse,
                               static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream);
+}
+
+int g4attn_decode_split_cache(const g4attn_bf16* q, const g4attn_bf16* krot,
+                              const g4attn_bf16* vside, int L, g4attn_bf16* out, float* lse,
+                              void* workspace, size_t ws_bytes, int B, const g4attn_layer_cfg* cfg,
+                              g4attn_stream_t stream) {
+    int rc = check_decode(q, krot, nullptr, L, out, lse, B, cfg);
+    if (rc) return rc;
+    if (cfg->kv_is_k != 1 || rope_pairs(cfg) != 64) return G4ATTN_ERR_UNSUPPORTED;
+    if (B > 0 && L > 0 && !vside) return G4ATTN_ERR_INVALID_ARG;
+    if (vside && !aligned16(vside)) return G4ATTN_ERR_MISALIGNED;
+    if (B == 0) return G4ATTN_OK;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    const DecodePlan plan = decode_plan(B, L, cfg, dev->sms);
+    if (!workspace || ws_bytes < plan.total) return G4ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
+    return launch_decode_plan(q, krot, nullptr, L, L, 0, out, lse,
+                              static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream, vside);
 }
 
 size_t g4attn_decode_ring_workspace_size(int B, int L, int C, const g4attn_layer_cfg* cfg) {

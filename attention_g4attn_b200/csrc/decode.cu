@@ -172,7 +172,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int pair = blockIdx.x >> 1;
     const PairRange pr = pair_range(a, pair);
     const int n_items = pr.n_items;   // this pair's items
-    const int slots_per_tile = sep_v ? 2 * NSB : NSB;
+    // split cache: the key slots (already rotated) and one value slot for the rotated dims
+    const bool split = a.split_cache != 0;
+    const int slots_per_tile = sep_v ? 2 * NSB : (split ? NSB + 1 : NSB);
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NSLOT; ++i) {
@@ -211,6 +213,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             prefetch_tmap(&a.tm_k);
             if (sep_v) prefetch_tmap(&a.tm_v);
+            if (split) prefetch_tmap(&a.tm_vside);
             uint32_t q = 0;   // ring slots filled so far
             for (int it = 0; it < n_items && !*abort; ++it) {
                 const Item w = item_of(a, pair, pr, it);
@@ -230,6 +233,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             tma_load_4d(sm.ring[slot], map, &sm.full[slot], sb * 64, w.g, key, w.b);
                             tma_load_4d(sm.ring[slot] + kBoxBytes, map, &sm.full[slot],
                                         D / 2 + sb * 64, w.g, key, w.b);
+                            ++q;
+                        }
+                    }
+                    if (split && !*abort) {
+                        // pre-RoPE values of the rotated dims: first-half dims in rows k,
+                        // their partners (d/2 + ...) in rows 64 + k, like slot 0
+                        const int slot = q % NSLOT;
+                        if (mbar_wait(&sm.empty[slot], ((q / NSLOT) & 1) ^ 1, wc, abort)) {
+                            mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes);
+                            tma_load_4d(sm.ring[slot], &a.tm_vside, &sm.full[slot], 0, w.g, key, w.b);
+                            tma_load_4d(sm.ring[slot] + kBoxBytes, &a.tm_vside, &sm.full[slot], 64,
+                                        w.g, key, w.b);
                             ++q;
                         }
                     }
@@ -287,7 +302,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const uint32_t qv = sep_v ? pc.q + NSB : pc.q;
 #pragma unroll
                     for (int sb = 0; sb < NSB; ++sb) {
-                        const uint32_t slot = (qv + sb) % NSLOT;
+                        // split cache: slot 0's values come from the tile's extra slot
+                        const uint32_t slot = (split && sb == 0 ? pc.q + NSB : qv + sb) % NSLOT;
                         // 16 keys per step = two 8-row groups of 1024 B
                         mma4_pair(tm_o + sb * NS, d_ring_mn + slot * kSlotDesc, 2048 >> 4, pb,
                                   32 >> 4, idesc_o, pc.t == 0 ? 0u : 1u);
@@ -313,8 +329,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const uint64_t bd = d_q + ((REL && sb == 0 && (sc.g & 1)) ? 4 : sb) * kQDesc;
                         mma4_pair(tm_s, ad, 32 >> 4, bd, 32 >> 4, idesc_s, acc);
                         acc = 1;
-                        // score slots of a separate-value layer go back right away
-                        if (sep_v) mma_commit_pair(&sm.empty[slot]);
+                        // score slots of a separate-value layer (and the rotated key slot of a
+                        // split cache) go back right away
+                        if (sep_v || (split && sb == 0)) mma_commit_pair(&sm.empty[slot]);
                     }
                     mma_commit_pair(&sm.s_full[sc.g & 1]);
                     if (sc.t == sc.nt - 1) mma_commit_pair(&sm.q_free);   // q may be restaged

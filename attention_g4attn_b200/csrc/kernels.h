@@ -42,6 +42,11 @@ cudaError_t launch_wait_selftest(int* status, long long limit, cudaStream_t stre
 struct DecodeArgs {
     CUtensorMap tm_k;       // kcache [B, L or C, Hkv, d] as a 4-D map (d, Hkv, rows, B), box (64, 1, 64, 1)
     CUtensorMap tm_v;       // vcache, same geometry (kv_is_k == 0), else a copy of tm_k
+    // split cache (split_cache = 1): tm_k holds keys rotated to their positions, tm_vside the
+    // pre-RoPE values of the 2R = 128 rotated dims [B, L, Hkv, 128] (the value operand of
+    // slot 0; the other slots' dims are the same rotated or not); no key is turned
+    CUtensorMap tm_vside;
+    int split_cache;
     const uint16_t* q;      // [B, Hq, d], normalised and rotated
     float* part_o;          // [2S, B, Hq, d]
     float* part_ml;         // [2S, B, Hq, 2]  (running max in log2 units, sum)

@@ -161,6 +161,24 @@ G4ATTN_API int g4attn_decode_ring(const g4attn_bf16* q, const g4attn_bf16* kring
                                   const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
 
 /*
+ * Decode against the split cache layout of a keys-as-values layer with R = 64 rotated pairs
+ * (the global layers' p-RoPE: head_dim 512, p = 0.25): the keys are stored already rotated
+ * to their positions, plus a side copy of the pre-RoPE values of the 2R = 128 rotated dims:
+ * 1.25 * d elements per key instead of 2 * d for separate rotated keys and values, 37.5%
+ * less (the global-layer cache saving the Gemma 4 report quotes).  No key is turned on the
+ * fly; the values are the pre-RoPE keys as in g4attn_decode with kv_is_k = 1.
+ *   krot    [B, L, Hkv, d] bf16: normalised keys, rotated to their positions
+ *   vside   [B, L, Hkv, 128] bf16: the same keys' pre-RoPE dims [0, 64) then [d/2, d/2 + 64)
+ *   workspace / ws_bytes  >= g4attn_decode_workspace_size(B, L, cfg)
+ * Other arguments and results as in g4attn_decode.  Needs kv_is_k = 1 and R = 64
+ * (G4ATTN_ERR_UNSUPPORTED otherwise).
+ */
+G4ATTN_API int g4attn_decode_split_cache(const g4attn_bf16* q, const g4attn_bf16* krot,
+                                         const g4attn_bf16* vside, int L, g4attn_bf16* out,
+                                         float* lse, void* workspace, size_t ws_bytes, int B,
+                                         const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/*
  * Decode without a workspace and without allocating (the papers describe no such call;
  * it exists for callers that cannot allocate device memory: plugins whose host framework
  * owns every device allocation and hands them only input and output buffers, and services

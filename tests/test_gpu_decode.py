@@ -171,3 +171,41 @@ def test_decode_ring_rejects_bad_rings():
     kr = torch.zeros(1, 256, 8, 256, dtype=torch.bfloat16, device=dev)   # window 512 > C
     with pytest.raises(b.G4AttnError):
         b.g4attn_decode_ring(q, kr, kr.clone(), 10, b.LayerCfg.from_layer(LOCAL))
+
+
+# ------------------------------------------------------------------- split cache (37.5%)
+def _split_cache(k_pre, R, base):
+    """Rotated keys (each turned to its position, rounded to bf16) and the side copy of the
+    pre-RoPE rotated dims [0, R) and [d/2, d/2 + R) of a pre-RoPE bf16 cache."""
+    import bruteforce as bf
+    kf = bf.bf16_to_f64(oracle.bf16_bits(k_pre))
+    L, d = kf.shape[1], kf.shape[-1]
+    krot = torch.from_numpy(bf.rope_complex(kf, np.arange(L), R, base)).to(torch.bfloat16)
+    vside = torch.cat([k_pre[..., :R], k_pre[..., d // 2:d // 2 + R]], dim=-1).contiguous()
+    return krot, vside
+
+
+@pytest.mark.parametrize("L", [1, 129, 1000, 4097])
+def test_decode_split_cache_matches_keys_as_values(L):
+    b = binding()
+    dev = torch.device("cuda:0")
+    dec = synth.decode_inputs(2, L, 32, 4, 512, False, seed=70 + L)
+    krot, vside = _split_cache(dec.k, 64, GLOBAL.rope_base)
+    cfg = b.LayerCfg.from_layer(GLOBAL)
+    out, lse = b.g4attn_decode_split_cache(dec.q.to(dev), krot.to(dev), vside.to(dev), cfg,
+                                           want_lse=True)
+    torch.cuda.synchronize()
+    assert b.g4attn_device_status() == 0
+    ro, rl = oracle.decode(dec.q[:, 0], dec.k, None, ocfg(GLOBAL))
+    assert_parity(to_np(out.cpu())[:, 0], ro, "split cache L=%d out" % L)
+    assert_parity(to_np(lse.cpu()), rl, "split cache L=%d lse" % L)
+
+
+def test_decode_split_cache_needs_keys_as_values_and_r64():
+    b = binding()
+    dev = torch.device("cuda:0")
+    dec = synth.decode_inputs(1, 10, 16, 8, 256, False, seed=71)
+    z = torch.zeros(1, 10, 8, 128, dtype=torch.bfloat16, device=dev)
+    with pytest.raises(b.G4AttnError):   # local layer: R = 128
+        b.g4attn_decode_split_cache(dec.q.to(dev), dec.k.to(dev), z,
+                                    b.LayerCfg.from_layer(workloads.LOCAL_W512, kv_is_k=1))
