@@ -528,9 +528,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // from the start of the pair-tile, so its (cos, sin) are fixed per thread; the start
         // angle goes onto the query, which both CTAs' keys share in the pair MMA:
         // q' = R(-key0 theta) q, and q' . R((64 rank + rk) theta) k equals
-        // q . R((key0 + 64 rank + rk) theta) k.  rc / rs hold (cos, cos) / (sin, sin) of the
-        // column pairs (2m, 2m + 1) of this thread, as packed fp32 pairs.
-        float2 rc[REL ? 16 : 1], rs[REL ? 16 : 1];
+        // q . R((key0 + 64 rank + rk) theta) k.  rc / rs / rn hold cos / sin / -sin of the
+        // column pairs (2m, 2m + 1) of this thread as packed bf16 pairs: the turn runs on
+        // bf16x2 multiply-adds, 4 per pair of columns (fp32 math with its unpacking and
+        // repacking took 11 and sat on the per-tile chain, 6% of the decode rate)
+        __nv_bfloat162 rc[REL ? 16 : 1], rs[REL ? 16 : 1], rn[REL ? 16 : 1];
         float qx[REL ? QH : 1], qy[REL ? QH : 1];    // REL: pair rk of q, heads cp + 2j
         float2 bcs = make_float2(1.f, 0.f);          // REL: cos/sin of pair start * theta_rk
         float2 stp = make_float2(1.f, 0.f);          // REL: cos/sin of 128 * theta_rk
@@ -592,8 +594,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
                 if (i0 < R) turn(i0, s0, c0);
                 if (i0 + 1 < R) turn(i0 + 1, s1, c1);
-                rc[m] = make_float2(c0, c1);
-                rs[m] = make_float2(s0, s1);
+                rc[m] = __floats2bfloat162_rn(c0, c1);
+                rs[m] = __floats2bfloat162_rn(s0, s1);
+                rn[m] = __floats2bfloat162_rn(-s0, -s1);
             }
             if (rk < R) stp = sm.step_cs[rk];
         }
@@ -702,13 +705,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                 uint32_t* w2 = &x2.x;
 #pragma unroll
                                 for (int m = 0; m < 4; ++m) {
-                                    const float2 u = bf16x2_to_f2(w1[m]);
-                                    const float2 v = bf16x2_to_f2(w2[m]);
-                                    const float2 c = rc[4 * g8 + m], sn = rs[4 * g8 + m];
-                                    const float2 u2 = sub_f2(mul_f2(u, c), mul_f2(v, sn));
-                                    const float2 v2 = fma_f2(u, sn, mul_f2(v, c));
-                                    w1[m] = pack_bf16x2(u2.x, u2.y);
-                                    w2[m] = pack_bf16x2(v2.x, v2.y);
+                                    const __nv_bfloat162 u = *reinterpret_cast<const __nv_bfloat162*>(&w1[m]);
+                                    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&w2[m]);
+                                    const int i = 4 * g8 + m;
+                                    const __nv_bfloat162 u2 = __hfma2(u, rc[i], __hmul2(v, rn[i]));
+                                    const __nv_bfloat162 v2 = __hfma2(u, rs[i], __hmul2(v, rc[i]));
+                                    w1[m] = *reinterpret_cast<const uint32_t*>(&u2);
+                                    w2[m] = *reinterpret_cast<const uint32_t*>(&v2);
                                 }
                             }
                             *reinterpret_cast<uint4*>(dst + o1) = x1;
