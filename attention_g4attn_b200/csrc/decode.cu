@@ -788,12 +788,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
 }
 
-// Merge the partials of one (b, h): two per split, one from each CTA of the pair,
+// Merge the partials of one (b, h): two per segment, one from each CTA of the pair,
 //   out = sum_p 2^(m_p - M) O_p / sum_p 2^(m_p - M) l_p,   M = max_p m_p (log2 units).
-// Block (b h, 128-dim chunk), thread = one dim: the per-part weights are computed once per
-// block into shared memory, then every thread streams its dim of all the partials.
+// Block (b h, 128-dim chunk), thread = one dim.
 constexpr int kCombineThreads = 128;
-constexpr int kMaxParts = 1024;
+constexpr int kMaxParts = 1024;   // sanity bound on the partials per sequence
 
 __global__ void __launch_bounds__(kCombineThreads)
     decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
@@ -801,11 +800,8 @@ __global__ void __launch_bounds__(kCombineThreads)
     // the decode's last CTAs finish; the partials are read only after the decode grid has
     // completed and its writes are visible
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    __shared__ float wgt[kMaxParts];
-    __shared__ float red[kCombineThreads / 32];
-    __shared__ float bM, bDen;
     const int bh = blockIdx.x;   // b * Hq + h
-    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    const int tid = threadIdx.x;
     const size_t stride = (size_t)a.B * a.Hq;
     // the segments of this (b, h)'s sequence: one per pair whose tiles it spans
     int nseg = 0;
@@ -814,59 +810,23 @@ __global__ void __launch_bounds__(kCombineThreads)
         nseg = pair_of_tile(a, s0 + a.tiles_per_seq - 1) - pair_of_tile(a, s0) + 1;
     }
     const int parts = 2 * nseg;
-    // running maxima of the parts, and their largest
-    float mx = -INFINITY;
-    for (int s = tid; s < parts; s += kCombineThreads) {
-        const float m = a.part_ml[(s * stride + bh) * 2];
-        wgt[s] = m;
-        mx = fmaxf(mx, m);
-    }
-    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    if (lane == 0) red[wp] = mx;
-    __syncthreads();
-    if (tid == 0) {
-        float M = red[0];
-        for (int i = 1; i < kCombineThreads / 32; ++i) M = fmaxf(M, red[i]);
-        bM = M;
-    }
-    __syncthreads();
-    const float M = bM;
-    // weights 2^(m_p - M) and their sum with the running sums
-    float den = 0.f;
-    for (int s = tid; s < parts; s += kCombineThreads) {
-        const float m = wgt[s];
-        const float w = (m == -INFINITY) ? 0.f : exp2f(m - M);
-        wgt[s] = w;
-        den += w * a.part_ml[(s * stride + bh) * 2 + 1];
-    }
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    __syncthreads();   // red[] reuse
-    if (lane == 0) red[wp] = den;
-    __syncthreads();
-    if (tid == 0) {
-        float t = 0.f;
-        for (int i = 0; i < kCombineThreads / 32; ++i) t += red[i];
-        bDen = t;
-    }
-    __syncthreads();
-    const float dsum = bDen;
-    const float inv = dsum > 0.f ? 1.f / dsum : 0.f;
+    // a sequence has a few parts: every thread reads their (max, sum) itself (the same
+    // addresses across the block) and forms the weights, with no block-wide reduction
+    const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + bh;
+    float M = -INFINITY;
+    for (int s = 0; s < parts; ++s) M = fmaxf(M, ml[s * stride].x);
     const int c = blockIdx.y * kCombineThreads + tid;
-    if (c < a.d) {
-        const float* po = a.part_o + (size_t)bh * a.d + c;
-        const size_t ps = stride * a.d;
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-        int s = 0;
-        for (; s + 4 <= parts; s += 4) {
-            acc0 += wgt[s] * po[s * ps];
-            acc1 += wgt[s + 1] * po[(s + 1) * ps];
-            acc2 += wgt[s + 2] * po[(s + 2) * ps];
-            acc3 += wgt[s + 3] * po[(s + 3) * ps];
-        }
-        for (; s < parts; ++s) acc0 += wgt[s] * po[s * ps];
-        const float acc = (acc0 + acc1) + (acc2 + acc3);
-        a.out[(size_t)bh * a.d + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc * inv));
+    const float* po = a.part_o + (size_t)bh * a.d + c;
+    const size_t ps = stride * a.d;
+    float dsum = 0.f, acc = 0.f;
+    for (int s = 0; s < parts; ++s) {
+        const float2 p = ml[s * stride];
+        const float w = (p.x == -INFINITY) ? 0.f : exp2f(p.x - M);
+        dsum += w * p.y;
+        if (c < a.d) acc += w * po[s * ps];
     }
+    const float inv = dsum > 0.f ? 1.f / dsum : 0.f;
+    if (c < a.d) a.out[(size_t)bh * a.d + c] = __bfloat16_as_ushort(__float2bfloat16_rn(acc * inv));
     if (tid == 0 && blockIdx.y == 0 && a.lse)
         a.lse[bh] = dsum > 0.f ? (M + log2f(dsum)) * 0.6931471805599453f : -INFINITY;
 }
