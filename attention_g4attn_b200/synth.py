@@ -70,3 +70,30 @@ def decode_inputs(B, L, n_q_heads, n_kv_heads, head_dim, separate_v, seed, devic
     gamma_q = 1.0 + 0.1 * _randn((head_dim,), gen, device)
     gamma_k = 1.0 + 0.1 * _randn((head_dim,), gen, device)
     return LayerInputs(q, kcache, vcache, gamma_q.contiguous(), gamma_k.contiguous())
+
+
+@dataclass
+class ChunkInputs:
+    q: torch.Tensor                 # [B, Tn, Hq, d] raw queries of the chunk
+    k: torch.Tensor                 # [B, Tn, Hkv, d] raw keys of the chunk
+    v: Optional[torch.Tensor]       # [B, Tn, Hkv, d] raw values of the chunk
+    kcache: torch.Tensor            # [B, P, Hkv, d] cached (already normalised) keys
+    vcache: Optional[torch.Tensor]  # [B, P, Hkv, d] cached values
+    gamma_q: torch.Tensor
+    gamma_k: torch.Tensor
+
+
+def chunk_inputs(B, P, Tn, n_q_heads, n_kv_heads, head_dim, separate_v, seed, device="cpu"):
+    """One prefill chunk: raw q/k/v of Tn tokens (as layer_inputs) plus the cache of the P
+    earlier positions, N(0,1) bf16 values used as if already normalised (as decode_inputs)."""
+    gen = torch.Generator(device=device).manual_seed(int(seed))
+    q = _randn_bf16((B, Tn, n_q_heads, head_dim), gen, device)
+    k = _randn_bf16((B, Tn, n_kv_heads, head_dim), gen, device)
+    kcache = _randn_bf16((B, P, n_kv_heads, head_dim), gen, device)
+    v = vcache = None
+    if separate_v:
+        v = _randn_bf16((B, Tn, n_kv_heads, head_dim), gen, device)
+        vcache = _randn_bf16((B, P, n_kv_heads, head_dim), gen, device)
+    gamma_q = 1.0 + 0.1 * _randn((head_dim,), gen, device)
+    gamma_k = 1.0 + 0.1 * _randn((head_dim,), gen, device)
+    return ChunkInputs(q, k, v, kcache, vcache, gamma_q.contiguous(), gamma_k.contiguous())

@@ -13,5 +13,6 @@ from .oracle import (  # noqa: F401
     prefill_rows,
     decode,
     decode_ring,
+    prefill_chunk,
     bf16_bits,
 )

@@ -5,7 +5,7 @@ widens them exactly to double.  Outputs are float64 numpy arrays.
 """
 import ctypes
 import math
-from dataclasses import dataclass
+from dataclasses import dataclass, replace
 
 import numpy as np
 
@@ -195,3 +195,67 @@ def decode_ring(q, kring, vring, L: int, cfg: OracleCfg, nthreads: int = 0):
         if vb is not None:
             v_lin[:, p] = vb[:, p % C]
     return decode(q, k_lin, v_lin, cfg, nthreads=nthreads)
+
+
+def _widen(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns to float64, exactly (the bits are the top half of an fp32)."""
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def prefill_chunk(q, k, v, kcache, vcache, gamma_q, gamma_k, P: int, cfg: OracleCfg, rows=None):
+    """Prefill of one chunk of a longer prompt (the attention of Gemma 4 report section 2,
+    taken a chunk at a time against the cache the earlier chunks left).
+
+    The chunk's Tn tokens sit at positions P .. P+Tn-1.  Keys at positions j < P are the
+    cache rows 0 .. P-1 as stored (already normalised, not rotated); the chunk's keys get
+    QKNorm here.  Key j is turned to angle j and the query of chunk token t, after QKNorm,
+    to angle P + t.  Token t sees the keys j <= P + t, and on a window-W layer only those
+    with j > P + t - W.  Softmax of the scaled scores weighs the values: the unrotated key
+    (kv_is_k = 1), the rotated key (2), or the separate value (0: vcache rows 0 .. P-1, then
+    the chunk's v).
+
+    Written out as that definition; the scores and the weighted sums are float64 numpy
+    matrix products over all P + Tn keys of a (batch, head).
+    Returns (out [B, nrows, Hq, d], lse [B, Hq, nrows]) for the chunk tokens `rows`."""
+    qb, kb, cb = bf16_bits(q), bf16_bits(k), bf16_bits(kcache)
+    B, Tn, Hq, d = qb.shape
+    Hkv = cfg.n_kv_heads
+    G = Hq // Hkv
+    if cb.shape[1] < P:
+        raise ValueError("the cache holds fewer than P positions")
+    rows = np.arange(Tn) if rows is None else np.asarray(rows, dtype=np.int64)
+    # the chunk: queries normalised and turned to P + t, keys normalised (and turned)
+    qr, kh_new, kr_new = qknorm_rope(qb, kb, gamma_q, gamma_k, cfg, pos0=P)
+    if P > 0:
+        # the cached keys are used as stored: rotation only
+        _, kh_old, kr_old = qknorm_rope(None, cb[:, :P], None, None, replace(cfg, qk_norm=0))
+        kh = np.concatenate([kh_old, kh_new], axis=1)
+        kr = np.concatenate([kr_old, kr_new], axis=1)
+    else:
+        kh, kr = kh_new, kr_new
+    if cfg.kv_is_k == 1:
+        vals = kh
+    elif cfg.kv_is_k == 2:
+        vals = kr
+    else:
+        vb = _widen(bf16_bits(v))
+        vals = np.concatenate([_widen(bf16_bits(vcache)[:, :P]), vb], axis=1) if P > 0 else vb
+    scale = cfg.scale if cfg.scale is not None else 1.0 / math.sqrt(d)
+    pos_q = P + rows                                  # positions of the chunk rows asked for
+    pos_k = np.arange(P + Tn)
+    vis = pos_k[None, :] <= pos_q[:, None]
+    if cfg.window and cfg.window > 0:
+        vis &= pos_k[None, :] > pos_q[:, None] - cfg.window
+    out = np.zeros((B, len(rows), Hq, d))
+    lse = np.zeros((B, Hq, len(rows)))
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            s = scale * (qr[b, rows, h] @ kr[b, :, g].T)          # [nrows, P + Tn]
+            s = np.where(vis, s, -np.inf)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            den = e.sum(axis=1, keepdims=True)
+            out[b, :, h] = (e / den) @ vals[b, :, g]
+            lse[b, h] = m[:, 0] + np.log(den[:, 0])
+    return out, lse

@@ -383,3 +383,82 @@ def test_decode_ring_agrees_across_capacities_and_with_the_linear_cache():
                                  _ring_from_linear(vb, L, C), L, cfg)
         np.testing.assert_array_equal(got[0], ref[0])
         np.testing.assert_array_equal(got[1], ref[1])
+
+
+# --------------------------------------------------------------- chunked prefill
+def _direct_chunk(ch, P, cfg):
+    """Chunk attention computed directly, row by row, with the complex-number RoPE and an
+    explicit list of the visible positions of each query."""
+    R = int(np.floor(cfg.rope_p * cfg.head_dim / 2))
+    kc = bf.bf16_to_f64(_bits(ch.kcache))
+    kn = bf.bf16_to_f64(_bits(ch.k))
+    q = bf.bf16_to_f64(_bits(ch.q))
+    if cfg.qk_norm:
+        kn = bf.rms(kn, ch.gamma_k.double().numpy(), 1e-6)
+        q = bf.rms(q, ch.gamma_q.double().numpy(), 1e-6)
+    B, Tn, Hq, d = q.shape
+    khat = np.concatenate([kc, kn], axis=1)
+    krot = bf.rope_complex(khat, np.arange(P + Tn), R, cfg.rope_base)
+    qrot = bf.rope_complex(q, P + np.arange(Tn), R, cfg.rope_base)
+    if cfg.kv_is_k == 1:
+        vals = khat
+    elif cfg.kv_is_k == 2:
+        vals = krot
+    else:
+        vals = np.concatenate([bf.bf16_to_f64(_bits(ch.vcache)), bf.bf16_to_f64(_bits(ch.v))], axis=1)
+    G = Hq // cfg.n_kv_heads
+    out = np.zeros_like(q)
+    lse = np.zeros((B, Hq, Tn))
+    for b in range(B):
+        for h in range(Hq):
+            for t in range(Tn):
+                i = P + t
+                js = [j for j in range(i + 1) if cfg.window == 0 or j > i - cfg.window]
+                s = np.array([qrot[b, t, h] @ krot[b, j, h // G] for j in js]) / math.sqrt(d)
+                w = np.exp(s - s.max())
+                out[b, t, h] = (w / w.sum()) @ vals[b, js, h // G]
+                lse[b, h, t] = s.max() + math.log(w.sum())
+    return out, lse
+
+
+@pytest.mark.parametrize("P,Tn,W,kv_is_k,qk_norm,p", [
+    (0, 12, 0, 1, 1, 0.25), (20, 9, 0, 1, 1, 0.25), (33, 16, 8, 0, 1, 1.0),
+    (40, 7, 16, 2, 0, 1.0), (5, 30, 4, 1, 1, 1.0), (64, 3, 0, 0, 0, 0.5)])
+def test_prefill_chunk_matches_direct_attention(P, Tn, W, kv_is_k, qk_norm, p):
+    B, Hq, Hkv, d = 2, 4, 2, 32
+    ch = synth.chunk_inputs(B, P, Tn, Hq, Hkv, d, kv_is_k == 0, seed=60 + P + Tn)
+    cfg = _cfg(Hq, Hkv, d, p=p, base=1e4, window=W, kv_is_k=kv_is_k, qk_norm=qk_norm)
+    out, lse = oracle.prefill_chunk(ch.q, ch.k, ch.v, ch.kcache, ch.vcache, ch.gamma_q,
+                                    ch.gamma_k, P, cfg)
+    ref_o, ref_l = _direct_chunk(ch, P, cfg)
+    np.testing.assert_allclose(out, ref_o, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(lse, ref_l, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("P,Tn,W,kv_is_k", [(48, 16, 0, 1), (37, 27, 20, 0), (100, 1, 0, 2)])
+def test_prefill_chunk_equals_rows_of_the_full_prefill(P, Tn, W, kv_is_k):
+    # without QKNorm a cached key is the raw key itself, so a chunk at P must give the
+    # full-sequence prefill's rows P .. P+Tn-1
+    B, Hq, Hkv, d = 1, 8, 2, 64
+    inp = synth.layer_inputs(B, P + Tn, Hq, Hkv, d, kv_is_k == 0, seed=70 + P)
+    cfg = _cfg(Hq, Hkv, d, p=0.25, base=1e6, window=W, kv_is_k=kv_is_k, qk_norm=0)
+    rows = np.arange(P, P + Tn, dtype=np.int32)
+    ref_o, ref_l = oracle.prefill_rows(inp.q, inp.k, inp.v, None, None, cfg, rows)
+    v = None if inp.v is None else inp.v[:, P:]
+    vc = None if inp.v is None else inp.v[:, :P]
+    out, lse = oracle.prefill_chunk(inp.q[:, P:], inp.k[:, P:], v, inp.k[:, :P], vc, None, None,
+                                    P, cfg)
+    np.testing.assert_allclose(out, ref_o, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(lse, ref_l, atol=1e-12, rtol=0)
+
+
+def test_prefill_chunk_at_zero_is_the_prefill():
+    B, T, Hq, Hkv, d = 2, 40, 8, 1, 64
+    inp = synth.layer_inputs(B, T, Hq, Hkv, d, False, seed=75)
+    cfg = _cfg(Hq, Hkv, d, p=0.25, base=1e6, window=0, kv_is_k=1, qk_norm=1)
+    ref_o, ref_l = oracle.prefill_rows(inp.q, inp.k, None, inp.gamma_q, inp.gamma_k, cfg)
+    empty = torch.zeros((B, 0, Hkv, d), dtype=torch.bfloat16)
+    out, lse = oracle.prefill_chunk(inp.q, inp.k, None, empty, None, inp.gamma_q, inp.gamma_k,
+                                    0, cfg)
+    np.testing.assert_allclose(out, ref_o, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(lse, ref_l, atol=1e-12, rtol=0)
