@@ -89,6 +89,8 @@ def _load():
         "g4attn_qknorm_rope": (I, [P, P, P, P, P, P, P, I, I, LL, CFG, P]),
         "g4attn_prefill_workspace_size": (SZ, [I, I, CFG]),
         "g4attn_prefill": (I, [P, P, P, P, P, P, P, P, SZ, I, I, CFG, P]),
+        "g4attn_prefill_chunk_workspace_size": (SZ, [I, I, I, CFG]),
+        "g4attn_prefill_chunk": (I, [P, P, P, P, P, P, P, I, I, P, P, P, SZ, I, I, I, CFG, P]),
         "g4attn_decode_workspace_size": (SZ, [I, I, CFG]),
         "g4attn_decode": (I, [P, P, P, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_decode_noalloc": (I, [P, P, P, I, P, P, I, CFG, P]),
@@ -221,6 +223,38 @@ def g4attn_prefill(q, k, v, gamma_q, gamma_k, cfg: LayerCfg, out=None, lse=None,
                              _ptr(out), _ptr(lse), _ptr(workspace), workspace.numel(), B, T,
                              ctypes.byref(c), _stream(stream))
     _check(rc, "g4attn_prefill")
+    return out, lse
+
+
+def g4attn_prefill_chunk_workspace_size(B: int, P: int, Tn: int, cfg: LayerCfg) -> int:
+    c = cfg.c()
+    return _lib.g4attn_prefill_chunk_workspace_size(B, P, Tn, ctypes.byref(c))
+
+
+def g4attn_prefill_chunk(q, k, v, gamma_q, gamma_k, kcache, vcache, P: int, cfg: LayerCfg,
+                         ring=False, out=None, lse=None, want_lse=False, workspace=None,
+                         stream=None):
+    """Prefill of a chunk: q [B,Tn,Hq,d], k/v [B,Tn,Hkv,d] raw, at positions P..P+Tn-1,
+    against kcache/vcache [B, rows, Hkv, d] (normalised keys; position p in row p, or in
+    row p % rows with ring=True), which receive the chunk's keys and values.
+    Returns (out, lse)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (kcache, "kcache"), (vcache, "vcache")):
+        _bf16(t, n)
+    B, Tn = q.shape[0], q.shape[1]
+    rows = kcache.shape[1]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.n_q_heads, Tn), dtype=torch.float32, device=q.device)
+    c = cfg.c()
+    ws_bytes = _lib.g4attn_prefill_chunk_workspace_size(B, int(P), Tn, ctypes.byref(c))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    rc = _lib.g4attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma_q), _ptr(gamma_k),
+                                   _ptr(kcache), _ptr(vcache), rows, int(bool(ring)), _ptr(out),
+                                   _ptr(lse), _ptr(workspace), workspace.numel(), B, int(P), Tn,
+                                   ctypes.byref(c), _stream(stream))
+    _check(rc, "g4attn_prefill_chunk")
     return out, lse
 
 

@@ -3,7 +3,9 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -158,21 +160,25 @@ int encode_cs_rows(CUtensorMap* m, const float2* cs, int T, int R, int rows) {
 }
 
 struct PrefillWs {
-    size_t kn_off, kr_off, cs_off, total;
+    size_t kn_off, kr_off, cs_off, v_off, total;
     bool need_kn;
 };
 
-PrefillWs prefill_ws(int B, int T, const g4attn_layer_cfg* c) {
+// Workspace of an attention pass over Tk key rows per batch: the fp16 normalised keys
+// (pre-RoPE copy when some chunk is unrotated or the keys are the values, rotated copy),
+// the (cos, sin) table of the Tk positions and, with v_copy, a bf16 copy of the values.
+PrefillWs prefill_ws(int B, long long Tk, const g4attn_layer_cfg* c, bool v_copy = false) {
     PrefillWs w{};
     const int d = c->head_dim, R = rope_pairs(c);
     bool any_plain = false;
     for (int ch = 0; ch < d / 64; ++ch) any_plain |= !chunk_rotated(ch, d, R);
     w.need_kn = any_plain || c->kv_is_k == 1;
-    const size_t rows = (size_t)B * T * c->n_kv_heads * d * 2;
+    const size_t rows = (size_t)B * Tk * c->n_kv_heads * d * 2;
     w.kn_off = 0;
     w.kr_off = w.need_kn ? align256(rows) : 0;
     w.cs_off = w.kr_off + align256(rows);
-    w.total = w.cs_off + align256((size_t)T * (R > 0 ? R : 1) * sizeof(float2));
+    w.v_off = w.cs_off + align256((size_t)Tk * (R > 0 ? R : 1) * sizeof(float2));
+    w.total = w.v_off + (v_copy && c->kv_is_k == 0 ? align256(rows) : 0);
     return w;
 }
 
@@ -319,6 +325,80 @@ int check_ring(int C, const g4attn_layer_cfg* cfg) {
     return G4ATTN_OK;
 }
 
+// The fused flash-attention kernel over prepared key rows: kn / kr [B, Tk, Hkv, d] fp16
+// (kn may be null when no chunk needs it), v [B, Tk, Hkv, d] bf16 separate values or null,
+// cs [Tk, R] (cos, sin); query token t of the T in q sits at key row q_off + t.
+int launch_attention(const g4attn_bf16* q, const uint16_t* kn, const uint16_t* kr,
+                     const g4attn_bf16* v, const float2* cs, const float* gamma_q,
+                     g4attn_bf16* out, float* lse, int B, int T, int Tk, int q_off,
+                     const g4attn_layer_cfg* cfg, DeviceInfo* dev, cudaStream_t st) {
+    int rc;
+    const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
+    g4::PrefillArgs a{};
+    const uint16_t* kn_or_kr = kn ? kn : kr;
+    if ((rc = encode_rows(&a.tm_kr_s, kr, B, Tk, Hkv, d, true, 64))) return rc;
+    if ((rc = encode_rows(&a.tm_kn_s, kn_or_kr, B, Tk, Hkv, d, true, 64))) return rc;
+    if ((rc = encode_rows(&a.tm_kr_v, kr, B, Tk, Hkv, d, true, 128))) return rc;
+    if ((rc = encode_rows(&a.tm_kn_v, kn_or_kr, B, Tk, Hkv, d, true, 128))) return rc;
+    if (v) rc = encode_rows(&a.tm_v, v, B, Tk, Hkv, d, false, 128);
+    else rc = encode_rows(&a.tm_v, kn_or_kr, B, Tk, Hkv, d, true, 128);
+    if (rc) return rc;
+    const int G = cfg->n_q_heads / Hkv;
+    if ((rc = encode_q_tile(&a.tm_q, q, B, T, cfg->n_q_heads, d, G))) return rc;
+    {
+        // the (cos, sin) rows of a row tile go to shared memory by TMA when they fit the
+        // staging room (free during the prologue) and the row pitch suits TMA
+        const int R = rope_pairs(cfg), rows = 128 / G;
+        const size_t bytes = (size_t)rows * R * 8;
+        a.cs_tma = R > 0 && R % 2 == 0 && 2 * R <= 256 && rows <= 256 &&
+                   bytes <= g4::prefill_cs_stage_bytes(d);
+        if (a.cs_tma && (rc = encode_cs_rows(&a.tm_cs, cs, Tk, R, rows))) return rc;
+    }
+    a.q = q;
+    a.gamma_q = gamma_q;
+    a.rope_cs = cs;
+    a.out = out;
+    a.lse = lse;
+    a.B = B; a.T = T; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d;
+    a.Tk = Tk;
+    a.q_off = q_off;
+    a.G = G;
+    a.window = cfg->window;
+    a.rope = make_rope(cfg);
+    a.qk_norm = cfg->qk_norm;
+    a.eps = cfg->qk_norm_eps;
+    a.scale_log2 = cfg->scale * 1.4426950408889634f;
+    a.kv_is_k = cfg->kv_is_k;
+    a.wait_limit = g_wait_limit.load();
+    a.status = dev->status;
+    return cuda_status(g4::launch_prefill(a, st));
+}
+
+
+// Key rows of a prefill chunk: positions kb .. P + Tn - 1, where kb is the first position
+// any of the chunk's queries can see (0 on causal layers, P - W + 1 on window-W layers).
+struct ChunkFrame {
+    long long kb;
+    int Tk, q_off;
+};
+
+ChunkFrame chunk_frame(int P, int Tn, const g4attn_layer_cfg* c) {
+    ChunkFrame f{};
+    f.kb = c->window > 0 ? std::max(0, P - c->window + 1) : 0;
+    f.Tk = (int)(P + (long long)Tn - f.kb);
+    f.q_off = (int)(P - f.kb);
+    return f;
+}
+
+int check_chunk(int B, int P, int Tn, int cache_rows, int ring, const g4attn_layer_cfg* c) {
+    if (B < 0 || P < 0 || Tn < 0 || cache_rows <= 0) return G4ATTN_ERR_INVALID_ARG;
+    if ((long long)P + Tn > INT_MAX / 2) return G4ATTN_ERR_INVALID_ARG;
+    if (ring != 0 && ring != 1) return G4ATTN_ERR_INVALID_ARG;
+    if (!ring && (long long)P + Tn > cache_rows) return G4ATTN_ERR_INVALID_ARG;
+    if (ring && (c->window <= 0 || c->window > cache_rows)) return G4ATTN_ERR_INVALID_ARG;
+    return G4ATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -448,42 +528,90 @@ int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16
     if ((rc = cuda_status(g4::launch_qknorm_rope(ka, st)))) return rc;
 
     // 2) the fused flash-attention kernel
-    g4::PrefillArgs a{};
-    const uint16_t* kn_or_kr = kn ? kn : kr;
-    if ((rc = encode_rows(&a.tm_kr_s, kr, B, T, Hkv, d, true, 64))) return rc;
-    if ((rc = encode_rows(&a.tm_kn_s, kn_or_kr, B, T, Hkv, d, true, 64))) return rc;
-    if ((rc = encode_rows(&a.tm_kr_v, kr, B, T, Hkv, d, true, 128))) return rc;
-    if ((rc = encode_rows(&a.tm_kn_v, kn_or_kr, B, T, Hkv, d, true, 128))) return rc;
-    if (v) rc = encode_rows(&a.tm_v, v, B, T, Hkv, d, false, 128);
-    else rc = encode_rows(&a.tm_v, kn_or_kr, B, T, Hkv, d, true, 128);
+    return launch_attention(q, kn, kr, v, cs, gamma_q, out, lse, B, T, T, 0, cfg, dev, st);
+}
+
+size_t g4attn_prefill_chunk_workspace_size(int B, int P, int Tn, const g4attn_layer_cfg* cfg) {
+    if (check_cfg(cfg, true) || B < 0 || P < 0 || Tn < 0) return 0;
+    if ((long long)P + Tn > INT_MAX / 2) return 0;
+    return prefill_ws(B, chunk_frame(P, Tn, cfg).Tk, cfg, true).total;
+}
+
+int g4attn_prefill_chunk(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16* v,
+                         const float* gamma_q, const float* gamma_k, g4attn_bf16* kcache,
+                         g4attn_bf16* vcache, int cache_rows, int ring, g4attn_bf16* out,
+                         float* lse, void* workspace, size_t ws_bytes, int B, int P, int Tn,
+                         const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
+    int rc = check_cfg(cfg, true);
     if (rc) return rc;
-    const int G = cfg->n_q_heads / Hkv;
-    if ((rc = encode_q_tile(&a.tm_q, q, B, T, cfg->n_q_heads, d, G))) return rc;
-    {
-        // the (cos, sin) rows of a row tile go to shared memory by TMA when they fit the
-        // staging room (free during the prologue) and the row pitch suits TMA
-        const int R = rope_pairs(cfg), rows = 128 / G;
-        const size_t bytes = (size_t)rows * R * 8;
-        a.cs_tma = R > 0 && R % 2 == 0 && 2 * R <= 256 && rows <= 256 &&
-                   bytes <= g4::prefill_cs_stage_bytes(d);
-        if (a.cs_tma && (rc = encode_cs_rows(&a.tm_cs, cs, T, R, rows))) return rc;
+    if ((rc = check_chunk(B, P, Tn, cache_rows, ring, cfg))) return rc;
+    if ((long long)B * Tn == 0) return G4ATTN_OK;
+    if (!q || !k || !out || !kcache) return G4ATTN_ERR_INVALID_ARG;
+    const bool sep_v = cfg->kv_is_k == 0;
+    if (sep_v != (v != nullptr) || sep_v != (vcache != nullptr)) return G4ATTN_ERR_INVALID_ARG;
+    if (cfg->qk_norm && (!gamma_q || !gamma_k)) return G4ATTN_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, gamma_q, gamma_k, kcache, vcache, out, lse};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return G4ATTN_ERR_MISALIGNED;
+    const ChunkFrame f = chunk_frame(P, Tn, cfg);
+    const PrefillWs ws = prefill_ws(B, f.Tk, cfg, true);
+    if (!workspace || ws_bytes < ws.total) return G4ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* w = static_cast<uint8_t*>(workspace);
+    uint16_t* kn = ws.need_kn ? reinterpret_cast<uint16_t*>(w + ws.kn_off) : nullptr;
+    uint16_t* kr = reinterpret_cast<uint16_t*>(w + ws.kr_off);
+    float2* cs = reinterpret_cast<float2*>(w + ws.cs_off);
+    uint16_t* vf = sep_v ? reinterpret_cast<uint16_t*>(w + ws.v_off) : nullptr;
+
+    // the key rows of both passes land in one frame of Tk rows per batch, row = position - kb
+    g4::QkNormRopeArgs ka{};
+    ka.k_out = kn;
+    ka.krot_out = kr;
+    ka.cs_out = cs;
+    ka.v_out = vf;
+    ka.k_f16 = 1;
+    ka.B = B; ka.Hq = cfg->n_q_heads; ka.Hkv = cfg->n_kv_heads; ka.d = cfg->head_dim;
+    ka.rope = make_rope(cfg);
+    ka.eps = cfg->qk_norm_eps;
+    ka.out_rows = f.Tk;
+    ka.out_base = f.kb;
+
+    // 1) the cached positions kb .. P-1: stored normalised, so only turned (and widened)
+    if (P > f.kb) {
+        g4::QkNormRopeArgs ca = ka;
+        ca.k_in = kcache;
+        ca.v_in = vcache;
+        ca.in_rows = cache_rows;
+        ca.in_ring = ring ? cache_rows : 0;
+        ca.in_base = 0;
+        ca.pos0 = f.kb;
+        ca.T = (int)(P - f.kb);
+        ca.qk_norm = 0;
+        if ((rc = cuda_status(g4::launch_qknorm_rope(ca, st)))) return rc;
     }
-    a.q = q;
-    a.gamma_q = gamma_q;
-    a.rope_cs = cs;
-    a.out = out;
-    a.lse = lse;
-    a.B = B; a.T = T; a.Hq = cfg->n_q_heads; a.Hkv = Hkv; a.d = d;
-    a.G = cfg->n_q_heads / Hkv;
-    a.window = cfg->window;
-    a.rope = make_rope(cfg);
-    a.qk_norm = cfg->qk_norm;
-    a.eps = cfg->qk_norm_eps;
-    a.scale_log2 = cfg->scale * 1.4426950408889634f;
-    a.kv_is_k = cfg->kv_is_k;
-    a.wait_limit = g_wait_limit.load();
-    a.status = dev->status;
-    return cuda_status(g4::launch_prefill(a, st));
+    // 2) the chunk's own keys: QKNorm, RoPE, and appended to the cache (values too)
+    {
+        g4::QkNormRopeArgs na = ka;
+        na.k_in = k;
+        na.v_in = v;
+        na.gamma_k = gamma_k;
+        na.in_rows = Tn;
+        na.in_base = P;
+        na.pos0 = P;
+        na.T = Tn;
+        na.qk_norm = cfg->qk_norm;
+        na.kc_out = kcache;
+        na.vc_out = vcache;
+        na.kc_rows = cache_rows;
+        na.kc_ring = ring ? cache_rows : 0;
+        if ((rc = cuda_status(g4::launch_qknorm_rope(na, st)))) return rc;
+    }
+    // 3) attention of the chunk's queries (key row q_off + t) over the frame
+    return launch_attention(q, kn, kr, vf, cs, gamma_q, out, lse, B, Tn, f.Tk, f.q_off, cfg,
+                            dev, st);
 }
 
 size_t g4attn_decode_workspace_size(int B, int L, const g4attn_layer_cfg* cfg) {

@@ -27,6 +27,21 @@ struct QkNormRopeArgs {
     int k_f16;            // 1: k_out / krot_out are written as fp16 instead of bf16
     int B, T, Hq, Hkv, d;
     long long pos0;
+    // Row placement (all default to the dense [B, T, H, d] layout when zero).  Token t of
+    // batch b sits at position p = pos0 + t.
+    //  inputs  (q_in, k_in, v_in):  row b * in_rows + (in_ring ? p % in_ring : p - in_base)
+    //  outputs (q_out, k_out, krot_out, v_out, cs_out): row b * out_rows + p - out_base
+    //  cache copies (kc_out, vc_out): row b * kc_rows + (kc_ring ? p % kc_ring : p); with a
+    //  ring only the last kc_ring tokens are written (earlier ones would be overwritten)
+    int in_rows, in_ring;
+    long long in_base;
+    int out_rows;
+    long long out_base;
+    const uint16_t* v_in;  // optional values, copied unchanged to v_out / vc_out
+    uint16_t* v_out;
+    uint16_t* kc_out;      // optional bf16 copy of the normalised, unrotated keys
+    uint16_t* vc_out;
+    int kc_rows, kc_ring;
     Rope rope;
     int qk_norm;
     float eps;
@@ -78,7 +93,7 @@ cudaError_t decode_scratch_ptr(void** out);
 
 // Flash-attention prefill.
 struct PrefillArgs {
-    // 4-D maps over [B, T, Hkv, d] as (d, Hkv, T, B), 128-byte swizzle.  The *_s maps load
+    // 4-D maps over [B, Tk, Hkv, d] as (d, Hkv, Tk, B), 128-byte swizzle.  The *_s maps load
     // 64 dims x 64 keys (the score operand, half a key tile per CTA of a pair); the *_v
     // maps load 64 dims x 128 keys (the value operand).
     CUtensorMap tm_kn_s;    // normalised pre-RoPE keys (fp16)
@@ -87,14 +102,16 @@ struct PrefillArgs {
     CUtensorMap tm_kr_v;
     CUtensorMap tm_v;       // separate values (bf16, kv_is_k == 0), else a copy of tm_kn_v
     CUtensorMap tm_q;       // raw queries as (d, Hq, T, B), box (64, G, 128 / G, 1): one row tile
-    CUtensorMap tm_cs;      // rope_cs as fp32 (2R, T), box (2R, 128 / G); valid when cs_tma
+    CUtensorMap tm_cs;      // rope_cs as fp32 (2R, Tk), box (2R, 128 / G); valid when cs_tma
     int cs_tma;             // the (cos, sin) rows of a row tile are loaded by TMA
     const uint16_t* q;      // raw queries [B, T, Hq, d]
     const float* gamma_q;
-    const float2* rope_cs;  // [T, R] (cos, sin) of position t, pair i
+    const float2* rope_cs;  // [Tk, R] (cos, sin) of the position of key row t, pair i
     uint16_t* out;          // [B, T, Hq, d]
     float* lse;             // [B, Hq, T] or null
     int B, T, Hq, Hkv, d, G;
+    int Tk;      // key rows per batch in the key maps and the (cos, sin) table
+    int q_off;   // key row of the position of query token 0 (q_off + T <= Tk)
     int window;
     Rope rope;
     int qk_norm;

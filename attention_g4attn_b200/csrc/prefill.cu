@@ -120,8 +120,9 @@ __device__ __forceinline__ PairGeom pair_geom(const PrefillArgs& a, uint32_t ran
     const int mt = 2 * pr + (int)rank;
     g.m0 = mt * tpt;
     g.tq = min(tpt, a.T - g.m0);
-    const int first_tok = 2 * pr * tpt;
-    const int last_tok = min(a.T, (2 * pr + 2) * tpt) - 1;
+    // key rows of the pair's first and last query tokens
+    const int first_tok = a.q_off + 2 * pr * tpt;
+    const int last_tok = a.q_off + min(a.T, (2 * pr + 2) * tpt) - 1;
     int k_first = 0;
     if (a.window > 0) k_first = max(0, first_tok - a.window + 1);
     g.j_lo = k_first / kBN;
@@ -194,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive_expect_tx(&sm.q_full, (uint32_t)(NCH * 16384) + cs_bytes);
                 for (int c = 0; c < NCH; ++c)
                     tma_load_4d(sm.q[c], &a.tm_q, &sm.q_full, c * 64, pg.g * a.G, pg.m0, pg.b);
-                if (a.cs_tma) tma_load_2d(cs_stage, &a.tm_cs, &sm.q_full, 0, pg.m0);
+                if (a.cs_tma) tma_load_2d(cs_stage, &a.tm_cs, &sm.q_full, 0, a.q_off + pg.m0);
             }
             uint32_t q = 0;
             for (int n = 0; n < ntiles && !*abort; ++n) {
@@ -400,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 gv[k] = a.qk_norm ? a.gamma_q[half + i0 + k] : 1.f;
             }
             const float2* const cs_smem = reinterpret_cast<const float2*>(cs_stage);
-            const float2* const cs_glob = a.rope_cs + (size_t)pg.m0 * R;
+            const float2* const cs_glob = a.rope_cs + (size_t)(a.q_off + pg.m0) * R;
             const bool rot_lane = i0 < R;
             const int lgG = __ffs(G) - 1;          // G divides 128 (host check): a power of two
             ok_pro = group_all(mbar_wait(&sm.q_full, 0, wc, abort), kBarWG, 128);
@@ -517,8 +518,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // ---- main loop
         const int tok_r = pg.m0 + row / G;          // token of this row
+        const int kr_r = a.q_off + tok_r;           // key row of its position (mask bound)
         const bool row_valid = (row / G) < pg.tq;
-        const int t_first = pg.m0, t_last = pg.m0 + pg.tq - 1;
+        const int t_first = a.q_off + pg.m0, t_last = t_first + pg.tq - 1;
         const float c2 = a.scale_log2;              // > 0 (checked on the host)
         // rows past the end of the sequence hold zero queries; a finite reference keeps
         // their (never stored) P finite on the unmasked path
@@ -556,7 +558,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool need_mask = (key0 + kBN - 1 > t_first) ||
                                    (a.window > 0 && key0 <= t_last - a.window);
             float psum = 0.f, alpha = 1.f;
-            const int lo_r = a.window > 0 ? tok_r - a.window + 1 : 0;
+            const int lo_r = a.window > 0 ? kr_r - a.window + 1 : 0;
             // fast path: a finite reference max in every row of the warp: one pass over S
             // with the current reference; for head_dim 256 masked keys (outside the causal
             // band or the window) are dropped element by element, head_dim 512 (registers
@@ -585,8 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float s0 = __uint_as_float(cur[e]), s1 = __uint_as_float(cur[e + 1]);
                         if constexpr (MASK) {
                             const int j = key0 + b * 32 + e;
-                            if (!(j <= tok_r && j >= lo_r)) s0 = -INFINITY;
-                            if (!(j + 1 <= tok_r && j + 1 >= lo_r)) s1 = -INFINITY;
+                            if (!(j <= kr_r && j >= lo_r)) s0 = -INFINITY;
+                            if (!(j + 1 <= kr_r && j + 1 >= lo_r)) s1 = -INFINITY;
                         }
                         mxr = fmaxf(mxr, fmaxf(s0, s1));
                         const float p0 = ex2_approx(fmaf(s0, c2, negm));
@@ -637,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             float sv = __uint_as_float(cur[e]);
                             if constexpr (MASK) {
                                 const int j = key0 + b * 32 + e;
-                                if (!(j <= tok_r && j >= lo_r)) sv = -INFINITY;
+                                if (!(j <= kr_r && j >= lo_r)) sv = -INFINITY;
                             }
                             mx = fmaxf(mx, sv);
                         }
@@ -689,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     #pragma unroll
                         for (int e = 0; e < 32; ++e) {
                             const int j = key0 + b * 32 + e;
-                            const bool vis = !need_mask || (j <= tok_r && j >= lo_r);
+                            const bool vis = !need_mask || (j <= kr_r && j >= lo_r);
                             mx = fmaxf(mx, vis ? __uint_as_float(sv[e]) * c2 : -INFINITY);
                         }
                     }
@@ -711,7 +713,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     #pragma unroll
                             for (int u = 0; u < 2; ++u) {
                                 const int j = key0 + b * 32 + e + u;
-                                const bool vis = row_valid && (!need_mask || (j <= tok_r && j >= lo_r));
+                                const bool vis = row_valid && (!need_mask || (j <= kr_r && j >= lo_r));
                                 pv[u] = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, negm)) : 0.f;
                             }
                             if constexpr (PF16) {

@@ -66,23 +66,42 @@ __global__ void __launch_bounds__(kThreads) qknorm_rope_kernel(QkNormRopeArgs a)
     extern __shared__ float2 cs[];   // [R] (cos, sin) of this token's position
     const int d = 64 * E;
     const int half = d / 2;
-    const long long bt = blockIdx.x;
-    const int t = (int)(bt % a.T);
+    const int b = (int)(blockIdx.x / a.T);
+    const int t = (int)(blockIdx.x % a.T);
     const long long pos = a.pos0 + t;
+    // rows of this token in the inputs, the outputs and the cache copies
+    const long long in_row = (long long)b * a.in_rows + (a.in_ring ? pos % a.in_ring : pos - a.in_base);
+    const long long out_row = (long long)b * a.out_rows + (pos - a.out_base);
+    const bool kc_live = !a.kc_ring || t >= a.T - a.kc_ring;   // not overwritten by a later token
+    const long long kc_row = (long long)b * a.kc_rows + (a.kc_ring ? pos % a.kc_ring : pos);
     for (int i = threadIdx.x; i < a.rope.R; i += kThreads) {
         cs[i] = rope_cos_sin(pos, i, d, a.rope.log2_base);
-        if (a.cs_out && bt < a.T) a.cs_out[(size_t)t * a.rope.R + i] = cs[i];
+        if (a.cs_out && b == 0) a.cs_out[(size_t)(pos - a.out_base) * a.rope.R + i] = cs[i];
     }
     __syncthreads();
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nq = a.q_in ? a.Hq : 0;
-    const int nrows = nq + (a.k_in ? a.Hkv : 0);
-    for (int r = warp; r < nrows; r += kThreads / 32) {
+    const int nk = a.k_in ? a.Hkv : 0;
+    const int nv = a.v_in ? a.Hkv : 0;
+    for (int r = warp; r < nq + nk + nv; r += kThreads / 32) {
+        if (r >= nq + nk) {   // values: a plain copy of the row
+            const int h = r - nq - nk;
+            const uint16_t* src = a.v_in + (in_row * a.Hkv + h) * (long long)d;
+            uint16_t* dst = a.v_out ? a.v_out + (out_row * a.Hkv + h) * (long long)d : nullptr;
+            uint16_t* cdst = a.vc_out && kc_live ? a.vc_out + (kc_row * a.Hkv + h) * (long long)d
+                                                 : nullptr;
+            for (int c = lane; c < d / 8; c += 32) {
+                const uint4 x = reinterpret_cast<const uint4*>(src)[c];
+                if (dst) reinterpret_cast<uint4*>(dst)[c] = x;
+                if (cdst) reinterpret_cast<uint4*>(cdst)[c] = x;
+            }
+            continue;
+        }
         const bool is_q = r < nq;
         const int h = is_q ? r : r - nq;
-        const uint16_t* src = is_q ? a.q_in + (bt * a.Hq + h) * (long long)d
-                                   : a.k_in + (bt * a.Hkv + h) * (long long)d;
+        const uint16_t* src = is_q ? a.q_in + (in_row * a.Hq + h) * (long long)d
+                                   : a.k_in + (in_row * a.Hkv + h) * (long long)d;
         const float* gamma = is_q ? a.gamma_q : a.gamma_k;
         float x0[E], x1[E];
         load_bf16<E>(src + lane * E, x0);
@@ -102,12 +121,17 @@ __global__ void __launch_bounds__(kThreads) qknorm_rope_kernel(QkNormRopeArgs a)
         }
         const bool f16 = !is_q && a.k_f16;
         if (!is_q && a.k_out) {
-            uint16_t* dst = a.k_out + (bt * a.Hkv + h) * (long long)d;
+            uint16_t* dst = a.k_out + (out_row * a.Hkv + h) * (long long)d;
             store_row_half<E>(dst + lane * E, x0, f16);
             store_row_half<E>(dst + half + lane * E, x1, f16);
         }
-        uint16_t* rdst = is_q ? (a.q_out ? a.q_out + (bt * a.Hq + h) * (long long)d : nullptr)
-                              : (a.krot_out ? a.krot_out + (bt * a.Hkv + h) * (long long)d
+        if (!is_q && a.kc_out && kc_live) {
+            uint16_t* dst = a.kc_out + (kc_row * a.Hkv + h) * (long long)d;
+            store_bf16<E>(dst + lane * E, x0);
+            store_bf16<E>(dst + half + lane * E, x1);
+        }
+        uint16_t* rdst = is_q ? (a.q_out ? a.q_out + (out_row * a.Hq + h) * (long long)d : nullptr)
+                              : (a.krot_out ? a.krot_out + (out_row * a.Hkv + h) * (long long)d
                                             : nullptr);
         if (rdst) {
 #pragma unroll
@@ -128,9 +152,18 @@ __global__ void __launch_bounds__(kThreads) qknorm_rope_kernel(QkNormRopeArgs a)
 
 }  // namespace
 
-cudaError_t launch_qknorm_rope(const QkNormRopeArgs& a, cudaStream_t stream) {
-    const long long blocks = (long long)a.B * a.T;
+cudaError_t launch_qknorm_rope(const QkNormRopeArgs& in, cudaStream_t stream) {
+    const long long blocks = (long long)in.B * in.T;
     if (blocks == 0) return cudaSuccess;
+    QkNormRopeArgs a = in;   // zero placement fields: the dense [B, T, H, d] layout
+    if (a.in_rows == 0 && a.in_ring == 0) {
+        a.in_rows = a.T;
+        a.in_base = a.pos0;
+    }
+    if (a.out_rows == 0) {
+        a.out_rows = a.T;
+        a.out_base = a.pos0;
+    }
     const size_t smem = sizeof(float2) * (size_t)(a.rope.R > 0 ? a.rope.R : 1);
     switch (a.d) {
         case 512: qknorm_rope_kernel<8><<<(unsigned)blocks, kThreads, smem, stream>>>(a); break;

@@ -247,6 +247,53 @@ def time_local_ring_decode(device, stream, reps=10):
             "gbs": nbytes / t / 1e9}
 
 
+def time_chunked_prefill(device, stream, chunk=4096, reps=3):
+    """The global layer's T = 32768 prefill (32 q / 4 kv heads, d 512, causal) fed as
+    chunks of `chunk` tokens, each against the linear cache the earlier chunks wrote
+    (g4attn_prefill_chunk): the time of the whole sequence of calls, and of the last chunk
+    (the 4096 queries at positions 28672 .. 32767 against all 32768 keys)."""
+    import torch
+    from attention_g4attn_b200 import binding as b, synth, workloads
+    ly = workloads.GLOBAL_8TO1
+    T = 32768
+    inp = synth.layer_inputs(1, T, ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False, seed=21,
+                             device=device)
+    cfg = b.LayerCfg.from_layer(ly)
+    gq, gk = inp.gamma_q.to(device), inp.gamma_k.to(device)
+    kc = torch.empty((1, T, ly.n_kv_heads, ly.head_dim), dtype=torch.bfloat16, device=device)
+    out = torch.empty_like(inp.q)
+    ws = torch.empty(b.g4attn_prefill_chunk_workspace_size(1, T - chunk, chunk, cfg),
+                     dtype=torch.uint8, device=device)
+    cuts = list(range(0, T + 1, chunk))
+    pieces = [(P, inp.q[:, P:P + chunk], inp.k[:, P:P + chunk], out[:, P:P + chunk])
+              for P in cuts[:-1]]
+
+    def one(P, q, k, o):
+        b.g4attn_prefill_chunk(q, k, None, gq, gk, kc, None, P, cfg, out=o, workspace=ws,
+                               stream=stream)
+
+    def timed(calls):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for c in calls:
+            one(*c)
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
+    for _ in range(2):
+        timed(pieces)
+    t_all = statistics.median([timed(pieces) for _ in range(reps)])
+    t_last = statistics.median([timed(pieces[-1:]) for _ in range(reps)])
+    assert b.g4attn_device_status(stream) == 0
+    flops_all = 4.0 * ly.head_dim * ly.n_q_heads * workloads.visible_pairs(T, 0)
+    P = T - chunk
+    flops_last = 4.0 * ly.head_dim * ly.n_q_heads * (chunk * P + chunk * (chunk + 1) / 2)
+    return {"workload": "global_prefill_T32768_in_chunks_of_%d_h32x4_d512" % chunk,
+            "ms_all_chunks": t_all * 1e3, "tflops_all_chunks": flops_all / t_all / 1e12,
+            "ms_last_chunk": t_last * 1e3, "tflops_last_chunk": flops_last / t_last / 1e12}
+
+
 # --------------------------------------------------------------------------- CPU oracle
 
 def oracle_sample(max_seconds=20.0, seed=0):
@@ -465,6 +512,9 @@ def main():
             extra["global_decode_L131072"]["gbs"] / hbm_peak
         extra["local_decode_ring"] = time_local_ring_decode(device, stream)
         extra["local_decode_ring"]["frac_of_hbm"] = extra["local_decode_ring"]["gbs"] / hbm_peak
+        extra["chunked_prefill"] = time_chunked_prefill(device, stream)
+        extra["chunked_prefill"]["frac_of_sustained"] = \
+            extra["chunked_prefill"]["tflops_all_chunks"] / tf_peak
 
     # end to end through the public API with host buffers (pinned), copies inside the region
     e2e = None

@@ -117,6 +117,42 @@ G4ATTN_API int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const 
                    int B, int T, const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
 
 /*
+ * Chunked prefill (the serving form of the prefill in report section 2: a long prompt goes
+ * through in chunks, each against the cache the earlier chunks left): Tn new tokens at
+ * positions P .. P+Tn-1 attend causally, and within the window W = cfg->window on
+ * sliding-window layers, to the P earlier positions held in the cache and to the chunk
+ * itself.  The chunk's normalised keys (and its raw values) are then in the cache, so the
+ * next chunk, or g4attn_decode, continues from position P + Tn.
+ *   q, k, v   the chunk's raw queries [B, Tn, Hq, d], keys and values [B, Tn, Hkv, d]
+ *             (v as in g4attn_prefill: non-NULL exactly when kv_is_k == 0)
+ *   kcache    [B, cache_rows, Hkv, d] bf16: normalised, NOT rotated keys, the layout
+ *             g4attn_decode reads.  Read: positions max(0, P-W+1) .. P-1 (all P on causal
+ *             layers).  Written: positions P .. P+Tn-1 (RMS(k) * gamma_k, rounded to bf16)
+ *   vcache    [B, cache_rows, Hkv, d] bf16 separate values (kv_is_k == 0), else NULL;
+ *             same rows read and written, the chunk's v copied unchanged
+ *   ring      0: linear cache, position p in row p, needs cache_rows >= P + Tn;
+ *             1: ring buffer, position p in row p % cache_rows, for window layers with
+ *             0 < W <= cache_rows; of a chunk longer than the ring only its last
+ *             cache_rows positions are written
+ *   out       [B, Tn, Hq, d] bf16 (written);  lse [B, Hq, Tn] fp32 or NULL
+ *   workspace / ws_bytes  >= g4attn_prefill_chunk_workspace_size(B, P, Tn, cfg),
+ *             256-byte aligned (fp16 key rows of the visible positions, their (cos, sin)
+ *             table, and a copy of the visible values when kv_is_k == 0)
+ * P = 0 is g4attn_prefill plus the cache write.  B = 0 or Tn = 0 is a no-op (nothing is
+ * written).  Arguments out of range return G4ATTN_ERR_INVALID_ARG before any launch.
+ * The cache must not overlap q, k, v, out or the workspace.
+ */
+G4ATTN_API size_t g4attn_prefill_chunk_workspace_size(int B, int P, int Tn,
+                                                      const g4attn_layer_cfg* cfg);
+G4ATTN_API int g4attn_prefill_chunk(const g4attn_bf16* q, const g4attn_bf16* k,
+                                    const g4attn_bf16* v, const float* gamma_q,
+                                    const float* gamma_k, g4attn_bf16* kcache,
+                                    g4attn_bf16* vcache, int cache_rows, int ring,
+                                    g4attn_bf16* out, float* lse, void* workspace,
+                                    size_t ws_bytes, int B, int P, int Tn,
+                                    const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/*
  * Bytes of device workspace g4attn_decode needs for (B, L, cfg): fp32 partial outputs
  * and softmax statistics of the split-KV pass.  Returns 0 for an invalid configuration.
  */

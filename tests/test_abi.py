@@ -192,3 +192,51 @@ def test_binding_refuses_host_tensors(b):
     with pytest.raises(b.G4AttnError):
         b.g4attn_prefill(q, k, None, g, g, b.LayerCfg(8, 1, 512, 0.25, 1e6), out=q.clone(),
                          workspace=torch.zeros(16, dtype=torch.uint8))
+
+
+def test_prefill_chunk_workspace_covers_the_visible_positions(b):
+    # causal layer: every earlier position is visible, so the key rows are those of a
+    # prefill of P + Tn tokens
+    g = b.LayerCfg(32, 4, 512, 0.25, 1e6, 0, None, 1)
+    assert b.g4attn_prefill_chunk_workspace_size(1, 30000, 2768, g) == \
+        b.g4attn_prefill_workspace_size(1, 32768, g)
+    # window 512: positions P-511 .. P+Tn-1, plus a copy of their values
+    loc = b.LayerCfg(16, 8, 256, 1.0, 1e4, 512, None, 0)
+    Tk = 511 + 100
+    rows = 2 * Tk * 8 * 256 * 2
+    assert b.g4attn_prefill_chunk_workspace_size(2, 3000, 100, loc) == \
+        2 * _align(rows) + _align(Tk * 128 * 8)
+    Tk = 300 + 100   # P < W: all P earlier positions
+    rows = 2 * Tk * 8 * 256 * 2
+    assert b.g4attn_prefill_chunk_workspace_size(2, 300, 100, loc) == \
+        2 * _align(rows) + _align(Tk * 128 * 8)
+    assert b.g4attn_prefill_chunk_workspace_size(1, -1, 10, g) == 0
+
+
+def _call_chunk(lib, b, cfg, v=None, kc=0x7000, vc=None, rows=1 << 20, ring=0, ws=0x100000,
+                ws_bytes=1 << 40, B=1, P=100, Tn=16):
+    c = cfg.c()
+    Pt, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.g4attn_prefill_chunk
+    f.restype = I
+    f.argtypes = [Pt, Pt, Pt, Pt, Pt, Pt, Pt, I, I, Pt, Pt, Pt, ctypes.c_size_t, I, I, I,
+                  ctypes.POINTER(type(c)), Pt]
+    return f(0x1000, 0x2000, v, 0x3000, 0x4000, kc, vc, rows, ring, 0x5000, None, ws, ws_bytes,
+             B, P, Tn, ctypes.byref(c), None)
+
+
+def test_prefill_chunk_argument_checks_without_gpu(lib, b):
+    g = b.LayerCfg(8, 1, 512, 0.25, 1e6)
+    loc = b.LayerCfg(16, 8, 256, 1.0, 1e4, 512, None, 0)
+    E = b.G4ATTN_ERR_INVALID_ARG
+    assert _call_chunk(lib, b, g, rows=115) == E                     # linear cache < P + Tn
+    assert _call_chunk(lib, b, g, rows=512, ring=1) == E             # ring without a window
+    assert _call_chunk(lib, b, loc, v=0x6000, vc=0x8000, rows=256, ring=1) == E   # W > ring
+    assert _call_chunk(lib, b, g, ring=2) == E
+    assert _call_chunk(lib, b, g, P=-1) == E
+    assert _call_chunk(lib, b, g, vc=0x8000) == E                    # K=V layer: no values
+    assert _call_chunk(lib, b, loc, v=0x6000) == E                   # values but no value cache
+    assert _call_chunk(lib, b, g, kc=None) == E
+    assert _call_chunk(lib, b, g, kc=0x7008) == b.G4ATTN_ERR_MISALIGNED
+    assert _call_chunk(lib, b, g, ws_bytes=16) == b.G4ATTN_ERR_WORKSPACE
+    assert _call_chunk(lib, b, g, Tn=0) == b.G4ATTN_OK               # empty chunk: no-op
