@@ -70,9 +70,9 @@ struct __align__(1024) DecodeSmem {
     uint8_t ring[C::NSLOT][kSlotBytes];
     uint8_t side[2][kSlotBytes];       // turned slot 0 of tiles j & 1 (values = pre-RoPE keys)
     // this CTA's half of the B operand of S^T per slot (NH rows: queries over the first
-    // half of d in CTA 0, the second half in CTA 1), K-major, swizzled; q[4] is the second
-    // copy of slot 0's operand, which the relative rotation rewrites per tile (tile j uses
-    // copy j & 1)
+    // half of d in CTA 0, the second half in CTA 1), K-major, swizzled; q[4] (and, head_dim
+    // 256, q[3]) are second copies of slot 0's (slot 1's) operand, which the relative
+    // rotation rewrites per tile (tile j uses copy j & 1)
     uint8_t q[5][NH * 128];
     uint8_t p[2][NH * 128];            // this CTA's half of the B operand of O^T: its P^T
     float xs[2][64][C::HH];            // score halves handed to the other half's threads
@@ -148,12 +148,20 @@ __device__ __forceinline__ void mma4_pair(uint32_t d, uint64_t a, uint32_t a_ste
 
 constexpr uint32_t kSlotDesc = kSlotBytes >> 4;   // one ring slot, in descriptor units
 
+
+// The q operand copy that tile parity `odd` of rotated slot sb reads.
+__host__ __device__ constexpr int q_copy(int sb, bool odd) { return odd ? (sb == 0 ? 4 : 3) : sb; }
+
 // D: head dim; NH: query heads per KV head handled by the softmax (8 or 16, >= G);
-// REL: relative rotation (values are not the rotated key and R <= 64).
-template <int D, int NH, bool REL>
+// RS: slots turned by the relative rotation (0: absolute angles).  One slot (R <= 64, values
+// not the rotated key) is the p-RoPE of the global layers; two (R <= 128, head_dim 256,
+// separate values, at most 8 query heads per kv head) the full RoPE of the local layers.
+template <int D, int NH, int RS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a) {
     using C = DecodeCfg<NH>;
+    constexpr bool REL = RS > 0;
+    static_assert(RS < 2 || (D == 256 && NH == 8), "two relative slots: head_dim 256, NH 8");
     constexpr int NSB = D / 128;    // slots per tile and tensor
     constexpr int NS = C::NS, HH = C::HH, NSLOT = C::NSLOT;
     extern __shared__ uint8_t smem_raw[];
@@ -326,7 +334,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         const bool rot = sb < nrot;
                         const uint64_t ad = (rot && side_rot) ? d_side + (sc.g & 1) * kSlotDesc
                                                               : d_ring_k + slot * kSlotDesc;
-                        const uint64_t bd = d_q + ((REL && sb == 0 && (sc.g & 1)) ? 4 : sb) * kQDesc;
+                        const uint64_t bd =
+                            d_q + (REL && sb < nrot ? q_copy(sb, sc.g & 1) : sb) * kQDesc;
                         mma4_pair(tm_s, ad, 32 >> 4, bd, 32 >> 4, idesc_s, acc);
                         acc = 1;
                         // score slots of a separate-value layer (and the rotated key slot of a
@@ -524,21 +533,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int G = a.G;
         constexpr int QV = NH * NSB * 8 / 128;        // 16-byte pieces of q staged per thread
         constexpr int QH = NH / 2;                    // REL: heads cp, cp + 2, ... of pair rk
+        constexpr int NRS = REL ? RS : 1;             // REL: rotated slots served
         // Relative rotation (REL): key row rk of this CTA sits at angle (64 rank + rk) theta_i
         // from the start of the pair-tile, so its (cos, sin) are fixed per thread; the start
         // angle goes onto the query, which both CTAs' keys share in the pair MMA:
         // q' = R(-key0 theta) q, and q' . R((64 rank + rk) theta) k equals
-        // q . R((key0 + 64 rank + rk) theta) k.  rc / rs / rn hold cos / sin / -sin of the
-        // column pairs (2m, 2m + 1) of this thread as packed bf16 pairs: the turn runs on
-        // bf16x2 multiply-adds, 4 per pair of columns (fp32 math with its unpacking and
-        // repacking took 11 and sat on the per-tile chain, 6% of the decode rate)
-        __nv_bfloat162 rc[REL ? 16 : 1], rs[REL ? 16 : 1], rn[REL ? 16 : 1];
-        float qx[REL ? QH : 1], qy[REL ? QH : 1];    // REL: pair rk of q, heads cp + 2j
-        float2 bcs = make_float2(1.f, 0.f);          // REL: cos/sin of pair start * theta_rk
-        float2 stp = make_float2(1.f, 0.f);          // REL: cos/sin of 128 * theta_rk
+        // q . R((key0 + 64 rank + rk) theta) k.  rc / rs hold cos / sin of the column pairs
+        // (2m, 2m + 1) of this thread (rotated slot r: pairs 64 r + 32 cp + 2m) as packed bf16
+        // pairs: the turn runs on bf16x2 multiply-adds, 4 per pair of columns (fp32 math with
+        // its unpacking and repacking took 11 and sat on the per-tile chain, 6% of the decode
+        // rate).  With 10 warps a thread gets at most 168 registers: with two slots -sin is
+        // formed per use (5 operations) rather than held, and the query pairs stay packed.
+        __nv_bfloat162 rc[REL ? 16 * NRS : 1], rs[REL ? 16 * NRS : 1];
+        __nv_bfloat162 rn[NRS == 1 && REL ? 16 : 1];  // -sin (one slot)
+        __nv_bfloat162 qxy[NRS][REL ? QH : 1];       // REL: pair 64 r + rk of q (x, y)
+        float2 bcs[NRS], stp[NRS];                   // REL: cos/sin of pair start * theta and
+                                                     // of 128 * theta, pair 64 r + rk
         // the next item's queries and start angles, fetched one tile ahead of their use
         uint4 qpre[QV];
-        float qxp[REL ? QH : 1], qyp[REL ? QH : 1];
+        __nv_bfloat162 qxyp[NRS][REL ? QH : 1];
         float2 bpre[2];
         auto prefetch = [&](int it2) {
             const Item w2 = item_of(a, pair, pr, it2);
@@ -556,19 +569,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             if constexpr (REL) {
 #pragma unroll
-                for (int j = 0; j < QH; ++j) {
-                    const int h = cp + 2 * j;
-                    const bool on = h < G && rk < R;
-                    qxp[j] = on ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                      qg + (size_t)h * D + rk))
-                                : 0.f;
-                    qyp[j] = on ? __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
-                                      qg + (size_t)h * D + D / 2 + rk))
-                                : 0.f;
+                for (int r = 0; r < NRS; ++r) {
+                    const int i = 64 * r + rk;   // this thread's pair in rotated slot r
+#pragma unroll
+                    for (int j = 0; j < QH; ++j) {
+                        const int h = cp + 2 * j;
+                        const bool on = h < G && i < R;
+                        const __nv_bfloat16 z = __float2bfloat16_rn(0.f);
+                        qxyp[r][j] = __halves2bfloat162(
+                            on ? *reinterpret_cast<const __nv_bfloat16*>(qg + (size_t)h * D + i) : z,
+                            on ? *reinterpret_cast<const __nv_bfloat16*>(qg + (size_t)h * D + D / 2 + i)
+                               : z);
+                    }
+                    // q' turns by the start of the pair-tile (shared by both CTAs)
+                    bpre[r] = i < R ? rope_cos_sin((long long)w2.k0, i, D, a.rope.log2_base)
+                                    : make_float2(1.f, 0.f);
                 }
-                // q' turns by the start of the pair-tile (shared by both CTAs)
-                bpre[0] = rk < R ? rope_cos_sin((long long)w2.k0, rk, D, a.rope.log2_base)
-                                 : make_float2(1.f, 0.f);
             } else {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
@@ -589,16 +605,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 __sincosf(x, &sn, &cs);
             };
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const int i0 = 32 * cp + 2 * m;
+            for (int m = 0; m < 16 * NRS; ++m) {
+                const int i0 = 64 * (m / 16) + 32 * cp + 2 * (m % 16);
                 float s0 = 0.f, c0 = 1.f, s1 = 0.f, c1 = 1.f;
                 if (i0 < R) turn(i0, s0, c0);
                 if (i0 + 1 < R) turn(i0 + 1, s1, c1);
                 rc[m] = __floats2bfloat162_rn(c0, c1);
                 rs[m] = __floats2bfloat162_rn(s0, s1);
-                rn[m] = __floats2bfloat162_rn(-s0, -s1);
+                if constexpr (NRS == 1) rn[m] = __floats2bfloat162_rn(-s0, -s1);
             }
-            if (rk < R) stp = sm.step_cs[rk];
+        }
+#pragma unroll
+        for (int r = 0; r < NRS; ++r) {
+            bcs[r] = make_float2(1.f, 0.f);
+            stp[r] = (REL && 64 * r + rk < R) ? sm.step_cs[64 * r + rk] : make_float2(1.f, 0.f);
         }
         uint32_t q = 0, gt = 0, item_n = 0;
         bool ok = true;
@@ -620,23 +640,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 if (!ok) break;
                 if (t == 0) {
-                    // stage this CTA's half of the queries' B operand; slot 0's operand goes
-                    // to both of its copies
+                    // stage this CTA's half of the queries' B operand; the operands of the
+                    // relatively rotated slots go to both of their copies
 #pragma unroll
                     for (int j = 0; j < QV; ++j) {
                         const int e = t128 + 128 * j;
                         const int h = e / (NSB * 8), sb = (e / 8) % NSB, c8 = e % 8;
                         *reinterpret_cast<uint4*>(sm.q[sb] + sw128_offset(h, c8 * 8)) = qpre[j];
-                        if (sb == 0)
-                            *reinterpret_cast<uint4*>(sm.q[4] + sw128_offset(h, c8 * 8)) = qpre[j];
+                        if (REL && sb < NRS)
+                            *reinterpret_cast<uint4*>(sm.q[q_copy(sb, true)] +
+                                                      sw128_offset(h, c8 * 8)) = qpre[j];
                     }
                     if constexpr (REL) {
 #pragma unroll
-                        for (int j = 0; j < QH; ++j) {
-                            qx[j] = qxp[j];
-                            qy[j] = qyp[j];
+                        for (int r = 0; r < NRS; ++r) {
+#pragma unroll
+                            for (int j = 0; j < QH; ++j) qxy[r][j] = qxyp[r][j];
+                            bcs[r] = bpre[r];
                         }
-                        bcs = bpre[0];
                     } else {
 #pragma unroll
                         for (int j = 0; j < 2; ++j)
@@ -653,9 +674,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     // start angle of this CTA's tile: exact (fp64-reduced) at the first tile
                     // of an item, then advanced by one pair-tile (128 keys) per step
                     if constexpr (REL) {
-                        if (t > 0)
-                            bcs = make_float2(bcs.x * stp.x - bcs.y * stp.y,
-                                              bcs.x * stp.y + bcs.y * stp.x);
+                        if (t > 0) {
+#pragma unroll
+                            for (int r = 0; r < NRS; ++r)
+                                bcs[r] = make_float2(bcs[r].x * stp[r].x - bcs[r].y * stp[r].y,
+                                                     bcs[r].x * stp[r].y + bcs[r].y * stp[r].x);
+                        }
                     } else if (t > 0) {
                         for (int i = t128; i < R; i += 128) {
                             const float2 b0 = sm.base_cs[i], st = sm.step_cs[i];
@@ -668,54 +692,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 if (R > 0) {
                     if constexpr (REL) {
-                        // this CTA's half of q' = R(-key0 theta) q on pair rk, key0 the start
-                        // of the pair-tile (first-half dim in CTA 0, second-half dim in CTA 1),
-                        // into copy gt & 1 of slot 0's operand (R <= 64: all rotated dims sit
-                        // in slot 0)
-                        uint8_t* qd = sm.q[(gt & 1) ? 4 : 0];
-                        if (rk < R) {
 #pragma unroll
-                            for (int j = 0; j < QH; ++j) {
-                                const int h = cp + 2 * j;
-                                if (h < G) {
-                                    const float v = rank == 0 ? qx[j] * bcs.x + qy[j] * bcs.y
-                                                              : qy[j] * bcs.x - qx[j] * bcs.y;
-                                    *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(h, rk)) =
-                                        __float2bfloat16_rn(v);
+                        for (int r = 0; r < NRS; ++r) {
+                            if (r >= nrot) break;
+                            // this CTA's half of q' = R(-key0 theta) q on pair 64 r + rk, key0
+                            // the start of the pair-tile (first-half dim in CTA 0, second-half
+                            // dim in CTA 1), into copy gt & 1 of rotated slot r's operand
+                            uint8_t* qd = sm.q[q_copy(r, gt & 1)];
+                            if (64 * r + rk < R) {
+#pragma unroll
+                                for (int j = 0; j < QH; ++j) {
+                                    const int h = cp + 2 * j;
+                                    if (h < G) {
+                                        const float2 b = bcs[r];
+                                        const float2 xy = __bfloat1622float2(qxy[r][j]);
+                                        const float v = rank == 0 ? xy.x * b.x + xy.y * b.y
+                                                                  : xy.y * b.x - xy.x * b.y;
+                                        *reinterpret_cast<__nv_bfloat16*>(qd + sw128_offset(h, rk)) =
+                                            __float2bfloat16_rn(v);
+                                    }
                                 }
                             }
-                        }
-                        // keys: R(rk theta) on the rotated pairs of row rk (dims in row rk,
-                        // their partners in row 64 + rk of slot 0)
-                        uint8_t* src = sm.ring[qk % NSLOT];
-                        uint8_t* dst = side_rot ? sm.side[gt & 1] : src;
+                            // keys: R(rk theta) on the rotated pairs of row rk (dims in row rk,
+                            // their partners in row 64 + rk of slot r)
+                            uint8_t* src = sm.ring[(qk + r) % NSLOT];
+                            uint8_t* dst = side_rot ? sm.side[gt & 1] : src;
 #pragma unroll
-                        for (int g8 = 0; g8 < 4; ++g8) {
-                            const int col = 32 * cp + 8 * g8;
-                            const bool rotg = col < R;
-                            if (!side_rot && !rotg) continue;   // in place: nothing to copy
-                            const uint32_t o1 = sw128_offset(rk, col);
-                            const uint32_t o2 = sw128_offset(64 + rk, col);
-                            uint4 x1 = *reinterpret_cast<const uint4*>(src + o1);
-                            uint4 x2 = *reinterpret_cast<const uint4*>(src + o2);
-                            if (rotg) {
-                                // pairs whose cos/sin are (1, 0) turn into themselves, so the
-                                // columns at or past R need no special case
-                                uint32_t* w1 = &x1.x;
-                                uint32_t* w2 = &x2.x;
+                            for (int g8 = 0; g8 < 4; ++g8) {
+                                const int col = 32 * cp + 8 * g8;
+                                const bool rotg = 64 * r + col < R;
+                                if (!side_rot && !rotg) continue;   // in place: nothing to copy
+                                const uint32_t o1 = sw128_offset(rk, col);
+                                const uint32_t o2 = sw128_offset(64 + rk, col);
+                                uint4 x1 = *reinterpret_cast<const uint4*>(src + o1);
+                                uint4 x2 = *reinterpret_cast<const uint4*>(src + o2);
+                                if (rotg) {
+                                    // pairs whose cos/sin are (1, 0) turn into themselves, so
+                                    // the columns at or past R need no special case
+                                    uint32_t* w1 = &x1.x;
+                                    uint32_t* w2 = &x2.x;
 #pragma unroll
-                                for (int m = 0; m < 4; ++m) {
-                                    const __nv_bfloat162 u = *reinterpret_cast<const __nv_bfloat162*>(&w1[m]);
-                                    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&w2[m]);
-                                    const int i = 4 * g8 + m;
-                                    const __nv_bfloat162 u2 = __hfma2(u, rc[i], __hmul2(v, rn[i]));
-                                    const __nv_bfloat162 v2 = __hfma2(u, rs[i], __hmul2(v, rc[i]));
-                                    w1[m] = *reinterpret_cast<const uint32_t*>(&u2);
-                                    w2[m] = *reinterpret_cast<const uint32_t*>(&v2);
+                                    for (int m = 0; m < 4; ++m) {
+                                        const __nv_bfloat162 u = *reinterpret_cast<const __nv_bfloat162*>(&w1[m]);
+                                        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&w2[m]);
+                                        const int i = 16 * r + 4 * g8 + m;
+                                        __nv_bfloat162 u2;
+                                        if constexpr (NRS == 1) u2 = __hfma2(u, rc[i], __hmul2(v, rn[i]));
+                                        else u2 = __hfma2(u, rc[i], __hneg2(__hmul2(v, rs[i])));
+                                        const __nv_bfloat162 v2 = __hfma2(u, rs[i], __hmul2(v, rc[i]));
+                                        w1[m] = *reinterpret_cast<const uint32_t*>(&u2);
+                                        w2[m] = *reinterpret_cast<const uint32_t*>(&v2);
+                                    }
                                 }
+                                *reinterpret_cast<uint4*>(dst + o1) = x1;
+                                *reinterpret_cast<uint4*>(dst + o2) = x2;
                             }
-                            *reinterpret_cast<uint4*>(dst + o1) = x1;
-                            *reinterpret_cast<uint4*>(dst + o2) = x2;
                         }
                     } else {
                         // absolute angles: angle(key0 + rk) = angle(key0) + rk * theta_i
@@ -831,25 +862,29 @@ __global__ void __launch_bounds__(kCombineThreads)
         a.lse[bh] = dsum > 0.f ? (M + log2f(dsum)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int D, int NH, bool REL>
+template <int D, int NH, int RS>
 cudaError_t run_decode(const DecodeArgs& a, int grid, cudaStream_t stream) {
     const size_t smem = sizeof(DecodeSmem<NH>) + 1024;
     static_assert(sizeof(DecodeSmem<NH>) + 1024 <= 227 * 1024, "decode shared memory");
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NH, REL>,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NH, RS>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_kernel<D, NH, REL><<<grid, kThreads, smem, stream>>>(a);
+    decode_kernel<D, NH, RS><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
 template <int D>
 cudaError_t dispatch_decode(const DecodeArgs& a, int grid, cudaStream_t stream) {
-    const bool rel = a.kv_is_k != 2 && a.rope.R <= 64;
-    if (a.G <= 8)
-        return rel ? run_decode<D, 8, true>(a, grid, stream)
-                   : run_decode<D, 8, false>(a, grid, stream);
-    return rel ? run_decode<D, 16, true>(a, grid, stream)
-               : run_decode<D, 16, false>(a, grid, stream);
+    // relative rotation: a side buffer holds one turned slot per tile, so the pre-RoPE-value
+    // layers (kv_is_k 1) take it for one rotated slot only
+    const bool rel1 = a.kv_is_k != 2 && a.rope.R <= 64;
+    if (a.G <= 8) {
+        if (rel1) return run_decode<D, 8, 1>(a, grid, stream);
+        if constexpr (D == 256)
+            if (a.kv_is_k == 0 && a.rope.R <= 128) return run_decode<D, 8, 2>(a, grid, stream);
+        return run_decode<D, 8, 0>(a, grid, stream);
+    }
+    return rel1 ? run_decode<D, 16, 1>(a, grid, stream) : run_decode<D, 16, 0>(a, grid, stream);
 }
 
 }  // namespace

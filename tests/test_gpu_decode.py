@@ -63,6 +63,21 @@ def test_decode_local_layer_shape():
     check(dec, loc, what="decode local")
 
 
+@pytest.mark.parametrize("p,L,window,Hq,Hkv", [
+    (1.0, 9000, 0, 16, 8),      # full RoPE, two turned slots, 70 pair-tiles per sequence
+    (0.75, 3001, 1024, 16, 8),  # R = 96: slot 1 turned in part
+    (0.5, 2500, 700, 16, 8),    # R = 64: one turned slot
+    (1.0, 1800, 1024, 32, 2),   # 16 query heads per kv head: the absolute-angle path
+])
+def test_decode_head_dim_256_rotation_variants(p, L, window, Hq, Hkv):
+    # the relative rotation turns up to two slots at head_dim 256 (separate values); each
+    # variant against the oracle
+    ly = workloads.with_layer(workloads.LOCAL_W1024, rope_p=p, window=window, n_q_heads=Hq,
+                              n_kv_heads=Hkv)
+    dec = synth.decode_inputs(2, L, Hq, Hkv, 256, True, seed=int(100 * p) + L)
+    check(dec, ly, what="decode d256 p=%.2f L=%d W=%d G=%d" % (p, L, window, Hq // Hkv))
+
+
 def test_decode_empty_cache():
     b = binding()
     dev = torch.device("cuda:0")
