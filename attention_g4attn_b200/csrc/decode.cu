@@ -85,7 +85,8 @@ struct __align__(1024) DecodeSmem {
     uint64_t full[C::NSLOT];           // this CTA's loads landed
     uint64_t empty[C::NSLOT];          // the pair's MMAs are done with the slot
     // per-tile barriers come in pairs (tile j uses [j & 1], phase (j >> 1) & 1): a waiter is
-    // never more than one phase of a barrier behind.  rot_ready and p_full live in the first
+    // never more than one phase of a barrier behind (the rotation warps wait for S(j - 2)
+    // before they arrive on rot_ready for tile j).  rot_ready and p_full live in the first
     // CTA and count one arrival from each CTA.
     uint64_t s_full[2], p_full[2], pv_done[2], rot_ready[2];
     uint64_t q_free, drain;            // once per item: all its scores done / teardown
@@ -155,13 +156,14 @@ __host__ __device__ constexpr int q_copy(int sb, bool odd) { return odd ? (sb ==
 // D: head dim; NH: query heads per KV head handled by the softmax (8 or 16, >= G);
 // RS: slots turned by the relative rotation (0: absolute angles).  One slot (R <= 64, values
 // not the rotated key) is the p-RoPE of the global layers; two (R <= 128, head_dim 256,
-// separate values, at most 8 query heads per kv head) the full RoPE of the local layers.
+// separate values, at most 4 query heads per kv head) the full RoPE of the local layers.
 template <int D, int NH, int RS>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a) {
     using C = DecodeCfg<NH>;
     constexpr bool REL = RS > 0;
     static_assert(RS < 2 || (D == 256 && NH == 8), "two relative slots: head_dim 256, NH 8");
+    // (the host takes RS = 2 only for G <= 4)
     constexpr int NSB = D / 128;    // slots per tile and tensor
     constexpr int NS = C::NS, HH = C::HH, NSLOT = C::NSLOT;
     extern __shared__ uint8_t smem_raw[];
@@ -532,7 +534,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int cp = t128 >> 6;                     // columns [32 cp, 32 cp + 32)
         const int G = a.G;
         constexpr int QV = NH * NSB * 8 / 128;        // 16-byte pieces of q staged per thread
-        constexpr int QH = NH / 2;                    // REL: heads cp, cp + 2, ... of pair rk
+        // REL: heads cp, cp + 2, ... of pair rk (two turned slots: at most 4 query heads per
+        // kv head, which keeps the per-thread state within the register budget)
+        constexpr int QH = RS == 2 ? 2 : NH / 2;
         constexpr int NRS = REL ? RS : 1;             // REL: rotated slots served
         // Relative rotation (REL): key row rk of this CTA sits at angle (64 rank + rk) theta_i
         // from the start of the pair-tile, so its (cos, sin) are fixed per thread; the start
@@ -630,11 +634,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 q += slots_per_tile;
                 // before rewriting the B operands: the first tile of an item needs every
                 // score product of the previous item complete (it restages all of q), a
-                // later tile only the one that last read its side buffer and q copy (gt - 2)
+                // later tile only the one that last read its side buffer and q copy (gt - 2).
+                // The wait on S(gt - 2) also keeps this role less than two tiles ahead of
+                // the issuer on the paired rot_ready barriers, whatever the ring depth (a
+                // head_dim 256 keys-as-values layer has 2 slots per tile, 5.5 tiles of ring)
                 if (t == 0 && item_n > 0) {
                     ok = group_all(mbar_wait(&sm.q_free, (item_n - 1) & 1, wc, abort), kBarRot,
                                    128);
-                } else if (t > 0 && R > 0 && gt > 1) {
+                } else if (t > 0 && gt > 1) {
                     ok = group_all(mbar_wait(&sm.s_full[gt & 1], ((gt - 2) >> 1) & 1, wc, abort),
                                    kBarRot, 128);
                 }
@@ -666,9 +673,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 // fetch the next item's queries now: the loads fly during this tile's work
                 if (t == nt - 1 && it + 1 < n_items) prefetch(it + 1);
-                // the slots with rotated pairs first: they are turned while the rest land
+                // the slots with rotated pairs first: they are turned while the rest land (the
+                // relative rotation turns its first slot while its second one lands)
                 bool got = true;
-                for (int k = 0; k < nrot && got; ++k)
+                const int nfirst = REL ? (nrot > 0 ? 1 : 0) : nrot;
+                for (int k = 0; k < nfirst && got; ++k)
                     got = mbar_wait(&sm.full[(qk + k) % NSLOT], ((qk + k) / NSLOT) & 1, wc, abort);
                 if (R > 0) {
                     // start angle of this CTA's tile: exact (fp64-reduced) at the first tile
@@ -695,6 +704,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int r = 0; r < NRS; ++r) {
                             if (r >= nrot) break;
+                            if (r > 0) {   // the next rotated slot, landed while slot r-1 turned
+                                const uint32_t k = qk + r;
+                                got = group_all(mbar_wait(&sm.full[k % NSLOT], (k / NSLOT) & 1,
+                                                          wc, abort),
+                                                kBarRot, 128);
+                                if (!got) break;
+                            }
                             // this CTA's half of q' = R(-key0 theta) q on pair 64 r + rk, key0
                             // the start of the pair-tile (first-half dim in CTA 0, second-half
                             // dim in CTA 1), into copy gt & 1 of rotated slot r's operand
@@ -881,7 +897,8 @@ cudaError_t dispatch_decode(const DecodeArgs& a, int grid, cudaStream_t stream) 
     if (a.G <= 8) {
         if (rel1) return run_decode<D, 8, 1>(a, grid, stream);
         if constexpr (D == 256)
-            if (a.kv_is_k == 0 && a.rope.R <= 128) return run_decode<D, 8, 2>(a, grid, stream);
+            if (a.kv_is_k == 0 && a.rope.R <= 128 && a.G <= 4)
+                return run_decode<D, 8, 2>(a, grid, stream);
         return run_decode<D, 8, 0>(a, grid, stream);
     }
     return rel1 ? run_decode<D, 16, 1>(a, grid, stream) : run_decode<D, 16, 0>(a, grid, stream);

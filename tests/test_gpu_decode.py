@@ -68,6 +68,8 @@ def test_decode_local_layer_shape():
     (0.75, 3001, 1024, 16, 8),  # R = 96: slot 1 turned in part
     (0.5, 2500, 700, 16, 8),    # R = 64: one turned slot
     (1.0, 1800, 1024, 32, 2),   # 16 query heads per kv head: the absolute-angle path
+    (1.0, 1500, 1024, 32, 4),   # 8 query heads per kv head: the absolute-angle path too
+    (1.0, 1400, 512, 16, 4),    # 4 query heads per kv head: two turned slots
 ])
 def test_decode_head_dim_256_rotation_variants(p, L, window, Hq, Hkv):
     # the relative rotation turns up to two slots at head_dim 256 (separate values); each
