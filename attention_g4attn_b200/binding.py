@@ -97,6 +97,8 @@ def _load():
         "g4attn_decode_ring_workspace_size": (SZ, [I, I, I, CFG]),
         "g4attn_decode_ring": (I, [P, P, P, I, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_decode_split_cache": (I, [P, P, P, I, P, P, P, SZ, I, CFG, P]),
+        "g4attn_decode_rotated_workspace_size": (SZ, [I, I, I, CFG]),
+        "g4attn_decode_rotated": (I, [P, P, P, I, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_status_string": (ctypes.c_char_p, [I]),
         "g4attn_device_status": (I, [P]),
         "g4attn_set_wait_limit": (LL, [LL]),
@@ -231,13 +233,17 @@ def g4attn_prefill_chunk_workspace_size(B: int, P: int, Tn: int, cfg: LayerCfg) 
     return _lib.g4attn_prefill_chunk_workspace_size(B, P, Tn, ctypes.byref(c))
 
 
+G4ATTN_CACHE_RING = 1
+G4ATTN_CACHE_ROTATED = 2
+
+
 def g4attn_prefill_chunk(q, k, v, gamma_q, gamma_k, kcache, vcache, P: int, cfg: LayerCfg,
-                         ring=False, out=None, lse=None, want_lse=False, workspace=None,
-                         stream=None):
+                         ring=False, rotated=False, out=None, lse=None, want_lse=False,
+                         workspace=None, stream=None):
     """Prefill of a chunk: q [B,Tn,Hq,d], k/v [B,Tn,Hkv,d] raw, at positions P..P+Tn-1,
-    against kcache/vcache [B, rows, Hkv, d] (normalised keys; position p in row p, or in
-    row p % rows with ring=True), which receive the chunk's keys and values.
-    Returns (out, lse)."""
+    against kcache/vcache [B, rows, Hkv, d] (normalised keys, turned to their positions
+    with rotated=True; position p in row p, or in row p % rows with ring=True), which
+    receive the chunk's keys and values.  Returns (out, lse)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (kcache, "kcache"), (vcache, "vcache")):
         _bf16(t, n)
     B, Tn = q.shape[0], q.shape[1]
@@ -251,7 +257,9 @@ def g4attn_prefill_chunk(q, k, v, gamma_q, gamma_k, kcache, vcache, P: int, cfg:
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
     rc = _lib.g4attn_prefill_chunk(_ptr(q), _ptr(k), _ptr(v), _ptr(gamma_q), _ptr(gamma_k),
-                                   _ptr(kcache), _ptr(vcache), rows, int(bool(ring)), _ptr(out),
+                                   _ptr(kcache), _ptr(vcache), rows,
+                                   (G4ATTN_CACHE_RING if ring else 0) |
+                                   (G4ATTN_CACHE_ROTATED if rotated else 0), _ptr(out),
                                    _ptr(lse), _ptr(workspace), workspace.numel(), B, int(P), Tn,
                                    ctypes.byref(c), _stream(stream))
     _check(rc, "g4attn_prefill_chunk")
@@ -303,6 +311,35 @@ def g4attn_decode_ring(q, kring, vring, L: int, cfg: LayerCfg, out=None, lse=Non
                                  _ptr(lse), _ptr(workspace), workspace.numel(), B,
                                  ctypes.byref(c), _stream(stream))
     _check(rc, "g4attn_decode_ring")
+    return out, lse
+
+
+def g4attn_decode_rotated_workspace_size(B: int, L: int, C: int, cfg: LayerCfg) -> int:
+    c = cfg.c()
+    return _lib.g4attn_decode_rotated_workspace_size(B, L, C, ctypes.byref(c))
+
+
+def g4attn_decode_rotated(q, krot, vcache, L: int, cfg: LayerCfg, ring=False, out=None,
+                          lse=None, want_lse=False, workspace=None, stream=None):
+    """Decode one token at position L-1 against keys stored turned to their positions and
+    separate values: krot/vcache [B, L, Hkv, d], or ring caches [B, C, Hkv, d] (row p % C)
+    with ring=True."""
+    for t, n in ((q, "q"), (krot, "krot"), (vcache, "vcache")):
+        _bf16(t, n)
+    B = krot.shape[0]
+    C = krot.shape[1] if ring else 0
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.n_q_heads), dtype=torch.float32, device=q.device)
+    c = cfg.c()
+    ws_bytes = _lib.g4attn_decode_rotated_workspace_size(B, int(L), C, ctypes.byref(c))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    rc = _lib.g4attn_decode_rotated(_ptr(q), _ptr(krot), _ptr(vcache), int(L), C, _ptr(out),
+                                    _ptr(lse), _ptr(workspace), workspace.numel(), B,
+                                    ctypes.byref(c), _stream(stream))
+    _check(rc, "g4attn_decode_rotated")
     return out, lse
 
 

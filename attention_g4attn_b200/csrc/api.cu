@@ -274,7 +274,7 @@ int launch_decode_plan(const g4attn_bf16* q, const g4attn_bf16* kcache,
                        const g4attn_bf16* vcache, int L, int rows, int ring, g4attn_bf16* out,
                        float* lse, uint8_t* w, const DecodePlan& plan, int B,
                        const g4attn_layer_cfg* cfg, const DeviceInfo* dev, g4attn_stream_t stream,
-                       const g4attn_bf16* vside = nullptr) {
+                       const g4attn_bf16* vside = nullptr, bool keys_rotated = false) {
     g4::DecodeArgs a{};
     const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
     int rc;
@@ -310,6 +310,7 @@ int launch_decode_plan(const g4attn_bf16* q, const g4attn_bf16* kcache,
         a.split_cache = 1;
         a.rope.R = 0;
     }
+    if (keys_rotated) a.rope.R = 0;   // keys stored turned to their positions: no turning
     a.scale_log2 = cfg->scale * 1.4426950408889634f;
     a.kv_is_k = cfg->kv_is_k;
     a.wait_limit = g_wait_limit.load();
@@ -390,10 +391,12 @@ ChunkFrame chunk_frame(int P, int Tn, const g4attn_layer_cfg* c) {
     return f;
 }
 
-int check_chunk(int B, int P, int Tn, int cache_rows, int ring, const g4attn_layer_cfg* c) {
+int check_chunk(int B, int P, int Tn, int cache_rows, int flags, const g4attn_layer_cfg* c) {
     if (B < 0 || P < 0 || Tn < 0 || cache_rows <= 0) return G4ATTN_ERR_INVALID_ARG;
     if ((long long)P + Tn > INT_MAX / 2) return G4ATTN_ERR_INVALID_ARG;
-    if (ring != 0 && ring != 1) return G4ATTN_ERR_INVALID_ARG;
+    if (flags & ~(G4ATTN_CACHE_RING | G4ATTN_CACHE_ROTATED)) return G4ATTN_ERR_INVALID_ARG;
+    if ((flags & G4ATTN_CACHE_ROTATED) && c->kv_is_k != 0) return G4ATTN_ERR_INVALID_ARG;
+    const bool ring = (flags & G4ATTN_CACHE_RING) != 0;
     if (!ring && (long long)P + Tn > cache_rows) return G4ATTN_ERR_INVALID_ARG;
     if (ring && (c->window <= 0 || c->window > cache_rows)) return G4ATTN_ERR_INVALID_ARG;
     return G4ATTN_OK;
@@ -539,12 +542,14 @@ size_t g4attn_prefill_chunk_workspace_size(int B, int P, int Tn, const g4attn_la
 
 int g4attn_prefill_chunk(const g4attn_bf16* q, const g4attn_bf16* k, const g4attn_bf16* v,
                          const float* gamma_q, const float* gamma_k, g4attn_bf16* kcache,
-                         g4attn_bf16* vcache, int cache_rows, int ring, g4attn_bf16* out,
+                         g4attn_bf16* vcache, int cache_rows, int cache_flags, g4attn_bf16* out,
                          float* lse, void* workspace, size_t ws_bytes, int B, int P, int Tn,
                          const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
     int rc = check_cfg(cfg, true);
     if (rc) return rc;
-    if ((rc = check_chunk(B, P, Tn, cache_rows, ring, cfg))) return rc;
+    if ((rc = check_chunk(B, P, Tn, cache_rows, cache_flags, cfg))) return rc;
+    const bool ring = (cache_flags & G4ATTN_CACHE_RING) != 0;
+    const bool rotated = (cache_flags & G4ATTN_CACHE_ROTATED) != 0;
     if ((long long)B * Tn == 0) return G4ATTN_OK;
     if (!q || !k || !out || !kcache) return G4ATTN_ERR_INVALID_ARG;
     const bool sep_v = cfg->kv_is_k == 0;
@@ -579,7 +584,9 @@ int g4attn_prefill_chunk(const g4attn_bf16* q, const g4attn_bf16* k, const g4att
     ka.out_rows = f.Tk;
     ka.out_base = f.kb;
 
-    // 1) the cached positions kb .. P-1: stored normalised, so only turned (and widened)
+    // 1) the cached positions kb .. P-1: stored normalised, so only turned (and widened); a
+    //    cache of turned keys is only widened (its (cos, sin) rows are not needed: the
+    //    queries sit at rows q_off and later)
     if (P > f.kb) {
         g4::QkNormRopeArgs ca = ka;
         ca.k_in = kcache;
@@ -590,6 +597,7 @@ int g4attn_prefill_chunk(const g4attn_bf16* q, const g4attn_bf16* k, const g4att
         ca.pos0 = f.kb;
         ca.T = (int)(P - f.kb);
         ca.qk_norm = 0;
+        if (rotated) ca.rope.R = 0;
         if ((rc = cuda_status(g4::launch_qknorm_rope(ca, st)))) return rc;
     }
     // 2) the chunk's own keys: QKNorm, RoPE, and appended to the cache (values too)
@@ -607,6 +615,7 @@ int g4attn_prefill_chunk(const g4attn_bf16* q, const g4attn_bf16* k, const g4att
         na.vc_out = vcache;
         na.kc_rows = cache_rows;
         na.kc_ring = ring ? cache_rows : 0;
+        na.kc_rot = rotated ? 1 : 0;
         if ((rc = cuda_status(g4::launch_qknorm_rope(na, st)))) return rc;
     }
     // 3) attention of the chunk's queries (key row q_off + t) over the frame
@@ -681,6 +690,36 @@ int g4attn_decode_ring(const g4attn_bf16* q, const g4attn_bf16* kring, const g4a
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
     return launch_decode_plan(q, kring, vring, L, C, C, out, lse,
                               static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream);
+}
+
+size_t g4attn_decode_rotated_workspace_size(int B, int L, int C, const g4attn_layer_cfg* cfg) {
+    if (check_cfg(cfg, true) || B < 0 || L < 0 || C < 0) return 0;
+    if (C > 0 && check_ring(C, cfg)) return 0;
+    DeviceInfo* dev = nullptr;
+    int sms = 148;
+    if (current_device(&dev) == G4ATTN_OK) sms = dev->sms;
+    else cudaGetLastError();
+    return decode_plan(B, L, cfg, sms, 0, C).total;
+}
+
+int g4attn_decode_rotated(const g4attn_bf16* q, const g4attn_bf16* krot,
+                          const g4attn_bf16* vcache, int L, int C, g4attn_bf16* out, float* lse,
+                          void* workspace, size_t ws_bytes, int B, const g4attn_layer_cfg* cfg,
+                          g4attn_stream_t stream) {
+    int rc = check_decode(q, krot, vcache, L, out, lse, B, cfg);
+    if (rc) return rc;
+    if (cfg->kv_is_k != 0) return G4ATTN_ERR_UNSUPPORTED;   // the values must be their own
+    if (C < 0) return G4ATTN_ERR_INVALID_ARG;
+    if (C > 0 && (rc = check_ring(C, cfg))) return rc;
+    if (B == 0) return G4ATTN_OK;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    const DecodePlan plan = decode_plan(B, L, cfg, dev->sms, 0, C);
+    if (!workspace || ws_bytes < plan.total) return G4ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
+    return launch_decode_plan(q, krot, vcache, L, C > 0 ? C : L, C, out, lse,
+                              static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream,
+                              nullptr, true);
 }
 
 // Decode with no workspace argument and no allocation: the split partials go to the

@@ -39,9 +39,10 @@ struct QkNormRopeArgs {
     long long out_base;
     const uint16_t* v_in;  // optional values, copied unchanged to v_out / vc_out
     uint16_t* v_out;
-    uint16_t* kc_out;      // optional bf16 copy of the normalised, unrotated keys
-    uint16_t* vc_out;
+    uint16_t* kc_out;      // optional bf16 copy of the normalised keys: unrotated, or
+    uint16_t* vc_out;      // turned to their positions when kc_rot is set
     int kc_rows, kc_ring;
+    int kc_rot;
     Rope rope;
     int qk_norm;
     float eps;

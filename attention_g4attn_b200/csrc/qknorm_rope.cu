@@ -125,15 +125,17 @@ __global__ void __launch_bounds__(kThreads) qknorm_rope_kernel(QkNormRopeArgs a)
             store_row_half<E>(dst + lane * E, x0, f16);
             store_row_half<E>(dst + half + lane * E, x1, f16);
         }
-        if (!is_q && a.kc_out && kc_live) {
-            uint16_t* dst = a.kc_out + (kc_row * a.Hkv + h) * (long long)d;
-            store_bf16<E>(dst + lane * E, x0);
-            store_bf16<E>(dst + half + lane * E, x1);
+        uint16_t* const kc_dst = !is_q && a.kc_out && kc_live
+                                     ? a.kc_out + (kc_row * a.Hkv + h) * (long long)d
+                                     : nullptr;
+        if (kc_dst && !a.kc_rot) {
+            store_bf16<E>(kc_dst + lane * E, x0);
+            store_bf16<E>(kc_dst + half + lane * E, x1);
         }
         uint16_t* rdst = is_q ? (a.q_out ? a.q_out + (out_row * a.Hq + h) * (long long)d : nullptr)
                               : (a.krot_out ? a.krot_out + (out_row * a.Hkv + h) * (long long)d
                                             : nullptr);
-        if (rdst) {
+        if (rdst || (kc_dst && a.kc_rot)) {
 #pragma unroll
             for (int e = 0; e < E; ++e) {
                 const int i = lane * E + e;
@@ -144,8 +146,14 @@ __global__ void __launch_bounds__(kThreads) qknorm_rope_kernel(QkNormRopeArgs a)
                     x1[e] = u * c.y + w * c.x;
                 }
             }
-            store_row_half<E>(rdst + lane * E, x0, f16);
-            store_row_half<E>(rdst + half + lane * E, x1, f16);
+            if (rdst) {
+                store_row_half<E>(rdst + lane * E, x0, f16);
+                store_row_half<E>(rdst + half + lane * E, x1, f16);
+            }
+            if (kc_dst && a.kc_rot) {
+                store_bf16<E>(kc_dst + lane * E, x0);
+                store_bf16<E>(kc_dst + half + lane * E, x1);
+            }
         }
     }
 }

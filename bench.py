@@ -217,10 +217,11 @@ def time_decode_128k(device, stream, reps=5):
     return {"workload": wl.name, "ms": t * 1e3, "gbs": wl.cache_bytes() / t / 1e9}
 
 
-def time_local_ring_decode(device, stream, reps=10):
+def time_local_ring_decode(device, stream, reps=10, rotated=False):
     """Decode step of the block's local layer (32 q / 16 kv heads, d 256, window 1024,
     separate values) for 16 sequences at position 65535, against ring caches of 1024 rows:
-    the keys and values of the window, each read once."""
+    the keys and values of the window, each read once.  rotated: the ring holds the keys
+    turned to their positions (g4attn_decode_rotated), so none is turned on the fly."""
     import torch
     from attention_g4attn_b200 import binding as b, synth, workloads
     ly = workloads.LOCAL_W1024
@@ -231,20 +232,27 @@ def time_local_ring_decode(device, stream, reps=10):
     ws = torch.empty(b.g4attn_decode_ring_workspace_size(B, L, C, cfg), dtype=torch.uint8,
                      device=device)
     out = torch.empty_like(d.q)
+    def call():
+        if rotated:
+            b.g4attn_decode_rotated(d.q, d.k, d.v, L, cfg, ring=True, out=out, workspace=ws,
+                                    stream=stream)
+        else:
+            b.g4attn_decode_ring(d.q, d.k, d.v, L, cfg, out=out, workspace=ws, stream=stream)
+
     for _ in range(3):
-        b.g4attn_decode_ring(d.q, d.k, d.v, L, cfg, out=out, workspace=ws, stream=stream)
+        call()
     ts = []
     for _ in range(reps):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        b.g4attn_decode_ring(d.q, d.k, d.v, L, cfg, out=out, workspace=ws, stream=stream)
+        call()
         e1.record(stream)
         e1.synchronize()
         ts.append(e0.elapsed_time(e1) / 1e3)
     t = statistics.median(ts)
     nbytes = 2.0 * B * ly.n_kv_heads * ly.window * ly.head_dim * 2
-    return {"workload": "local_decode_ring_B16_pos65535_C1024_h32x16_d256_w1024", "ms": t * 1e3,
-            "gbs": nbytes / t / 1e9}
+    name = "local_decode_ring%s_B16_pos65535_C1024_h32x16_d256_w1024" % ("_turned_keys" if rotated else "")
+    return {"workload": name, "ms": t * 1e3, "gbs": nbytes / t / 1e9}
 
 
 def time_chunked_prefill(device, stream, chunk=4096, reps=3):
@@ -512,6 +520,9 @@ def main():
             extra["global_decode_L131072"]["gbs"] / hbm_peak
         extra["local_decode_ring"] = time_local_ring_decode(device, stream)
         extra["local_decode_ring"]["frac_of_hbm"] = extra["local_decode_ring"]["gbs"] / hbm_peak
+        extra["local_decode_ring_turned_keys"] = time_local_ring_decode(device, stream, rotated=True)
+        extra["local_decode_ring_turned_keys"]["frac_of_hbm"] = \
+            extra["local_decode_ring_turned_keys"]["gbs"] / hbm_peak
         extra["chunked_prefill"] = time_chunked_prefill(device, stream)
         extra["chunked_prefill"]["frac_of_sustained"] = \
             extra["chunked_prefill"]["tflops_all_chunks"] / tf_peak

@@ -125,15 +125,21 @@ G4ATTN_API int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const 
  * next chunk, or g4attn_decode, continues from position P + Tn.
  *   q, k, v   the chunk's raw queries [B, Tn, Hq, d], keys and values [B, Tn, Hkv, d]
  *             (v as in g4attn_prefill: non-NULL exactly when kv_is_k == 0)
- *   kcache    [B, cache_rows, Hkv, d] bf16: normalised, NOT rotated keys, the layout
- *             g4attn_decode reads.  Read: positions max(0, P-W+1) .. P-1 (all P on causal
- *             layers).  Written: positions P .. P+Tn-1 (RMS(k) * gamma_k, rounded to bf16)
+ *   kcache    [B, cache_rows, Hkv, d] bf16: normalised keys, NOT rotated (the layout
+ *             g4attn_decode reads) or, with G4ATTN_CACHE_ROTATED, turned to their positions
+ *             (the layout g4attn_decode_rotated reads).  Read: positions max(0, P-W+1) ..
+ *             P-1 (all P on causal layers).  Written: positions P .. P+Tn-1 (RMS(k) *
+ *             gamma_k, turned when ROTATED, rounded to bf16)
  *   vcache    [B, cache_rows, Hkv, d] bf16 separate values (kv_is_k == 0), else NULL;
  *             same rows read and written, the chunk's v copied unchanged
- *   ring      0: linear cache, position p in row p, needs cache_rows >= P + Tn;
- *             1: ring buffer, position p in row p % cache_rows, for window layers with
- *             0 < W <= cache_rows; of a chunk longer than the ring only its last
- *             cache_rows positions are written
+ *   cache_flags  0 or a combination of
+ *             G4ATTN_CACHE_RING: position p in row p % cache_rows (window layers with
+ *               0 < W <= cache_rows; of a chunk longer than the ring only its last
+ *               cache_rows positions are written); without it position p is in row p and
+ *               cache_rows >= P + Tn
+ *             G4ATTN_CACHE_ROTATED: the keys are stored turned (separate-value layers only,
+ *               kv_is_k == 0: a keys-as-values cache must hold the unrotated keys, which
+ *               are its values)
  *   out       [B, Tn, Hq, d] bf16 (written);  lse [B, Hq, Tn] fp32 or NULL
  *   workspace / ws_bytes  >= g4attn_prefill_chunk_workspace_size(B, P, Tn, cfg),
  *             256-byte aligned (fp16 key rows of the visible positions, their (cos, sin)
@@ -144,10 +150,12 @@ G4ATTN_API int g4attn_prefill(const g4attn_bf16* q, const g4attn_bf16* k, const 
  */
 G4ATTN_API size_t g4attn_prefill_chunk_workspace_size(int B, int P, int Tn,
                                                       const g4attn_layer_cfg* cfg);
+#define G4ATTN_CACHE_RING 1
+#define G4ATTN_CACHE_ROTATED 2
 G4ATTN_API int g4attn_prefill_chunk(const g4attn_bf16* q, const g4attn_bf16* k,
                                     const g4attn_bf16* v, const float* gamma_q,
                                     const float* gamma_k, g4attn_bf16* kcache,
-                                    g4attn_bf16* vcache, int cache_rows, int ring,
+                                    g4attn_bf16* vcache, int cache_rows, int cache_flags,
                                     g4attn_bf16* out, float* lse, void* workspace,
                                     size_t ws_bytes, int B, int P, int Tn,
                                     const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
@@ -213,6 +221,27 @@ G4ATTN_API int g4attn_decode_split_cache(const g4attn_bf16* q, const g4attn_bf16
                                          const g4attn_bf16* vside, int L, g4attn_bf16* out,
                                          float* lse, void* workspace, size_t ws_bytes, int B,
                                          const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/*
+ * Decode of a separate-value layer against a cache of keys stored turned to their positions
+ * (the local layers' cache: their values are a tensor of their own, so nothing needs the
+ * unrotated key).  Same operation as g4attn_decode (C = 0) or g4attn_decode_ring (C > 0),
+ * but no key is turned on the fly:
+ *   krot    [B, L or C, Hkv, d] bf16: normalised keys, key of position p turned to angle p
+ *           (g4attn_qknorm_rope's krot_out, or g4attn_prefill_chunk with
+ *           G4ATTN_CACHE_ROTATED); linear (row p) when C == 0, ring (row p % C) when C > 0
+ *   vcache  [B, L or C, Hkv, d] bf16 values, same rows
+ *   C       0, or the ring's rows under the rules of g4attn_decode_ring
+ *   workspace / ws_bytes  >= g4attn_decode_rotated_workspace_size(B, L, C, cfg)
+ * Other arguments and results as in g4attn_decode.  kv_is_k != 0 returns
+ * G4ATTN_ERR_UNSUPPORTED.
+ */
+G4ATTN_API size_t g4attn_decode_rotated_workspace_size(int B, int L, int C,
+                                                       const g4attn_layer_cfg* cfg);
+G4ATTN_API int g4attn_decode_rotated(const g4attn_bf16* q, const g4attn_bf16* krot,
+                                     const g4attn_bf16* vcache, int L, int C, g4attn_bf16* out,
+                                     float* lse, void* workspace, size_t ws_bytes, int B,
+                                     const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
 
 /*
  * Decode without a workspace and without allocating (the papers describe no such call;

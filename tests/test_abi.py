@@ -232,7 +232,9 @@ def test_prefill_chunk_argument_checks_without_gpu(lib, b):
     assert _call_chunk(lib, b, g, rows=115) == E                     # linear cache < P + Tn
     assert _call_chunk(lib, b, g, rows=512, ring=1) == E             # ring without a window
     assert _call_chunk(lib, b, loc, v=0x6000, vc=0x8000, rows=256, ring=1) == E   # W > ring
-    assert _call_chunk(lib, b, g, ring=2) == E
+    assert _call_chunk(lib, b, g, ring=2) == E                       # turned keys: K=V layer
+    assert _call_chunk(lib, b, g, ring=4) == E                       # unknown flag
+    assert _call_chunk(lib, b, loc, v=0x6000, vc=0x8000, ring=8) == E
     assert _call_chunk(lib, b, g, P=-1) == E
     assert _call_chunk(lib, b, g, vc=0x8000) == E                    # K=V layer: no values
     assert _call_chunk(lib, b, loc, v=0x6000) == E                   # values but no value cache
@@ -240,3 +242,26 @@ def test_prefill_chunk_argument_checks_without_gpu(lib, b):
     assert _call_chunk(lib, b, g, kc=0x7008) == b.G4ATTN_ERR_MISALIGNED
     assert _call_chunk(lib, b, g, ws_bytes=16) == b.G4ATTN_ERR_WORKSPACE
     assert _call_chunk(lib, b, g, Tn=0) == b.G4ATTN_OK               # empty chunk: no-op
+
+
+def test_decode_rotated_workspace_and_checks_without_gpu(lib, b):
+    loc = b.LayerCfg(16, 8, 256, 1.0, 1e4, 512, None, 0)
+    assert b.g4attn_decode_rotated_workspace_size(4, 5000, 0, loc) == \
+        b.g4attn_decode_workspace_size(4, 5000, loc)
+    assert b.g4attn_decode_rotated_workspace_size(4, 5000, 1024, loc) == \
+        b.g4attn_decode_ring_workspace_size(4, 5000, 1024, loc)
+    assert b.g4attn_decode_rotated_workspace_size(4, 5000, 100, loc) == 0   # C % 64 != 0
+    assert b.g4attn_decode_rotated_workspace_size(4, 5000, -64, loc) == 0
+    Pt, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.g4attn_decode_rotated
+    f.restype = I
+    g = b.LayerCfg(32, 4, 512, 0.25, 1e6).c()
+    lc = loc.c()
+    f.argtypes = [Pt, Pt, Pt, I, I, Pt, Pt, Pt, ctypes.c_size_t, I, ctypes.POINTER(type(g)), Pt]
+    # keys-as-values layer: its cache holds unrotated keys
+    assert f(0x1000, 0x2000, None, 16, 0, 0x4000, None, 0x10000, 1 << 30, 1, ctypes.byref(g),
+             None) == b.G4ATTN_ERR_UNSUPPORTED
+    assert f(0x1000, 0x2000, 0x3000, 16, 100, 0x4000, None, 0x10000, 1 << 30, 1,
+             ctypes.byref(lc), None) == b.G4ATTN_ERR_INVALID_ARG              # bad ring
+    assert f(0x1000, 0x2000, None, 16, 0, 0x4000, None, 0x10000, 1 << 30, 1, ctypes.byref(lc),
+             None) == b.G4ATTN_ERR_INVALID_ARG                                # values missing

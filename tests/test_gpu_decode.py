@@ -226,3 +226,47 @@ def test_decode_split_cache_needs_keys_as_values_and_r64():
     with pytest.raises(b.G4AttnError):   # local layer: R = 128
         b.g4attn_decode_split_cache(dec.q.to(dev), dec.k.to(dev), z,
                                     b.LayerCfg.from_layer(workloads.LOCAL_W512, kv_is_k=1))
+
+
+# ------------------------------------------- cache of turned keys (separate-value layers)
+def _turned(k_pre, R, base):
+    """Each cached key turned to its position (complex-number RoPE in fp64, rounded to bf16)."""
+    import bruteforce as bf
+    kf = bf.bf16_to_f64(oracle.bf16_bits(k_pre))
+    return torch.from_numpy(bf.rope_complex(kf, np.arange(kf.shape[1]), R, base)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("L,C", [(1, 0), (700, 0), (3000, 0), (300, 512), (1500, 1024),
+                                 (5000, 512)])
+def test_decode_rotated_cache(L, C):
+    # against the definition (scores on the stored keys as they are: the oracle without
+    # rotation) and against the decode of the unrotated cache (within the bf16 rounding of the
+    # stored keys)
+    b = binding()
+    dev = torch.device("cuda:0")
+    dec = synth.decode_inputs(2, L, LOCAL.n_q_heads, LOCAL.n_kv_heads, LOCAL.head_dim, True,
+                              seed=90 + L + C)
+    R = oracle.rope_pairs(LOCAL.head_dim, LOCAL.rope_p)
+    krot = _turned(dec.k, R, LOCAL.rope_base)
+    kc, vc = (krot, dec.v) if C == 0 else (_ring(krot, L, C), _ring(dec.v, L, C))
+    cfg = b.LayerCfg.from_layer(LOCAL)
+    out, lse = b.g4attn_decode_rotated(dec.q.to(dev), kc.to(dev), vc.to(dev), L, cfg,
+                                       ring=C > 0, want_lse=True)
+    torch.cuda.synchronize()
+    assert b.g4attn_device_status() == 0
+    go, gl = to_np(out.cpu())[:, 0], to_np(lse.cpu())
+    what = "turned-key decode L=%d C=%d" % (L, C)
+    ro, rl = oracle.decode(dec.q[:, 0], krot, dec.v, ocfg(LOCAL, rope_p=0.0))
+    assert_parity(go, ro, what + " out")
+    assert_parity(gl, rl, what + " lse")
+    ro2, rl2 = oracle.decode(dec.q[:, 0], dec.k, dec.v, ocfg(LOCAL))
+    assert_parity(go, ro2, what + " out vs unrotated cache")
+    assert_parity(gl, rl2, what + " lse vs unrotated cache")
+
+
+def test_decode_rotated_refuses_keys_as_values():
+    b = binding()
+    dev = torch.device("cuda:0")
+    dec = synth.decode_inputs(1, 10, 32, 4, 512, False, seed=91)
+    with pytest.raises(b.G4AttnError):
+        b.g4attn_decode_rotated(dec.q.to(dev), dec.k.to(dev), None, 10, b.LayerCfg.from_layer(GLOBAL))

@@ -36,33 +36,46 @@ def _cache(lin_bits, P, rows, ring):
     return c
 
 
-def _run_chunk(ch, ly, P, rows, ring):
+def _turned(k_pre, R, base):
+    """Keys turned to their positions (complex-number RoPE in fp64, rounded to bf16)."""
+    import bruteforce as bf
+    kf = bf.bf16_to_f64(_bits(k_pre))
+    return torch.from_numpy(bf.rope_complex(kf, np.arange(kf.shape[1]), R, base)).to(torch.bfloat16)
+
+
+def _run_chunk(ch, ly, P, rows, ring, rotated=False):
     b = binding()
     cfg = b.LayerCfg.from_layer(ly)
-    kc = _from_bits(_cache(_bits(ch.kcache), P, rows, ring)).to(DEV)
+    kpre = ch.kcache
+    if rotated:
+        kpre = _turned(kpre, oracle.rope_pairs(ly.head_dim, ly.rope_p), ly.rope_base)
+    kc = _from_bits(_cache(_bits(kpre), P, rows, ring)).to(DEV)
     vc = None
     if ch.vcache is not None:
         vc = _from_bits(_cache(_bits(ch.vcache), P, rows, ring)).to(DEV)
     v = None if ch.v is None else ch.v.to(DEV)
     out, lse = b.g4attn_prefill_chunk(ch.q.to(DEV), ch.k.to(DEV), v, ch.gamma_q.to(DEV),
                                       ch.gamma_k.to(DEV), kc, vc, P, cfg, ring=ring,
-                                      want_lse=True)
+                                      rotated=rotated, want_lse=True)
     torch.cuda.synchronize()
     assert b.g4attn_device_status() == 0
     return out.cpu(), lse.cpu(), kc.cpu(), None if vc is None else vc.cpu()
 
 
-def _check_appended(ch, ly, P, Tn, rows, ring, kc, vc, before_k, before_v):
-    """Rows of positions P .. P+Tn-1 hold RMS(k) * gamma_k rounded to bf16 (and v as
-    given); every other row is as it was."""
-    _, kh, _ = oracle.qknorm_rope(None, ch.k, None, ch.gamma_k, ocfg(ly), pos0=P)
+def _check_appended(ch, ly, P, Tn, rows, ring, kc, vc, before_k, before_v, rotated=False):
+    """Rows of positions P .. P+Tn-1 hold RMS(k) * gamma_k (turned to its position when
+    rotated) rounded to bf16, and v as given; every other row is as it was."""
+    _, kh, kr = oracle.qknorm_rope(None, ch.k, None, ch.gamma_k, ocfg(ly), pos0=P)
+    if rotated:
+        kh = kr
     got_k, got_v = _bits(kc), None if vc is None else _bits(vc)
     written = set()
     for t in range(max(0, Tn - rows) if ring else 0, Tn):
         r = (P + t) % rows if ring else P + t
         written.add(r)
         g = to_np(_from_bits(got_k[:, r]))
-        np.testing.assert_allclose(g, kh[:, t], rtol=2.0 ** -8, atol=1e-30)
+        # one bf16 rounding, plus the fp32 turn's error on components that cancel
+        np.testing.assert_allclose(g, kh[:, t], rtol=2.0 ** -8, atol=1e-5 if rotated else 1e-30)
         if vc is not None:
             np.testing.assert_array_equal(got_v[:, r], _bits(ch.v)[:, t])
     keep = [r for r in range(rows) if r not in written]
@@ -71,18 +84,21 @@ def _check_appended(ch, ly, P, Tn, rows, ring, kc, vc, before_k, before_v):
         np.testing.assert_array_equal(got_v[:, keep], before_v[:, keep])
 
 
-def _chunk_case(ly, B, P, Tn, rows, ring, seed):
+def _chunk_case(ly, B, P, Tn, rows, ring, seed, rotated=False):
     ch = synth.chunk_inputs(B, P, Tn, ly.n_q_heads, ly.n_kv_heads, ly.head_dim, ly.separate_v,
                             seed=seed)
-    out, lse, kc, vc = _run_chunk(ch, ly, P, rows, ring)
+    out, lse, kc, vc = _run_chunk(ch, ly, P, rows, ring, rotated)
     ro, rl = oracle.prefill_chunk(ch.q, ch.k, ch.v, ch.kcache, ch.vcache, ch.gamma_q,
                                   ch.gamma_k, P, ocfg(ly))
     what = "chunk P=%d Tn=%d rows=%d ring=%d" % (P, Tn, rows, ring)
     assert_parity(to_np(out), ro, what + " out")
     assert_parity(to_np(lse), rl, what + " lse")
-    before_k = _cache(_bits(ch.kcache), P, rows, ring)
+    kpre = ch.kcache
+    if rotated:
+        kpre = _turned(kpre, oracle.rope_pairs(ly.head_dim, ly.rope_p), ly.rope_base)
+    before_k = _cache(_bits(kpre), P, rows, ring)
     before_v = None if ch.vcache is None else _cache(_bits(ch.vcache), P, rows, ring)
-    _check_appended(ch, ly, P, Tn, rows, ring, kc, vc, before_k, before_v)
+    _check_appended(ch, ly, P, Tn, rows, ring, kc, vc, before_k, before_v, rotated)
 
 
 @pytest.mark.parametrize("P,Tn", [(0, 200), (128, 128), (300, 77), (1000, 256), (4097, 130),
@@ -113,16 +129,24 @@ def test_local_chunk_ring_cache(P, Tn, C):
     _chunk_case(LOCAL, 1, P, Tn, C, True, 300 + P + C)
 
 
+@pytest.mark.parametrize("P,Tn,C", [(700, 300, 0), (1500, 300, 512), (600, 1100, 512)])
+def test_local_chunk_turned_key_cache(P, Tn, C):
+    # the cache holds keys turned to their positions: read as stored, appended turned; the
+    # oracle works on the unrotated cache (within the bf16 rounding of the turned keys)
+    _chunk_case(LOCAL, 1, P, Tn, C if C else P + Tn, C > 0, 400 + P, rotated=True)
+
+
 def test_local_chunk_keys_as_values_window():
     ly = workloads.with_layer(LOCAL, kv_is_k=1, window=100)
     _chunk_case(ly, 1, 450, 200, 700, False, 9)
 
 
-@pytest.mark.parametrize("ly,cuts,ring_rows", [
-    (GLOBAL, (0, 700, 1300, 2000), 0),
-    (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 0),
-    (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 320)])
-def test_prompt_in_chunks_matches_the_full_prefill(ly, cuts, ring_rows):
+@pytest.mark.parametrize("ly,cuts,ring_rows,rotated", [
+    (GLOBAL, (0, 700, 1300, 2000), 0, False),
+    (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 0, False),
+    (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 320, False),
+    (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 320, True)])
+def test_prompt_in_chunks_matches_the_full_prefill(ly, cuts, ring_rows, rotated):
     # a prompt fed in chunks, each against the cache the previous chunks wrote, gives the
     # full-sequence prefill (the cache rounds the normalised keys to bf16: within the bar)
     b = binding()
@@ -140,7 +164,7 @@ def test_prompt_in_chunks_matches_the_full_prefill(ly, cuts, ring_rows):
         o, l = b.g4attn_prefill_chunk(inp.q[:, sl].contiguous().to(DEV),
                                       inp.k[:, sl].contiguous().to(DEV), v,
                                       inp.gamma_q.to(DEV), inp.gamma_k.to(DEV), kc, vc, P, cfg,
-                                      ring=bool(ring_rows), want_lse=True)
+                                      ring=bool(ring_rows), rotated=rotated, want_lse=True)
         outs.append(o.cpu())
         lses.append(l.cpu())
     torch.cuda.synchronize()
@@ -149,3 +173,16 @@ def test_prompt_in_chunks_matches_the_full_prefill(ly, cuts, ring_rows):
     ro, rl = oracle.prefill_rows(inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, ocfg(ly))
     assert_parity(to_np(out), ro, "chunked prompt out")
     assert_parity(to_np(lse), rl, "chunked prompt lse")
+    if ring_rows and rotated:
+        # the next token's decode against the cache the chunks left (turned keys, ring)
+        gen = torch.Generator().manual_seed(5)
+        qn = torch.randn((1, 1, ly.n_q_heads, ly.head_dim), generator=gen).to(torch.bfloat16)
+        o, l = b.g4attn_decode_rotated(qn.to(DEV), kc, vc, T, cfg, ring=True, want_lse=True)
+        torch.cuda.synchronize()
+        assert b.g4attn_device_status() == 0
+        # the oracle's cache: the normalised keys of the whole prompt (exact, unrotated)
+        _, kh, _ = oracle.qknorm_rope(None, inp.k, None, inp.gamma_k, ocfg(ly))
+        kh_bits = oracle.bf16_bits(torch.from_numpy(kh).to(torch.bfloat16))
+        ro, rl = oracle.decode(qn[:, 0], kh_bits, inp.v, ocfg(ly))
+        assert_parity(to_np(o.cpu())[:, 0], ro, "decode after chunks out")
+        assert_parity(to_np(l.cpu()), rl, "decode after chunks lse")
