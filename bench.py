@@ -356,6 +356,10 @@ CASES = {
     "local_prefill_T16384": ("prefill", dict(B=1, T=16384, layer="LOCAL_W1024")),
     "global_decode_L8192": ("decode", dict(B=16, L=8192, layer="GLOBAL_8TO1")),
     "global_decode_L32768": ("decode", dict(B=16, L=32768, layer="GLOBAL_8TO1")),
+    # the local layer's decode at position 65535 over rings of 1024 rows (1.07 GB of window)
+    "local_decode_ring_B64": ("ring", dict(B=64, L=65536, C=1024, layer="LOCAL_W1024")),
+    "local_decode_ring_turned_B64": ("ring_turned", dict(B=64, L=65536, C=1024,
+                                                         layer="LOCAL_W1024")),
 }
 
 
@@ -380,6 +384,23 @@ def run_case(name, steps, warmup):
                              workspace=ws, stream=stream)
         work = 4.0 * ly.head_dim * ly.n_q_heads * p["B"] * workloads.visible_pairs(p["T"], ly.window)
         unit = "TFLOP/s"
+    elif kind in ("ring", "ring_turned"):
+        # the ring's rows are random draws: any ring content is a valid cache
+        d = synth.decode_inputs(p["B"], p["C"], ly.n_q_heads, ly.n_kv_heads, ly.head_dim, True,
+                                seed=3, device=dev)
+        ws = torch.empty(b.g4attn_decode_ring_workspace_size(p["B"], p["L"], p["C"], cfg),
+                         dtype=torch.uint8, device=dev)
+        out = torch.empty_like(d.q)
+
+        def call():
+            if kind == "ring":
+                b.g4attn_decode_ring(d.q, d.k, d.v, p["L"], cfg, out=out, workspace=ws,
+                                     stream=stream)
+            else:
+                b.g4attn_decode_rotated(d.q, d.k, d.v, p["L"], cfg, ring=True, out=out,
+                                        workspace=ws, stream=stream)
+        work = float(2 * p["B"] * ly.n_kv_heads * ly.window * ly.head_dim * 2) * 1e3   # -> GB/s
+        unit = "GB/s"
     else:
         d = synth.decode_inputs(p["B"], p["L"], ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False,
                                 seed=3, device=dev)
