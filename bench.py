@@ -255,6 +255,45 @@ def time_local_ring_decode(device, stream, reps=10, rotated=False):
     return {"workload": name, "ms": t * 1e3, "gbs": nbytes / t / 1e9}
 
 
+def time_decode_graph(device, reps=20):
+    """The global decode step (B=16, L=32768) captured once in a CUDA graph and replayed back
+    to back: the per-step time without host launch overhead (serving loops replay a captured
+    decode step)."""
+    import torch
+    from attention_g4attn_b200 import binding as b, synth, workloads
+    ly = workloads.GLOBAL_8TO1
+    B, L = 16, 32768
+    d = synth.decode_inputs(B, L, ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False, seed=7,
+                            device=device)
+    cfg = b.LayerCfg.from_layer(ly)
+    ws = torch.empty(b.g4attn_decode_workspace_size(B, L, cfg), dtype=torch.uint8, device=device)
+    out = torch.empty_like(d.q)
+    side = torch.cuda.Stream(device)
+    side.wait_stream(torch.cuda.current_stream(device))
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            b.g4attn_decode(d.q, d.k, None, cfg, out=out, workspace=ws)
+    torch.cuda.current_stream(device).wait_stream(side)
+    torch.cuda.synchronize(device)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        b.g4attn_decode(d.q, d.k, None, cfg, out=out, workspace=ws)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    e1.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    assert b.g4attn_device_status() == 0
+    del g
+    return {"workload": "global_decode_B16_L32768_h32x4_d512_cuda_graph_replay", "ms": t * 1e3,
+            "gbs": B * ly.n_kv_heads * L * ly.head_dim * 2 / t / 1e9}
+
+
 def time_chunked_prefill(device, stream, chunk=4096, reps=3):
     """The global layer's T = 32768 prefill (32 q / 4 kv heads, d 512, causal) fed as
     chunks of `chunk` tokens, each against the linear cache the earlier chunks wrote
@@ -544,6 +583,9 @@ def main():
         extra["local_decode_ring_turned_keys"] = time_local_ring_decode(device, stream, rotated=True)
         extra["local_decode_ring_turned_keys"]["frac_of_hbm"] = \
             extra["local_decode_ring_turned_keys"]["gbs"] / hbm_peak
+        extra["global_decode_L32768_graph"] = time_decode_graph(device)
+        extra["global_decode_L32768_graph"]["frac_of_hbm"] = \
+            extra["global_decode_L32768_graph"]["gbs"] / hbm_peak
         extra["chunked_prefill"] = time_chunked_prefill(device, stream)
         extra["chunked_prefill"]["frac_of_sustained"] = \
             extra["chunked_prefill"]["tflops_all_chunks"] / tf_peak
