@@ -14,5 +14,8 @@ from .oracle import (  # noqa: F401
     decode,
     decode_ring,
     prefill_chunk,
+    quantize_int8,
+    dequantize_int8,
+    decode_int8,
     bf16_bits,
 )

@@ -278,6 +278,10 @@ typedef struct {
     const uint16_t* q;
     const uint16_t* kc;
     const uint16_t* vc;
+    const int8_t* kq;   /* int8 cache (kq != NULL): element = scale of its row * code */
+    const float* ks;
+    const int8_t* vq;
+    const float* vs;
     const g4o_cfg* cfg;
     const int32_t* bg;  /* optional list of b * Hkv + g items; NULL = all */
     int nbg, B, L, R;
@@ -286,13 +290,27 @@ typedef struct {
     atomic_long next;
 } decode_job;
 
+/* Row (b, j, g) of the key (v = 0) or value (v = 1) cache, widened exactly to double: a bf16
+ * element, or the row's fp32 scale times an int8 code. */
+static void cache_row(const decode_job* J, int v, int b, int g, int64_t j, double* dst) {
+    int d = J->cfg->head_dim, Hkv = J->cfg->n_kv_heads;
+    size_t row = ((size_t)b * J->L + (size_t)j) * Hkv + g;
+    size_t off = row * (size_t)d;
+    if (J->kq) {
+        const int8_t* code = v ? J->vq : J->kq;
+        double sc = (double)(v ? J->vs : J->ks)[row];
+        for (int c = 0; c < d; ++c) dst[c] = sc * (double)code[off + c];
+    } else {
+        const uint16_t* src = v ? J->vc : J->kc;
+        for (int c = 0; c < d; ++c) dst[c] = bf16_to_double(src[off + c]);
+    }
+}
+
 /* Key j of the cache, as the score side (rotated to position j) and the value side. */
 static void decode_key(const decode_job* J, int b, int g, int64_t j, double* kh, double* kr) {
     const g4o_cfg* cfg = J->cfg;
-    int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
-    size_t off = (((size_t)b * J->L + (size_t)j) * Hkv + g) * (size_t)d;
-    for (int c = 0; c < d; ++c) kh[c] = bf16_to_double(J->kc[off + c]);
-    g4o_rope(kh, d, J->R, cfg->rope_base, j, kr);
+    cache_row(J, 0, b, g, j, kh);
+    g4o_rope(kh, cfg->head_dim, J->R, cfg->rope_base, j, kr);
 }
 
 static void* decode_worker(void* arg) {
@@ -344,8 +362,7 @@ static void* decode_worker(void* arg) {
             const double* vj = kh;
             if (cfg->kv_is_k == 2) vj = kr;
             if (cfg->kv_is_k == 0) {
-                size_t off = (((size_t)b * J->L + (size_t)j) * Hkv + g) * (size_t)d;
-                for (int c = 0; c < d; ++c) kr[c] = bf16_to_double(J->vc[off + c]);
+                cache_row(J, 1, b, g, j, kr);
                 vj = kr;
             }
             for (int hl = 0; hl < G; ++hl) {
@@ -362,6 +379,25 @@ static void* decode_worker(void* arg) {
     return NULL;
 }
 
+static int decode_run(decode_job* J, int nthreads) {
+    int nt = online_cores(nthreads);
+    int work = J->bg ? J->nbg : J->B * J->cfg->n_kv_heads;
+    if (work == 0) return 0;
+    if (nt > work) nt = work;
+    pthread_t* th = malloc(sizeof(pthread_t) * (size_t)nt);
+    for (int t = 0; t < nt; ++t) pthread_create(&th[t], NULL, decode_worker, J);
+    for (int t = 0; t < nt; ++t) pthread_join(th[t], NULL);
+    free(th);
+    return 0;
+}
+
+static int check_items(const int32_t* bg, int nbg, int B, const g4o_cfg* cfg) {
+    if (bg)
+        for (int i = 0; i < nbg; ++i)
+            if (bg[i] < 0 || bg[i] >= B * cfg->n_kv_heads) return -1;
+    return 0;
+}
+
 int g4o_decode(const uint16_t* q, const uint16_t* kcache, const uint16_t* vcache,
                int B, int L, const g4o_cfg* cfg, const int32_t* bg, int nbg,
                int nthreads, double* out, double* lse) {
@@ -369,18 +405,22 @@ int g4o_decode(const uint16_t* q, const uint16_t* kcache, const uint16_t* vcache
     if (cfg->kv_is_k == 0 && !vcache && L > 0) return -1;
     if (B == 0) return 0;
     if (!q || !out || (L > 0 && !kcache)) return -1;
-    if (bg)
-        for (int i = 0; i < nbg; ++i)
-            if (bg[i] < 0 || bg[i] >= B * cfg->n_kv_heads) return -1;
-    int nt = online_cores(nthreads);
-    int work = bg ? nbg : B * cfg->n_kv_heads;
-    if (work == 0) return 0;
-    if (nt > work) nt = work;
-    decode_job J = {q, kcache, vcache, cfg, bg, nbg, B, L,
+    if (check_items(bg, nbg, B, cfg)) return -1;
+    decode_job J = {q, kcache, vcache, NULL, NULL, NULL, NULL, cfg, bg, nbg, B, L,
                     g4o_rope_pairs(cfg->head_dim, cfg->rope_p), out, lse, 0};
-    pthread_t* th = malloc(sizeof(pthread_t) * (size_t)nt);
-    for (int t = 0; t < nt; ++t) pthread_create(&th[t], NULL, decode_worker, &J);
-    for (int t = 0; t < nt; ++t) pthread_join(th[t], NULL);
-    free(th);
-    return 0;
+    return decode_run(&J, nthreads);
+}
+
+int g4o_decode_int8(const uint16_t* q, const int8_t* kcodes, const float* kscales,
+                    const int8_t* vcodes, const float* vscales, int B, int L,
+                    const g4o_cfg* cfg, const int32_t* bg, int nbg, int nthreads,
+                    double* out, double* lse) {
+    if (!cfg_valid(cfg) || B < 0 || L < 0 || nbg < 0) return -1;
+    if (cfg->kv_is_k == 0 && (!vcodes || !vscales) && L > 0) return -1;
+    if (B == 0) return 0;
+    if (!q || !out || (L > 0 && (!kcodes || !kscales))) return -1;
+    if (check_items(bg, nbg, B, cfg)) return -1;
+    decode_job J = {q, NULL, NULL, kcodes, kscales, vcodes, vscales, cfg, bg, nbg, B, L,
+                    g4o_rope_pairs(cfg->head_dim, cfg->rope_p), out, lse, 0};
+    return decode_run(&J, nthreads);
 }

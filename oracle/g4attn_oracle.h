@@ -82,6 +82,14 @@ int g4o_decode(const uint16_t* q, const uint16_t* kcache, const uint16_t* vcache
                int B, int L, const g4o_cfg* cfg, const int32_t* bg, int nbg,
                int nthreads, double* out, double* lse);
 
+/* Decode against an int8 cache (the same operation as g4o_decode): element c of row (b, j, g)
+ * is scales[(b * L + j) * Hkv + g] * codes[((b * L + j) * Hkv + g) * d + c], exact in double.
+ * vcodes / vscales are the separate values (kv_is_k = 0), else NULL. */
+int g4o_decode_int8(const uint16_t* q, const int8_t* kcodes, const float* kscales,
+                    const int8_t* vcodes, const float* vscales, int B, int L,
+                    const g4o_cfg* cfg, const int32_t* bg, int nbg, int nthreads,
+                    double* out, double* lse);
+
 #ifdef __cplusplus
 }
 #endif

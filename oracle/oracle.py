@@ -72,6 +72,9 @@ def _load():
         lib.g4o_decode.argtypes = [P, P, P, ctypes.c_int, ctypes.c_int, ctypes.POINTER(_Cfg),
                                    P, ctypes.c_int, ctypes.c_int, P, P]
         lib.g4o_decode.restype = ctypes.c_int
+        lib.g4o_decode_int8.argtypes = [P, P, P, P, P, ctypes.c_int, ctypes.c_int,
+                                        ctypes.POINTER(_Cfg), P, ctypes.c_int, ctypes.c_int, P, P]
+        lib.g4o_decode_int8.restype = ctypes.c_int
         _lib = lib
     return _lib
 
@@ -258,4 +261,49 @@ def prefill_chunk(q, k, v, kcache, vcache, gamma_q, gamma_k, P: int, cfg: Oracle
             den = e.sum(axis=1, keepdims=True)
             out[b, :, h] = (e / den) @ vals[b, :, g]
             lse[b, h] = m[:, 0] + np.log(den[:, 0])
+    return out, lse
+
+
+def quantize_int8(x):
+    """int8 cache of a bf16 cache [..., d]: one scale per row (the last axis), symmetric.
+
+    The pages count the KV cache in int8 (Gemma 4 report, memory table) but give no scheme;
+    the reading taken: scale = max_c |x_c| / 127 and code_c = round(x_c / scale) (half to
+    even), clamped to [-127, 127]; a row of zeros has scale 0 and codes 0.  These steps take
+    integer decisions, so they run in IEEE fp32 (each operation rounded to nearest), the
+    precision the device quantiser uses, and the codes and scales are exact to compare.
+    Returns (codes int8 [..., d], scales float32 [...])."""
+    xf = _widen(bf16_bits(x)).astype(np.float32)          # exact: bf16 values fit fp32
+    amax = np.max(np.abs(xf), axis=-1)
+    scales = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(scales > 0, scales, np.float32(1.0)).astype(np.float32)
+    ratio = (xf / safe[..., None]).astype(np.float32)
+    codes = np.clip(np.rint(ratio), -127, 127)
+    codes = np.where(scales[..., None] > 0, codes, 0).astype(np.int8)
+    return codes, scales
+
+
+def dequantize_int8(codes, scales):
+    """scale * code per element, in float64 (exact)."""
+    return np.asarray(scales, np.float64)[..., None] * np.asarray(codes, np.float64)
+
+
+def decode_int8(q, kcodes, kscales, vcodes, vscales, cfg: OracleCfg, items=None, nthreads: int = 0):
+    """decode() against an int8 cache: codes [B, L, Hkv, d] int8 and scales [B, L, Hkv] fp32
+    (values likewise when kv_is_k = 0); each element is scale * code, exact in double."""
+    qb = bf16_bits(q)
+    kq = np.ascontiguousarray(kcodes, np.int8)
+    ks = np.ascontiguousarray(kscales, np.float32)
+    vq = None if vcodes is None else np.ascontiguousarray(vcodes, np.int8)
+    vs = None if vscales is None else np.ascontiguousarray(vscales, np.float32)
+    B, L = kq.shape[0], kq.shape[1]
+    out = np.full((B, cfg.n_q_heads, cfg.head_dim), np.nan)
+    lse = np.full((B, cfg.n_q_heads), np.nan)
+    it = None if items is None else np.ascontiguousarray(items, dtype=np.int32)
+    c = cfg.c()
+    rc = _load().g4o_decode_int8(_ptr(qb), _ptr(kq), _ptr(ks), _ptr(vq), _ptr(vs), B, L,
+                                 ctypes.byref(c), _ptr(it), 0 if it is None else len(it),
+                                 nthreads, _ptr(out), _ptr(lse))
+    if rc != 0:
+        raise ValueError("oracle int8 decode rejected its arguments (%d)" % rc)
     return out, lse

@@ -462,3 +462,69 @@ def test_prefill_chunk_at_zero_is_the_prefill():
                                     0, cfg)
     np.testing.assert_allclose(out, ref_o, atol=1e-13, rtol=0)
     np.testing.assert_allclose(lse, ref_l, atol=1e-12, rtol=0)
+
+
+# --------------------------------------------------------------- int8 cache
+def test_quantize_int8_exact_rows():
+    # rows whose values are exact multiples of a power-of-two scale: the codes are those
+    # multiples; half-way quotients go to the even neighbour; a zero row has scale 0
+    x = torch.tensor([[127, -64, 0, 1], [0, 0, 0, 0], [127, 0.5, 1.5, 2.5], [-127, -0.5, -1.5, 3]],
+                     dtype=torch.float32).mul(0.125).to(torch.bfloat16)
+    codes, scales = oracle.quantize_int8(x)
+    np.testing.assert_array_equal(scales, np.array([0.125, 0.0, 0.125, 0.125], np.float32))
+    np.testing.assert_array_equal(codes, np.array([[127, -64, 0, 1], [0, 0, 0, 0], [127, 0, 2, 2],
+                                                   [-127, 0, -2, 3]], np.int8))
+
+
+def test_quantize_int8_bounds_on_random_rows():
+    gen = torch.Generator().manual_seed(81)
+    x = (torch.randn((3, 50, 2, 256), generator=gen) * torch.rand((3, 50, 2, 1), generator=gen) * 4)
+    x = x.to(torch.bfloat16)
+    codes, scales = oracle.quantize_int8(x)
+    xf = bf.bf16_to_f64(_bits(x))
+    assert codes.dtype == np.int8 and scales.dtype == np.float32
+    assert np.all(np.abs(codes.astype(np.int32)) <= 127)
+    # the largest magnitude of every row lands on +-127, and scale = max |x| / 127 (one fp32 rounding)
+    assert np.all(np.max(np.abs(codes.astype(np.int32)), axis=-1) == 127)
+    np.testing.assert_allclose(scales, np.max(np.abs(xf), axis=-1) / 127.0, rtol=2.0 ** -23)
+    # dequantised within half a step, plus the fp32 quotient's rounding: |x / s| <= 127 with
+    # relative error 2^-24, so the code is within 0.5 + 127 * 2^-24 < 0.5 + 2^-17 steps
+    err = np.abs(oracle.dequantize_int8(codes, scales) - xf)
+    assert np.all(err <= scales[..., None] * (0.5 + 2.0 ** -17) + 1e-30)
+
+
+def test_decode_int8_equals_decode_on_a_representable_cache():
+    # power-of-two scales and int8 codes give values bf16 holds exactly: the int8 decode and the
+    # bf16 decode of the same values are the same computation
+    B, L, Hq, Hkv, d = 2, 77, 8, 2, 64
+    rng = np.random.default_rng(82)
+    for kv_is_k in (1, 0):
+        kc = rng.integers(-127, 128, size=(B, L, Hkv, d)).astype(np.int8)
+        ks = np.exp2(rng.integers(-6, 2, size=(B, L, Hkv))).astype(np.float32)
+        vc = rng.integers(-127, 128, size=(B, L, Hkv, d)).astype(np.int8) if kv_is_k == 0 else None
+        vs = np.exp2(rng.integers(-6, 2, size=(B, L, Hkv))).astype(np.float32) if kv_is_k == 0 else None
+        kb = torch.from_numpy(oracle.dequantize_int8(kc, ks)).to(torch.bfloat16)
+        vb = None if vc is None else torch.from_numpy(oracle.dequantize_int8(vc, vs)).to(torch.bfloat16)
+        assert np.array_equal(bf.bf16_to_f64(_bits(kb)), oracle.dequantize_int8(kc, ks))
+        q = torch.from_numpy(rng.standard_normal((B, Hq, d))).to(torch.bfloat16)
+        cfg = _cfg(Hq, Hkv, d, p=0.25, base=1e6, window=30 if kv_is_k == 0 else 0, kv_is_k=kv_is_k)
+        a = oracle.decode(q, kb, vb, cfg)
+        c = oracle.decode_int8(q, kc, ks, vc, vs, cfg)
+        np.testing.assert_array_equal(a[0], c[0])
+        np.testing.assert_array_equal(a[1], c[1])
+
+
+def test_decode_int8_stays_close_to_the_bf16_cache():
+    # quantising a N(0,1) cache moves each element by at most half a step (max|x|/254): the
+    # decode output moves by about a percent (a dropped scale or a transposed index moves it
+    # by order one)
+    B, L, Hq, Hkv, d = 2, 300, 8, 2, 128
+    dec = synth.decode_inputs(B, L, Hq, Hkv, d, True, seed=83)
+    cfg = _cfg(Hq, Hkv, d, p=1.0, base=1e4, window=0, kv_is_k=0)
+    ref_o, ref_l = oracle.decode(dec.q[:, 0], dec.k, dec.v, cfg)
+    kc, ks = oracle.quantize_int8(dec.k)
+    vc, vs = oracle.quantize_int8(dec.v)
+    o, l = oracle.decode_int8(dec.q[:, 0], kc, ks, vc, vs, cfg)
+    rel = np.linalg.norm(o - ref_o) / np.linalg.norm(ref_o)
+    assert 1e-4 < rel < 3e-2
+    assert np.max(np.abs(l - ref_l)) < 5e-2
