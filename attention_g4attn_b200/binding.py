@@ -99,6 +99,7 @@ def _load():
         "g4attn_decode_split_cache": (I, [P, P, P, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_decode_rotated_workspace_size": (SZ, [I, I, I, CFG]),
         "g4attn_decode_rotated": (I, [P, P, P, I, I, P, P, P, SZ, I, CFG, P]),
+        "g4attn_quantize_int8": (I, [P, P, P, LL, I, P]),
         "g4attn_status_string": (ctypes.c_char_p, [I]),
         "g4attn_device_status": (I, [P]),
         "g4attn_set_wait_limit": (LL, [LL]),
@@ -341,6 +342,21 @@ def g4attn_decode_rotated(q, krot, vcache, L: int, cfg: LayerCfg, ring=False, ou
                                     ctypes.byref(c), _stream(stream))
     _check(rc, "g4attn_decode_rotated")
     return out, lse
+
+
+def g4attn_quantize_int8(x, codes=None, scales=None, stream=None):
+    """int8 cache of a bf16 cache x [..., d] (d 128, 256 or 512), one fp32 scale per row of d:
+    returns (codes int8 [..., d], scales fp32 [...])."""
+    _bf16(x, "x")
+    d = x.shape[-1]
+    rows = x.numel() // d if d else 0
+    if codes is None:
+        codes = torch.empty(x.shape, dtype=torch.int8, device=x.device)
+    if scales is None:
+        scales = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    rc = _lib.g4attn_quantize_int8(_ptr(x), _ptr(codes), _ptr(scales), rows, d, _stream(stream))
+    _check(rc, "g4attn_quantize_int8")
+    return codes, scales
 
 
 def g4attn_decode_split_cache(q, krot, vside, cfg: LayerCfg, out=None, lse=None, want_lse=False,

@@ -14,6 +14,12 @@
 #include "g4attn.h"
 #include "kernels.h"
 
+namespace g4 {
+// int8 KV cache writer (quant.cu): rows of d bf16 elements -> d int8 codes + one fp32 scale
+cudaError_t launch_quantize_int8(const uint16_t* x, int8_t* codes, float* scales, long long rows,
+                                 int d, cudaStream_t stream);
+}  // namespace g4
+
 namespace {
 
 __device__ int g_device_status = 0;   // written by bounded waits that give up
@@ -720,6 +726,20 @@ int g4attn_decode_rotated(const g4attn_bf16* q, const g4attn_bf16* krot,
     return launch_decode_plan(q, krot, vcache, L, C > 0 ? C : L, C, out, lse,
                               static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream,
                               nullptr, true);
+}
+
+int g4attn_quantize_int8(const g4attn_bf16* x, int8_t* codes, float* scales, long long rows,
+                         int d, g4attn_stream_t stream) {
+    if (rows < 0 || (d != 128 && d != 256 && d != 512)) return G4ATTN_ERR_INVALID_ARG;
+    if (rows == 0) return G4ATTN_OK;
+    if (!x || !codes || !scales) return G4ATTN_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(codes) || (reinterpret_cast<uintptr_t>(scales) & 3u))
+        return G4ATTN_ERR_MISALIGNED;
+    DeviceInfo* dev = nullptr;
+    int rc;
+    if ((rc = current_device(&dev))) return rc;
+    return cuda_status(g4::launch_quantize_int8(x, codes, scales, rows, d,
+                                                reinterpret_cast<cudaStream_t>(stream)));
 }
 
 // Decode with no workspace argument and no allocation: the split partials go to the

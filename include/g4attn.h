@@ -244,6 +244,22 @@ G4ATTN_API int g4attn_decode_rotated(const g4attn_bf16* q, const g4attn_bf16* kr
                                      const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
 
 /*
+ * int8 KV cache writer.  The Gemma 4 report's memory table counts the KV cache in int8; the
+ * scheme is not on the pages, and the one built here is symmetric with one fp32 scale per row
+ * (a position of one kv head):
+ *   scale = max_c |x_c| / 127,  code_c = round-half-even(x_c / scale) clamped to [-127, 127],
+ * both divisions IEEE fp32 rounded to nearest; a row of zeros has scale 0 and codes 0.  The
+ * element the cache stands for is scale * code.
+ *   x       [rows, d] bf16 (e.g. a [B, L, Hkv, d] cache: rows = B * L * Hkv), 16-byte aligned
+ *   codes   [rows, d] int8 (written), 16-byte aligned
+ *   scales  [rows] fp32 (written)
+ *   d       128, 256 or 512
+ * rows = 0 is a no-op; a bad d or null pointer returns G4ATTN_ERR_INVALID_ARG.
+ */
+G4ATTN_API int g4attn_quantize_int8(const g4attn_bf16* x, int8_t* codes, float* scales,
+                                    long long rows, int d, g4attn_stream_t stream);
+
+/*
  * Decode without a workspace and without allocating (the papers describe no such call;
  * it exists for callers that cannot allocate device memory: plugins whose host framework
  * owns every device allocation and hands them only input and output buffers, and services

@@ -265,3 +265,16 @@ def test_decode_rotated_workspace_and_checks_without_gpu(lib, b):
              ctypes.byref(lc), None) == b.G4ATTN_ERR_INVALID_ARG              # bad ring
     assert f(0x1000, 0x2000, None, 16, 0, 0x4000, None, 0x10000, 1 << 30, 1, ctypes.byref(lc),
              None) == b.G4ATTN_ERR_INVALID_ARG                                # values missing
+
+
+def test_quantize_int8_argument_checks_without_gpu(lib, b):
+    Pt = ctypes.c_void_p
+    f = lib.g4attn_quantize_int8
+    f.restype = ctypes.c_int
+    f.argtypes = [Pt, Pt, Pt, ctypes.c_longlong, ctypes.c_int, Pt]
+    assert f(0x1000, 0x2000, 0x3000, 10, 384, None) == b.G4ATTN_ERR_INVALID_ARG   # d
+    assert f(0x1000, 0x2000, 0x3000, -1, 512, None) == b.G4ATTN_ERR_INVALID_ARG
+    assert f(None, 0x2000, 0x3000, 10, 512, None) == b.G4ATTN_ERR_INVALID_ARG
+    assert f(0x1008, 0x2000, 0x3000, 10, 512, None) == b.G4ATTN_ERR_MISALIGNED
+    assert f(0x1000, 0x2000, 0x3002, 10, 512, None) == b.G4ATTN_ERR_MISALIGNED
+    assert f(None, None, None, 0, 512, None) == b.G4ATTN_OK                       # empty
