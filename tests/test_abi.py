@@ -278,3 +278,20 @@ def test_quantize_int8_argument_checks_without_gpu(lib, b):
     assert f(0x1008, 0x2000, 0x3000, 10, 512, None) == b.G4ATTN_ERR_MISALIGNED
     assert f(0x1000, 0x2000, 0x3002, 10, 512, None) == b.G4ATTN_ERR_MISALIGNED
     assert f(None, None, None, 0, 512, None) == b.G4ATTN_OK                       # empty
+
+
+def test_header_compiles_as_plain_c(tmp_path):
+    # the boundary is a C ABI: the public header must stand alone in a C99 translation unit
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_header.c"
+    src.write_text('#include "g4attn.h"\n'
+                   "int probe(void) { g4attn_layer_cfg c; (void)c; "
+                   "return G4ATTN_CACHE_RING | G4ATTN_CACHE_ROTATED; }\n")
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", os.path.dirname(HEADER),
+                        "-c", str(src), "-o", str(tmp_path / "use_header.o")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
