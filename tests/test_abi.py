@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -295,3 +296,25 @@ def test_header_compiles_as_plain_c(tmp_path):
                         "-c", str(src), "-o", str(tmp_path / "use_header.o")],
                        capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_prefill_chunk_frame_over_random_chunks(b, seed):
+    # the frame holds the positions any chunk query can see: from max(0, P - W + 1) (0 when
+    # causal) to P + Tn - 1; its workspace is the fp16 key copies, the (cos, sin) table and,
+    # with separate values, a bf16 value copy of those rows
+    rng = np.random.default_rng(seed)
+    layers = [b.LayerCfg(32, 4, 512, 0.25, 1e6, 0, None, 1),       # global: pre-RoPE + rotated
+              b.LayerCfg(16, 8, 256, 1.0, 1e4, 512, None, 0),      # local: rotated + values
+              b.LayerCfg(16, 8, 256, 0.5, 1e4, 100, None, 1)]      # both copies, K=V
+    for _ in range(25):
+        c = layers[rng.integers(len(layers))]
+        B, P, Tn = int(rng.integers(1, 4)), int(rng.integers(0, 5000)), int(rng.integers(1, 3000))
+        W, d, Hkv, kvk = c.window, c.head_dim, c.n_kv_heads, c.kv_is_k
+        kb = max(0, P - W + 1) if W > 0 else 0
+        Tk = P + Tn - kb
+        R = int(c.rope_p * d / 2)
+        rows = _align(B * Tk * Hkv * d * 2)
+        need_kn = kvk == 1 or R < d // 2
+        want = (2 if need_kn else 1) * rows + _align(Tk * max(R, 1) * 8) + (rows if kvk == 0 else 0)
+        assert b.g4attn_prefill_chunk_workspace_size(B, P, Tn, c) == want, (B, P, Tn, W)
