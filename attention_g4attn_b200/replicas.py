@@ -40,3 +40,30 @@ def init_from_env(backend: str = "nccl", timeout_s: int = 120):
     import torch.distributed as dist
     dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
     return dist, rank, world, local_rank
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(n: int, argv: Sequence[str], port: Optional[int] = None,
+                 timeout_s: Optional[float] = None, env: Optional[dict] = None) -> int:
+    """Run `python argv...` as `n` local ranks under torch.distributed.run (rendezvous on
+    127.0.0.1) and return its exit status.  The ranks inherit stdout / stderr, so the line
+    rank 0 prints reaches the caller's stdout unchanged."""
+    import os
+    import subprocess
+    import sys
+    if n < 1:
+        raise ValueError("need at least one rank")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           "--nproc-per-node=%d" % n, "--master-addr=127.0.0.1",
+           "--master-port=%d" % (port or free_port())] + list(argv)
+    e = dict(os.environ if env is None else env)
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "LOCAL_WORLD_SIZE", "MASTER_ADDR",
+              "MASTER_PORT", "GROUP_RANK", "ROLE_RANK", "TORCHELASTIC_RUN_ID"):
+        e.pop(k, None)
+    return subprocess.run(cmd, env=e, timeout=timeout_s).returncode

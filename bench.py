@@ -9,9 +9,10 @@ One step = one pass of the whole hot path on synthetic data shaped like the page
 their device time); the decode half of the metric (cache GB/s) rides along in `decode`.
 Inputs are larger than L2 (126 MB), so no flush is needed between steps.
 
---impl reference times the fp64 CPU oracle on a bounded sample of the same workload.
-Multi-GPU (torchrun): every rank runs an independent replica (weak scaling, no collective
-on the data path); timing is the max over ranks.
+--impl reference times the fp64 CPU oracle on the host cores, each step a bounded sample of
+the same workload.  Multi-GPU: `--gpus N` runs N ranks (under torchrun, or re-launched as N
+processes of torch.distributed.run when started plainly); every rank runs an independent
+replica (weak scaling, no collective on the data path) and the timing is the max over ranks.
 """
 import argparse
 import hashlib
@@ -48,71 +49,145 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
+TRAFFIC_JSON = os.path.join(ROOT, "profiles", "prefill_global_T65536_traffic.json")
+
+
 def recorded_traffic(kernel_hash):
-    """DRAM bytes per launch of the global prefill kernel from the committed ncu summary,
-    valid only while the kernel sources still hash to the recorded value."""
-    p = os.path.join(ROOT, "profiles", "prefill_global_T65536_traffic.md")
-    if not os.path.exists(p):
+    """DRAM bytes per launch of the global prefill kernel from the committed ncu record
+    (profiles/prefill_global_T65536_traffic.json), valid only while the kernel sources still
+    hash to the value recorded there."""
+    try:
+        with open(TRAFFIC_JSON) as f:
+            rec = json.load(f)
+    except (OSError, ValueError):
         return None
-    vals = {}
-    with open(p) as f:
-        for line in f:
-            if ":" in line and line.strip().startswith("- "):
-                k, v = line.strip()[2:].split(":", 1)
-                vals[k.strip()] = v.strip()
-    if vals.get("kernel_source_hash") != kernel_hash:
+    if rec.get("kernel_source_hash") != kernel_hash:
         return None
     try:
-        return float(vals["dram_bytes_per_full_launch"])
-    except (KeyError, ValueError):
+        return float(rec["dram_bytes_per_full_launch"])
+    except (KeyError, TypeError, ValueError):
         return None
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
-    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event reasons of one GPU, sampled every 50 ms for the whole
+    run in a background thread (NVML, read-only; `nvidia-smi` queries when NVML is missing).
+    `window()` marks a stretch of wall-clock time; `summary(w)` covers the samples inside it."""
+    # NVML clock-event reason bits (nvml.h: clocks event reasons)
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
+    SMI_FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index):
-        self.index = index
-        self.samples = []
+    def __init__(self, cuda_index):
+        self.cuda_index = cuda_index
+        self.samples = []          # (time, sm_mhz, max_mhz, watts, reasons)
         self._stop = threading.Event()
         self._thr = None
+        self._nvml = None
+        self._handle = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._handle = self._find_handle(pynvml, cuda_index)
+        except Exception:
+            self._nvml = None
+
+    @staticmethod
+    def _find_handle(pynvml, cuda_index):
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(cuda_index).uuid)
+            return pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:
+            return pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+
+    def _sample_nvml(self):
+        n, h = self._nvml, self._handle
+        sm = n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)
+        mx = n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)
+        w = n.nvmlDeviceGetPowerUsage(h) / 1000.0
+        get = getattr(n, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            n.nvmlDeviceGetCurrentClocksThrottleReasons
+        bits = int(get(h))
+        return (float(sm), float(mx), w, sorted(k for k, b in self.REASONS.items() if bits & b))
+
+    def _sample_smi(self):
+        out = subprocess.run(["nvidia-smi", "-i", str(self.cuda_index),
+                              "--query-gpu=" + self.SMI_FIELDS, "--format=csv,noheader,nounits"],
+                             capture_output=True, text=True, timeout=5)
+        p = [x.strip() for x in out.stdout.strip().split(",")]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        return (float(p[0]), float(p[1]), float(p[2]) if p[2].replace(".", "").isdigit() else None,
+                sorted(names[i] for i in range(4) if p[3 + i].lower() == "active"))
 
     def _run(self):
         while not self._stop.is_set():
             try:
-                out = subprocess.run(
-                    ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                     "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=5)
-                parts = [x.strip() for x in out.stdout.strip().split(",")]
-                if len(parts) >= 7:
-                    self.samples.append(parts)
+                s = self._sample_nvml() if self._nvml else self._sample_smi()
+                self.samples.append((time.time(),) + s)
             except Exception:
                 pass
-            self._stop.wait(0.2)
+            self._stop.wait(0.05 if self._nvml else 0.2)
 
-    def __enter__(self):
+    def start(self):
         self._thr = threading.Thread(target=self._run, daemon=True)
         self._thr.start()
         return self
 
-    def __exit__(self, *exc):
+    def stop(self):
         self._stop.set()
-        self._thr.join(timeout=10)
+        if self._thr:
+            self._thr.join(timeout=10)
 
-    def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
-        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for s in self.samples for i in range(4)
-                          if s[3 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(self.samples)}
+    class _Window:
+        def __init__(self):
+            self.t0 = self.t1 = None
+
+        def __enter__(self):
+            self.t0 = time.time()
+            return self
+
+        def __exit__(self, *exc):
+            self.t1 = time.time()
+
+    def window(self):
+        return self._Window()
+
+    def summary(self, w=None):
+        s = [x for x in self.samples if w is None or (w.t0 <= x[0] <= (w.t1 or time.time()))]
+        if not s:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(x[1] for x in s),
+                "sm_min_mhz": min(x[1] for x in s),
+                "sm_max_mhz": max(x[2] for x in s),
+                "reasons": sorted({r for x in s for r in x[4]}),
+                "samples": len(s),
+                "source": "nvml" if self._nvml else "nvidia-smi"}
+
+
+def timed_calls(call, stream, min_seconds=0.5, min_reps=5, max_reps=5000):
+    """Back-to-back calls on `stream`, each bracketed by CUDA events, until `min_seconds` of
+    device time: the median per-call seconds and the number of calls."""
+    import torch
+    evs = []
+    total = 0.0
+    while len(evs) < max_reps and (len(evs) < min_reps or total < min_seconds):
+        batch = []
+        for _ in range(min_reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            call()
+            e1.record(stream)
+            batch.append((e0, e1))
+        batch[-1][1].synchronize()
+        for e0, e1 in batch:
+            total += e0.elapsed_time(e1) / 1e3
+        evs.extend(batch)
+    ts = [e0.elapsed_time(e1) / 1e3 for e0, e1 in evs]
+    return statistics.median(ts), len(ts)
 
 
 # --------------------------------------------------------------------------- workload
@@ -164,7 +239,7 @@ def run_step(S, stream, ev=None):
 LAUNCHES_PER_STEP = 6 * 2 + 2   # per layer: key pre-pass + flash kernel; decode + combine
 
 
-def time_global_32k(device, stream, reps=3):
+def time_global_32k(device, stream):
     """Global-layer prefill at T=32768 alone (the workload of the prefill target)."""
     import torch
     from attention_g4attn_b200 import binding as b, synth, workloads
@@ -176,52 +251,42 @@ def time_global_32k(device, stream, reps=3):
     ws = torch.empty(b.g4attn_prefill_workspace_size(wl.B, wl.T, cfg), dtype=torch.uint8,
                      device=device)
     out = torch.empty_like(inp.q)
+
+    def call():
+        b.g4attn_prefill(inp.q, inp.k, None, inp.gamma_q, inp.gamma_k, cfg, out=out,
+                         workspace=ws, stream=stream)
     for _ in range(2):
-        b.g4attn_prefill(inp.q, inp.k, None, inp.gamma_q, inp.gamma_k, cfg, out=out,
-                         workspace=ws, stream=stream)
-    ts = []
-    for _ in range(reps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        b.g4attn_prefill(inp.q, inp.k, None, inp.gamma_q, inp.gamma_k, cfg, out=out,
-                         workspace=ws, stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1) / 1e3)
-    t = statistics.median(ts)
-    return {"workload": wl.name, "ms": t * 1e3, "tflops": wl.flops() / t / 1e12}
+        call()
+    t, n = timed_calls(call, stream, min_seconds=1.0, min_reps=3)
+    return {"workload": wl.name, "ms": t * 1e3, "calls": n, "tflops": wl.flops() / t / 1e12}
 
 
-def time_decode_128k(device, stream, reps=5):
+def time_decode(device, stream, wl, seed):
+    """Global-layer decode step (K=V bf16 cache), back-to-back calls."""
     import torch
-    from attention_g4attn_b200 import binding as b, synth, workloads
-    wl = workloads.GLOBAL_DECODE_128K
+    from attention_g4attn_b200 import binding as b, synth
     ly = wl.layer
     d = synth.decode_inputs(wl.B, wl.L, ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False,
-                            seed=8, device=device)
+                            seed=seed, device=device)
     cfg = b.LayerCfg.from_layer(ly)
     ws = torch.empty(b.g4attn_decode_workspace_size(wl.B, wl.L, cfg), dtype=torch.uint8,
                      device=device)
     out = torch.empty_like(d.q)
+
+    def call():
+        b.g4attn_decode(d.q, d.k, None, cfg, out=out, workspace=ws, stream=stream)
     for _ in range(3):
-        b.g4attn_decode(d.q, d.k, None, cfg, out=out, workspace=ws, stream=stream)
-    ts = []
-    for _ in range(reps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        b.g4attn_decode(d.q, d.k, None, cfg, out=out, workspace=ws, stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1) / 1e3)
-    t = statistics.median(ts)
-    return {"workload": wl.name, "ms": t * 1e3, "gbs": wl.cache_bytes() / t / 1e9}
+        call()
+    t, n = timed_calls(call, stream, min_seconds=0.5)
+    return {"workload": wl.name, "ms": t * 1e3, "calls": n, "gbs": wl.cache_bytes() / t / 1e9}
 
 
-def time_local_ring_decode(device, stream, reps=10, rotated=False):
+def time_local_ring_decode(device, stream, rotated=False):
     """Decode step of the block's local layer (32 q / 16 kv heads, d 256, window 1024,
     separate values) for 16 sequences at position 65535, against ring caches of 1024 rows:
     the keys and values of the window, each read once.  rotated: the ring holds the keys
-    turned to their positions (g4attn_decode_rotated), so none is turned on the fly."""
+    turned to their positions (g4attn_decode_rotated, the local layers' serving layout), so
+    none is turned on the fly."""
     import torch
     from attention_g4attn_b200 import binding as b, synth, workloads
     ly = workloads.LOCAL_W1024
@@ -232,6 +297,7 @@ def time_local_ring_decode(device, stream, reps=10, rotated=False):
     ws = torch.empty(b.g4attn_decode_ring_workspace_size(B, L, C, cfg), dtype=torch.uint8,
                      device=device)
     out = torch.empty_like(d.q)
+
     def call():
         if rotated:
             b.g4attn_decode_rotated(d.q, d.k, d.v, L, cfg, ring=True, out=out, workspace=ws,
@@ -241,21 +307,13 @@ def time_local_ring_decode(device, stream, reps=10, rotated=False):
 
     for _ in range(3):
         call()
-    ts = []
-    for _ in range(reps):
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        call()
-        e1.record(stream)
-        e1.synchronize()
-        ts.append(e0.elapsed_time(e1) / 1e3)
-    t = statistics.median(ts)
+    t, n = timed_calls(call, stream, min_seconds=0.3)
     nbytes = 2.0 * B * ly.n_kv_heads * ly.window * ly.head_dim * 2
     name = "local_decode_ring%s_B16_pos65535_C1024_h32x16_d256_w1024" % ("_turned_keys" if rotated else "")
-    return {"workload": name, "ms": t * 1e3, "gbs": nbytes / t / 1e9}
+    return {"workload": name, "ms": t * 1e3, "calls": n, "gbs": nbytes / t / 1e9}
 
 
-def time_decode_graph(device, reps=20):
+def time_decode_graph(device, reps=1000):
     """The global decode step (B=16, L=32768) captured once in a CUDA graph and replayed back
     to back: the per-step time without host launch overhead (serving loops replay a captured
     decode step)."""
@@ -291,7 +349,7 @@ def time_decode_graph(device, reps=20):
     assert b.g4attn_device_status() == 0
     del g
     return {"workload": "global_decode_B16_L32768_h32x4_d512_cuda_graph_replay", "ms": t * 1e3,
-            "gbs": B * ly.n_kv_heads * L * ly.head_dim * 2 / t / 1e9}
+            "calls": reps, "gbs": B * ly.n_kv_heads * L * ly.head_dim * 2 / t / 1e9}
 
 
 def time_chunked_prefill(device, stream, chunk=4096, reps=3):
@@ -343,47 +401,100 @@ def time_chunked_prefill(device, stream, chunk=4096, reps=3):
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def oracle_sample(max_seconds=20.0, seed=0):
-    """Time the fp64 oracle on a bounded sample of the step: query rows of the global layer
-    of the block (all 32 heads) against their full causal prefix of T=65536 keys.  Only the
-    sampled query rows are drawn (the rest of q stays untouched zero pages); keys are drawn
-    in full.  Returns (TFLOP/s, info, seconds)."""
-    import numpy as np
-    import torch
-    import oracle
-    from attention_g4attn_b200 import workloads
+class OracleSample:
+    """The fp64 CPU oracle on a bounded sample of the step: `rows` query rows (all 32 heads)
+    of the block's global layer (T=65536, causal), each against its full prefix, key
+    normalisation included.  The keys are drawn once; every call draws its own rows
+    (positions uniform in [T/2, T)) and their queries from `seed`."""
 
-    blk = workloads.BLOCK_5TO1_64K
-    ly = blk.layers[5]
-    gen = torch.Generator().manual_seed(1234 + seed)
-    k = torch.randn((blk.B, blk.T, ly.n_kv_heads, ly.head_dim), generator=gen).bfloat16()
-    kb = oracle.bf16_bits(k)
-    gq = (1.0 + 0.1 * torch.randn(ly.head_dim, generator=gen)).numpy()
-    gk = (1.0 + 0.1 * torch.randn(ly.head_dim, generator=gen)).numpy()
-    qb = np.zeros((blk.B, blk.T, ly.n_q_heads, ly.head_dim), np.uint16)
-    cfg = oracle.OracleCfg(ly.n_q_heads, ly.n_kv_heads, ly.head_dim, ly.rope_p, ly.rope_base,
-                           ly.window, ly.scale, ly.kv_is_k, ly.qk_norm, ly.qk_norm_eps)
-    rng = np.random.default_rng(seed)
-    nrows = 1
-    flops = 0.0
-    done_rows = 0
-    t_total = 0.0
-    while t_total < max_seconds and nrows <= 64:
-        rows = np.sort(rng.integers(blk.T // 2, blk.T, size=nrows)).astype(np.int32)
+    def __init__(self, rows=8):
+        import numpy as np
+        import torch
+        import oracle
+        from attention_g4attn_b200 import workloads
+        self.np, self.torch, self.oracle = np, torch, oracle
+        self.blk = workloads.BLOCK_5TO1_64K
+        self.ly = ly = self.blk.layers[5]
+        self.rows = rows
+        gen = torch.Generator().manual_seed(1234)
+        k = torch.randn((self.blk.B, self.blk.T, ly.n_kv_heads, ly.head_dim), generator=gen).bfloat16()
+        self.kb = oracle.bf16_bits(k)
+        self.gq = (1.0 + 0.1 * torch.randn(ly.head_dim, generator=gen)).numpy()
+        self.gk = (1.0 + 0.1 * torch.randn(ly.head_dim, generator=gen)).numpy()
+        self.qb = np.zeros((self.blk.B, self.blk.T, ly.n_q_heads, ly.head_dim), np.uint16)
+        self.cfg = oracle.OracleCfg(ly.n_q_heads, ly.n_kv_heads, ly.head_dim, ly.rope_p,
+                                    ly.rope_base, ly.window, ly.scale, ly.kv_is_k, ly.qk_norm,
+                                    ly.qk_norm_eps)
+
+    def step(self, seed):
+        """One sample: returns (FLOPs, seconds)."""
+        np, torch, ly, T = self.np, self.torch, self.ly, self.blk.T
+        rng = np.random.default_rng(seed)
+        rows = np.sort(rng.choice(np.arange(T // 2, T), size=self.rows, replace=False)).astype(np.int32)
+        gen = torch.Generator().manual_seed(10_000 + seed)
         for r in rows:
-            qr = torch.randn((blk.B, ly.n_q_heads, ly.head_dim), generator=gen).bfloat16()
-            qb[:, r] = oracle.bf16_bits(qr)
+            qr = torch.randn((self.blk.B, ly.n_q_heads, ly.head_dim), generator=gen).bfloat16()
+            self.qb[:, r] = self.oracle.bf16_bits(qr)
         t0 = time.perf_counter()
-        oracle.prefill_rows(qb, kb, None, gq, gk, cfg, rows)
-        t_total += time.perf_counter() - t0
-        flops += float(sum(4.0 * ly.head_dim * ly.n_q_heads * (int(r) + 1) for r in rows))
-        done_rows += nrows
-        nrows *= 2
+        self.oracle.prefill_rows(self.qb, self.kb, None, self.gq, self.gk, self.cfg, rows)
+        secs = time.perf_counter() - t0
+        flops = float(sum(4.0 * ly.head_dim * ly.n_q_heads * (int(r) + 1) for r in rows))
+        return flops, secs
+
+    def describe(self, steps, seconds):
+        return ("%d steps x %d query rows x %d heads of the block's global layer (T=65536, "
+                "positions uniform in [T/2, T), causal prefix of each row, key normalisation "
+                "included), %.1f s of oracle time"
+                % (steps, self.rows, self.ly.n_q_heads, seconds))
+
+
+def reference_arm(args, rank):
+    """--impl reference: the fp64 oracle (the only reference implementation of the pages'
+    method) on the host cores.  Each step is one bounded sample of the workload (OracleSample);
+    `warmup` untimed steps, then `steps` timed ones.  Under torchrun only rank 0 runs."""
+    if rank != 0:
+        return
+    steps, warmup = max(args.steps, 1), max(args.warmup, 0)
+    sampler = OracleSample(rows=8)
+    for w in range(warmup):
+        sampler.step(seed=w)
+    flops = secs = 0.0
+    for k in range(steps):
+        f, s = sampler.step(seed=1000 + k)
+        flops += f
+        secs += s
+    v = flops / secs / 1e12
     cores = os.cpu_count() or 1
-    info = {"kind": "oracle", "cores": cores,
-            "sample": "%d query rows x 32 heads of the block's global layer (T=65536, causal "
-                      "prefix of each row, key normalisation included)" % done_rows}
-    return flops / t_total / 1e12, info, t_total
+    info = {"kind": "oracle", "cores": cores, "value": v, "unit": "TFLOP/s",
+            "sample": sampler.describe(steps, secs)}
+    line = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": steps, "warmup": warmup, "ms_per_step": secs * 1e3 / steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "block_5local_1global_T65536+global_decode_B16_L32768",
+                       "step": "one sample of %d query rows x %d heads of the global layer"
+                               % (sampler.rows, sampler.ly.n_q_heads),
+                       "sample": info["sample"], "rows_per_step": sampler.rows,
+                       "heads": sampler.ly.n_q_heads, "oracle_seconds": secs},
+            "impl": "reference", "cpu_baseline": info,
+            "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def cpu_baseline(max_seconds=15.0):
+    """The oracle timed on a bounded sample (rank 0, one GPU): OracleSample steps until about
+    `max_seconds` of oracle time."""
+    sampler = OracleSample(rows=8)
+    flops = secs = 0.0
+    n = 0
+    while secs < max_seconds and n < 64:
+        f, s = sampler.step(seed=2000 + n)
+        flops += f
+        secs += s
+        n += 1
+    return {"kind": "oracle", "cores": os.cpu_count() or 1, "value": flops / secs / 1e12,
+            "unit": "TFLOP/s", "sample": sampler.describe(n, secs)}
 
 
 # --------------------------------------------------------------------------- main
@@ -475,39 +586,31 @@ def main():
     ap.add_argument("--impl", default="g4attn", choices=["g4attn", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
     args = ap.parse_args()
     if args.case:
         run_case(args.case, max(args.steps, 1), max(args.warmup, 0))
         return
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-
     if args.impl == "reference":
-        if rank != 0:
-            return
-        v, info, secs = oracle_sample(max_seconds=20.0)
-        steps = max(args.steps, 1)
-        info["value"] = v
-        line = {"metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus,
-                "steps": steps, "warmup": args.warmup, "ms_per_step": secs * 1e3,
-                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f64", "data": "synthetic",
-                "config": {"workload": "block_5local_1global_T65536+global_decode_B16_L32768",
-                           "sample": info["sample"]},
-                "impl": "reference", "cpu_baseline": info,
-                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line))
+        reference_arm(args, int(os.environ.get("RANK", "0")))
         return
 
-    import torch
     from attention_g4attn_b200 import replicas
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: run this same command as --gpus ranks under torch.distributed.run
+        sys.exit(replicas.launch_ranks(args.gpus, [os.path.abspath(__file__)] + sys.argv[1:]))
+    world_env = int(os.environ.get("WORLD_SIZE", "1"))
+    if world_env != args.gpus:
+        print("bench.py: --gpus %d but WORLD_SIZE=%d" % (args.gpus, world_env), file=sys.stderr)
+        sys.exit(2)
+
+    import torch
     dist, rank, world, local_rank = replicas.init_from_env("nccl")
     torch.cuda.set_device(local_rank)
     device = torch.device("cuda", local_rank)
     from attention_g4attn_b200 import binding as b  # noqa: F401  (fails loudly without the .so)
+    clk = ClockSampler(local_rank).start()
 
     stream = torch.cuda.Stream(device)
     with torch.cuda.stream(stream):
@@ -525,7 +628,7 @@ def main():
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local_rank) as clk:
+    with clk.window() as w_main:
         t_start.record(stream)
         for k in range(args.steps):
             run_step(S, stream, ev[k])
@@ -545,70 +648,80 @@ def main():
     dec_gbs = replicas.job_rate(dec.cache_bytes() * args.steps, dec_s, world, 1e9)
     peaks, peak_src = load_peaks()
     tf_peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    tf_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     hbm_peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
 
-    # dominant kernel: the global layer of the block (about 93% of the step's FLOPs)
+    # dominant kernel: the global layer of the block (about 93% of the step's FLOPs), timed
+    # by CUDA events on its launching stream
     g_inp, g_cfg, g_ws, g_out = S["layers"][5]
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    gt = []
-    for _ in range(3):
-        e0.record(stream)
+
+    def g_call():
         b.g4attn_prefill(g_inp.q, g_inp.k, None, g_inp.gamma_q, g_inp.gamma_k, g_cfg, out=g_out,
                          workspace=g_ws, stream=stream)
-        e1.record(stream)
-        e1.synchronize()
-        gt.append(e0.elapsed_time(e1) / 1e3)
-    g_s = statistics.median(gt)
+    with clk.window() as w_roof:
+        g_s, g_n = timed_calls(g_call, stream, min_seconds=0.4, min_reps=3)
     from attention_g4attn_b200 import workloads
     g_flops = 4.0 * 512 * 32 * blk.B * workloads.visible_pairs(blk.T, 0)
     khash = kernel_source_hash()
     roofline = {"bound": "tensor", "achieved": g_flops / g_s / 1e12, "peak": tf_peak,
                 "unit": "TFLOP/s", "frac": g_flops / g_s / 1e12 / tf_peak,
                 "traffic": recorded_traffic(khash),
+                "algorithmic_flops_per_launch": g_flops, "launch_ms": g_s * 1e3,
+                "launches_timed": g_n,
                 "kernel": "prefill_kernel<512> (+ key pre-pass) on the block's global layer",
-                "peak_source": "%s bf16_tflops_sustained" % peak_src}
+                "peak_source": "%s bf16_tflops_sustained" % peak_src,
+                "clocks": clk.summary(w_roof)}
 
     extra = {}
-    if rank == 0:
-        extra["global_prefill_T32768"] = time_global_32k(device, stream)
-        extra["global_prefill_T32768"]["frac_of_sustained"] = \
-            extra["global_prefill_T32768"]["tflops"] / tf_peak
+    if rank == 0 and not args.no_extras:
+        def run_extra(name, fn, frac_key, num_key, peak):
+            with clk.window() as w:
+                r = fn()
+            r[frac_key] = r[num_key] / peak
+            r["clocks"] = clk.summary(w)
+            extra[name] = r
+        run_extra("global_prefill_T32768", lambda: time_global_32k(device, stream),
+                  "frac_of_sustained", "tflops", tf_peak)
         extra["global_prefill_T32768"]["frac_of_burst"] = \
-            extra["global_prefill_T32768"]["tflops"] / float(peaks.get("bf16_tflops", 1590.0))
-        extra["global_decode_L131072"] = time_decode_128k(device, stream)
-        extra["global_decode_L131072"]["frac_of_hbm"] = \
-            extra["global_decode_L131072"]["gbs"] / hbm_peak
-        extra["local_decode_ring"] = time_local_ring_decode(device, stream)
-        extra["local_decode_ring"]["frac_of_hbm"] = extra["local_decode_ring"]["gbs"] / hbm_peak
-        extra["local_decode_ring_turned_keys"] = time_local_ring_decode(device, stream, rotated=True)
-        extra["local_decode_ring_turned_keys"]["frac_of_hbm"] = \
-            extra["local_decode_ring_turned_keys"]["gbs"] / hbm_peak
-        extra["global_decode_L32768_graph"] = time_decode_graph(device)
-        extra["global_decode_L32768_graph"]["frac_of_hbm"] = \
-            extra["global_decode_L32768_graph"]["gbs"] / hbm_peak
-        extra["chunked_prefill"] = time_chunked_prefill(device, stream)
-        extra["chunked_prefill"]["frac_of_sustained"] = \
-            extra["chunked_prefill"]["tflops_all_chunks"] / tf_peak
+            extra["global_prefill_T32768"]["tflops"] / tf_burst
+        run_extra("global_decode_L32768_alone",
+                  lambda: time_decode(device, stream, workloads.GLOBAL_DECODE_32K, 8),
+                  "frac_of_hbm", "gbs", hbm_peak)
+        run_extra("global_decode_L131072",
+                  lambda: time_decode(device, stream, workloads.GLOBAL_DECODE_128K, 8),
+                  "frac_of_hbm", "gbs", hbm_peak)
+        run_extra("global_decode_L32768_graph", lambda: time_decode_graph(device),
+                  "frac_of_hbm", "gbs", hbm_peak)
+        run_extra("local_decode_ring", lambda: time_local_ring_decode(device, stream),
+                  "frac_of_hbm", "gbs", hbm_peak)
+        run_extra("local_decode_ring_turned_keys",
+                  lambda: time_local_ring_decode(device, stream, rotated=True),
+                  "frac_of_hbm", "gbs", hbm_peak)
+        run_extra("chunked_prefill", lambda: time_chunked_prefill(device, stream),
+                  "frac_of_sustained", "tflops_all_chunks", tf_peak)
 
     # end to end through the public API with host buffers (pinned), copies inside the region
     e2e = None
     if not args.no_e2e:
         try:
-            e2e = run_e2e(S, stream, device, steps=min(args.steps, 2))
+            with clk.window() as w_e2e:
+                e2e = run_e2e(S, stream, device, steps=min(args.steps, 2))
         except RuntimeError as exc:   # pinned host memory refused
             e2e = {"error": str(exc)[:200]}
     if e2e is not None and "error" not in e2e:
         e2e["seconds"] = replicas.max_over_ranks([e2e["seconds"]], dist, device)[0]
         e2e = {"value": replicas.job_rate(flops_step * e2e["steps"], e2e["seconds"], world, 1e12),
                "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
-               "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"]}
+               "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],
+               "ms_per_step": e2e["seconds"] * 1e3 / e2e["steps"],
+               "overlap": "host-to-device copies on one stream, kernels on a second, "
+                          "device-to-host copies on a third, ordered per layer by events",
+               "clocks": clk.summary(w_e2e)}
+    clk.stop()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, info, _ = oracle_sample(max_seconds=15.0)
-        info["value"] = v
-        info["unit"] = "TFLOP/s"
-        cpu = info
+        cpu = cpu_baseline(max_seconds=15.0)
 
     if dist:
         dist.barrier()
@@ -624,11 +737,13 @@ def main():
                    "prefill": "5 x (32q/16kv, d256, window 1024, RoPE 1e4, separate v) + "
                               "1 x (32q/4kv, d512, p-RoPE 0.25 @ 1e6, K=V, causal), B=1, T=65536",
                    "decode": "B=16, 32q/4kv, d512, K=V cache L=32768",
-                   "l2": "inputs larger than L2, no flush", "parallelism": "replicas"},
+                   "l2": "inputs larger than L2, no flush",
+                   "parallelism": "replicas" if world == 1 else "replicas x%d" % world},
         "decode": {"value": dec_gbs, "unit": "GB/s", "frac": dec_gbs / world / hbm_peak,
-                   "peak": hbm_peak, "peak_source": "%s hbm_gbs" % peak_src},
+                   "peak": hbm_peak, "peak_source": "%s hbm_gbs" % peak_src,
+                   "ms_per_step": dec_s * 1e3 / args.steps},
         "roofline": roofline,
-        "clocks": clk.summary(),
+        "clocks": clk.summary(w_main),
         "gpu_launches": LAUNCHES_PER_STEP * args.steps,
         "device_status": status,
         "e2e": e2e,
@@ -640,45 +755,71 @@ def main():
 
 def run_e2e(S, stream, device, steps):
     """The same step through the public API with inputs in pinned host memory: every step
-    copies its inputs host->device, runs, and copies the outputs device->host."""
+    copies each layer's inputs host->device, runs the layer, and copies its output
+    device->host.  Copies in and out run on streams of their own, so layer i+1's inputs and
+    layer i-1's output cross PCIe while layer i computes; events order each layer's buffers
+    (its inputs are overwritten only after its previous compute, its output only after the
+    previous copy out)."""
     import torch
     from attention_g4attn_b200 import binding as b
 
     def pin(t):
         return None if t is None else t.to("cpu").pin_memory()
 
-    host = []
+    units = []   # (host inputs, device inputs, host out, device out, launch)
     h2d = d2h = 0
     for inp, cfg, ws, out in S["layers"]:
-        hq, hk, hv = pin(inp.q), pin(inp.k), pin(inp.v)
+        hin = [pin(t) for t in (inp.q, inp.k, inp.v)]
         ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        host.append((hq, hk, hv, ho))
-        h2d += sum(t.numel() * t.element_size() for t in (hq, hk, hv) if t is not None)
+
+        def launch(inp=inp, cfg=cfg, ws=ws, out=out):
+            b.g4attn_prefill(inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, cfg, out=out,
+                             workspace=ws, stream=stream)
+        units.append((hin, [inp.q, inp.k, inp.v], ho, out, launch))
+        h2d += sum(t.numel() * t.element_size() for t in hin if t is not None)
         d2h += ho.numel() * ho.element_size()
     d = S["dinp"]
-    hdq, hdk = pin(d.q), pin(d.k)
+    hin = [pin(d.q), pin(d.k)]
     hdo = torch.empty(S["dout"].shape, dtype=S["dout"].dtype).pin_memory()
-    h2d += hdq.numel() * 2 + hdk.numel() * 2
-    d2h += hdo.numel() * 2
+
+    def dlaunch():
+        b.g4attn_decode(d.q, d.k, None, S["dcfg"], out=S["dout"], workspace=S["dws"],
+                        stream=stream)
+    units.append((hin, [d.q, d.k], hdo, S["dout"], dlaunch))
+    h2d += sum(t.numel() * t.element_size() for t in hin)
+    d2h += hdo.numel() * hdo.element_size()
+
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    n = len(units)
+    in_ready = [torch.cuda.Event() for _ in range(n)]
+    computed = [torch.cuda.Event() for _ in range(n)]
+    drained = [torch.cuda.Event() for _ in range(n)]
     torch.cuda.synchronize()
     t0 = time.perf_counter()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    with torch.cuda.stream(stream):
-        for _ in range(steps):
-            for (inp, cfg, ws, out), (hq, hk, hv, ho) in zip(S["layers"], host):
-                inp.q.copy_(hq, non_blocking=True)
-                inp.k.copy_(hk, non_blocking=True)
-                if hv is not None:
-                    inp.v.copy_(hv, non_blocking=True)
-                b.g4attn_prefill(inp.q, inp.k, inp.v, inp.gamma_q, inp.gamma_k, cfg, out=out,
-                                 workspace=ws, stream=stream)
-                ho.copy_(out, non_blocking=True)
-            d.q.copy_(hdq, non_blocking=True)
-            d.k.copy_(hdk, non_blocking=True)
-            b.g4attn_decode(d.q, d.k, None, S["dcfg"], out=S["dout"], workspace=S["dws"],
-                            stream=stream)
-            hdo.copy_(S["dout"], non_blocking=True)
+    s_in.wait_event(e0)
+    s_out.wait_event(e0)
+    for s in range(steps):
+        for i, (hin, din, ho, dout, launch) in enumerate(units):
+            if s > 0:
+                s_in.wait_event(computed[i])      # the previous step's layer i read its inputs
+            with torch.cuda.stream(s_in):
+                for h, dv in zip(hin, din):
+                    if h is not None:
+                        dv.copy_(h, non_blocking=True)
+            in_ready[i].record(s_in)
+            stream.wait_event(in_ready[i])
+            if s > 0:
+                stream.wait_event(drained[i])     # the previous output of layer i is on the host
+            launch()
+            computed[i].record(stream)
+            s_out.wait_event(computed[i])
+            with torch.cuda.stream(s_out):
+                ho.copy_(dout, non_blocking=True)
+            drained[i].record(s_out)
+    stream.wait_stream(s_in)
+    stream.wait_stream(s_out)
     e1.record(stream)
     e1.synchronize()
     secs = e0.elapsed_time(e1) / 1e3

@@ -52,3 +52,33 @@ def test_single_process_is_a_no_op():
     assert replicas.job_rate(10.0, 2.0, 1) == 5.0
     with pytest.raises(ValueError):
         replicas.job_rate(1.0, 0.0, 1)
+
+
+def test_launcher_runs_n_ranks(tmp_path):
+    """bench.py --gpus N started without torchrun re-launches itself through
+    replicas.launch_ranks: N local ranks under torch.distributed.run, rendezvous on
+    127.0.0.1.  Here with 2 gloo ranks of a small child script on CPU."""
+    import json
+    from attention_g4attn_b200 import replicas
+    child = os.path.join(os.path.dirname(os.path.abspath(__file__)), "replica_child.py")
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    rc = replicas.launch_ranks(2, [child, str(tmp_path)], timeout_s=240, env=env)
+    assert rc == 0
+    res = [json.load(open(tmp_path / ("rank%d.json" % r))) for r in range(2)]
+    for r, x in enumerate(res):
+        assert x["rank"] == r and x["world"] == 2 and x["local_rank"] == r
+        assert x["master"] == "127.0.0.1"
+        assert x["got"] == [2.0, 3.0]
+        assert x["rate"] == pytest.approx(2 * 10.0 / 2.0)
+
+
+def test_bench_refuses_a_rank_count_that_disagrees_with_gpus():
+    """Under torchrun, bench.py checks that WORLD_SIZE equals --gpus before any GPU work."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, WORLD_SIZE="2", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "4"],
+                       env=env, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 2
+    assert "WORLD_SIZE=2" in r.stderr
