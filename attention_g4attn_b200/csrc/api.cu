@@ -32,7 +32,9 @@ struct DeviceInfo {
     bool probed = false;
     bool supported = false;
     int sms = 0;
-    int* status = nullptr;   // device address of g_device_status
+    unsigned long long ctx_id = 0;   // id of the context the addresses below belong to
+    int* status = nullptr;           // device address of g_device_status
+    void* scratch = nullptr;         // device address of the no-alloc decode's scratch
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -41,9 +43,37 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
 EncodeTiledFn g_encode = nullptr;
+CtxGetCurrentFn g_ctx_current = nullptr;
+CtxGetIdFn g_ctx_id = nullptr;
 
-// Probe the current device once: compute capability 10.0, SM count, status word address.
+template <typename F>
+F driver_fn(const char* name) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        return reinterpret_cast<F>(fn);
+    cudaGetLastError();
+    return nullptr;
+}
+
+// Unique id of the current CUDA context (0 if it cannot be read).  Device addresses of the
+// library's __device__ variables belong to a context: after cudaDeviceReset the runtime
+// creates a new primary context and the module's variables move, so addresses are cached
+// together with this id and looked up again when it changes.
+unsigned long long current_ctx_id() {
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!g_ctx_current || !g_ctx_id || g_ctx_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Probe the current device: compute capability 10.0, SM count, and the device addresses of
+// the status word and the no-alloc scratch (once per device and context).
 int current_device(DeviceInfo** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -51,6 +81,11 @@ int current_device(DeviceInfo** out) {
         return G4ATTN_ERR_CUDA;
     }
     std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+        g_encode = driver_fn<EncodeTiledFn>("cuTensorMapEncodeTiled");
+        g_ctx_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+        g_ctx_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+    }
     DeviceInfo& d = g_dev[dev];
     if (!d.probed) {
         d.probed = true;
@@ -58,26 +93,23 @@ int current_device(DeviceInfo** out) {
         cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
         cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
-        d.supported = (major == 10 && minor == 0);
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) {
-            cudaGetLastError();
-            d.supported = false;
-        }
-        d.status = static_cast<int*>(p);
-        if (!g_encode) {
-            void* fn = nullptr;
-            cudaDriverEntryPointQueryResult q;
-            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
-                    cudaSuccess &&
-                q == cudaDriverEntryPointSuccess)
-                g_encode = reinterpret_cast<EncodeTiledFn>(fn);
-            else
-                cudaGetLastError();
-        }
-        if (!g_encode) d.supported = false;
+        d.supported = (major == 10 && minor == 0) && g_encode != nullptr;
+        cudaGetLastError();
     }
     if (!d.supported) return G4ATTN_ERR_UNSUPPORTED;
+    const unsigned long long ctx = current_ctx_id();
+    if (!d.status || ctx == 0 || ctx != d.ctx_id) {
+        void* p = nullptr;
+        void* s = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess ||
+            g4::decode_scratch_ptr(&s) != cudaSuccess) {
+            cudaGetLastError();
+            return G4ATTN_ERR_CUDA;
+        }
+        d.status = static_cast<int*>(p);
+        d.scratch = s;
+        d.ctx_id = ctx;
+    }
     *out = &d;
     return G4ATTN_OK;
 }
@@ -759,14 +791,16 @@ int g4attn_decode_noalloc(const g4attn_bf16* q, const g4attn_bf16* kcache,
     if (align256(per_split * cfg->head_dim * sizeof(float)) + align256(per_split * 2 * sizeof(float)) >
         cap)
         return G4ATTN_ERR_TOO_LARGE;
+    // the most CTA pairs whose partials fit: every pair count from the full split down is
+    // tried (a count that divides the sequences evenly can fit where its neighbours cut
+    // sequences in two), so the decode keeps as many SMs as the scratch allows
     DecodePlan plan = decode_plan(B, L, cfg, dev->sms);
-    while (plan.total > cap && plan.n_pairs > 1)   // fewer pairs, fewer segments, until they fit
-        plan = decode_plan(B, L, cfg, dev->sms, plan.n_pairs / 2);
+    for (int p = plan.n_pairs - 1; plan.total > cap && p >= 1; --p)
+        plan = decode_plan(B, L, cfg, dev->sms, p);
     if (plan.total > cap) return G4ATTN_ERR_TOO_LARGE;
-    void* scratch = nullptr;
-    if (g4::decode_scratch_ptr(&scratch) != cudaSuccess) return cuda_status(cudaErrorUnknown);
+    if (!dev->scratch) return G4ATTN_ERR_CUDA;
     return launch_decode_plan(q, kcache, vcache, L, L, 0, out, lse,
-                              static_cast<uint8_t*>(scratch), plan, B, cfg, dev, stream);
+                              static_cast<uint8_t*>(dev->scratch), plan, B, cfg, dev, stream);
 }
 
 }  // extern "C"

@@ -38,8 +38,6 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
-#include <mutex>
-
 #include "kernels.h"
 #include "rope.cuh"
 #include "sm100.cuh"
@@ -918,24 +916,14 @@ static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBy
 
 size_t decode_scratch_bytes() { return kDecodeScratchBytes; }
 
+// The array's device address in the current device's context.  The caller (api.cu) calls
+// this at set-up, once per device and context, with that device current, and caches the
+// result with the context's id.
 cudaError_t decode_scratch_ptr(void** out) {
-    constexpr int kMaxDev = 64;
-    static void* ptr[kMaxDev] = {};
-    static bool ready[kMaxDev] = {};
-    static std::mutex mu;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDev) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lk(mu);
-    if (!ready[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_decode_scratch);
-        if (e != cudaSuccess) return e;
-        ptr[dev] = p;
-        ready[dev] = true;
-    }
-    *out = ptr[dev];
+    *out = p;
     return cudaSuccess;
 }
 

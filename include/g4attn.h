@@ -249,7 +249,9 @@ G4ATTN_API int g4attn_decode_rotated(const g4attn_bf16* q, const g4attn_bf16* kr
  * (a position of one kv head):
  *   scale = max_c |x_c| / 127,  code_c = round-half-even(x_c / scale) clamped to [-127, 127],
  * both divisions IEEE fp32 rounded to nearest; a row of zeros has scale 0 and codes 0.  The
- * element the cache stands for is scale * code.
+ * element the cache stands for is scale * code.  Inputs are expected finite (normalised keys
+ * are); a row holding an infinity or a NaN is written with scale NaN and codes 0, so each of
+ * its elements reads back as NaN.
  *   x       [rows, d] bf16 (e.g. a [B, L, Hkv, d] cache: rows = B * L * Hkv), 16-byte aligned
  *   codes   [rows, d] int8 (written), 16-byte aligned
  *   scales  [rows] fp32 (written)
@@ -267,12 +269,14 @@ G4ATTN_API int g4attn_quantize_int8(const g4attn_bf16* x, int8_t* codes, float* 
  * g4attn_decode minus the workspace: the split-KV partials live in a fixed 8 MiB device
  * array inside the library, which every device that loads the library holds until the
  * process exits.  The call allocates nothing.
- *   - The number of CTA pairs (and with it the segments each sequence is split into) is
- *     lowered until the partials fit; if even one segment per sequence needs more than
+ *   - The call keeps the largest number of CTA pairs (and with it of segments each sequence
+ *     is split into) whose partials fit; if even one segment per sequence needs more than
  *     8 MiB (2 * B * Hq * (head_dim + 2) * 4 bytes > 8 MiB: the kernel keeps two partials
  *     per segment), the call returns G4ATTN_ERR_TOO_LARGE and launches nothing.
- *   - The first call on a device looks up the array's device address (once per device,
- *     with that device current); make that first call before any stream capture.
+ *   - The array's device address is looked up at set-up: by the first g4attn call on a
+ *     device (any entry point), with that device current, and again if the device's CUDA
+ *     context changes (after cudaDeviceReset).  Make that first call before any stream
+ *     capture.
  *   - All calls share the one array and it keeps the last call's partials.  Nothing in it
  *     needs to start at zero (every partial is written before it is read), but calls that
  *     overlap on the GPU (different streams, or several host threads) race on it: order
