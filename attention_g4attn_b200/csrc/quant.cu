@@ -4,7 +4,9 @@
 // The Gemma 4 report's memory table counts the KV cache in int8 without giving the scheme;
 // the one built here: scale = max |x| / 127, code = round-half-even(x / scale), clamped; a
 // row of zeros keeps scale 0 and codes 0.  Both integer decisions use IEEE fp32 division
-// rounded to nearest, so the codes are reproducible on any IEEE machine.
+// rounded to nearest, so the codes are reproducible on any IEEE machine.  A row holding an
+// infinity or a NaN has no such scale: it gets scale NaN and codes 0, so every element it
+// stands for (scale * code) reads as NaN rather than as a wrong finite value.
 //
 // Memory-bound: one warp per row, each lane a contiguous run of d/32 elements (vector loads of
 // 8-32 bytes, stores of 4-16 bytes), the row maximum by warp shuffles.
@@ -67,15 +69,20 @@ __global__ void __launch_bounds__(kQuantThreads)
         }
     }
     float amax = 0.f;
+    bool finite = true;
 #pragma unroll
-    for (int i = 0; i < E; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    for (int i = 0; i < E; ++i) {
+        amax = fmaxf(amax, fabsf(v[i]));
+        finite &= isfinite(v[i]);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = __fdiv_rn(amax, 127.0f);
+    finite = __all_sync(0xffffffffu, finite);
+    const float s = finite ? __fdiv_rn(amax, 127.0f) : __int_as_float(0x7fc00000);   // NaN
     int c[E];
 #pragma unroll
     for (int i = 0; i < E; ++i) {
-        float r = s > 0.f ? rintf(__fdiv_rn(v[i], s)) : 0.f;
+        float r = s > 0.f ? rintf(__fdiv_rn(v[i], s)) : 0.f;   // NaN scale: codes 0
         r = fminf(fmaxf(r, -127.f), 127.f);
         c[i] = (int)r;
     }

@@ -272,13 +272,20 @@ def quantize_int8(x):
     even), clamped to [-127, 127]; a row of zeros has scale 0 and codes 0.  These steps take
     integer decisions, so they run in IEEE fp32 (each operation rounded to nearest), the
     precision the device quantiser uses, and the codes and scales are exact to compare.
+    A row holding an infinity or a NaN (outside the reading: max|x|/127 is not a scale)
+    gets scale NaN and codes 0.
     Returns (codes int8 [..., d], scales float32 [...])."""
     xf = _widen(bf16_bits(x)).astype(np.float32)          # exact: bf16 values fit fp32
-    amax = np.max(np.abs(xf), axis=-1)
+    finite = np.all(np.isfinite(xf), axis=-1)
+    amax = np.max(np.abs(np.where(np.isfinite(xf), xf, np.float32(0))), axis=-1)
     scales = (amax / np.float32(127.0)).astype(np.float32)
+    # a row holding an infinity or a NaN has no finite max|x|: scale NaN, codes 0, so every
+    # element it stands for reads as NaN
+    scales = np.where(finite, scales, np.float32(np.nan)).astype(np.float32)
     safe = np.where(scales > 0, scales, np.float32(1.0)).astype(np.float32)
-    ratio = (xf / safe[..., None]).astype(np.float32)
-    codes = np.clip(np.rint(ratio), -127, 127)
+    with np.errstate(invalid="ignore"):
+        ratio = (xf / safe[..., None]).astype(np.float32)
+        codes = np.clip(np.rint(ratio), -127, 127)
     codes = np.where(scales[..., None] > 0, codes, 0).astype(np.int8)
     return codes, scales
 

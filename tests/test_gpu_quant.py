@@ -43,6 +43,16 @@ def test_quantize_int8_special_rows():
     _check(x.to(torch.bfloat16))
 
 
+def test_quantize_int8_non_finite_rows():
+    # rows holding +inf, -inf or NaN get scale NaN and codes 0 on both sides
+    d = 128
+    x = torch.randn((5, d), generator=torch.Generator().manual_seed(5))
+    x[0, 3] = float("inf")
+    x[2, 100] = float("-inf")
+    x[4, 0] = float("nan")
+    _check(x.to(torch.bfloat16))
+
+
 def test_quantize_int8_full_size_global_cache():
     # the global decode workload's cache (B=16, L=32768, 4 kv heads, d 512), rows sampled
     b = binding()

@@ -476,6 +476,21 @@ def test_quantize_int8_exact_rows():
                                                    [-127, 0, -2, 3]], np.int8))
 
 
+def test_quantize_int8_non_finite_rows():
+    # a row holding +inf, -inf or NaN has no finite max|x|: scale NaN, codes 0 (every element it
+    # stands for reads as NaN); the finite rows around it are untouched
+    x = torch.tensor([[1.0, float("inf"), 2.0, -3.0], [127, -64, 0, 1],
+                      [float("-inf"), 0, 0, 0], [0.5, float("nan"), 0, 0]],
+                     dtype=torch.float32).to(torch.bfloat16)
+    codes, scales = oracle.quantize_int8(x)
+    assert np.isnan(scales[0]) and np.isnan(scales[2]) and np.isnan(scales[3])
+    assert scales[1] == np.float32(1.0)
+    np.testing.assert_array_equal(codes[[0, 2, 3]], np.zeros((3, 4), np.int8))
+    np.testing.assert_array_equal(codes[1], np.array([127, -64, 0, 1], np.int8))
+    deq = oracle.dequantize_int8(codes, scales)
+    assert np.all(np.isnan(deq[[0, 2, 3]])) and np.all(np.isfinite(deq[1]))
+
+
 def test_quantize_int8_bounds_on_random_rows():
     gen = torch.Generator().manual_seed(81)
     x = (torch.randn((3, 50, 2, 256), generator=gen) * torch.rand((3, 50, 2, 1), generator=gen) * 4)
