@@ -1,5 +1,5 @@
 """Per-config report: GPU time and roofline fraction, oracle time, and parity for the five
-named workloads (needs a CUDA device: `python tests/report_configs.py`; prints a markdown table).
+named workloads (needs a CUDA device: `python report_configs.py`; prints a markdown table).
 
 GPU: CUDA events on the launching stream, 3 warm-up calls, median of 10 timed calls (3 for the
 T=65536 layers), inputs resident in device memory.  Oracle: the fp64 CPU oracle on all host
@@ -17,8 +17,9 @@ import time
 import numpy as np
 import torch
 
-sys.path.insert(0, os.path.dirname(os.path.abspath(__file__)))
-sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+sys.path.insert(0, os.path.join(ROOT, "tests"))   # the parity helpers the GPU tests use
 
 import oracle  # noqa: E402
 from attention_g4attn_b200 import binding as b, synth, workloads  # noqa: E402

@@ -92,7 +92,7 @@ def test_global_prefill_32k_sampled():
     check_prefill(inp, ly, rows=sample_rows(wl.T, 0, n_random=8), what=wl.name)
 
 
-@pytest.mark.parametrize("layer_idx", [0, 5])
+@pytest.mark.parametrize("layer_idx", [0, 1, 2, 3, 4, 5])
 def test_block_5to1_layers_sampled(layer_idx):
     wl = workloads.BLOCK_5TO1_64K
     ly = wl.layers[layer_idx]
