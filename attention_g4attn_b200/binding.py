@@ -100,6 +100,8 @@ def _load():
         "g4attn_decode_rotated_workspace_size": (SZ, [I, I, I, CFG]),
         "g4attn_decode_rotated": (I, [P, P, P, I, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_quantize_int8": (I, [P, P, P, LL, I, P]),
+        "g4attn_decode_int8_workspace_size": (SZ, [I, I, I, CFG]),
+        "g4attn_decode_int8": (I, [P, P, P, P, P, I, I, P, P, P, SZ, I, CFG, P]),
         "g4attn_status_string": (ctypes.c_char_p, [I]),
         "g4attn_device_status": (I, [P]),
         "g4attn_set_wait_limit": (LL, [LL]),
@@ -357,6 +359,41 @@ def g4attn_quantize_int8(x, codes=None, scales=None, stream=None):
     rc = _lib.g4attn_quantize_int8(_ptr(x), _ptr(codes), _ptr(scales), rows, d, _stream(stream))
     _check(rc, "g4attn_quantize_int8")
     return codes, scales
+
+
+def g4attn_decode_int8_workspace_size(B: int, L: int, C: int, cfg: LayerCfg) -> int:
+    c = cfg.c()
+    return _lib.g4attn_decode_int8_workspace_size(B, L, C, ctypes.byref(c))
+
+
+def g4attn_decode_int8(q, kcodes, kscales, vcodes, vscales, L: int, cfg: LayerCfg, ring=False,
+                       out=None, lse=None, want_lse=False, workspace=None, stream=None):
+    """Decode one token at position L-1 against an int8 cache: codes [B, L, Hkv, d] int8 and
+    scales [B, L, Hkv] fp32 (g4attn_quantize_int8's layout), keys not rotated; values likewise
+    when kv_is_k == 0, else vcodes / vscales None.  ring=True: ring caches of C rows (row
+    p % C)."""
+    _bf16(q, "q")
+    for t, n in ((kcodes, "kcodes"), (vcodes, "vcodes")):
+        if t is not None and t.dtype != torch.int8:
+            raise G4AttnError(G4ATTN_ERR_INVALID_ARG, n + " must be int8")
+    for t, n in ((kscales, "kscales"), (vscales, "vscales")):
+        if t is not None and t.dtype != torch.float32:
+            raise G4AttnError(G4ATTN_ERR_INVALID_ARG, n + " must be float32")
+    B = kcodes.shape[0]
+    C = kcodes.shape[1] if ring else 0
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, cfg.n_q_heads), dtype=torch.float32, device=q.device)
+    c = cfg.c()
+    ws_bytes = _lib.g4attn_decode_int8_workspace_size(B, int(L), C, ctypes.byref(c))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    rc = _lib.g4attn_decode_int8(_ptr(q), _ptr(kcodes), _ptr(kscales), _ptr(vcodes),
+                                 _ptr(vscales), int(L), C, _ptr(out), _ptr(lse), _ptr(workspace),
+                                 workspace.numel(), B, ctypes.byref(c), _stream(stream))
+    _check(rc, "g4attn_decode_int8")
+    return out, lse
 
 
 def g4attn_decode_split_cache(q, krot, vside, cfg: LayerCfg, out=None, lse=None, want_lse=False,

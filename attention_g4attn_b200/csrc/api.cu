@@ -172,6 +172,20 @@ int encode_rows(CUtensorMap* m, const void* base, int B, int T, int H, int d, bo
     return r == CUDA_SUCCESS ? G4ATTN_OK : G4ATTN_ERR_CUDA;
 }
 
+// 4-D map over an int8 cache [B, T, H, d] as (d, H, T, B), box (64, 1, 64, 1) (64-byte rows),
+// 64-byte swizzle, zero fill; `T_phys` as in encode_rows.
+int encode_rows_i8(CUtensorMap* m, const void* base, int B, int T, int H, int d, int T_phys) {
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)d, (cuuint64_t)H * d, (cuuint64_t)T_phys * H * d};
+    cuuint32_t box[4] = {64, 1, 64, 1};
+    cuuint32_t es[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims,
+                          strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? G4ATTN_OK : G4ATTN_ERR_CUDA;
+}
+
 // 4-D map over the raw queries [B, T, Hq, d] as (d, Hq, T, B) with box (64, G, 128 / G, 1):
 // one box is a 64-dim chunk of a packed row tile (row = token * G + head), 128-byte swizzle.
 int encode_q_tile(CUtensorMap* m, const void* q, int B, int T, int Hq, int d, int G) {
@@ -312,15 +326,29 @@ int launch_decode_plan(const g4attn_bf16* q, const g4attn_bf16* kcache,
                        const g4attn_bf16* vcache, int L, int rows, int ring, g4attn_bf16* out,
                        float* lse, uint8_t* w, const DecodePlan& plan, int B,
                        const g4attn_layer_cfg* cfg, const DeviceInfo* dev, g4attn_stream_t stream,
-                       const g4attn_bf16* vside = nullptr, bool keys_rotated = false) {
+                       const g4attn_bf16* vside = nullptr, bool keys_rotated = false,
+                       const int8_t* kcodes = nullptr, const float* kscale = nullptr,
+                       const int8_t* vcodes = nullptr, const float* vscale = nullptr) {
     g4::DecodeArgs a{};
     const int d = cfg->head_dim, Hkv = cfg->n_kv_heads;
     int rc;
     if (L > 0) {
         const int seen = L < rows ? L : rows;   // rows that hold positions
-        if ((rc = encode_rows(&a.tm_k, kcache, B, seen, Hkv, d, false, 64, rows))) return rc;
-        if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, seen, Hkv, d, false, 64, rows)))
-            return rc;
+        if (kcodes) {
+            if ((rc = encode_rows_i8(&a.tm_k, kcodes, B, seen, Hkv, d, rows))) return rc;
+            if ((rc = encode_rows_i8(&a.tm_v, vcodes ? vcodes : kcodes, B, seen, Hkv, d, rows)))
+                return rc;
+        } else {
+            if ((rc = encode_rows(&a.tm_k, kcache, B, seen, Hkv, d, false, 64, rows))) return rc;
+            if ((rc = encode_rows(&a.tm_v, vcache ? vcache : kcache, B, seen, Hkv, d, false, 64,
+                                  rows)))
+                return rc;
+        }
+    }
+    if (kcodes) {
+        a.int8 = 1;
+        a.kscale = kscale;
+        a.vscale = vscale ? vscale : kscale;
     }
     a.q = q;
     a.part_o = reinterpret_cast<float*>(w + plan.o_off);
@@ -683,6 +711,36 @@ int g4attn_decode(const g4attn_bf16* q, const g4attn_bf16* kcache, const g4attn_
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
     return launch_decode_plan(q, kcache, vcache, L, L, 0, out, lse,
                               static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream);
+}
+
+size_t g4attn_decode_int8_workspace_size(int B, int L, int C, const g4attn_layer_cfg* cfg) {
+    return g4attn_decode_rotated_workspace_size(B, L, C, cfg);
+}
+
+int g4attn_decode_int8(const g4attn_bf16* q, const int8_t* kcodes, const float* kscales,
+                       const int8_t* vcodes, const float* vscales, int L, int C,
+                       g4attn_bf16* out, float* lse, void* workspace, size_t ws_bytes, int B,
+                       const g4attn_layer_cfg* cfg, g4attn_stream_t stream) {
+    // the bf16 decode's checks, on the code tensors' pointers
+    int rc = check_decode(q, reinterpret_cast<const g4attn_bf16*>(kcodes),
+                          reinterpret_cast<const g4attn_bf16*>(vcodes), L, out, lse, B, cfg);
+    if (rc) return rc;
+    if (cfg->n_q_heads / cfg->n_kv_heads > 8) return G4ATTN_ERR_UNSUPPORTED;
+    if ((vcodes != nullptr) != (vscales != nullptr)) return G4ATTN_ERR_INVALID_ARG;
+    if (B > 0 && L > 0 && !kscales) return G4ATTN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(kscales) & 3u) || (reinterpret_cast<uintptr_t>(vscales) & 3u))
+        return G4ATTN_ERR_MISALIGNED;
+    if (C < 0) return G4ATTN_ERR_INVALID_ARG;
+    if (C > 0 && (rc = check_ring(C, cfg))) return rc;
+    if (B == 0) return G4ATTN_OK;
+    DeviceInfo* dev = nullptr;
+    if ((rc = current_device(&dev))) return rc;
+    const DecodePlan plan = decode_plan(B, L, cfg, dev->sms, 0, C);
+    if (!workspace || ws_bytes < plan.total) return G4ATTN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return G4ATTN_ERR_MISALIGNED;
+    return launch_decode_plan(q, nullptr, nullptr, L, C > 0 ? C : L, C, out, lse,
+                              static_cast<uint8_t*>(workspace), plan, B, cfg, dev, stream,
+                              nullptr, false, kcodes, kscales, vcodes, vscales);
 }
 
 int g4attn_decode_split_cache(const g4attn_bf16* q, const g4attn_bf16* krot,

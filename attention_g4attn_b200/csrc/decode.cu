@@ -54,18 +54,38 @@ constexpr int kBarSM = 1;            // named barrier of the softmax warpgroup
 constexpr int kBarRot = 2;           // named barrier of the rotation warpgroup
 constexpr float kLazyMax = 8.0f;     // log2 units: headroom of the lazy reference max
 
-template <int NH>
+constexpr int kStageBytes = 8192;    // int8 staging slot: 64 keys x 64 dims of each half
+
+// I8: the cache holds int8 codes with one fp32 scale per row.  The codes land by TMA in a
+// staging ring (64-byte rows, 64-byte swizzle) and the rotation warps widen them into the
+// bf16 ring slots the MMAs read (exact: |code| <= 127 needs 8 bits), so the ring is shorter
+// (two tiles) to make room for the staging slots.
+template <int NH, bool I8>
 struct DecodeCfg {
     static constexpr int NS = 2 * NH;                // N of both MMAs (the pair's B rows)
     static constexpr int HH = NH / 2;                // heads finished by each half of the rows
-    static constexpr int NSLOT = NH == 8 ? 11 : 10;  // ring slots of 16 KB
+    static constexpr int NSLOT = I8 ? 8 : (NH == 8 ? 11 : 10);   // ring slots of 16 KB
+    static constexpr int NSTG = I8 ? 6 : 0;          // int8 staging slots of 8 KB
     static constexpr uint32_t TMEM_COLS = NH == 8 ? 128 : 256;   // 2 S^T + D/128 O^T blocks
 };
 
-template <int NH>
-struct __align__(1024) DecodeSmem {
-    using C = DecodeCfg<NH>;
-    uint8_t ring[C::NSLOT][kSlotBytes];
+template <int NSTG>
+struct DecodeStage {
+    uint8_t stage[NSTG][kStageBytes];
+    uint64_t stage_full[NSTG];         // a staging slot's codes landed
+    uint64_t stage_empty[NSTG];        // the rotation warps have widened it
+};
+template <>
+struct DecodeStage<0> {};
+
+// The MMA operands (ring, side buffers, q, P) must start on 1024-byte boundaries: the
+// 128-byte swizzle of the hardware is a function of the shared-memory address, and the
+// offsets computed here (sw128_offset) assume each tile starts on such a boundary.  The
+// staging base class ends with its barriers, so the ring is aligned explicitly.
+template <int NH, bool I8>
+struct __align__(1024) DecodeSmem : DecodeStage<DecodeCfg<NH, I8>::NSTG> {
+    using C = DecodeCfg<NH, I8>;
+    alignas(1024) uint8_t ring[C::NSLOT][kSlotBytes];
     uint8_t side[2][kSlotBytes];       // turned slot 0 of tiles j & 1 (values = pre-RoPE keys)
     // this CTA's half of the B operand of S^T per slot (NH rows: queries over the first
     // half of d in CTA 0, the second half in CTA 1), K-major, swizzled; q[4] (and, head_dim
@@ -151,21 +171,46 @@ constexpr uint32_t kSlotDesc = kSlotBytes >> 4;   // one ring slot, in descripto
 // The q operand copy that tile parity `odd` of rotated slot sb reads.
 __host__ __device__ constexpr int q_copy(int sb, bool odd) { return odd ? (sb == 0 ? 4 : 3) : sb; }
 
+// Sixteen int8 codes (one 16-byte piece of a staging row) as sixteen bf16, exactly: each
+// code c is biased to the byte u = c + 128, placed in the low mantissa bits of the fp32
+// 2^23 (0x4B0000uu = 2^23 + u), and 2^23 + 128 is subtracted, which leaves c exact in fp32;
+// its upper half is then c as a bf16 (c needs at most 8 significant bits).
+__device__ __forceinline__ void widen_i8x16(uint4 in, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {in.x ^ 0x80808080u, in.y ^ 0x80808080u, in.z ^ 0x80808080u,
+                           in.w ^ 0x80808080u};
+    uint32_t o[8];
+    const float2 bias = make_float2(8388736.0f, 8388736.0f);   // 2^23 + 128
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f01 = sub_f2(make_float2(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7540)),
+                                              __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7541))),
+                                  bias);
+        const float2 f23 = sub_f2(make_float2(__uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7542)),
+                                              __uint_as_float(__byte_perm(w[i], 0x4B000000u, 0x7543))),
+                                  bias);
+        o[2 * i] = __byte_perm(__float_as_uint(f01.x), __float_as_uint(f01.y), 0x7632);
+        o[2 * i + 1] = __byte_perm(__float_as_uint(f23.x), __float_as_uint(f23.y), 0x7632);
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
 // D: head dim; NH: query heads per KV head handled by the softmax (8 or 16, >= G);
 // RS: slots turned by the relative rotation (0: absolute angles).  One slot (R <= 64, values
 // not the rotated key) is the p-RoPE of the global layers; two (R <= 128, head_dim 256,
 // separate values, at most 4 query heads per kv head) the full RoPE of the local layers.
-template <int D, int NH, int RS>
+// I8: an int8 cache (codes and per-row scales), widened to bf16 in shared memory.
+template <int D, int NH, int RS, bool I8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a) {
-    using C = DecodeCfg<NH>;
+    using C = DecodeCfg<NH, I8>;
     constexpr bool REL = RS > 0;
     static_assert(RS < 2 || (D == 256 && NH == 8), "two relative slots: head_dim 256, NH 8");
     // (the host takes RS = 2 only for G <= 4)
     constexpr int NSB = D / 128;    // slots per tile and tensor
     constexpr int NS = C::NS, HH = C::HH, NSLOT = C::NSLOT;
     extern __shared__ uint8_t smem_raw[];
-    DecodeSmem<NH>& sm = *reinterpret_cast<DecodeSmem<NH>*>(
+    DecodeSmem<NH, I8>& sm = *reinterpret_cast<DecodeSmem<NH, I8>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const WaitCtl wc{a.wait_limit, a.status};
@@ -197,6 +242,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         mbar_init(&sm.q_free, 1);
         mbar_init(&sm.drain, 1);
+        if constexpr (I8) {
+            for (int i = 0; i < C::NSTG; ++i) {
+                mbar_init(&sm.stage_full[i], 1);
+                mbar_init(&sm.stage_empty[i], 1);
+            }
+        }
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -218,7 +269,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
-        if (lane == 0) {
+        if (I8 && lane == 0) {
+            if constexpr (I8) {
+                // the int8 codes of each slot (rows k: dims [64 sb, 64 sb + 64) of key k; rows
+                // 64 + k: the same dims of the second half) into the staging ring
+                prefetch_tmap(&a.tm_k);
+                if (sep_v) prefetch_tmap(&a.tm_v);
+                uint32_t q = 0;   // staging slots filled so far
+                for (int it = 0; it < n_items && !*abort; ++it) {
+                    const Item w = item_of(a, pair, pr, it);
+                    const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
+                    for (int t = 0; t < nt && !*abort; ++t) {
+                        const int kpos = w.k0 + t * kPairKeys + (int)rank * kTileKeys;
+                        const int key = a.ring > 0 ? kpos % a.ring : kpos;
+                        for (int pass = 0; pass < (sep_v ? 2 : 1) && !*abort; ++pass) {
+                            const CUtensorMap* map = pass ? &a.tm_v : &a.tm_k;
+                            for (int sb = 0; sb < NSB; ++sb) {
+                                const int st = q % C::NSTG;
+                                if (!mbar_wait(&sm.stage_empty[st], ((q / C::NSTG) & 1) ^ 1, wc,
+                                               abort))
+                                    break;
+                                mbar_arrive_expect_tx(&sm.stage_full[st], kStageBytes);
+                                tma_load_4d(sm.stage[st], map, &sm.stage_full[st], sb * 64, w.g,
+                                            key, w.b);
+                                tma_load_4d(sm.stage[st] + kStageBytes / 2, map, &sm.stage_full[st],
+                                            D / 2 + sb * 64, w.g, key, w.b);
+                                ++q;
+                            }
+                        }
+                    }
+                }
+                if (*abort) {
+                    const uint32_t first = q > (uint32_t)C::NSTG ? q - C::NSTG : 0;
+                    for (uint32_t k = first; k < q; ++k)
+                        mbar_wait_drain(&sm.stage_full[k % C::NSTG], (k / C::NSTG) & 1);
+                }
+            }
+        } else if (lane == 0) {
             prefetch_tmap(&a.tm_k);
             if (sep_v) prefetch_tmap(&a.tm_v);
             if (split) prefetch_tmap(&a.tm_vside);
@@ -385,6 +472,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool good = j < 0 || mbar_wait(&sm.pv_done[j & 1], (j >> 1) & 1, wc, abort);
             return group_all(good, kBarSM, 128);
         };
+        // I8: the fp32 scales of this thread's key in tile t of item w (key, then value
+        // scale; the value scale is the key's when the values are the keys).  They are
+        // fetched one tile ahead of their use.
+        auto scale_of = [&](const Item& w, int t) -> float2 {
+            float2 r = make_float2(0.f, 0.f);
+            if constexpr (I8) {
+                const int pos = w.k0 + t * kPairKeys + (int)rank * kTileKeys + key;
+                if (pos < w.k1) {
+                    const int rows = a.ring > 0 ? a.ring : a.L;
+                    const size_t idx =
+                        ((size_t)w.b * rows + (a.ring > 0 ? pos % a.ring : pos)) * a.Hkv + w.g;
+                    r.x = __ldg(a.kscale + idx);
+                    r.y = sep_v ? __ldg(a.vscale + idx) : r.x;
+                }
+            }
+            return r;
+        };
+        float2 scl_next = make_float2(0.f, 0.f);
+        if (I8 && n_items > 0) scl_next = scale_of(item_of(a, pair, pr, 0), 0);
         for (int it = 0; it < n_items && ok; ++it) {
             const Item w = item_of(a, pair, pr, it);
             const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
@@ -395,6 +501,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 l_part[j] = 0.f;
             }
             for (int t = 0; t < nt; ++t, ++gt) {
+                const float2 scl = scl_next;
+                if constexpr (I8) {
+                    if (t + 1 < nt) scl_next = scale_of(w, t + 1);
+                    else if (it + 1 < n_items) scl_next = scale_of(item_of(a, pair, pr, it + 1), 0);
+                }
                 ok = group_all(mbar_wait(&sm.s_full[gt & 1], (gt >> 1) & 1, wc, abort), kBarSM,
                                128);
                 if (!ok) break;
@@ -409,13 +520,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < HH; ++j) sm.xs[hf ^ 1][key][j] = hf ? sp[j] : sp[HH + j];
                 group_sync(kBarSM, 128);
                 const bool valid = key0 + key < w.k1 && key0 + key >= w.lo;
+                // int8 cache: the key's score is its scale times the product with its codes
+                const float c2k = I8 ? c2 * scl.x : c2;
                 float x[HH];
                 bool big = false;
 #pragma unroll
                 for (int j = 0; j < HH; ++j) {
                     const int h = hf * HH + j;
                     const float sc = (hf ? sp[HH + j] : sp[j]) + sm.xs[hf][key][j];
-                    x[j] = (valid && h < G) ? sc * c2 : -INFINITY;
+                    x[j] = (valid && h < G) ? sc * c2k : -INFINITY;
                     big |= x[j] > m_run[j] + kLazyMax;
                 }
                 // lazy reference max: only when some score of the tile exceeds the running
@@ -477,9 +590,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int j = 0; j < HH; ++j) {
                         const float p = (x[j] == -INFINITY) ? 0.f : ex2_approx(x[j] - m_run[j]);
-                        const __nv_bfloat16 pr = __float2bfloat16_rn(p);
-                        // the running sum uses the rounded weight the MMA sees
-                        l_part[j] = l_part[j] * alpha[j] + __bfloat162float(pr);
+                        // int8 cache: the value operand holds the codes, so the weight carries
+                        // the value's scale (bf16 keeps fp32's exponent range)
+                        const __nv_bfloat16 pr = __float2bfloat16_rn(I8 ? p * scl.y : p);
+                        // the running sum uses the rounded weight the MMA sees (int8: the
+                        // unrounded weight, the scale being folded into the rounded one)
+                        l_part[j] = l_part[j] * alpha[j] + (I8 ? p : __bfloat162float(pr));
                         *reinterpret_cast<__nv_bfloat16*>(pb + sw128_offset(hf * HH + j, key)) = pr;
                     }
                 }
@@ -671,12 +787,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 // fetch the next item's queries now: the loads fly during this tile's work
                 if (t == nt - 1 && it + 1 < n_items) prefetch(it + 1);
-                // the slots with rotated pairs first: they are turned while the rest land (the
-                // relative rotation turns its first slot while its second one lands)
                 bool got = true;
-                const int nfirst = REL ? (nrot > 0 ? 1 : 0) : nrot;
-                for (int k = 0; k < nfirst && got; ++k)
-                    got = mbar_wait(&sm.full[(qk + k) % NSLOT], ((qk + k) / NSLOT) & 1, wc, abort);
+                if constexpr (I8) {
+                    // widen the tile's int8 slots into its bf16 ring slots, each once the MMAs
+                    // are done with that ring slot: thread (rk, cp) takes rows rk and 64 + rk
+                    // (the two halves of key rk), dims [32 cp, 32 cp + 32) of the slot.  The
+                    // staging rows are 64 bytes with the 64-byte swizzle (16-byte piece c of
+                    // row r at piece c ^ ((r >> 1) & 3)), conflict-free for 8 consecutive rows.
+                    // Each staging slot goes back to the producer as soon as it is widened (a
+                    // tile can have more slots than the staging ring: separate values at
+                    // head_dim 512 take 8).
+                    for (int k = 0; k < slots_per_tile && got; ++k) {
+                        const uint32_t sq = qk + k;
+                        got = mbar_wait(&sm.stage_full[sq % C::NSTG], (sq / C::NSTG) & 1, wc, abort) &&
+                              mbar_wait(&sm.empty[sq % NSLOT], ((sq / NSLOT) & 1) ^ 1, wc, abort);
+                        if (!group_all(got, kBarRot, 128)) {
+                            got = false;
+                            break;
+                        }
+                        const uint8_t* src = sm.stage[sq % C::NSTG];
+                        uint8_t* dst = sm.ring[sq % NSLOT];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int row = 64 * h + rk;
+#pragma unroll
+                            for (int c = 0; c < 2; ++c) {
+                                const int piece = 2 * cp + c;   // dims [16 piece, 16 piece + 16)
+                                const uint4 w8 = *reinterpret_cast<const uint4*>(
+                                    src + row * 64 + ((piece ^ ((row >> 1) & 3)) << 4));
+                                uint4 lo, hi;
+                                widen_i8x16(w8, lo, hi);
+                                *reinterpret_cast<uint4*>(dst + sw128_offset(row, 16 * piece)) = lo;
+                                *reinterpret_cast<uint4*>(dst + sw128_offset(row, 16 * piece + 8)) = hi;
+                            }
+                        }
+                        // every thread's reads of the staging slot are done (and, after the
+                        // last slot, every widened row is in place for the turns below)
+                        group_sync(kBarRot, 128);
+                        if (t128 == 0) mbar_arrive(&sm.stage_empty[sq % C::NSTG]);
+                    }
+                } else {
+                    // the slots with rotated pairs first: they are turned while the rest land
+                    // (the relative rotation turns its first slot while its second one lands)
+                    const int nfirst = REL ? (nrot > 0 ? 1 : 0) : nrot;
+                    for (int k = 0; k < nfirst && got; ++k)
+                        got = mbar_wait(&sm.full[(qk + k) % NSLOT], ((qk + k) / NSLOT) & 1, wc,
+                                        abort);
+                }
                 if (R > 0) {
                     // start angle of this CTA's tile: exact (fp64-reduced) at the first tile
                     // of an item, then advanced by one pair-tile (128 keys) per step
@@ -702,7 +859,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
                         for (int r = 0; r < NRS; ++r) {
                             if (r >= nrot) break;
-                            if (r > 0) {   // the next rotated slot, landed while slot r-1 turned
+                            if (!I8 && r > 0) {   // the next rotated slot, landed while slot r-1 turned
                                 const uint32_t k = qk + r;
                                 got = group_all(mbar_wait(&sm.full[k % NSLOT], (k / NSLOT) & 1,
                                                           wc, abort),
@@ -807,7 +964,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     }
                 }
                 // every slot of the tile has landed (the MMA issuer relies on this barrier)
-                for (int k = nrot; k < slots_per_tile && got; ++k)
+                for (int k = nrot; !I8 && k < slots_per_tile && got; ++k)
                     got = mbar_wait(&sm.full[(qk + k) % NSLOT], ((qk + k) / NSLOT) & 1, wc, abort);
                 // the tile's operands are in place: one arrival per CTA on the first CTA
                 fence_proxy_async_smem();
@@ -876,30 +1033,33 @@ __global__ void __launch_bounds__(kCombineThreads)
         a.lse[bh] = dsum > 0.f ? (M + log2f(dsum)) * 0.6931471805599453f : -INFINITY;
 }
 
-template <int D, int NH, int RS>
+template <int D, int NH, int RS, bool I8>
 cudaError_t run_decode(const DecodeArgs& a, int grid, cudaStream_t stream) {
-    const size_t smem = sizeof(DecodeSmem<NH>) + 1024;
-    static_assert(sizeof(DecodeSmem<NH>) + 1024 <= 227 * 1024, "decode shared memory");
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NH, RS>,
+    using Smem = DecodeSmem<NH, I8>;
+    const size_t smem = sizeof(Smem) + 1024;
+    static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "decode shared memory");
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NH, RS, I8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    decode_kernel<D, NH, RS><<<grid, kThreads, smem, stream>>>(a);
+    decode_kernel<D, NH, RS, I8><<<grid, kThreads, smem, stream>>>(a);
     return cudaGetLastError();
 }
 
-template <int D>
+template <int D, bool I8>
 cudaError_t dispatch_decode(const DecodeArgs& a, int grid, cudaStream_t stream) {
     // relative rotation: a side buffer holds one turned slot per tile, so the pre-RoPE-value
     // layers (kv_is_k 1) take it for one rotated slot only
     const bool rel1 = a.kv_is_k != 2 && a.rope.R <= 64;
     if (a.G <= 8) {
-        if (rel1) return run_decode<D, 8, 1>(a, grid, stream);
+        if (rel1) return run_decode<D, 8, 1, I8>(a, grid, stream);
         if constexpr (D == 256)
             if (a.kv_is_k == 0 && a.rope.R <= 128 && a.G <= 4)
-                return run_decode<D, 8, 2>(a, grid, stream);
-        return run_decode<D, 8, 0>(a, grid, stream);
+                return run_decode<D, 8, 2, I8>(a, grid, stream);
+        return run_decode<D, 8, 0, I8>(a, grid, stream);
     }
-    return rel1 ? run_decode<D, 16, 1>(a, grid, stream) : run_decode<D, 16, 0>(a, grid, stream);
+    if constexpr (I8) return cudaErrorInvalidValue;   // int8 caches: at most 8 query heads per kv head
+    else return rel1 ? run_decode<D, 16, 1, false>(a, grid, stream)
+                     : run_decode<D, 16, 0, false>(a, grid, stream);
 }
 
 }  // namespace
@@ -932,9 +1092,17 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     if (a.n_pairs > 0 && a.total_tiles > 0) {
         // one cluster of two CTAs per pair of the stream-K split
         const int grid = 2 * a.n_pairs;
-        cudaError_t e = a.d == 512 ? dispatch_decode<512>(a, grid, stream)
-                        : a.d == 256 ? dispatch_decode<256>(a, grid, stream)
-                                     : cudaErrorInvalidValue;
+        cudaError_t e;
+        if (a.int8) {
+            if (a.split_cache || a.G > 8) return cudaErrorInvalidValue;
+            e = a.d == 512 ? dispatch_decode<512, true>(a, grid, stream)
+                : a.d == 256 ? dispatch_decode<256, true>(a, grid, stream)
+                             : cudaErrorInvalidValue;
+        } else {
+            e = a.d == 512 ? dispatch_decode<512, false>(a, grid, stream)
+                : a.d == 256 ? dispatch_decode<256, false>(a, grid, stream)
+                             : cudaErrorInvalidValue;
+        }
         if (e != cudaSuccess) return e;
     }
     if (a.B * a.Hq > 0) {

@@ -63,6 +63,12 @@ struct DecodeArgs {
     // slot 0; the other slots' dims are the same rotated or not); no key is turned
     CUtensorMap tm_vside;
     int split_cache;
+    // int8 cache (int8 = 1): tm_k / tm_v map the int8 codes [B, L or C, Hkv, d] as (d, Hkv,
+    // rows, B) with box (64, 1, 64, 1) and 64-byte swizzle; element = scale of its row * code,
+    // the scales fp32 [B, L or C, Hkv] (kscale; vscale for separate values)
+    int int8;
+    const float* kscale;
+    const float* vscale;
     const uint16_t* q;      // [B, Hq, d], normalised and rotated
     float* part_o;          // [2S, B, Hq, d]
     float* part_ml;         // [2S, B, Hq, 2]  (running max in log2 units, sum)

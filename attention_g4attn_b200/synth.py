@@ -97,3 +97,20 @@ def chunk_inputs(B, P, Tn, n_q_heads, n_kv_heads, head_dim, separate_v, seed, de
     gamma_q = 1.0 + 0.1 * _randn((head_dim,), gen, device)
     gamma_k = 1.0 + 0.1 * _randn((head_dim,), gen, device)
     return ChunkInputs(q, k, v, kcache, vcache, gamma_q.contiguous(), gamma_k.contiguous())
+
+
+def int8_cache(B, L, n_kv_heads, head_dim, seed, device="cpu"):
+    """A random int8 cache in g4attn_quantize_int8's layout, drawn directly (for the sizes
+    where quantising a drawn bf16 cache on the host would be slow), with the statistics of a
+    quantised N(0,1) cache of head_dim 256-512 (row maximum about 3.3, so scale about 0.026 and
+    codes about N(0, 38^2)): codes = clamp(round(38 N(0,1)), -127, 127) int8 [B, L, Hkv, d],
+    scales = 0.026 (1 + 0.05 N(0,1)) fp32 [B, L, Hkv]; the elements scale * code are then
+    close to N(0,1)."""
+    gen = torch.Generator(device=device).manual_seed(int(seed))
+    codes = torch.empty((B, L, n_kv_heads, head_dim), dtype=torch.int8, device=device)
+    flat = codes.view(-1)
+    for i in range(0, flat.numel(), _CHUNK):
+        m = min(_CHUNK, flat.numel() - i)
+        flat[i:i + m] = torch.round(38.0 * _randn((m,), gen, device)).clamp_(-127, 127).to(torch.int8)
+    scales = 0.026 * (1.0 + 0.05 * _randn((B, L, n_kv_heads), gen, device))
+    return codes, scales.contiguous()

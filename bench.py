@@ -281,6 +281,32 @@ def time_decode(device, stream, wl, seed):
     return {"workload": wl.name, "ms": t * 1e3, "calls": n, "gbs": wl.cache_bytes() / t / 1e9}
 
 
+def time_decode_int8(device, stream, wl, seed):
+    """The global decode step against an int8 cache (codes + one fp32 scale per row, the
+    layout g4attn_quantize_int8 writes): GB/s of the int8 bytes read (codes and scales)."""
+    import torch
+    from attention_g4attn_b200 import binding as b, synth
+    ly = wl.layer
+    kc, ks = synth.int8_cache(wl.B, wl.L, ly.n_kv_heads, ly.head_dim, seed=seed, device=device)
+    q = synth.decode_inputs(wl.B, 1, ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False,
+                            seed=seed, device=device).q
+    cfg = b.LayerCfg.from_layer(ly)
+    ws = torch.empty(b.g4attn_decode_int8_workspace_size(wl.B, wl.L, 0, cfg), dtype=torch.uint8,
+                     device=device)
+    out = torch.empty_like(q)
+
+    def call():
+        b.g4attn_decode_int8(q, kc, ks, None, None, wl.L, cfg, out=out, workspace=ws,
+                             stream=stream)
+    for _ in range(3):
+        call()
+    t, n = timed_calls(call, stream, min_seconds=0.5)
+    nbytes = float(kc.numel() + 4 * ks.numel())
+    return {"workload": wl.name.replace("global_decode", "global_decode_int8"), "ms": t * 1e3,
+            "calls": n, "gbs": nbytes / t / 1e9, "bytes": nbytes,
+            "bf16_equivalent_gbs": wl.cache_bytes() / t / 1e9}
+
+
 def time_local_ring_decode(device, stream, rotated=False):
     """Decode step of the block's local layer (32 q / 16 kv heads, d 256, window 1024,
     separate values) for 16 sequences at position 65535, against ring caches of 1024 rows:
@@ -510,6 +536,8 @@ CASES = {
     "local_decode_ring_B64": ("ring", dict(B=64, L=65536, C=1024, layer="LOCAL_W1024")),
     "local_decode_ring_turned_B64": ("ring_turned", dict(B=64, L=65536, C=1024,
                                                          layer="LOCAL_W1024")),
+    "global_decode_int8_L32768": ("decode_int8", dict(B=16, L=32768, layer="GLOBAL_8TO1")),
+    "global_decode_int8_L8192": ("decode_int8", dict(B=16, L=8192, layer="GLOBAL_8TO1")),
 }
 
 
@@ -550,6 +578,19 @@ def run_case(name, steps, warmup):
                 b.g4attn_decode_rotated(d.q, d.k, d.v, p["L"], cfg, ring=True, out=out,
                                         workspace=ws, stream=stream)
         work = float(2 * p["B"] * ly.n_kv_heads * ly.window * ly.head_dim * 2) * 1e3   # -> GB/s
+        unit = "GB/s"
+    elif kind == "decode_int8":
+        kc, ks = synth.int8_cache(p["B"], p["L"], ly.n_kv_heads, ly.head_dim, seed=3, device=dev)
+        q = synth.decode_inputs(p["B"], 1, ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False,
+                                seed=3, device=dev).q
+        ws = torch.empty(b.g4attn_decode_int8_workspace_size(p["B"], p["L"], 0, cfg),
+                         dtype=torch.uint8, device=dev)
+        out = torch.empty_like(q)
+
+        def call():
+            b.g4attn_decode_int8(q, kc, ks, None, None, p["L"], cfg, out=out, workspace=ws,
+                                 stream=stream)
+        work = float(kc.numel() + 4 * ks.numel()) * 1e3   # -> GB/s
         unit = "GB/s"
     else:
         d = synth.decode_inputs(p["B"], p["L"], ly.n_q_heads, ly.n_kv_heads, ly.head_dim, False,
@@ -691,6 +732,12 @@ def main():
                   lambda: time_decode(device, stream, workloads.GLOBAL_DECODE_128K, 8),
                   "frac_of_hbm", "gbs", hbm_peak)
         run_extra("global_decode_L32768_graph", lambda: time_decode_graph(device),
+                  "frac_of_hbm", "gbs", hbm_peak)
+        run_extra("global_decode_int8_L32768",
+                  lambda: time_decode_int8(device, stream, workloads.GLOBAL_DECODE_32K, 18),
+                  "frac_of_hbm", "gbs", hbm_peak)
+        run_extra("global_decode_int8_L131072",
+                  lambda: time_decode_int8(device, stream, workloads.GLOBAL_DECODE_128K, 18),
                   "frac_of_hbm", "gbs", hbm_peak)
         run_extra("local_decode_ring", lambda: time_local_ring_decode(device, stream),
                   "frac_of_hbm", "gbs", hbm_peak)

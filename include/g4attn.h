@@ -262,6 +262,33 @@ G4ATTN_API int g4attn_quantize_int8(const g4attn_bf16* x, int8_t* codes, float* 
                                     long long rows, int d, g4attn_stream_t stream);
 
 /*
+ * Decode against an int8 KV cache (the Gemma 4 report's memory table counts the KV cache in
+ * int8: papers.ananclaw.com explainer, section on long context and memory).  The cache is
+ * the one g4attn_quantize_int8 writes: codes [rows, d] int8 and one fp32 scale per row (a
+ * position of one kv head), each element standing for scale * code.  Same operation as
+ * g4attn_decode (C = 0) or g4attn_decode_ring (C > 0) on that cache:
+ *   q        [B, 1, Hq, d] bf16: the new queries, normalised and rotated to position L-1
+ *   kcodes   [B, L or C, Hkv, d] int8 and kscales [B, L or C, Hkv] fp32: normalised keys, NOT
+ *            rotated (turned on the fly, as in g4attn_decode)
+ *   vcodes / vscales  the same layout for separate values (kv_is_k == 0), else both NULL
+ *   C        0 (linear cache, row = position) or the ring's rows under g4attn_decode_ring's
+ *            rules (row = position % C)
+ *   out, lse as in g4attn_decode
+ *   workspace / ws_bytes  >= g4attn_decode_int8_workspace_size(B, L, C, cfg), 256-byte aligned
+ * The query stays bf16; the codes are widened to bf16 inside the kernel (exact), each key's
+ * scale multiplies its score and each value's scale its softmax weight.  kv_is_k 0, 1 and 2
+ * are served; at most 8 query heads per kv head (G4ATTN_ERR_UNSUPPORTED otherwise).  codes
+ * must be 16-byte aligned, scales 4-byte aligned.  L = 0 writes out = 0 and lse = -inf.
+ */
+G4ATTN_API size_t g4attn_decode_int8_workspace_size(int B, int L, int C,
+                                                    const g4attn_layer_cfg* cfg);
+G4ATTN_API int g4attn_decode_int8(const g4attn_bf16* q, const int8_t* kcodes,
+                                  const float* kscales, const int8_t* vcodes,
+                                  const float* vscales, int L, int C, g4attn_bf16* out,
+                                  float* lse, void* workspace, size_t ws_bytes, int B,
+                                  const g4attn_layer_cfg* cfg, g4attn_stream_t stream);
+
+/*
  * Decode without a workspace and without allocating (the papers describe no such call;
  * it exists for callers that cannot allocate device memory: plugins whose host framework
  * owns every device allocation and hands them only input and output buffers, and services

@@ -281,6 +281,40 @@ def test_quantize_int8_argument_checks_without_gpu(lib, b):
     assert f(None, None, None, 0, 512, None) == b.G4ATTN_OK                       # empty
 
 
+def test_decode_int8_argument_checks_without_gpu(lib, b):
+    loc = b.LayerCfg(32, 16, 256, 1.0, 1e4, 1024, None, 0)
+    glb = b.LayerCfg(32, 4, 512, 0.25, 1e6)
+    # same split-KV partials as the bf16 decode of the same geometry
+    assert b.g4attn_decode_int8_workspace_size(16, 32768, 0, glb) == \
+        b.g4attn_decode_workspace_size(16, 32768, glb)
+    assert b.g4attn_decode_int8_workspace_size(16, 65536, 1024, loc) == \
+        b.g4attn_decode_ring_workspace_size(16, 65536, 1024, loc)
+    assert b.g4attn_decode_int8_workspace_size(16, 65536, 1000, loc) == 0   # C % 64 != 0
+    Pt, I = ctypes.c_void_p, ctypes.c_int
+    f = lib.g4attn_decode_int8
+    f.restype = I
+    g, lc = glb.c(), loc.c()
+    f.argtypes = [Pt, Pt, Pt, Pt, Pt, I, I, Pt, Pt, Pt, ctypes.c_size_t, I,
+                  ctypes.POINTER(type(g)), Pt]
+    ws = (0x100000, 1 << 30)
+    # keys as values: no value codes; separate values: both codes and scales
+    assert f(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 16, 0, 0x6000, None, *ws, 1,
+             ctypes.byref(g), None) == b.G4ATTN_ERR_INVALID_ARG
+    assert f(0x1000, 0x2000, 0x3000, 0x4000, None, 16, 1024, 0x6000, None, *ws, 1,
+             ctypes.byref(lc), None) == b.G4ATTN_ERR_INVALID_ARG
+    assert f(0x1000, 0x2000, None, None, None, 16, 0, 0x6000, None, *ws, 1,
+             ctypes.byref(g), None) == b.G4ATTN_ERR_INVALID_ARG               # key scales missing
+    assert f(0x1000, 0x2008, 0x3000, None, None, 16, 0, 0x6000, None, *ws, 1,
+             ctypes.byref(g), None) == b.G4ATTN_ERR_MISALIGNED                # codes
+    assert f(0x1000, 0x2000, 0x3002, None, None, 16, 0, 0x6000, None, *ws, 1,
+             ctypes.byref(g), None) == b.G4ATTN_ERR_MISALIGNED                # scales
+    assert f(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 16, 100, 0x6000, None, *ws, 1,
+             ctypes.byref(lc), None) == b.G4ATTN_ERR_INVALID_ARG              # bad ring
+    g16 = b.LayerCfg(32, 2, 512, 0.25, 1e6).c()                               # 16 q heads per kv head
+    assert f(0x1000, 0x2000, 0x3000, None, None, 16, 0, 0x6000, None, *ws, 1,
+             ctypes.byref(g16), None) == b.G4ATTN_ERR_UNSUPPORTED
+
+
 def test_header_compiles_as_plain_c(tmp_path):
     # the boundary is a C ABI: the public header must stand alone in a C99 translation unit
     import shutil
