@@ -54,37 +54,26 @@ constexpr int kBarSM = 1;            // named barrier of the softmax warpgroup
 constexpr int kBarRot = 2;           // named barrier of the rotation warpgroup
 constexpr float kLazyMax = 8.0f;     // log2 units: headroom of the lazy reference max
 
-constexpr int kStageBytes = 8192;    // int8 staging slot: 64 keys x 64 dims of each half
+// I8: the cache holds int8 codes with one fp32 scale per row.  A slot's codes (8 KB: 64-byte
+// rows, 64-byte swizzle) land by TMA in the upper half of its 16 KB ring slot, and the
+// rotation warps widen them in place into the bf16 layout the MMAs read (exact: |code| <=
+// 127 needs 8 bits), so the ring keeps its depth.
+constexpr int kCodeOff = kSlotBytes / 2;   // byte offset of a slot's int8 codes
 
-// I8: the cache holds int8 codes with one fp32 scale per row.  The codes land by TMA in a
-// staging ring (64-byte rows, 64-byte swizzle) and the rotation warps widen them into the
-// bf16 ring slots the MMAs read (exact: |code| <= 127 needs 8 bits), so the ring is shorter
-// (two tiles) to make room for the staging slots.
-template <int NH, bool I8>
+template <int NH>
 struct DecodeCfg {
     static constexpr int NS = 2 * NH;                // N of both MMAs (the pair's B rows)
     static constexpr int HH = NH / 2;                // heads finished by each half of the rows
-    static constexpr int NSLOT = I8 ? 8 : (NH == 8 ? 11 : 10);   // ring slots of 16 KB
-    static constexpr int NSTG = I8 ? 6 : 0;          // int8 staging slots of 8 KB
+    static constexpr int NSLOT = NH == 8 ? 11 : 10;  // ring slots of 16 KB
     static constexpr uint32_t TMEM_COLS = NH == 8 ? 128 : 256;   // 2 S^T + D/128 O^T blocks
 };
 
-template <int NSTG>
-struct DecodeStage {
-    uint8_t stage[NSTG][kStageBytes];
-    uint64_t stage_full[NSTG];         // a staging slot's codes landed
-    uint64_t stage_empty[NSTG];        // the rotation warps have widened it
-};
-template <>
-struct DecodeStage<0> {};
-
-// The MMA operands (ring, side buffers, q, P) must start on 1024-byte boundaries: the
-// 128-byte swizzle of the hardware is a function of the shared-memory address, and the
-// offsets computed here (sw128_offset) assume each tile starts on such a boundary.  The
-// staging base class ends with its barriers, so the ring is aligned explicitly.
-template <int NH, bool I8>
-struct __align__(1024) DecodeSmem : DecodeStage<DecodeCfg<NH, I8>::NSTG> {
-    using C = DecodeCfg<NH, I8>;
+// The MMA operands (ring, side buffers, q, P) start on 1024-byte boundaries: the hardware's
+// 128-byte swizzle is a function of the shared-memory address, and the offsets computed
+// here (sw128_offset) assume each tile starts on such a boundary.
+template <int NH>
+struct __align__(1024) DecodeSmem {
+    using C = DecodeCfg<NH>;
     alignas(1024) uint8_t ring[C::NSLOT][kSlotBytes];
     uint8_t side[2][kSlotBytes];       // turned slot 0 of tiles j & 1 (values = pre-RoPE keys)
     // this CTA's half of the B operand of S^T per slot (NH rows: queries over the first
@@ -171,7 +160,7 @@ constexpr uint32_t kSlotDesc = kSlotBytes >> 4;   // one ring slot, in descripto
 // The q operand copy that tile parity `odd` of rotated slot sb reads.
 __host__ __device__ constexpr int q_copy(int sb, bool odd) { return odd ? (sb == 0 ? 4 : 3) : sb; }
 
-// Sixteen int8 codes (one 16-byte piece of a staging row) as sixteen bf16, exactly: each
+// Sixteen int8 codes (one 16-byte piece of a code row) as sixteen bf16, exactly: each
 // code c is biased to the byte u = c + 128, placed in the low mantissa bits of the fp32
 // 2^23 (0x4B0000uu = 2^23 + u), and 2^23 + 128 is subtracted, which leaves c exact in fp32;
 // its upper half is then c as a bf16 (c needs at most 8 significant bits).
@@ -203,14 +192,14 @@ __device__ __forceinline__ void widen_i8x16(uint4 in, uint4& lo, uint4& hi) {
 template <int D, int NH, int RS, bool I8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ DecodeArgs a) {
-    using C = DecodeCfg<NH, I8>;
+    using C = DecodeCfg<NH>;
     constexpr bool REL = RS > 0;
     static_assert(RS < 2 || (D == 256 && NH == 8), "two relative slots: head_dim 256, NH 8");
     // (the host takes RS = 2 only for G <= 4)
     constexpr int NSB = D / 128;    // slots per tile and tensor
     constexpr int NS = C::NS, HH = C::HH, NSLOT = C::NSLOT;
     extern __shared__ uint8_t smem_raw[];
-    DecodeSmem<NH, I8>& sm = *reinterpret_cast<DecodeSmem<NH, I8>*>(
+    DecodeSmem<NH>& sm = *reinterpret_cast<DecodeSmem<NH>*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const WaitCtl wc{a.wait_limit, a.status};
@@ -242,12 +231,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         mbar_init(&sm.q_free, 1);
         mbar_init(&sm.drain, 1);
-        if constexpr (I8) {
-            for (int i = 0; i < C::NSTG; ++i) {
-                mbar_init(&sm.stage_full[i], 1);
-                mbar_init(&sm.stage_empty[i], 1);
-            }
-        }
         sm.abort = 0;
         fence_mbar_init();
     }
@@ -269,43 +252,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ---------------------------------------------------------------- TMA producer
-        if (I8 && lane == 0) {
-            if constexpr (I8) {
-                // the int8 codes of each slot (rows k: dims [64 sb, 64 sb + 64) of key k; rows
-                // 64 + k: the same dims of the second half) into the staging ring
-                prefetch_tmap(&a.tm_k);
-                if (sep_v) prefetch_tmap(&a.tm_v);
-                uint32_t q = 0;   // staging slots filled so far
-                for (int it = 0; it < n_items && !*abort; ++it) {
-                    const Item w = item_of(a, pair, pr, it);
-                    const int nt = ceil_div(w.k1 - w.k0, kPairKeys);
-                    for (int t = 0; t < nt && !*abort; ++t) {
-                        const int kpos = w.k0 + t * kPairKeys + (int)rank * kTileKeys;
-                        const int key = a.ring > 0 ? kpos % a.ring : kpos;
-                        for (int pass = 0; pass < (sep_v ? 2 : 1) && !*abort; ++pass) {
-                            const CUtensorMap* map = pass ? &a.tm_v : &a.tm_k;
-                            for (int sb = 0; sb < NSB; ++sb) {
-                                const int st = q % C::NSTG;
-                                if (!mbar_wait(&sm.stage_empty[st], ((q / C::NSTG) & 1) ^ 1, wc,
-                                               abort))
-                                    break;
-                                mbar_arrive_expect_tx(&sm.stage_full[st], kStageBytes);
-                                tma_load_4d(sm.stage[st], map, &sm.stage_full[st], sb * 64, w.g,
-                                            key, w.b);
-                                tma_load_4d(sm.stage[st] + kStageBytes / 2, map, &sm.stage_full[st],
-                                            D / 2 + sb * 64, w.g, key, w.b);
-                                ++q;
-                            }
-                        }
-                    }
-                }
-                if (*abort) {
-                    const uint32_t first = q > (uint32_t)C::NSTG ? q - C::NSTG : 0;
-                    for (uint32_t k = first; k < q; ++k)
-                        mbar_wait_drain(&sm.stage_full[k % C::NSTG], (k / C::NSTG) & 1);
-                }
-            }
-        } else if (lane == 0) {
+        if (lane == 0) {
             prefetch_tmap(&a.tm_k);
             if (sep_v) prefetch_tmap(&a.tm_v);
             if (split) prefetch_tmap(&a.tm_vside);
@@ -324,10 +271,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                             const int slot = q % NSLOT;
                             if (!mbar_wait(&sm.empty[slot], ((q / NSLOT) & 1) ^ 1, wc, abort))
                                 break;
-                            mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes);
-                            tma_load_4d(sm.ring[slot], map, &sm.full[slot], sb * 64, w.g, key, w.b);
-                            tma_load_4d(sm.ring[slot] + kBoxBytes, map, &sm.full[slot],
-                                        D / 2 + sb * 64, w.g, key, w.b);
+                            if constexpr (I8) {
+                                // int8 codes: rows k (first half) then 64 + k (second half),
+                                // 64 bytes each, in the slot's upper 8 KB
+                                mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes / 2);
+                                tma_load_4d(sm.ring[slot] + kCodeOff, map, &sm.full[slot], sb * 64,
+                                            w.g, key, w.b);
+                                tma_load_4d(sm.ring[slot] + kCodeOff + kBoxBytes / 2, map,
+                                            &sm.full[slot], D / 2 + sb * 64, w.g, key, w.b);
+                            } else {
+                                mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes);
+                                tma_load_4d(sm.ring[slot], map, &sm.full[slot], sb * 64, w.g, key,
+                                            w.b);
+                                tma_load_4d(sm.ring[slot] + kBoxBytes, map, &sm.full[slot],
+                                            D / 2 + sb * 64, w.g, key, w.b);
+                            }
                             ++q;
                         }
                     }
@@ -789,43 +747,48 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (t == nt - 1 && it + 1 < n_items) prefetch(it + 1);
                 bool got = true;
                 if constexpr (I8) {
-                    // widen the tile's int8 slots into its bf16 ring slots, each once the MMAs
-                    // are done with that ring slot: thread (rk, cp) takes rows rk and 64 + rk
-                    // (the two halves of key rk), dims [32 cp, 32 cp + 32) of the slot.  The
-                    // staging rows are 64 bytes with the 64-byte swizzle (16-byte piece c of
-                    // row r at piece c ^ ((r >> 1) & 3)), conflict-free for 8 consecutive rows.
-                    // Each staging slot goes back to the producer as soon as it is widened (a
-                    // tile can have more slots than the staging ring: separate values at
-                    // head_dim 512 take 8).
+                    // widen the tile's slots in place: thread (rk, cp) takes rows rk and 64 + rk
+                    // (the two halves of key rk), dims [32 cp, 32 cp + 32) of the slot.  Code row
+                    // r sits at kCodeOff + 64 r with the 64-byte swizzle (16-byte piece c at
+                    // piece c ^ ((r >> 1) & 3)), conflict-free for 8 consecutive rows.  The bf16
+                    // rows 64..127 overwrite the codes, so every thread reads its codes of the
+                    // slot before any thread writes.
                     for (int k = 0; k < slots_per_tile && got; ++k) {
                         const uint32_t sq = qk + k;
-                        got = mbar_wait(&sm.stage_full[sq % C::NSTG], (sq / C::NSTG) & 1, wc, abort) &&
-                              mbar_wait(&sm.empty[sq % NSLOT], ((sq / NSLOT) & 1) ^ 1, wc, abort);
-                        if (!group_all(got, kBarRot, 128)) {
-                            got = false;
-                            break;
-                        }
-                        const uint8_t* src = sm.stage[sq % C::NSTG];
-                        uint8_t* dst = sm.ring[sq % NSLOT];
+                        got = mbar_wait(&sm.full[sq % NSLOT], (sq / NSLOT) & 1, wc, abort);
+                        uint8_t* slotp = sm.ring[sq % NSLOT];
+                        uint4 w8[2][2];
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             const int row = 64 * h + rk;
 #pragma unroll
                             for (int c = 0; c < 2; ++c) {
                                 const int piece = 2 * cp + c;   // dims [16 piece, 16 piece + 16)
-                                const uint4 w8 = *reinterpret_cast<const uint4*>(
-                                    src + row * 64 + ((piece ^ ((row >> 1) & 3)) << 4));
-                                uint4 lo, hi;
-                                widen_i8x16(w8, lo, hi);
-                                *reinterpret_cast<uint4*>(dst + sw128_offset(row, 16 * piece)) = lo;
-                                *reinterpret_cast<uint4*>(dst + sw128_offset(row, 16 * piece + 8)) = hi;
+                                w8[h][c] = got ? *reinterpret_cast<const uint4*>(
+                                                     slotp + kCodeOff + row * 64 +
+                                                     ((piece ^ ((row >> 1) & 3)) << 4))
+                                               : make_uint4(0, 0, 0, 0);
                             }
                         }
-                        // every thread's reads of the staging slot are done (and, after the
-                        // last slot, every widened row is in place for the turns below)
-                        group_sync(kBarRot, 128);
-                        if (t128 == 0) mbar_arrive(&sm.stage_empty[sq % C::NSTG]);
+                        if (!group_all(got, kBarRot, 128)) {
+                            got = false;
+                            break;
+                        }
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            const int row = 64 * h + rk;
+#pragma unroll
+                            for (int c = 0; c < 2; ++c) {
+                                const int piece = 2 * cp + c;
+                                uint4 lo, hi;
+                                widen_i8x16(w8[h][c], lo, hi);
+                                *reinterpret_cast<uint4*>(slotp + sw128_offset(row, 16 * piece)) = lo;
+                                *reinterpret_cast<uint4*>(slotp + sw128_offset(row, 16 * piece + 8)) = hi;
+                            }
+                        }
                     }
+                    // every widened row is in place before the turns below read them
+                    got = group_all(got, kBarRot, 128);
                 } else {
                     // the slots with rotated pairs first: they are turned while the rest land
                     // (the relative rotation turns its first slot while its second one lands)
@@ -1035,7 +998,7 @@ __global__ void __launch_bounds__(kCombineThreads)
 
 template <int D, int NH, int RS, bool I8>
 cudaError_t run_decode(const DecodeArgs& a, int grid, cudaStream_t stream) {
-    using Smem = DecodeSmem<NH, I8>;
+    using Smem = DecodeSmem<NH>;
     const size_t smem = sizeof(Smem) + 1024;
     static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "decode shared memory");
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<D, NH, RS, I8>,
