@@ -25,9 +25,10 @@
 // head_dim 512: a 128 x 512 fp32 O fills all 512 TMEM columns, so S borrows columns
 // [128, 256): the softmax warps hold that quarter of O in registers while S lives there.
 //
-// Warp roles (192 threads per CTA): warp 0 TMA producer (both CTAs), warp 1 TMEM owner and,
-// in the leader CTA, the MMA issuer; warps 2..5 prologue / softmax / epilogue.  Every wait
-// is bounded; a CTA that gives up raises the abort flag of both CTAs of its pair.
+// Warp roles (320 threads per CTA): warp 0 TMA producer (both CTAs), warp 1 TMEM owner and,
+// in the leader CTA, the MMA issuer; warps 2..9 prologue / softmax / epilogue, two threads
+// per tile row (each half of the row's score and output columns).  Every wait is bounded; a
+// CTA that gives up raises the abort flag of both CTAs of its pair.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -39,12 +40,13 @@
 namespace g4 {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;
 constexpr int kBM = 128;               // packed query rows per CTA
 constexpr int kBN = 128;               // keys per tile (shared by the pair)
 constexpr int kSlot = 16384;           // ring slot: 64 keys x 128 dims (S) or 128 keys x 64 dims (V)
 constexpr uint32_t kTmemCols = 512;
-constexpr int kBarWG = 1;
+constexpr int kBarWG = 1;               // the eight row warps
+constexpr int kBarPair0 = 2;            // + lane quarter: the two warps of one quarter
 constexpr float kLazyMax = 8.0f;       // log2 units
 
 template <int D>
@@ -85,6 +87,7 @@ struct __align__(1024) PrefillSmem : PrefillPArea<D> {
     uint64_t s_free[2], s_full[2], p_full[2], pv_done[2];
     uint64_t q_full, q_ready, o_done, o1_done, drain;
     uint64_t pro_done;                     // this CTA's prologue is done with its staging area
+    float xchg[2][128];                    // a value of each row from each of its two threads
     uint32_t tmem_base;
     int abort;
 };
@@ -372,17 +375,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else {
         // ------------------------------------ prologue / softmax / correction / epilogue
-        const int t128 = threadIdx.x - 64;
-        const int wq = warp - 2;                  // 0..3 for the row-parallel prologue
-        const int quarter = warp & 3;             // TMEM lane quarter
-        const int row = quarter * 32 + lane;      // this thread's TMEM lane = tile row
+        // Eight warps.  Warps w and w + 4 share TMEM lane quarter w & 3, so the two threads of
+        // tile row r = 32 (w & 3) + lane sit in a pair of warps: thread (row, ch) takes the
+        // row's score columns [64 ch, 64 ch + 64) and output columns [D/2 ch, D/2 ch + D/2).
+        // Both keep the row's reference max (they update it from the same values), and they
+        // agree on it through a shared-memory exchange behind a 64-thread barrier of the pair.
+        const int t256 = threadIdx.x - 64;         // 0..255
+        const int wq = warp - 2;                   // 0..7
+        const int quarter = warp & 3;              // TMEM lane quarter
+        const int ch = wq >> 2;                    // column half of the row
+        const int row = quarter * 32 + lane;       // this thread's TMEM lane = tile row
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int bar_pair = kBarPair0 + quarter;  // the two warps of this lane quarter
         const int G = a.G;
 
         bool ok_pro = true;
         // ---- prologue: QKNorm + RoPE of the 128 packed rows, in place in shared memory.
         // The raw bf16 tile arrived by TMA (row r = token r / G, head r % G, the layout the
-        // MMAs read).  Warp wq turns rows [32 wq, 32 wq + 32) into normalised, rotated fp16
+        // MMAs read).  Warp wq turns rows [16 wq, 16 wq + 16) into normalised, rotated fp16
         // rows, one row at a time across the warp: lane l holds dims [H l, H l + H) and their
         // RoPE partners d/2 + [H l, H l + H), so both members of every rotated pair, their
         // gammas (in registers for the whole tile) and a contiguous run of the row's
@@ -404,13 +414,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float2* const cs_glob = a.rope_cs + (size_t)(a.q_off + pg.m0) * R;
             const bool rot_lane = i0 < R;
             const int lgG = __ffs(G) - 1;          // G divides 128 (host check): a power of two
-            ok_pro = group_all(mbar_wait(&sm.q_full, 0, wc, abort), kBarWG, 128);
+            ok_pro = group_all(mbar_wait(&sm.q_full, 0, wc, abort), kBarWG, 256);
             if (ok_pro) {
                 // NB rows per step, each stage over all of them, so the rows' load, warp-sum
                 // and square-root latencies overlap
                 constexpr int NB = H == 4 ? 8 : 4;
 #pragma unroll 1
-                for (int r0 = wq * 32; r0 < wq * 32 + 32; r0 += NB) {
+                for (int r0 = wq * 16; r0 < wq * 16 + 16; r0 += NB) {
                     float u[NB][H], v[NB][H];
 #pragma unroll
                     for (int j = 0; j < NB; ++j) {
@@ -509,8 +519,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             fence_proxy_async_smem();
-            group_sync(kBarWG, 128);
-            if (t128 == 0) {   // Q ready (and, head_dim 512, S free for tile 0)
+            group_sync(kBarWG, 256);
+            if (t256 == 0) {   // Q ready (and, head_dim 512, S free for tile 0)
                 mbar_arrive_remote(C::SWAP ? &sm.s_free[0] : &sm.q_ready, 0);
                 mbar_arrive(&sm.pro_done);   // the staged (cos, sin) rows are no longer read
             }
@@ -522,220 +532,136 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool row_valid = (row / G) < pg.tq;
         const int t_first = a.q_off + pg.m0, t_last = t_first + pg.tq - 1;
         const float c2 = a.scale_log2;              // > 0 (checked on the host)
+        const int lo_r = a.window > 0 ? kr_r - a.window + 1 : 0;
         // rows past the end of the sequence hold zero queries; a finite reference keeps
         // their (never stored) P finite on the unmasked path
-        float m_ref = row_valid ? -INFINITY : 0.f, l_sum = 0.f;
-        uint32_t o1[C::SWAP ? 128 : 1];
+        float m_ref = row_valid ? -INFINITY : 0.f, l_own = 0.f;
+        // head_dim 512: this thread's 64 columns of the O quarter that S borrows
+        uint32_t o1[C::SWAP ? 64 : 1];
         if constexpr (C::SWAP) {
 #pragma unroll
-            for (int i = 0; i < 128; ++i) o1[i] = 0u;
+            for (int i = 0; i < 64; ++i) o1[i] = 0u;
         }
+        // the row's value of v over both threads of the pair (both read the same two values)
+        auto pair_max = [&](float v) -> float {
+            sm.xchg[ch][row] = v;
+            group_sync(bar_pair, 64);
+            return fmaxf(sm.xchg[0][row], sm.xchg[1][row]);
+        };
         bool ok = ok_pro;
         for (int n = 0; n < ntiles && ok; ++n) {
             const int key0 = (pg.j_lo + n) * kBN;
+            const int keyc = key0 + 64 * ch;        // key of this thread's first column
             if constexpr (C::SWAP) {
                 if (n > 0) {
-                    // O[:, 128..255] leaves TMEM so S(n) can use those columns (block 0 of the
-                    // previous P.V is done; block 1 may still run, it does not touch them)
-                    ok = group_all(mbar_wait(&sm.o1_done, (n - 1) & 1, wc, abort), kBarWG, 128);
+                    // this thread's half of O[:, 128..255] leaves TMEM so S(n) can use those
+                    // columns (block 0 of the previous P.V is done; block 1 may still run, it
+                    // does not touch them)
+                    ok = group_all(mbar_wait(&sm.o1_done, (n - 1) & 1, wc, abort), kBarWG, 256);
                     if (!ok) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) tmem_ld32_nowait(tm_s + c * 32 + lane_off, o1 + c * 32);
+                    tmem_ld32_nowait(tm_s + 64 * ch + lane_off, o1);
+                    tmem_ld32_nowait(tm_s + 64 * ch + 32 + lane_off, o1 + 32);
                     tmem_ld_wait();
                     tc_fence_before();
-                    group_sync(kBarWG, 128);
-                    if (t128 == 0) mbar_arrive_remote(&sm.s_free[0], 0);
+                    group_sync(kBarWG, 256);
+                    if (t256 == 0) mbar_arrive_remote(&sm.s_free[0], 0);
                 }
             }
             const uint32_t sbuf = C::SWAP ? 0u : (uint32_t)(n & 1);
             const uint32_t tm_sn = tm_s + 128 * sbuf;   // this tile's S
             ok = group_all(C::SWAP ? mbar_wait(&sm.s_full[0], n & 1, wc, abort)
                                    : mbar_wait(&sm.s_full[sbuf], (n >> 1) & 1, wc, abort),
-                           kBarWG, 128);
+                           kBarWG, 256);
             if (!ok) break;
             tc_fence_after();
             const bool need_mask = (key0 + kBN - 1 > t_first) ||
                                    (a.window > 0 && key0 <= t_last - a.window);
             float psum = 0.f, alpha = 1.f;
-            const int lo_r = a.window > 0 ? kr_r - a.window + 1 : 0;
-            // fast path: a finite reference max in every row of the warp: one pass over S
-            // with the current reference; for head_dim 256 masked keys (outside the causal
-            // band or the window) are dropped element by element, head_dim 512 (registers
-            // full with the O quarter) takes masked tiles on the two-pass path
-            bool slow = (C::SWAP && need_mask) || !__all_sync(0xffffffffu, m_ref != -INFINITY);
-            bool fresh = false;   // the reference was set from this tile's row max
-            // head_dim 256: P(n) overwrites S(n) in tensor memory, so it waits in registers
-            // (packed pairs) until the pass is known to stand
-            uint32_t pw[C::SWAP ? 1 : 64];
-            // one pass over S with the current reference; MASK: drop keys outside the causal
-            // band or the window element by element (a separate copy of the loop, so unmasked
-            // tiles carry no per-element test)
-            auto one_pass = [&](auto mask_tag, float negm, float& mxr) {
+            // head_dim 256: P(n) waits in registers (packed pairs) until the pass stands, then
+            // overwrites the first 64 columns of S(n) in tensor memory
+            uint32_t pw[C::SWAP ? 1 : 32];
+            // one pass over this thread's 64 scores with reference -negm (log2 units): P
+            // (rounded to the format of V) to the P buffer (head_dim 512) or pw (head_dim 256),
+            // its sum to ps, the largest visible raw score to mxr; MASK drops keys outside the
+            // causal band or the window (a separate copy of the loop, so unmasked tiles test
+            // nothing)
+            auto pass = [&](auto mask_tag, float negm, float& ps, float& mxr) {
                 constexpr bool MASK = decltype(mask_tag)::value;
                 uint32_t sa[32], sb[32];
-                tmem_ld32_nowait(tm_sn + lane_off, sa);
+                tmem_ld32_nowait(tm_sn + 64 * ch + lane_off, sa);
+                tmem_ld32_nowait(tm_sn + 64 * ch + 32 + lane_off, sb);
                 tmem_ld_wait();
 #pragma unroll
-                for (int b = 0; b < 4; ++b) {
-                    uint32_t* cur = (b & 1) ? sb : sa;
-                    uint32_t* nxt = (b & 1) ? sa : sb;
-                    if (b < 3) tmem_ld32_nowait(tm_sn + (b + 1) * 32 + lane_off, nxt);
+                for (int bb = 0; bb < 2; ++bb) {
+                    const uint32_t* cur = bb ? sb : sa;
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
                         float s0 = __uint_as_float(cur[e]), s1 = __uint_as_float(cur[e + 1]);
                         if constexpr (MASK) {
-                            const int j = key0 + b * 32 + e;
-                            if (!(j <= kr_r && j >= lo_r)) s0 = -INFINITY;
-                            if (!(j + 1 <= kr_r && j + 1 >= lo_r)) s1 = -INFINITY;
+                            const int j = keyc + bb * 32 + e;
+                            if (!(row_valid && j <= kr_r && j >= lo_r)) s0 = -INFINITY;
+                            if (!(row_valid && j + 1 <= kr_r && j + 1 >= lo_r)) s1 = -INFINITY;
                         }
                         mxr = fmaxf(mxr, fmaxf(s0, s1));
                         const float p0 = ex2_approx(fmaf(s0, c2, negm));
                         const float p1 = ex2_approx(fmaf(s1, c2, negm));
                         if constexpr (PF16) {
                             w[e / 2] = pack_f16x2(p0, p1);
-                            psum += p0 + p1;
+                            ps += p0 + p1;
                         } else {
                             const __nv_bfloat162 h = __floats2bfloat162_rn(p0, p1);
                             const float2 f = __bfloat1622float2(h);
-                            psum += f.x + f.y;
+                            ps += f.x + f.y;
                             w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
                         }
                     }
                     if constexpr (C::SWAP) {
-                        uint8_t* pb = sm.p[sbuf][b >> 1];
-                        const int col = (b & 1) * 32;
+                        // keys 64 ch .. 64 ch + 63 are P chunk ch
+                        uint8_t* pb = sm.p[0][ch];
 #pragma unroll
                         for (int k = 0; k < 4; ++k)
-                            *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8 * k)) =
+                            *reinterpret_cast<uint4*>(pb + sw128_offset(row, bb * 32 + 8 * k)) =
                                 make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
                     } else {
 #pragma unroll
-                        for (int k = 0; k < 16; ++k) pw[16 * b + k] = w[k];
+                        for (int k = 0; k < 16; ++k) pw[16 * bb + k] = w[k];
                     }
-                    if (b < 3) tmem_ld_wait();
                 }
             };
-            for (;;) {
-            if (slow && !(C::SWAP && need_mask)) {
-                // first tile of a row (or, head_dim 256, a jump of the max): the row max of
-                // the visible scores sets the reference, then the one-pass loop below runs
-                // with it.  A row with no visible key here keeps a -inf reference; its masked
-                // scores give P = 0 whatever the stand-in.
-                auto max_pass = [&](auto mask_tag) -> float {
-                    constexpr bool MASK = decltype(mask_tag)::value;
-                    uint32_t sa[32], sb[32];
-                    float mx = -INFINITY;
-                    tmem_ld32_nowait(tm_sn + lane_off, sa);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int b = 0; b < 4; ++b) {
-                        uint32_t* cur = (b & 1) ? sb : sa;
-                        uint32_t* nxt = (b & 1) ? sa : sb;
-                        if (b < 3) tmem_ld32_nowait(tm_sn + (b + 1) * 32 + lane_off, nxt);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            float sv = __uint_as_float(cur[e]);
-                            if constexpr (MASK) {
-                                const int j = key0 + b * 32 + e;
-                                if (!(j <= kr_r && j >= lo_r)) sv = -INFINITY;
-                            }
-                            mx = fmaxf(mx, sv);
-                        }
-                        if (b < 3) tmem_ld_wait();
-                    }
-                    return mx * c2;
-                };
-                float mx;
-                if constexpr (C::SWAP) mx = max_pass(std::false_type{});   // unmasked here
-                else mx = need_mask ? max_pass(std::true_type{}) : max_pass(std::false_type{});
-                if (!row_valid) mx = -INFINITY;
-                if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
-                    alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
-                    m_ref = mx;
-                }
-                slow = false;
-                fresh = true;
-            }
-            if (!slow) {
+            auto run = [&](float negm, float& ps, float& mxr) {
+                if (need_mask) pass(std::true_type{}, negm, ps, mxr);
+                else pass(std::false_type{}, negm, ps, mxr);
+            };
+            {
+                // one pass with the current reference; the row's largest score over both
+                // threads decides whether the reference moves (it moves only when a score
+                // exceeds it by more than the lazy headroom, or while it is -inf), and then
+                // the pass runs again with the new one
                 float mxr = -INFINITY;
-                const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
-                if (!C::SWAP && need_mask) one_pass(std::true_type{}, negm, mxr);
-                else one_pass(std::false_type{}, negm, mxr);
-                // the reference stays unless this tile's max exceeds it by more than 2^8
-                if (!fresh) {
-                    slow = __any_sync(0xffffffffu, mxr * c2 > m_ref + kLazyMax);
-                    if (slow) psum = 0.f;
-                    // head_dim 256: S is intact (P still in registers): the max pass again
-                    if constexpr (!C::SWAP)
-                        if (slow) continue;
-                }
-            }
-            break;
-            }
-            if constexpr (!C::SWAP) {
-                // P(n) over the first 64 columns of S(n): the A operand of the value product
-#pragma unroll
-                for (int b = 0; b < 4; ++b) tmem_st16_u32(tm_sn + 16 * b + lane_off, pw + 16 * b);
-            }
-            if constexpr (C::SWAP) {   // head_dim 512: masked tiles and jumps of the max
-                if (slow) {
-                    // two passes with masks: row max, then P with a (lazily) updated reference
-                    float mx = -INFINITY;
-    #pragma unroll 1
-                    for (int b = 0; b < 4; ++b) {
-                        uint32_t sv[32];
-                        tmem_ld32_nowait(tm_sn + b * 32 + lane_off, sv);
-                        tmem_ld_wait();
-    #pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int j = key0 + b * 32 + e;
-                            const bool vis = !need_mask || (j <= kr_r && j >= lo_r);
-                            mx = fmaxf(mx, vis ? __uint_as_float(sv[e]) * c2 : -INFINITY);
-                        }
-                    }
-                    if (!row_valid) mx = -INFINITY;
-                    if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
+                run(m_ref == -INFINITY ? 0.f : -m_ref, psum, mxr);
+                const float mx = pair_max(mxr * c2);
+                const bool jump = mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY);
+                // the warps of the pair hold the same rows: the same decision in both
+                if (__any_sync(0xffffffffu, jump)) {
+                    if (jump) {
                         alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
                         m_ref = mx;
                     }
-                    const float negm = (m_ref == -INFINITY) ? 0.f : -m_ref;
-    #pragma unroll 1
-                    for (int b = 0; b < 4; ++b) {
-                        uint32_t sv[32];
-                        tmem_ld32_nowait(tm_sn + b * 32 + lane_off, sv);
-                        tmem_ld_wait();
-                        uint32_t w[16];
-    #pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            float pv[2];
-    #pragma unroll
-                            for (int u = 0; u < 2; ++u) {
-                                const int j = key0 + b * 32 + e + u;
-                                const bool vis = row_valid && (!need_mask || (j <= kr_r && j >= lo_r));
-                                pv[u] = vis ? ex2_approx(fmaf(__uint_as_float(sv[e + u]), c2, negm)) : 0.f;
-                            }
-                            if constexpr (PF16) {
-                                w[e / 2] = pack_f16x2(pv[0], pv[1]);
-                                psum += pv[0] + pv[1];
-                            } else {
-                                const __nv_bfloat162 h = __floats2bfloat162_rn(pv[0], pv[1]);
-                                const float2 f = __bfloat1622float2(h);
-                                psum += f.x + f.y;
-                                w[e / 2] = *reinterpret_cast<const uint32_t*>(&h);
-                            }
-                        }
-                        uint8_t* pb = sm.p[sbuf][b >> 1];
-                        const int col = (b & 1) * 32;
-    #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            *reinterpret_cast<uint4*>(pb + sw128_offset(row, col + 8 * k)) =
-                                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-                    }
+                    psum = 0.f;
+                    run(m_ref == -INFINITY ? 0.f : -m_ref, psum, mxr);
+                    // head_dim 256: P overwrites S columns the partner thread reads
+                    if constexpr (!C::SWAP) group_sync(bar_pair, 64);
                 }
             }
-            l_sum = l_sum * alpha + psum;
+            if constexpr (!C::SWAP) {
+                // P(n) as packed pairs over the first 64 columns of S(n): this thread's 64 keys
+                // are columns [32 ch, 32 ch + 32), the A operand of the value product
+                tmem_st16_u32(tm_sn + 32 * ch + lane_off, pw);
+                tmem_st16_u32(tm_sn + 32 * ch + 16 + lane_off, pw + 16);
+            }
+            l_own = l_own * alpha + psum;
             // correction of the accumulator when a finite reference max moved (rare: a row
             // whose reference was still -inf has an all-zero accumulator); with two S
             // buffers the value product of the tile before may still be running
@@ -744,10 +670,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     *abort = 1;
                 if constexpr (C::SWAP) {
 #pragma unroll
-                    for (int i = 0; i < 128; ++i) o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
+                    for (int i = 0; i < 64; ++i) o1[i] = __float_as_uint(__uint_as_float(o1[i]) * alpha);
                 }
-                for (int c = 0; c < D / 32; ++c) {
-                    if (C::SWAP && c >= 4 && c < 8) continue;   // that quarter is in o1
+                // this thread's output columns [D/2 ch, D/2 ch + D/2) (head_dim 512: less the
+                // quarter in o1)
+                for (int c = (D / 64) * ch; c < (D / 64) * (ch + 1); ++c) {
+                    if (C::SWAP && c >= 4 && c < 8) continue;
                     uint32_t o[32];
                     tmem_ld32_nowait(tm_o + c * 32 + lane_off, o);
                     tmem_ld_wait();
@@ -755,34 +683,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                     tmem_st32_nowait(tm_o + c * 32 + lane_off, o);
                 }
-                tmem_st_wait();
             }
             if constexpr (C::SWAP) {
-                // put O[:, 128..255] back for the P.V product
-#pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_st32_nowait(tm_s + c * 32 + lane_off, o1 + c * 32);
-                tmem_st_wait();
+                // this thread's half of O[:, 128..255] back for the P.V product
+                tmem_st32_nowait(tm_s + 64 * ch + lane_off, o1);
+                tmem_st32_nowait(tm_s + 64 * ch + 32 + lane_off, o1 + 32);
             }
-            if constexpr (!C::SWAP) tmem_st_wait();   // P (and any rescaled O) in TMEM
+            tmem_st_wait();   // P, O quarter and any rescaled O in TMEM
             fence_proxy_async_smem();
             tc_fence_before();
-            group_sync(kBarWG, 128);
-            if (t128 == 0) mbar_arrive_remote(&sm.p_full[sbuf], 0);
+            group_sync(kBarWG, 256);
+            if (t256 == 0) mbar_arrive_remote(&sm.p_full[sbuf], 0);
         }
         // ---- epilogue
         if (ok) {
-            ok = group_all(mbar_wait(&sm.o_done, 0, wc, abort), kBarWG, 128);   // once per CTA
+            ok = group_all(mbar_wait(&sm.o_done, 0, wc, abort), kBarWG, 256);   // once per CTA
         }
         if (ok) {
             tc_fence_after();
+            // the row's sum over both threads (the end-of-tile barrier above ordered the last
+            // exchange's reads before this write)
+            sm.xchg[ch][row] = l_own;
+            group_sync(bar_pair, 64);
+            const float l_sum = sm.xchg[0][row] + sm.xchg[1][row];
             const float inv = l_sum > 0.f ? 1.f / l_sum : 0.f;
             const int h = pg.g * G + row % G;
-            uint16_t* dst = a.out + (((size_t)pg.b * a.T + tok_r) * a.Hq + h) * D;
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32_nowait(tm_o + c * 32 + lane_off, o);
+            uint16_t* dst = a.out + (((size_t)pg.b * a.T + tok_r) * a.Hq + h) * D + (D / 2) * ch;
+            const uint32_t tcol = tm_o + (D / 2) * ch + lane_off;
+            // the next block of O loads while the current one is converted and stored
+            uint32_t oa[32], ob[32];
+            tmem_ld32_nowait(tcol, oa);
+#pragma unroll 1
+            for (int c = 0; c < D / 64; c += 2) {
                 tmem_ld_wait();
-                if (row_valid) {
+                tmem_ld32_nowait(tcol + (c + 1) * 32, ob);
+                auto store = [&](const uint32_t* o, int cc) {
+                    if (!row_valid) return;
                     uint32_t w[16];
 #pragma unroll
                     for (int e = 0; e < 32; e += 2)
@@ -790,11 +726,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                __uint_as_float(o[e + 1]) * inv);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        *reinterpret_cast<uint4*>(dst + c * 32 + 8 * k) =
+                        *reinterpret_cast<uint4*>(dst + cc * 32 + 8 * k) =
                             make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-                }
+                };
+                store(oa, c);
+                tmem_ld_wait();
+                if (c + 2 < D / 64) tmem_ld32_nowait(tcol + (c + 2) * 32, oa);
+                store(ob, c + 1);
             }
-            if (row_valid && a.lse)
+            if (row_valid && a.lse && ch == 0)
                 a.lse[((size_t)pg.b * a.Hq + h) * a.T + tok_r] =
                     l_sum > 0.f ? (m_ref + log2f(l_sum)) * 0.6931471805599453f : -INFINITY;
         }
