@@ -88,6 +88,8 @@ struct __align__(1024) PrefillSmem : PrefillPArea<D> {
     uint64_t q_full, q_ready, o_done, o1_done, drain;
     uint64_t pro_done;                     // this CTA's prologue is done with its staging area
     float xchg[2][128];                    // a value of each row from each of its two threads
+    uint32_t issued;                       // ring positions this CTA's producer filled
+    uint32_t peer_issued;                  // leader only: the same count of the other CTA
     uint32_t tmem_base;
     int abort;
 };
@@ -241,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                          pg.b);
                     }
             }
+            sm.issued = q;   // read at teardown, after __syncthreads
         }
     } else if (warp == 1) {
         // ------------------------------------------------ MMA issuer (leader CTA only)
@@ -741,19 +744,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     // -------------------------------------------------------------------- teardown
-    // A CTA that gave up tells its peer, so the peer's waits end promptly too.
-    __syncthreads();
-    if (*abort && threadIdx.x == 0) {
-        st_shared_remote_u32((const void*)&sm.abort, rank ^ 1u, 1u);
-        // copies this CTA started must land before its shared memory is freed: the query
-        // tile on its own barrier; the key/value slots complete on the pair leader's
-        // barrier, which this CTA cannot observe, so it gives them a settle time (copies
-        // land in microseconds)
-        mbar_wait_drain(&sm.q_full, 0);
-        spin_ns(100000);
+    // A CTA that gave up tells its peer, so the peer's waits end promptly too, and the
+    // other CTA tells the leader how many ring positions it filled.
+    __syncthreads();   // every role is done: neither producer issues another copy
+    if (threadIdx.x == 0) {
+        if (*abort) st_shared_remote_u32((const void*)&sm.abort, rank ^ 1u, 1u);
+        if (!leader) st_shared_remote_u32((const void*)&sm.peer_issued, 0u, sm.issued);
     }
     tc_fence_before();
     cluster_sync();
+    if (*abort && threadIdx.x == 0) {
+        // Every copy either CTA started must land before either frees its shared memory.
+        // The query tile completes on this CTA's own barrier.  The key / value halves of
+        // both CTAs complete on the leader's ring barriers, which the leader settles: a
+        // position filled by one CTA only gets the other half's bytes counted as arrived
+        // (and, if the leader never armed it, is armed first), so every phase completes
+        // exactly when the copies that were issued have landed.  A slot is refilled only
+        // after both halves of its previous position were consumed, so positions below
+        // the last NSLOT have landed already.
+        mbar_wait_drain(&sm.q_full, 0);
+        if (leader) {
+            const uint32_t mine = sm.issued, peer = sm.peer_issued;
+            const uint32_t hi = mine > peer ? mine : peer;
+            const uint32_t lo = hi > (uint32_t)NSLOT ? hi - (uint32_t)NSLOT : 0u;
+            for (uint32_t k = lo; k < hi; ++k) {
+                uint64_t* bar = &sm.full[k % NSLOT];
+                if (k >= mine) {            // only the other CTA filled it
+                    mbar_arrive_expect_tx(bar, 2 * kSlot);
+                    mbar_complete_tx(bar, kSlot);
+                } else if (k >= peer) {     // only the leader filled it
+                    mbar_complete_tx(bar, kSlot);
+                }
+                mbar_wait_drain(bar, (k / NSLOT) & 1);
+            }
+        }
+    }
+    tc_fence_before();
+    cluster_sync();   // the leader's settled copies have landed in both CTAs
     if (leader && warp == 1 && lane == 0) {
         // every MMA of the pair must be complete before either CTA frees its columns
         mma_commit_pair(&sm.drain);
