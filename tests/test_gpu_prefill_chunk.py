@@ -145,7 +145,10 @@ def test_local_chunk_keys_as_values_window():
     (GLOBAL, (0, 700, 1300, 2000), 0, False),
     (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 0, False),
     (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 320, False),
-    (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 320, True)])
+    (workloads.with_layer(LOCAL, window=256), (0, 300, 301, 900, 1500), 320, True),
+    # the 5:1 block's local layer (32 q / 16 kv heads, d 256, window 1024) in its serving
+    # layout: a ring of 1024 rows holding turned keys, then a decode step
+    (workloads.LOCAL_W1024, (0, 1500, 2600, 3000), 1024, True)])
 def test_prompt_in_chunks_matches_the_full_prefill(ly, cuts, ring_rows, rotated):
     # a prompt fed in chunks, each against the cache the previous chunks wrote, gives the
     # full-sequence prefill (the cache rounds the normalised keys to bf16: within the bar)
