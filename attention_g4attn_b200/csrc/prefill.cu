@@ -461,12 +461,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 gu[kk] = a.qk_norm ? __ldg(a.gamma_q + i0 + kk) : 1.f;
                 gv[kk] = a.qk_norm ? __ldg(a.gamma_q + half + i0 + kk) : 1.f;
             }
+            // NB rows per step, each stage over all of them, so the rows' load, warp-sum and
+            // square-root latencies overlap (8 rows at head_dim 256 spill registers beside the
+            // state the next item's epilogue keeps)
+            constexpr int NB = 4;
+            // head_dim 256: the (cos, sin) of the lane's pairs at the warp's first token come
+            // from the table (L2, read before the query wait); from one token to the next they
+            // turn by theta_i <= 1 rad (its cos and sin in fp32; angle addition, at most 15
+            // steps: ~1e-6 rad)
+            const bool turn4 = H == 4 && rot_lane && i0 + 4 <= R;
+            float2 cr[H == 4 ? 4 : 1], stp[H == 4 ? 4 : 1];
+            if constexpr (H == 4) {
+                const int tok0 = (wq * 16) >> lgG;
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) {
+                    cr[kk] = make_float2(1.f, 0.f);
+                    stp[kk] = make_float2(1.f, 0.f);
+                    if (turn4) {
+                        const float th =
+                            exp2f(-(2.f * (float)(i0 + kk) / (float)D) * (float)a.rope.log2_base);
+                        sincosf(th, &stp[kk].y, &stp[kk].x);
+                    }
+                }
+                if (turn4 && tok0 < pq.tq) {
+                    const float4* g = reinterpret_cast<const float4*>(cs_glob + (size_t)tok0 * R + i0);
+                    const float4 lo = __ldg(g), hi = __ldg(g + 1);
+                    cr[0] = make_float2(lo.x, lo.y);
+                    cr[1] = make_float2(lo.z, lo.w);
+                    cr[2] = make_float2(hi.x, hi.y);
+                    cr[3] = make_float2(hi.z, hi.w);
+                }
+            }
             const bool good = group_all(mbar_wait(&sm.q_full, k & 1, wc, abort), kBarWG, 256);
             if (good) {
-                // NB rows per step, each stage over all of them, so the rows' load, warp-sum
-                // and square-root latencies overlap (8 rows at head_dim 256 spill registers
-                // beside the state the next item's epilogue keeps)
-                constexpr int NB = 4;
 #pragma unroll 1
                 for (int r0 = wq * 16; r0 < wq * 16 + 16; r0 += NB) {
                     float u[NB][H], v[NB][H];
@@ -526,14 +553,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             float2 c[H];
                             bool have = false;
                             if constexpr (H == 4) {
-                                if (i0 + 4 <= R) {
-                                    // head_dim 256: the lane's 32 bytes of the table row (L2)
-                                    const float4* g = reinterpret_cast<const float4*>(cs_glob + cso);
-                                    const float4 lo = __ldg(g), hi = __ldg(g + 1);
-                                    c[0] = make_float2(lo.x, lo.y);
-                                    c[1] = make_float2(lo.z, lo.w);
-                                    c[2 % H] = make_float2(hi.x, hi.y);
-                                    c[3 % H] = make_float2(hi.z, hi.w);
+                                if (turn4) {
+#pragma unroll
+                                    for (int kk = 0; kk < 4; ++kk) c[kk] = cr[kk];
                                     have = true;
                                 }
                             }
@@ -563,6 +585,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                             *reinterpret_cast<uint4*>(qv + off) =
                                 make_uint4(pack_f16x2(v[j][0], v[j][1]), pack_f16x2(v[j][2], v[j][3]),
                                            pack_f16x2(v[j][4], v[j][5]), pack_f16x2(v[j][6], v[j][7]));
+                        }
+                        if constexpr (H == 4) {
+                            // the next row's token: one theta_i further
+                            if (((r + 1) >> lgG) != (r >> lgG)) {
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    cr[kk] = make_float2(cr[kk].x * stp[kk].x - cr[kk].y * stp[kk].y,
+                                                         cr[kk].x * stp[kk].y + cr[kk].y * stp[kk].x);
+                            }
                         }
                     }
                 }
@@ -782,6 +813,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int h = pg.g * G + row % G;
                 uint16_t* dst = a.out + (((size_t)pg.b * a.T + tok_r) * a.Hq + h) * D + (D / 2) * ch;
                 const uint32_t tcol = tm_o + (D / 2) * ch + lane_off;
+                const bool out32 = (reinterpret_cast<uintptr_t>(a.out) & 31) == 0;
                 // the next block of O loads while the current one is converted and stored
                 uint32_t oa[32], ob[32];
                 tmem_ld32_nowait(tcol, oa);
@@ -796,10 +828,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int e = 0; e < 32; e += 2)
                             w[e / 2] = pack_bf16x2(__uint_as_float(o[e]) * inv,
                                                    __uint_as_float(o[e + 1]) * inv);
+                        if (out32) {
+                            // whole 32-byte sectors per lane: a row's pieces are 64 B apart
+                            // from the warp's other rows, so 16-byte stores wrote half sectors
+                            st_global_v8(dst + cc * 32, w);
+                            st_global_v8(dst + cc * 32 + 16, w + 8);
+                        } else {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            *reinterpret_cast<uint4*>(dst + cc * 32 + 8 * k) =
-                                make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                            for (int k = 0; k < 4; ++k)
+                                *reinterpret_cast<uint4*>(dst + cc * 32 + 8 * k) =
+                                    make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                        }
                     };
                     store(oa, c);
                     tmem_ld_wait();
