@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (turn4) {
                         const float th =
                             exp2f(-(2.f * (float)(i0 + kk) / (float)D) * (float)a.rope.log2_base);
-                        sincosf(th, &stp[kk].y, &stp[kk].x);
+                        __sincosf(th, &stp[kk].y, &stp[kk].x);
                     }
                 }
                 if (turn4 && tok0 < pq.tq) {
@@ -727,12 +727,48 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (need_mask) pass(std::true_type{}, negm, ps, mxr);
                     else pass(std::false_type{}, negm, ps, mxr);
                 };
-                {
+                // the largest visible raw score of this thread's 64 columns, no exponentials
+                auto scan = [&](auto mask_tag, float& mxr) {
+                    constexpr bool MASK = decltype(mask_tag)::value;
+                    uint32_t sa[32], sb[32];
+                    tmem_ld32_nowait(tm_sn + 64 * ch + lane_off, sa);
+                    tmem_ld32_nowait(tm_sn + 64 * ch + 32 + lane_off, sb);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int bb = 0; bb < 2; ++bb) {
+                        const uint32_t* cur = bb ? sb : sa;
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            float s0 = __uint_as_float(cur[e]);
+                            if constexpr (MASK) {
+                                const int j = keyc + bb * 32 + e;
+                                if (!(row_valid && j <= kr_r && j >= lo_r)) s0 = -INFINITY;
+                            }
+                            mxr = fmaxf(mxr, s0);
+                        }
+                    }
+                };
+                float mxr = -INFINITY;
+                if (C::PERSIST && __any_sync(0xffffffffu, m_ref == -INFINITY)) {
+                    // rows without a reference yet (their first visible keys): the row's largest
+                    // score over both threads first, then one pass with it.  head_dim 256 only:
+                    // there one tile in ten is an item's first; the head_dim-512 loop measured
+                    // slower with the branch
+                    if (need_mask) scan(std::true_type{}, mxr);
+                    else scan(std::false_type{}, mxr);
+                    const float mx = pair_max(mxr * c2);
+                    if (mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY)) {
+                        alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mx);
+                        m_ref = mx;
+                    }
+                    run(m_ref == -INFINITY ? 0.f : -m_ref, psum, mxr);
+                    // head_dim 256: P overwrites S columns the partner thread reads
+                    if constexpr (!C::SWAP) group_sync(bar_pair, 64);
+                } else {
                     // one pass with the current reference; the row's largest score over both
                     // threads decides whether the reference moves (it moves only when a score
                     // exceeds it by more than the lazy headroom, or while it is -inf), and then
                     // the pass runs again with the new one
-                    float mxr = -INFINITY;
                     run(m_ref == -INFINITY ? 0.f : -m_ref, psum, mxr);
                     const float mx = pair_max(mxr * c2);
                     const bool jump = mx > m_ref + kLazyMax || (m_ref == -INFINITY && mx != -INFINITY);
