@@ -752,7 +752,8 @@ def main():
     if not args.no_e2e:
         try:
             with clk.window() as w_e2e:
-                e2e = run_e2e(S, stream, device, steps=min(args.steps, 2))
+                e2e = run_e2e(S, stream, device, steps=max(args.steps, 1),
+                              warmup=min(max(args.warmup, 0), 1))
         except RuntimeError as exc:   # pinned host memory refused
             e2e = {"error": str(exc)[:200]}
     if e2e is not None and "error" not in e2e:
@@ -760,6 +761,7 @@ def main():
         e2e = {"value": replicas.job_rate(flops_step * e2e["steps"], e2e["seconds"], world, 1e12),
                "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
                "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],
+               "warmup": e2e["warmup"],
                "ms_per_step": e2e["seconds"] * 1e3 / e2e["steps"],
                "overlap": "host-to-device copies on one stream, kernels on a second, "
                           "device-to-host copies on a third, ordered per layer by events",
@@ -800,13 +802,15 @@ def main():
     print(json.dumps(line))
 
 
-def run_e2e(S, stream, device, steps):
+def run_e2e(S, stream, device, steps, warmup):
     """The same step through the public API with inputs in pinned host memory: every step
     copies each layer's inputs host->device, runs the layer, and copies its output
     device->host.  Copies in and out run on streams of their own, so layer i+1's inputs and
     layer i-1's output cross PCIe while layer i computes; events order each layer's buffers
     (its inputs are overwritten only after its previous compute, its output only after the
-    previous copy out)."""
+    previous copy out).  Like the device-timed steps: `warmup` untimed steps, then `steps`
+    timed ones between synchronizes (the first timed step's copies have nothing to overlap
+    with; later steps' copies overlap the step before)."""
     import torch
     from attention_g4attn_b200 import binding as b
 
@@ -841,36 +845,42 @@ def run_e2e(S, stream, device, steps):
     in_ready = [torch.cuda.Event() for _ in range(n)]
     computed = [torch.cuda.Event() for _ in range(n)]
     drained = [torch.cuda.Event() for _ in range(n)]
+
+    def run(nsteps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for s in range(nsteps):
+            for i, (hin, din, ho, dout, launch) in enumerate(units):
+                if s > 0:
+                    s_in.wait_event(computed[i])      # the previous step's layer i read its inputs
+                with torch.cuda.stream(s_in):
+                    for h, dv in zip(hin, din):
+                        if h is not None:
+                            dv.copy_(h, non_blocking=True)
+                in_ready[i].record(s_in)
+                stream.wait_event(in_ready[i])
+                if s > 0:
+                    stream.wait_event(drained[i])     # the previous output of layer i is on the host
+                launch()
+                computed[i].record(stream)
+                s_out.wait_event(computed[i])
+                with torch.cuda.stream(s_out):
+                    ho.copy_(dout, non_blocking=True)
+                drained[i].record(s_out)
+        stream.wait_stream(s_in)
+        stream.wait_stream(s_out)
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1) / 1e3
+
+    if warmup > 0:
+        run(warmup)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    s_in.wait_event(e0)
-    s_out.wait_event(e0)
-    for s in range(steps):
-        for i, (hin, din, ho, dout, launch) in enumerate(units):
-            if s > 0:
-                s_in.wait_event(computed[i])      # the previous step's layer i read its inputs
-            with torch.cuda.stream(s_in):
-                for h, dv in zip(hin, din):
-                    if h is not None:
-                        dv.copy_(h, non_blocking=True)
-            in_ready[i].record(s_in)
-            stream.wait_event(in_ready[i])
-            if s > 0:
-                stream.wait_event(drained[i])     # the previous output of layer i is on the host
-            launch()
-            computed[i].record(stream)
-            s_out.wait_event(computed[i])
-            with torch.cuda.stream(s_out):
-                ho.copy_(dout, non_blocking=True)
-            drained[i].record(s_out)
-    stream.wait_stream(s_in)
-    stream.wait_stream(s_out)
-    e1.record(stream)
-    e1.synchronize()
-    secs = e0.elapsed_time(e1) / 1e3
-    return {"seconds": secs, "steps": steps, "h2d": h2d, "d2h": d2h,
+    secs = run(steps)
+    return {"seconds": secs, "steps": steps, "warmup": warmup, "h2d": h2d, "d2h": d2h,
             "wall": time.perf_counter() - t0}
 
 
