@@ -62,9 +62,10 @@ struct PrefillCfg {
     // memory of P buffers goes to the ring (10 slots, 2.5 tiles)
     static constexpr int NSLOT = (D == 512) ? 4 : 10;
     static constexpr uint32_t S_COL = (D == 512) ? 128 : 256;
-    // head_dim 256: two S buffers (columns 256 and 384, S_COL), so the scores of tile n + 1
-    // are computed while the softmax works on tile n; P(n) overwrites the first 64 columns of
+    // head_dim 256: two S buffers (columns 256 and 384), so the scores of tile n + 1 are
+    // computed while the softmax works on tile n; P(n) overwrites the first 64 columns of
     // S(n) as packed bf16 / fp16 and is the tensor-memory A operand of P.V
+    static constexpr int NBUF = (D == 512) ? 1 : 2;
     // head_dim 256: the CTA pair loops over row-tile items (persistent), the ring running on
     // from one item to the next; head_dim 512 takes one item per pair
     static constexpr bool PERSIST = (D == 256);
@@ -87,9 +88,9 @@ struct __align__(1024) PrefillSmem : PrefillPArea<D> {
     uint8_t ring[PrefillCfg<D>::NSLOT][kSlot];
     uint64_t full[PrefillCfg<D>::NSLOT];   // used in the leader: both CTAs' bytes land here
     uint64_t empty[PrefillCfg<D>::NSLOT];  // per CTA, released by the leader's MMA commits
-    // per S buffer (head_dim 256: tile n uses [n & 1]); s_free / p_full / q_ready / o_free
-    // count one arrival per CTA; the once-per-item barriers (q_full, q_ready, q_free, o_done,
-    // o_free) complete one phase per item
+    // per buffer (tile n uses [n % NBUF]); s_free / p_full / q_ready / o_free count one
+    // arrival per CTA; the once-per-item barriers (q_full, q_ready, q_free, o_done, o_free)
+    // complete one phase per item
     uint64_t s_free[2], s_full[2], p_full[2], pv_done[2];
     uint64_t q_full, q_ready, o_done, o1_done, drain;
     uint64_t q_free;                       // the item's score products are done with q
