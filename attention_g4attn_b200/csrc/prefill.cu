@@ -16,9 +16,11 @@
 //   per key tile of 128 keys (causal / sliding-window tiles outside the band are skipped):
 //     S  = Q K^T        M=256 N=128, fp32 in TMEM; rotated 64-dim chunks come from the
 //                       rotated key copy, the others from the pre-RoPE copy
-//     softmax           thread = row: masked row max with a lazy reference (it only moves
-//                       when the tile max exceeds it by more than 2^8), P = exp2 rounded to
-//                       the format of V into shared memory, running sum of the rounded P
+//     softmax           two threads per row: masked row max with a lazy reference (it only
+//                       moves when the tile max exceeds it by more than 2^8), P = exp2
+//                       rounded to the format of V (head_dim 512: into shared memory;
+//                       head_dim 256: into tensor memory over its scores), running sum of the
+//                       rounded P
 //     O += P V          M=256 N=256 per 256-dim block, V read MN-major; V is the pre-RoPE
 //                       key (keys reused as values), the rotated key, or the caller's values
 //   epilogue  O / l -> bf16 rows; lse = (m + log2 l) ln 2
@@ -62,9 +64,9 @@ struct PrefillCfg {
     // memory of P buffers goes to the ring (10 slots, 2.5 tiles)
     static constexpr int NSLOT = (D == 512) ? 4 : 10;
     static constexpr uint32_t S_COL = (D == 512) ? 128 : 256;
-    // head_dim 256: two S buffers (columns 256 and 384), so the scores of tile n + 1 are
-    // computed while the softmax works on tile n; P(n) overwrites the first 64 columns of
-    // S(n) as packed bf16 / fp16 and is the tensor-memory A operand of P.V
+    // head_dim 256: two S buffers (NBUF; columns 256 and 384), so the scores of tile n + 1
+    // are computed while the softmax works on tile n; P(n) overwrites the first 64 columns
+    // of S(n) as packed bf16 / fp16 and is the tensor-memory A operand of P.V
     static constexpr int NBUF = (D == 512) ? 1 : 2;
     // head_dim 256: the CTA pair loops over row-tile items (persistent), the ring running on
     // from one item to the next; head_dim 512 takes one item per pair

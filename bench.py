@@ -41,11 +41,34 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def _code_lines(text):
+    """The lines of a C++ source without its // comments and blank lines (a // inside a
+    string literal, i.e. after an odd number of quotes on the line, is kept)."""
+    out = []
+    for line in text.splitlines():
+        cut = len(line)
+        start = 0
+        while True:
+            i = line.find("//", start)
+            if i < 0:
+                break
+            if line.count('"', 0, i) % 2 == 0:
+                cut = i
+                break
+            start = i + 2
+        code = line[:cut].rstrip()
+        if code.strip():
+            out.append(code)
+    return out
+
+
 def kernel_source_hash():
+    """Hash of the global prefill kernel's code (its sources less comments and blank lines),
+    so that a recorded DRAM-traffic figure stays attached to the code it was measured on."""
     h = hashlib.sha256()
     for name in ("prefill.cu", "sm100.cuh", "kernels.h"):
-        with open(os.path.join(ROOT, "attention_g4attn_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "attention_g4attn_b200", "csrc", name), encoding="utf-8") as f:
+            h.update("\n".join(_code_lines(f.read())).encode())
     return h.hexdigest()[:16]
 
 
