@@ -26,11 +26,11 @@
 //   epilogue  O / l -> bf16 rows; lse = (m + log2 l) ln 2
 // head_dim 512: a 128 x 512 fp32 O fills all 512 TMEM columns, so S borrows columns
 // [128, 256): the softmax warps hold that quarter of O in registers while S lives there.
-// head_dim 256 (the sliding-window layers: a pair's window spans only 9-10 key tiles): the
-// launch holds as many pairs as fit at once, each looping over row-tile items, so a pair
-// pays its set-up once, loads the next item's queries while the current item's last
-// scores are used, and turns them before writing the current output, while the tensor
-// core starts the next item's scores.
+// head_dim 256 (the model's local layers, whose window spans only 9-10 key tiles per pair;
+// causal head_dim-256 launches take the same path): the launch holds as many pairs as fit
+// at once, each looping over row-tile items, so a pair pays its set-up once, loads the next
+// item's queries while the current item's last scores are used, and turns them before
+// writing the current output, while the tensor core starts the next item's scores.
 //
 // Warp roles (320 threads per CTA): warp 0 TMA producer (both CTAs), warp 1 TMEM owner and,
 // in the leader CTA, the MMA issuer; warps 2..9 prologue / softmax / epilogue, two threads
