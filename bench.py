@@ -737,7 +737,9 @@ def main():
                 "clocks": clk.summary(w_roof)}
 
     extra = {}
-    if rank == 0 and not args.no_extras:
+    # single-GPU extras: under N ranks the others would wait at the next reduction while rank 0
+    # ran them
+    if rank == 0 and world == 1 and not args.no_extras:
         def run_extra(name, fn, frac_key, num_key, peak):
             with clk.window() as w:
                 r = fn()
@@ -779,8 +781,14 @@ def main():
                               warmup=min(max(args.warmup, 0), 1))
         except RuntimeError as exc:   # pinned host memory refused
             e2e = {"error": str(exc)[:200]}
+    if e2e is not None:
+        # every rank takes the same reduction, a rank whose leg failed included (as +inf)
+        ok = "error" not in e2e
+        secs = replicas.max_over_ranks([e2e["seconds"] if ok else math.inf], dist, device)[0]
+        if ok and not math.isfinite(secs):
+            e2e = {"error": "the end-to-end leg failed on another rank"}
     if e2e is not None and "error" not in e2e:
-        e2e["seconds"] = replicas.max_over_ranks([e2e["seconds"]], dist, device)[0]
+        e2e["seconds"] = secs
         e2e = {"value": replicas.job_rate(flops_step * e2e["steps"], e2e["seconds"], world, 1e12),
                "unit": "TFLOP/s", "h2d_bytes_per_step": e2e["h2d"],
                "d2h_bytes_per_step": e2e["d2h"], "steps": e2e["steps"],
